@@ -1,0 +1,19 @@
+"""fp64 CPU oracle for the LoRA-adapted linear layer (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg use
+this package.  It shares no code with the CUDA library and imports nothing from it.
+"""
+from .lora_oracle import (  # noqa: F401
+    bf16_round_bits,
+    bf16_to_f64,
+    fp16_to_f64,
+    lora_forward,
+    lora_backward,
+    lora_forward_rows,
+    lora_backward_rows,
+    dequant_blockwise4,
+    quantize_blockwise4,
+    nearest_codes,
+    lora_merge,
+    weight_f64,
+)

@@ -1,0 +1,209 @@
+"""Plain fp64 CPU oracle for the LoRA-adapted linear layer.
+
+TEST INFRASTRUCTURE ONLY.  This module is what the CUDA library is checked against.
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import it; the library (``qlora_linear_b200``) never does, and this module
+imports nothing from the library.
+
+What it computes (the method is exact, so the oracle is the plain definition):
+
+* Forward of a linear layer with a frozen weight ``W:[N,K]`` and a rank-``r``
+  adapter ``A:[r,K]``, ``B:[N,r]`` scaled by ``s = alpha/r``::
+
+      XA = X·Aᵀ                  [M,r]
+      Y  = X·Wᵀ + s·XA·Bᵀ        [M,N]
+
+  The adapter product is bracketed skinny-first, so the ``N×K`` matrix ``B·A`` is
+  never built ("Unsloth vs PyTorch: The ONLY Video You Need to Understand the
+  Difference", transcript 1:35-2:00, on associativity and the skinny adapter).
+* Backward with ``W`` frozen (no ``dW``), derived by hand rather than by autograd
+  (same page, transcript 0:43-1:35; "Unsloth" wiki entry, Theory, second bullet)::
+
+      dYB = dY·B                 [M,r]
+      dX  = dY·W + s·dYB·A       [M,K]
+      dB  = s·dYᵀ·XA             [N,r]
+      dA  = s·dYBᵀ·X             [r,K]
+
+* The 4-bit blockwise weight ("Rev vs unsloth", fused quantized-LoRA paragraph;
+  "Unsloth vs The Stack v2", quantized fine-tuning paragraph): packed codes
+  ``[N, K/2]`` (element ``2j`` in the low nibble, ``2j+1`` in the high nibble),
+  one fp16 absmax per 64 contiguous elements of the row-major weight and a
+  16-entry float32 codebook.  One element dequantizes to
+  ``bf16_rn(fp32_rn(codebook[code] * absmax))``.
+* Merge of the adapter into the weight ("Rev vs unsloth", GGUF export paragraph;
+  "Unsloth vs The Stack v2", merge paragraph): ``W' = W + s·B·A``.
+
+Everything runs in fp64 on the exact values of the bf16 / fp16 / fp32 inputs;
+matrix products use numpy's fp64 ``matmul`` as a library primitive, with no
+blocking or reordering beyond the formulas above.
+
+Parity pins: every function here is pinned by a CPU test against something other
+than itself (brute force on tiny integer inputs, associativity and merge
+invariants, the B = 0 and W = 0 special cases, finite differences, an exhaustive
+codebook round trip).  No function is left unpinned.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# storage types -> fp64 (exact widening)
+# ----------------------------------------------------------------------------
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64, exactly (bf16 is the top half of fp32)."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def fp16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """IEEE half bit patterns (uint16) -> float64, exactly."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def bf16_round_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (8 significant bits, ties to even); uint16 bits.
+
+    Written from the definition: split ``x = m·2^e`` with ``0.5 <= |m| < 1``, keep
+    ``round_half_even(m·2^8)`` and rescale.  Valid for zero and normal values, which
+    is the whole domain this oracle meets (products of fp32 codebook levels and
+    normal fp16 scales); subnormal inputs are rejected.
+    """
+    v = np.asarray(x, dtype=np.float32).astype(np.float64)
+    if not np.all(np.isfinite(v)):
+        raise ValueError("bf16_round_bits: non-finite input")
+    tiny = np.abs(v) < np.float64(np.finfo(np.float32).tiny)
+    if np.any(tiny & (v != 0)):
+        raise ValueError("bf16_round_bits: subnormal input")
+    m, e = np.frexp(v)
+    q = np.rint(m * 256.0)  # numpy rint rounds half to even
+    r = np.ldexp(q, e - 8)
+    r32 = r.astype(np.float32)  # exact: r has <= 8 significant bits
+    if not np.all(np.isfinite(r32)):
+        raise ValueError("bf16_round_bits: overflow")
+    return (r32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# 4-bit blockwise format
+# ----------------------------------------------------------------------------
+
+BLOCK = 64
+
+
+def _unpack_codes(codes: np.ndarray, N: int, K: int) -> np.ndarray:
+    """[N, K/2] packed bytes -> [N, K] codes; element 2j is the low nibble of byte j."""
+    c = np.asarray(codes, dtype=np.uint8).reshape(N, K // 2)
+    out = np.empty((N, K), dtype=np.uint8)
+    out[:, 0::2] = c & 0x0F
+    out[:, 1::2] = c >> 4
+    return out
+
+
+def dequant_blockwise4(codes: np.ndarray, absmax: np.ndarray, codebook: np.ndarray,
+                       N: int, K: int) -> np.ndarray:
+    """Dequantize the 4-bit blockwise weight to bf16 bit patterns ``[N, K]``.
+
+    Element ``(n, k)`` has code ``c`` and lies in block ``b = (n*K + k) // 64`` of the
+    row-major weight; its value is ``bf16_rn(fp32_rn(codebook[c] * absmax[b]))``.
+    The fp64 product of an fp32 level and an fp16 scale is exact, so rounding it to
+    float32 gives the correctly rounded fp32 product.
+    """
+    if K % BLOCK:
+        raise ValueError("K must be a multiple of 64")
+    c = _unpack_codes(codes, N, K)
+    level = np.asarray(codebook, dtype=np.float32).astype(np.float64)[c]
+    scale = fp16_to_f64(np.asarray(absmax).reshape(-1)[: N * K // BLOCK]).reshape(N, K // BLOCK)
+    prod = level * np.repeat(scale, BLOCK, axis=1)
+    return bf16_round_bits(prod.astype(np.float32))
+
+
+def nearest_codes(values: np.ndarray, scales: np.ndarray, codebook: np.ndarray) -> np.ndarray:
+    """Code of the nearest level for each value of each block.
+
+    ``values`` is ``[nblocks, 64]``, ``scales`` (fp64) is ``[nblocks]``.  Each value
+    takes ``argmin_i |v/scale - codebook[i]|``, ties to the lower index; a block
+    whose scale is zero takes code 7 everywhere.
+    """
+    v = np.asarray(values, dtype=np.float64)
+    scale = np.asarray(scales, dtype=np.float64)
+    cb = np.asarray(codebook, dtype=np.float32).astype(np.float64)
+    safe = np.where(scale > 0, scale, 1.0)
+    dist = np.abs(v[..., None] / safe[:, None, None] - cb)
+    code = np.argmin(dist, axis=-1).astype(np.uint8)  # first minimum = lower index
+    code[scale == 0] = 7
+    return code
+
+
+def quantize_blockwise4(W: np.ndarray, codebook: np.ndarray):
+    """Quantize an ``[N, K]`` weight to the 4-bit blockwise format.
+
+    Per block of 64 contiguous elements: ``scale = fp16_rn(max |w|)`` and each
+    element takes its nearest level (:func:`nearest_codes`).
+    Returns ``(codes uint8 [N, K/2], absmax uint16 [N*K/64])``.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    N, K = W.shape
+    if K % BLOCK:
+        raise ValueError("K must be a multiple of 64")
+    blocks = W.reshape(N * K // BLOCK, BLOCK)
+    scale16 = np.max(np.abs(blocks), axis=1).astype(np.float16)
+    code = nearest_codes(blocks, scale16.astype(np.float64), codebook).reshape(N, K)
+    packed = (code[:, 0::2] | (code[:, 1::2] << 4)).astype(np.uint8)
+    return packed, scale16.view(np.uint16)
+
+
+def weight_f64(inputs: dict) -> np.ndarray:
+    """The frozen weight of an input dict as fp64 ``[N, K]`` (dequantized if 4-bit)."""
+    if inputs.get("W") is not None:
+        return bf16_to_f64(inputs["W"])
+    case = inputs["case"]
+    bits = dequant_blockwise4(inputs["codes"], inputs["absmax"], inputs["codebook"], case.N, case.K)
+    return bf16_to_f64(bits)
+
+
+# ----------------------------------------------------------------------------
+# the layer
+# ----------------------------------------------------------------------------
+
+
+def lora_forward(X: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float):
+    """Forward: returns ``(Y, XA)`` with ``XA = X·Aᵀ`` and ``Y = X·Wᵀ + s·XA·Bᵀ`` (fp64)."""
+    X, W, A, B = (np.asarray(t, dtype=np.float64) for t in (X, W, A, B))
+    XA = X @ A.T
+    Y = X @ W.T + s * (XA @ B.T)
+    return Y, XA
+
+
+def lora_backward(dY: np.ndarray, X: np.ndarray, W: np.ndarray, A: np.ndarray,
+                  B: np.ndarray, s: float) -> dict:
+    """Backward with frozen ``W``: returns dict with ``dX, dA, dB`` and the skinny
+    intermediates ``XA = X·Aᵀ``, ``dYB = dY·B`` (all fp64)."""
+    dY, X, W, A, B = (np.asarray(t, dtype=np.float64) for t in (dY, X, W, A, B))
+    XA = X @ A.T
+    dYB = dY @ B
+    dX = dY @ W + s * (dYB @ A)
+    dB = s * (dY.T @ XA)
+    dA = s * (dYB.T @ X)
+    return {"dX": dX, "dA": dA, "dB": dB, "XA": XA, "dYB": dYB}
+
+
+def lora_forward_rows(X_rows: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray,
+                      s: float):
+    """Rows of ``(Y, XA)`` for a subset of the tokens (each output row depends only on
+    its own input row)."""
+    return lora_forward(X_rows, W, A, B, s)
+
+
+def lora_backward_rows(dY_rows: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray,
+                       s: float) -> np.ndarray:
+    """Rows of ``dX`` for a subset of the tokens: ``dX[m] = dY[m]·W + s·(dY[m]·B)·A``."""
+    dY_rows, W, A, B = (np.asarray(t, dtype=np.float64) for t in (dY_rows, W, A, B))
+    return dY_rows @ W + s * ((dY_rows @ B) @ A)
+
+
+def lora_merge(W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:
+    """Merged weight ``W' = W + s·B·A`` (fp64, ``[N, K]``)."""
+    W, A, B = (np.asarray(t, dtype=np.float64) for t in (W, A, B))
+    return W + s * (B @ A)

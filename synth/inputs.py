@@ -1,0 +1,180 @@
+"""Seeded synthetic inputs for the LoRA-adapted linear layer.
+
+Shapes follow the PyTorch ``Linear`` convention used throughout this project:
+``X:[M,K]``, ``W:[N,K]``, ``A:[r,K]``, ``B:[N,r]``, ``dY:[M,N]``.  Every tensor is
+stored the way the library takes it: bf16 tensors as ``uint16`` bit patterns, the
+4-bit weight as packed codes (``uint8 [N, K/2]``, element ``2j`` in the low nibble),
+one fp16 absmax per 64 contiguous elements (``uint16`` bit patterns) and a 16-entry
+float32 codebook.
+
+Value recipe (one seed per case, one independent stream per tensor and per 2^20-element
+chunk, so the result does not depend on the number of worker threads):
+
+* ``X ~ N(0, 1)``, ``dY ~ N(0, 1)``
+* ``W ~ N(0, 1/K)`` (variance ``1/K``)
+* ``A ~ U(-1/sqrt(K), 1/sqrt(K))``
+* ``B ~ N(0, 0.01)`` read as variance 0.01, i.e. standard deviation 0.1
+* 4-bit weight: codes uniform on ``{0..15}``; scale of block ``b`` is
+  ``fp16_rn((1.2 + 0.8 u_b)/sqrt(K))`` with ``u_b ~ U(0,1)``; codebook levels
+  ``(2i - 15)/15`` for ``i = 0..15`` rounded to float32 (16 symmetric levels in
+  ``[-1, 1]``).  With these, the 4-bit weight has rms close to ``1/sqrt(K)``, the
+  same as the bf16 weight.
+
+Every draw is rounded to the storage type (round to nearest even) and nothing else
+happens to it here.
+"""
+from __future__ import annotations
+
+import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+BASE_SEED = 20261202
+_CHUNK = 1 << 20
+
+# tensor ids for the per-tensor random streams
+_TID = {"X": 1, "W": 2, "A": 3, "B": 4, "dY": 5, "codes": 6, "absmax": 7}
+
+
+def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16, nearest-even; returns the uint16 bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    r = ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+    nan = np.isnan(np.ascontiguousarray(x, dtype=np.float32))
+    if nan.any():
+        r[nan] = np.uint16(0x7FC0)
+    return r
+
+
+def f32_from_bf16_bits(b: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to float32 (exact)."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+@dataclasses.dataclass(frozen=True)
+class LoraCase:
+    """One LoRA-linear problem: sizes, format and seed."""
+
+    name: str
+    M: int
+    N: int
+    K: int
+    r: int
+    alpha: float
+    fmt: str  # "bf16" or "block4"
+    seed: int
+    x_seed: int | None = None  # lets two projections share one activation tensor
+
+    @property
+    def s(self) -> float:
+        return float(self.alpha) / float(self.r)
+
+    def with_M(self, M: int) -> "LoraCase":
+        return dataclasses.replace(self, M=M, name=f"{self.name}_M{M}")
+
+
+def _cases() -> dict[str, list[LoraCase]]:
+    b = BASE_SEED
+    c = {}
+    c["c0"] = [LoraCase("c0_tiny", 256, 512, 512, 8, 16.0, "bf16", b + 0)]
+    c["c1"] = [LoraCase("c1_attn", 8192, 4096, 4096, 16, 32.0, "bf16", b + 1)]
+    c["c2"] = [
+        LoraCase("c2_gate", 16384, 14336, 4096, 16, 32.0, "bf16", b + 2, x_seed=b + 2),
+        LoraCase("c2_up", 16384, 14336, 4096, 16, 32.0, "bf16", b + 2 + 100, x_seed=b + 2),
+        LoraCase("c2_down", 16384, 4096, 14336, 16, 32.0, "bf16", b + 2 + 200),
+    ]
+    c["c3"] = [LoraCase("c3_qlora", 8192, 14336, 4096, 16, 32.0, "block4", b + 3)]
+    sweep = []
+    i = 0
+    for fmt in ("bf16", "block4"):
+        for (K, N) in ((8192, 8192), (8192, 28672)):
+            for M in (512, 4096, 16384):
+                for r in (8, 16, 64, 128):
+                    sweep.append(LoraCase(f"c4_{fmt}_K{K}_N{N}_M{M}_r{r}", M, N, K, r, 2.0 * r, fmt,
+                                          b + 4 + 1000 * (i + 1)))
+                    i += 1
+    c["c4"] = sweep
+    return c
+
+
+CONFIGS: dict[str, list[LoraCase]] = _cases()
+
+
+def config_cases(name: str) -> list[LoraCase]:
+    return list(CONFIGS[name])
+
+
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def _fill(shape, seed: int, tid: int, draw) -> np.ndarray:
+    """Fill an array chunk by chunk; chunk i uses stream SeedSequence([seed, tid, i])."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = np.empty(n, dtype=np.uint16)
+    nchunks = (n + _CHUNK - 1) // _CHUNK
+
+    def work(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tid, i])))
+        out[lo:hi] = draw(g, hi - lo)
+
+    if nchunks <= 1:
+        for i in range(nchunks):
+            work(i)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(work, range(nchunks)))
+    return out.reshape(shape)
+
+
+def _normal_bf16(std: float):
+    def draw(g, n):
+        v = g.standard_normal(n, dtype=np.float32)
+        if std != 1.0:
+            v *= np.float32(std)
+        return bf16_bits_from_f32(v)
+    return draw
+
+
+def _uniform_bf16(lo: float, hi: float):
+    def draw(g, n):
+        v = g.random(n, dtype=np.float32) * np.float32(hi - lo) + np.float32(lo)
+        return bf16_bits_from_f32(v)
+    return draw
+
+
+def codebook_levels() -> np.ndarray:
+    """The 16 symmetric levels (2i-15)/15, i = 0..15, rounded to float32."""
+    return np.array([(2 * i - 15) / 15.0 for i in range(16)], dtype=np.float64).astype(np.float32)
+
+
+def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
+    """Draw the inputs of ``case``.  ``want`` limits which tensors are drawn."""
+    M, N, K, r = case.M, case.N, case.K, case.r
+    out: dict = {"case": case}
+    xs = case.x_seed if case.x_seed is not None else case.seed
+    if "X" in want:
+        out["X"] = _fill((M, K), xs, _TID["X"], _normal_bf16(1.0))
+    if "W" in want:
+        if case.fmt == "bf16":
+            out["W"] = _fill((N, K), case.seed, _TID["W"], _normal_bf16(1.0 / np.sqrt(K)))
+        else:
+            assert K % 64 == 0
+            g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([case.seed, _TID["codes"]])))
+            out["codes"] = g.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+            g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([case.seed, _TID["absmax"]])))
+            u = g.random(N * K // 64)
+            out["absmax"] = ((1.2 + 0.8 * u) / np.sqrt(K)).astype(np.float16).view(np.uint16)
+            out["codebook"] = codebook_levels()
+    if "A" in want:
+        a = 1.0 / np.sqrt(K)
+        out["A"] = _fill((r, K), case.seed, _TID["A"], _uniform_bf16(-a, a))
+    if "B" in want:
+        out["B"] = _fill((N, r), case.seed, _TID["B"], _normal_bf16(0.1))
+    if "dY" in want:
+        out["dY"] = _fill((M, N), case.seed, _TID["dY"], _normal_bf16(1.0))
+    return out

@@ -1,0 +1,316 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Each test checks an oracle function against brute force on tiny inputs, a closed
+form, an invariant of the mathematics, or an independent library routine, chosen so
+that a dropped term, a wrong sign or index, a transposed operand or a wrong scale
+fails at least one of them.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from synth import bf16_bits_from_f32, f32_from_bf16_bits
+from synth.inputs import codebook_levels
+
+
+# ---------------------------------------------------------------------------
+# brute force on tiny integer inputs (exact rational arithmetic, pure Python)
+# ---------------------------------------------------------------------------
+
+def _bf_matmul(a, b):
+    return [[sum(a[i][t] * b[t][j] for t in range(len(b))) for j in range(len(b[0]))]
+            for i in range(len(a))]
+
+
+def _bf_T(a):
+    return [list(r) for r in zip(*a)]
+
+
+def _bf_layer(X, W, A, B, dY, s):
+    """Forward and backward by the definition, with Python Fractions, one loop nest
+    per product, no numpy."""
+    M, K, N, r = len(X), len(X[0]), len(W), len(A)
+    # Y[m][n] = sum_k X[m][k] W[n][k] + s * sum_j (sum_k X[m][k] A[j][k]) B[n][j]
+    XA = [[sum(X[m][k] * A[j][k] for k in range(K)) for j in range(r)] for m in range(M)]
+    Y = [[sum(X[m][k] * W[n][k] for k in range(K)) + s * sum(XA[m][j] * B[n][j] for j in range(r))
+          for n in range(N)] for m in range(M)]
+    # L = sum_{m,n} dY[m][n] Y[m][n]; gradients of L by the chain rule written per element
+    dX = [[sum(dY[m][n] * (W[n][k] + s * sum(B[n][j] * A[j][k] for j in range(r)))
+               for n in range(N)) for k in range(K)] for m in range(M)]
+    dA = [[sum(dY[m][n] * s * B[n][j] * X[m][k] for m in range(M) for n in range(N))
+           for k in range(K)] for j in range(r)]
+    dB = [[sum(dY[m][n] * s * XA[m][j] for m in range(M)) for j in range(r)] for n in range(N)]
+    return Y, XA, dX, dA, dB
+
+
+def _ints(rng, shape, lo=-4, hi=5):
+    return rng.integers(lo, hi, size=shape).astype(np.int64)
+
+
+@pytest.mark.parametrize("alpha", [3, 16])
+def test_layer_matches_brute_force_exactly(alpha):
+    rng = np.random.default_rng(11)
+    M, K, N, r = 3, 5, 4, 2
+    X, W, A, B, dY = (_ints(rng, s) for s in [(M, K), (N, K), (r, K), (N, r), (M, N)])
+    s = Fraction(alpha, r)
+    Yb, XAb, dXb, dAb, dBb = _bf_layer(*(t.tolist() for t in (X, W, A, B, dY)), s)
+    Y, XA = O.lora_forward(X, W, A, B, float(s))
+    g = O.lora_backward(dY, X, W, A, B, float(s))
+    # small integers and s = alpha/2: every value is exact in fp64
+    assert np.array_equal(Y, np.array(Yb, dtype=np.float64))
+    assert np.array_equal(XA, np.array(XAb, dtype=np.float64))
+    assert np.array_equal(g["dX"], np.array(dXb, dtype=np.float64))
+    assert np.array_equal(g["dA"], np.array(dAb, dtype=np.float64))
+    assert np.array_equal(g["dB"], np.array(dBb, dtype=np.float64))
+    assert np.array_equal(g["XA"], XA)
+
+
+def test_brute_force_helper_is_a_plain_matmul():
+    # the brute-force forward reduces to a plain product when the adapter is zero
+    rng = np.random.default_rng(3)
+    X, W = _ints(rng, (2, 3)), _ints(rng, (4, 3))
+    Z = [[0, 0]] * 4
+    Yb = _bf_layer(X.tolist(), W.tolist(), [[0, 0, 0]] * 2, Z, [[0] * 4] * 2, 1)[0]
+    assert Yb == _bf_matmul(X.tolist(), _bf_T(W.tolist()))
+
+
+# ---------------------------------------------------------------------------
+# invariants on random fp64 inputs
+# ---------------------------------------------------------------------------
+
+def _rand(rng, M=37, K=48, N=29, r=6):
+    X = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K)) / np.sqrt(K)
+    A = rng.uniform(-1, 1, (r, K)) / np.sqrt(K)
+    B = rng.standard_normal((N, r)) * 0.1
+    dY = rng.standard_normal((M, N))
+    return X, W, A, B, dY
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+def test_associativity_and_merge_invariant():
+    """Bracketed forward equals the unbracketed X·(W + s·B·A)ᵀ, which is also X
+    times the merged weight."""
+    rng = np.random.default_rng(5)
+    X, W, A, B, dY = _rand(rng)
+    s = 2.5
+    Y, _ = O.lora_forward(X, W, A, B, s)
+    naive = X @ (W + s * (B @ A)).T
+    assert _rel(Y, naive) <= 1e-12
+    assert _rel(X @ O.lora_merge(W, A, B, s).T, naive) <= 1e-12
+    # the merged weight against its definition element by element
+    Wm = O.lora_merge(W, A, B, s)
+    n, k = 7, 11
+    assert abs(Wm[n, k] - (W[n, k] + s * sum(B[n, j] * A[j, k] for j in range(A.shape[0])))) < 1e-13
+
+
+def test_b_zero_reduces_to_plain_linear():
+    rng = np.random.default_rng(6)
+    X, W, A, B, dY = _rand(rng)
+    B0 = np.zeros_like(B)
+    s = 2.0
+    Y, XA = O.lora_forward(X, W, A, B0, s)
+    g = O.lora_backward(dY, X, W, A, B0, s)
+    assert np.array_equal(Y, X @ W.T)
+    assert np.array_equal(g["dX"], dY @ W)
+    assert np.array_equal(g["dA"], np.zeros_like(A))
+    # dB does not vanish: it is s·dYᵀ·XA
+    assert np.linalg.norm(g["dB"]) > 0
+    assert _rel(g["dB"], s * np.einsum("mn,mj->nj", dY, X @ A.T)) <= 1e-12
+    # merge with B = 0 gives W back exactly
+    assert np.array_equal(O.lora_merge(W, A, B0, s), W)
+
+
+def test_w_zero_leaves_the_low_rank_path():
+    rng = np.random.default_rng(7)
+    X, W, A, B, dY = _rand(rng)
+    s = 0.75
+    Y, _ = O.lora_forward(X, np.zeros_like(W), A, B, s)
+    assert _rel(Y, X @ (s * B @ A).T) <= 1e-12
+    g = O.lora_backward(dY, X, np.zeros_like(W), A, B, s)
+    assert _rel(g["dX"], dY @ (s * B @ A)) <= 1e-12
+
+
+def test_finite_differences():
+    """L = Σ dY ⊙ Y is linear in X, in A and in B separately, so central
+    differences are exact up to fp64 round-off."""
+    rng = np.random.default_rng(8)
+    M, K, N, r = 3, 5, 4, 2
+    X, W, A, B, dY = _rand(rng, M, K, N, r)
+    s = 1.7
+    g = O.lora_backward(dY, X, W, A, B, s)
+
+    def L(X_, A_, B_):
+        return float(np.sum(dY * O.lora_forward(X_, W, A_, B_, s)[0]))
+
+    h = 1e-3
+    for name, T, grad in (("X", X, g["dX"]), ("A", A, g["dA"]), ("B", B, g["dB"])):
+        fd = np.zeros_like(T)
+        for idx in np.ndindex(T.shape):
+            Tp, Tm = T.copy(), T.copy()
+            Tp[idx] += h
+            Tm[idx] -= h
+            args_p = {"X": X, "A": A, "B": B}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = Tp, Tm
+            fd[idx] = (L(args_p["X"], args_p["A"], args_p["B"]) - L(args_m["X"], args_m["A"], args_m["B"])) / (2 * h)
+        assert _rel(fd, grad) <= 1e-9, name
+
+
+def test_row_sampled_versions_match_full():
+    rng = np.random.default_rng(9)
+    X, W, A, B, dY = _rand(rng)
+    s = 2.0
+    Y, XA = O.lora_forward(X, W, A, B, s)
+    g = O.lora_backward(dY, X, W, A, B, s)
+    rows = np.array([0, 5, 17, 36])
+    Yr, XAr = O.lora_forward_rows(X[rows], W, A, B, s)
+    assert _rel(Yr, Y[rows]) <= 1e-14 and _rel(XAr, XA[rows]) <= 1e-14
+    assert _rel(O.lora_backward_rows(dY[rows], W, A, B, s), g["dX"][rows]) <= 1e-13
+
+
+# ---------------------------------------------------------------------------
+# storage types and the 4-bit format
+# ---------------------------------------------------------------------------
+
+def _bf16_nearest_even_fraction(x: float) -> float:
+    """Nearest bf16 to x (a normal float32) by exact rational comparison of the two
+    neighbouring 8-significant-bit values; ties go to the even significand."""
+    f = Fraction(x)
+    sign = -1 if f < 0 else 1
+    f = abs(f)
+    e = 0
+    while f >= 2:
+        f /= 2
+        e += 1
+    while f < 1:
+        f *= 2
+        e -= 1
+    lo = Fraction(int(f * 128), 128)
+    hi = lo + Fraction(1, 128)
+    dlo, dhi = f - lo, hi - f
+    if dlo < dhi or (dlo == dhi and int(lo * 128) % 2 == 0):
+        q = lo
+    else:
+        q = hi
+    return float(sign * q * Fraction(2) ** e)
+
+
+def test_bf16_rounding_against_exact_rationals_and_torch():
+    rng = np.random.default_rng(10)
+    x = (rng.standard_normal(4000) * np.exp(rng.uniform(-20, 20, 4000))).astype(np.float32)
+    # exact ties: 1 + 2^-8 -> 1 (even), 1 + 3·2^-8 -> 1 + 2^-6 (even), negatives too
+    ties = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 3 * (1 + 2 ** -8), 0.0],
+                    dtype=np.float32)
+    x = np.concatenate([x, ties])
+    bits = O.bf16_round_bits(x)
+    got = f32_from_bf16_bits(bits).astype(np.float64)
+    want = np.array([_bf16_nearest_even_fraction(float(v)) if v != 0 else 0.0 for v in x])
+    assert np.array_equal(got, want)
+    # an independent library path: torch's float32 -> bfloat16 conversion
+    tb = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bits, tb)
+    # the input generator's rounding agrees as well
+    assert np.array_equal(bits, bf16_bits_from_f32(x))
+
+
+def test_codebook_levels_are_correctly_rounded():
+    cb = codebook_levels()
+    assert cb.dtype == np.float32 and cb.shape == (16,)
+    for i, v in enumerate(cb):
+        exact = Fraction(2 * i - 15, 15)
+        # float32 neighbours of the exact level bracket it and v is the nearer one
+        below = np.nextafter(v, np.float32(-np.inf))
+        above = np.nextafter(v, np.float32(np.inf))
+        assert abs(Fraction(float(v)) - exact) <= abs(Fraction(float(below)) - exact)
+        assert abs(Fraction(float(v)) - exact) <= abs(Fraction(float(above)) - exact)
+    assert cb[0] == -1 and cb[15] == 1 and np.array_equal(cb, -cb[::-1])
+
+
+def test_dequant_hand_example_nibble_order_and_blocks():
+    """Two rows of 128 elements: byte j holds element 2j in its low nibble; each row
+    has two 64-element blocks with their own scale."""
+    N, K = 2, 128
+    cb = codebook_levels()
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    codes[0, 0] = 0x2F  # element 0 -> code 15 (+1.0), element 1 -> code 2 (-11/15)
+    codes[1, 40] = 0x70  # row 1, element 80 -> code 0 (-1.0), element 81 -> code 7 (-1/15)
+    scales = np.array([2.0, 4.0, 0.5, 8.0], dtype=np.float16)
+    bits = O.dequant_blockwise4(codes, scales.view(np.uint16), cb, N, K)
+    v = f32_from_bf16_bits(bits)
+    assert v[0, 0] == np.float32(2.0) * cb[15] == 2.0
+    want01 = f32_from_bf16_bits(bf16_bits_from_f32(np.float32(cb[2]) * np.float32(2.0)))
+    assert v[0, 1] == want01
+    assert v[0, 64] == f32_from_bf16_bits(bf16_bits_from_f32(np.float32(cb[0]) * np.float32(4.0)))
+    assert v[1, 80] == -8.0  # block 3 (row 1, second half), scale 8, level -1
+    assert v[1, 81] == f32_from_bf16_bits(bf16_bits_from_f32(cb[7] * np.float32(8.0)))
+    assert v[1, 0] == f32_from_bf16_bits(bf16_bits_from_f32(cb[0] * np.float32(0.5)))
+
+
+def test_dequant_against_torch_float32_product():
+    """Library cross-check: torch multiplies the fp32 level by the fp32 scale and
+    converts to bf16; the oracle's fp64 path must land on the same bits."""
+    rng = np.random.default_rng(12)
+    N, K = 64, 256
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = rng.uniform(1e-3, 30.0, N * K // 64).astype(np.float16)
+    cb = codebook_levels()
+    bits = O.dequant_blockwise4(codes, scales.view(np.uint16), cb, N, K)
+    c = np.empty((N, K), dtype=np.int64)
+    c[:, 0::2] = codes & 15
+    c[:, 1::2] = codes >> 4
+    lv = torch.from_numpy(cb)[torch.from_numpy(c)]
+    sc = torch.from_numpy(scales.astype(np.float32)).repeat_interleave(64).reshape(N, K)
+    tb = (lv * sc).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bits, tb)
+
+
+def test_codebook_round_trip_exhaustive():
+    """For every code and every positive normal fp16 scale, dequantizing and taking
+    the nearest level under the same scale gives the code back."""
+    cb = codebook_levels()
+    e = np.arange(1, 31, dtype=np.uint16)
+    m = np.arange(0, 1024, dtype=np.uint16)
+    sbits = ((e[:, None] << np.uint16(10)) | m[None, :]).reshape(-1)  # all positive normals
+    nS = sbits.size
+    for c in range(16):
+        # one block of 64 per scale, every element carrying code c
+        byte = np.uint8(c | (c << 4))
+        codes = np.full((nS, 32), byte, dtype=np.uint8)
+        bits = O.dequant_blockwise4(codes, sbits, cb, nS, 64)
+        vals = O.bf16_to_f64(bits)
+        back = O.nearest_codes(vals, O.fp16_to_f64(sbits), cb)
+        assert np.all(back == c), c
+
+
+def test_requantize_is_idempotent():
+    rng = np.random.default_rng(13)
+    N, K = 32, 192
+    W = rng.standard_normal((N, K)) / np.sqrt(K)
+    cb = codebook_levels()
+    q1, s1 = O.quantize_blockwise4(W, cb)
+    W1 = O.bf16_to_f64(O.dequant_blockwise4(q1, s1, cb, N, K))
+    q2, s2 = O.quantize_blockwise4(W1, cb)
+    W2 = O.bf16_to_f64(O.dequant_blockwise4(q2, s2, cb, N, K))
+    q3, s3 = O.quantize_blockwise4(W2, cb)
+    assert np.array_equal(q2, q3) and np.array_equal(s2, s3)
+    assert np.array_equal(W2, O.bf16_to_f64(O.dequant_blockwise4(q3, s3, cb, N, K)))
+    # quantization error is bounded by half a level spacing times the scale plus rounding
+    err = np.abs(W1 - W).reshape(-1, 64).max(axis=1)
+    assert np.all(err <= (1 / 15 + 2 ** -7) * O.fp16_to_f64(s1) + 1e-12)
+
+
+def test_zero_block_takes_code_seven():
+    cb = codebook_levels()
+    W = np.zeros((1, 64))
+    q, s = O.quantize_blockwise4(W, cb)
+    assert np.all(q == 0x77) and s[0] == 0
+    # level -1/15 times a zero scale is IEEE negative zero
+    d = O.dequant_blockwise4(q, s, cb, 1, 64)
+    assert np.all(O.bf16_to_f64(d) == 0.0) and np.all(d == 0x8000)
