@@ -1,0 +1,465 @@
+"""Benchmark: fused LoRA-linear forward + hand-derived backward on B200.
+
+One step = forward and backward of every projection of the workload (default: the
+Llama-8B MLP projections gate, up and down at M = 16384 tokens, r = 16, bf16 weight),
+with inputs resident in device memory.  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3] [--impl ours|reference]
+
+Multi-GPU (one process per GPU under torch.distributed.run): data parallel over tokens,
+every rank runs the full per-rank workload (weak scaling) and the adapter gradients dA
+and dB are summed across ranks with NCCL, the layer's one exchange step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LoRA linear fwd+bwd TFLOP/s & tokens/s; % of B200 BF16 tensor peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def workload(name: str):
+    from synth import CONFIGS
+    cases = CONFIGS[name]
+    desc = {
+        "c1": "Llama-8B attention projection, M=8192, K=N=4096, r=16, alpha=32, bf16 weight",
+        "c2": "Llama-8B MLP projections gate+up (K=4096,N=14336) and down (K=14336,N=4096), "
+              "M=16384, r=16, alpha=32, bf16 weight",
+        "c3": "QLoRA 4-bit blockwise weight K=4096 N=14336 (16-level codebook, fp16 absmax per 64), "
+              "M=8192, r=16, alpha=32",
+    }[name]
+    return cases, desc
+
+
+def case_flops(c) -> float:
+    """Algorithmic FLOPs of one forward + backward: 4MNK + 6Mr(N+K)."""
+    return 4.0 * c.M * c.N * c.K + 6.0 * c.M * c.r * (c.N + c.K)
+
+
+def gemm_flops(c) -> tuple[float, float]:
+    """Algorithmic FLOPs of the Y GEMM (2MNK + 2MNr) and of the dX GEMM (2MNK + 2MKr)."""
+    return 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.N * c.r, 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.K * c.r
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_uuid(dev) -> str:
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(dev.index if hasattr(dev, "index") else 0)
+
+
+# ---------------------------------------------------------------------------- oracle leg
+def oracle_sample(cases, tokens: int):
+    """Runs the fp64 oracle (as it stands) on the first `tokens` tokens of every
+    projection; returns (seconds, algorithmic flops of the sample)."""
+    import oracle as O
+    from synth import make_case
+    inputs = [make_case(c.with_M(tokens)) for c in cases]
+    t0 = time.perf_counter()
+    flops = 0.0
+    for inp in inputs:
+        c = inp["case"]
+        W = O.weight_f64(inp)
+        X, A, B, dY = (O.bf16_to_f64(inp[k]) for k in ("X", "A", "B", "dY"))
+        O.lora_forward(X, W, A, B, c.s)
+        O.lora_backward(dY, X, W, A, B, c.s)
+        flops += case_flops(c)
+    return time.perf_counter() - t0, flops
+
+
+def run_reference(args, cases, desc, rank, world):
+    if rank != 0:
+        return 0
+    tokens = args.cpu_tokens
+    for _ in range(args.warmup):
+        oracle_sample(cases, tokens)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        t, flops = oracle_sample(cases, tokens)
+        times.append(t)
+    total = sum(times)
+    val = args.steps * flops / total / 1e12
+    sample = f"first {tokens} tokens of each projection per step (full K and N), fp64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "tokens_per_step": tokens, "projections": [c.name for c in cases]},
+        "tokens_per_s": args.steps * tokens / total,
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- our leg
+def traffic_record():
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "qlora_linear_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def run_ours(args, cases, desc, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import qlora_linear_b200 as q
+    from synth.device import make_case_device
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    # ---- inputs resident in HBM (drawn on the device)
+    layers, data = [], []
+    x_cache = {}
+    for c in cases:
+        want = ["W", "A", "B", "dY"]
+        xkey = c.x_seed if c.x_seed is not None else (c.data_seed if c.data_seed is not None else c.seed)
+        xkey = (xkey, c.M, c.K)
+        if xkey not in x_cache:
+            want.append("X")
+        d = make_case_device(c, dev, rank=rank, want=tuple(want))
+        if "X" in d:
+            x_cache[xkey] = d["X"]
+        d["X"] = x_cache[xkey]
+        if c.fmt == "bf16":
+            W = q.LoraWeight(c.N, c.K, d["W"])
+        else:
+            W = q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
+        layer = q.LoraLinear(W, d["A"], d["B"], c.alpha)
+        layer.workspace(c.M)
+        out = {
+            "Y": torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev),
+            "XA": torch.empty((c.M, c.r), dtype=torch.bfloat16, device=dev),
+            "dX": torch.empty((c.M, c.K), dtype=torch.bfloat16, device=dev),
+            "dA": torch.empty((c.r, c.K), dtype=torch.bfloat16, device=dev),
+            "dB": torch.empty((c.N, c.r), dtype=torch.bfloat16, device=dev),
+        }
+        layers.append(layer)
+        data.append((d, out))
+    torch.cuda.synchronize()
+
+    def step(inputs=None):
+        for i, (layer, (d, o)) in enumerate(zip(layers, data)):
+            X = d["X"] if inputs is None else inputs[i]["X"]
+            dY = d["dY"] if inputs is None else inputs[i]["dY"]
+            layer.forward(X, Y=o["Y"], XA=o["XA"])
+            layer.backward(dY, X, o["XA"], out=(o["dX"], o["dA"], o["dB"]))
+            if world > 1:
+                dist.all_reduce(o["dA"])
+                dist.all_reduce(o["dB"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = q.lora_device_status(layers[0].workspace(cases[0].M))
+    if st != q.LORA_OK:
+        raise RuntimeError("device status after warm-up: " + q.status_string(st))
+
+    # ---- timed region: K steps, device time (CUDA events), max over ranks
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    time.sleep(0.3)
+    q.lora_timing_enable(True)
+    q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
+    q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
+    launches0 = q.lora_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = q.lora_launch_count() - launches0
+    q.lora_timing_enable(False)
+    fwd_ms, fwd_n = q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
+    bwd_ms, bwd_n = q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    for layer, c in zip(layers, cases):
+        st = q.lora_device_status(layer.workspace(c.M))
+        if st != q.LORA_OK:
+            raise RuntimeError("device status after timing: " + q.status_string(st))
+
+    flops_step = sum(case_flops(c) for c in cases)
+    tokens_step = cases[0].M
+    value = world * flops_step / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+
+    # ---- roofline of the dominant kernel (the tcgen05 GEMM: Y and dX launches)
+    gflops = sum(sum(gemm_flops(c)) for c in cases) * args.steps
+    g_ms = fwd_ms + bwd_ms
+    g_launches = fwd_n + bwd_n
+    achieved = gflops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    tr = traffic_record()
+    traffic = None
+    if tr and tr.get("source_hash") == source_hash() and tr.get("workload") == args.workload:
+        traffic = tr.get("bytes_per_launch")
+    roofline = {
+        "kernel": "lora_gemm_kernel (Y and dX GEMMs)",
+        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": achieved / peak if achieved else None, "traffic": traffic,
+        "peak_source": f"{peak_src} bf16 dense, sustained (kernel timed inside a long step)",
+        "launches": g_launches, "avg_launch_ms": g_ms / g_launches if g_launches else None,
+        "gemm_share_of_step": g_ms / (ms * args.steps) if ms > 0 else None,
+    }
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cases, layers, data, step, world, dev)
+
+    # ---- oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, fl = oracle_sample(cases, args.cpu_tokens)
+        cpu = {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"first {args.cpu_tokens} tokens of each projection (full K and N), fp64 numpy oracle, "
+                         f"{t:.1f} s", "tokens_per_s": args.cpu_tokens / t}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, drawn on device)",
+            "config": {"workload": desc, "tokens_per_rank_per_step": tokens_step,
+                       "global_batch_tokens": tokens_step * world, "r": cases[0].r,
+                       "projections": [c.name for c in cases], "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (step working set several GB >> 126 MB)"},
+            "tokens_per_s": world * tokens_step / (ms * 1e-3),
+            "pct_peak_burst": value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+            "pct_peak_sustained": value / world / peak,
+            "peak_source": peak_src,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, cases, layers, data, step, world, dev):
+    """Same metric through the public API with host buffers: each step copies that
+    step's inputs (X, dY and the adapter A, B) from pinned host memory and reads the
+    outputs (Y, dX, dA, dB) back; the frozen weight stays resident."""
+    import torch
+    import torch.distributed as dist
+
+    stream = torch.cuda.current_stream()
+    host_in, host_out, dev_in = [], [], []
+    h2d = d2h = 0
+    seen_x = {}
+    for (d, o) in data:
+        hx = seen_x.get(id(d["X"]))
+        if hx is None:
+            hx = d["X"].cpu().pin_memory()
+            seen_x[id(d["X"])] = hx
+            h2d += hx.numel() * 2
+        hi = {"X": hx, "dY": d["dY"].cpu().pin_memory(), "A": d["A"].cpu().pin_memory(),
+              "B": d["B"].cpu().pin_memory()}
+        h2d += (hi["dY"].numel() + hi["A"].numel() + hi["B"].numel()) * 2
+        host_in.append(hi)
+        dev_in.append({"X": torch.empty_like(d["X"]), "dY": torch.empty_like(d["dY"])})
+        ho = {k: torch.empty(o[k].shape, dtype=o[k].dtype).pin_memory() for k in ("Y", "dX", "dA", "dB")}
+        d2h += sum(v.numel() * 2 for v in ho.values())
+        host_out.append(ho)
+    xdev = {}
+
+    def e2e_step():
+        xdev.clear()
+        for i, (layer, (d, o)) in enumerate(zip(layers, data)):
+            hx = host_in[i]["X"]
+            if id(hx) not in xdev:
+                dev_in[i]["X"].copy_(hx, non_blocking=True)
+                xdev[id(hx)] = dev_in[i]["X"]
+            else:
+                dev_in[i]["X"] = xdev[id(hx)]
+            dev_in[i]["dY"].copy_(host_in[i]["dY"], non_blocking=True)
+            layer.A.copy_(host_in[i]["A"], non_blocking=True)
+            layer.B.copy_(host_in[i]["B"], non_blocking=True)
+        step(inputs=dev_in)
+        for i, (d, o) in enumerate(data):
+            for k in ("Y", "dX", "dA", "dB"):
+                host_out[i][k].copy_(o[k], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    steps = max(3, args.steps // 2)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    flops_step = sum(case_flops(c) for c in cases)
+    return {"value": world * flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+            "note": "inputs X, dY, A, B copied from pinned host memory and Y, dX, dA, dB read back every step; "
+                    "the frozen weight stays resident"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3"])
+    ap.add_argument("--cpu-tokens", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cases, desc = workload(args.workload)
+
+    if args.impl == "reference":
+        return run_reference(args, cases, desc, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, cases, desc, rank, world, local_rank)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

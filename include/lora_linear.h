@@ -1,0 +1,155 @@
+/*
+ * lora_linear.h — C ABI of liblora_linear.so: forward and hand-derived backward of a
+ * LoRA-adapted linear layer over a frozen weight (bf16 or 4-bit blockwise), for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operation.  A linear layer with frozen weight W:[N,K] and a trainable rank-r
+ * adapter A:[r,K], B:[N,r] scaled by s = alpha/r:
+ *
+ *     Y  = X·Wᵀ + s·(X·Aᵀ)·Bᵀ
+ *     dX = dY·W + s·(dY·B)·A        dB = s·dYᵀ·(X·Aᵀ)        dA = s·(dY·B)ᵀ·X
+ *
+ * The fused quantized-weight LoRA product and its replaced backward are described in
+ * "Rev vs unsloth" (fused quantized-LoRA paragraph) and "Unsloth vs The Stack v2"
+ * (LoRA kernel and quantized fine-tuning paragraphs); the hand derivation and the
+ * skinny-first bracketing, which never forms the N×K matrix B·A, in "Unsloth vs
+ * PyTorch: The ONLY Video You Need to Understand the Difference" (transcript
+ * 0:43-2:11).  W is frozen, so there is no dW.
+ *
+ * Conventions for every entry point:
+ *   - Shapes follow PyTorch Linear: X:[M,K], W:[N,K], A:[r,K], B:[N,r], Y:[M,N].  All
+ *     matrices are dense row-major with no padding (row pitch = columns × element size).
+ *   - bf16 means IEEE bfloat16 bit patterns (uint16).  Accumulation is fp32; every
+ *     bf16 output is the round-to-nearest-even of its fp32 value.
+ *   - Pointers named "device" must point to memory of the current CUDA device; the
+ *     library reads them on the GPU.  Pointers marked "host" are read on the CPU.
+ *   - Ownership: the caller owns every buffer.  The library allocates no memory; the
+ *     scratch it needs is the caller's workspace (lora_workspace_bytes()).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return after enqueueing.  Arguments are validated on the host before
+ *     anything is enqueued; on a validation error nothing is enqueued.
+ *   - Device pointers must be 16-byte aligned (LORA_ERR_ALIGNMENT otherwise).
+ *   - Results are deterministic: the same inputs give the same bits on every call.
+ *   - Limits: 8 <= r <= 128 with r % 8 == 0; K % 8 == 0 and N % 8 == 0 (bf16 weight)
+ *     or K % 64 == 0 and N % 8 == 0 (4-bit weight); M >= 0 (M == 0 is an empty batch);
+ *     s finite.  Sizes outside these give LORA_ERR_UNSUPPORTED (r, alignment of sizes)
+ *     or LORA_ERR_INVALID_ARG (negative or zero N/K, non-finite s, NULL pointers).
+ */
+#ifndef LORA_LINEAR_H
+#define LORA_LINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LORA_OK = 0,
+  LORA_ERR_INVALID_ARG = 1,     /* NULL pointer, bad size, non-finite s, bad enum */
+  LORA_ERR_ALIGNMENT = 2,       /* a device pointer is not 16-byte aligned */
+  LORA_ERR_UNSUPPORTED = 3,     /* sizes outside the limits above */
+  LORA_ERR_WORKSPACE = 4,       /* workspace NULL or smaller than lora_workspace_bytes() */
+  LORA_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed (launch error etc.) */
+  LORA_ERR_DEVICE_TIMEOUT = 6   /* a kernel gave up a bounded wait (read with lora_device_status) */
+} lora_status_t;
+
+typedef enum {
+  LORA_W_BF16 = 0,    /* data: bf16 [N,K] */
+  LORA_W_BLOCK4 = 1   /* data: uint8 [N,K/2] codes; absmax: fp16 [N*K/64]; codebook: fp32 [16] */
+} lora_wfmt_t;
+
+/*
+ * Frozen weight, logical shape [N,K], row-major.  All pointers are device pointers.
+ *
+ * LORA_W_BF16:   data = bf16 [N,K]; absmax and codebook are ignored (may be NULL).
+ * LORA_W_BLOCK4: the 4-bit blockwise format ("Rev vs unsloth", fused quantized-LoRA
+ *   paragraph: 4-bit frozen weights; "Unsloth vs The Stack v2", quantized fine-tuning
+ *   paragraph).  data = uint8 [N, K/2]: byte j of row n holds element 2j in its low
+ *   nibble and element 2j+1 in its high nibble (4-bit codes).  absmax = IEEE fp16
+ *   [N*K/64]: scale of block b = elements [64b, 64b+64) of the row-major flattened
+ *   weight (K % 64 == 0, so a block never straddles two rows).  codebook = fp32 [16]
+ *   levels.  Element value = bf16_rn(fp32_rn(codebook[code] * float(absmax[block]))),
+ *   computed as an fp32 multiply (never fused into an FMA) followed by a
+ *   round-to-nearest-even conversion to bf16.
+ */
+typedef struct {
+  int32_t fmt;            /* lora_wfmt_t */
+  int32_t reserved;       /* must be 0 */
+  int64_t N, K;
+  const void* data;
+  const void* absmax;
+  const float* codebook;
+} lora_weight_t;
+
+/*
+ * Bytes of device workspace the forward and backward need for these sizes (the same
+ * buffer serves both).  The workspace must be zero-filled once before its first use
+ * (it holds the device status word read by lora_device_status()); afterwards calls
+ * leave that word alone unless a kernel reports an error.  Returns 0 for invalid sizes.
+ */
+size_t lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int32_t fmt);
+
+/*
+ * Forward.  Computes XA = X·Aᵀ (saved for the backward) and Y = X·Wᵀ + s·XA·Bᵀ.
+ *   X  : device bf16 [M,K]          A : device bf16 [r,K]        B : device bf16 [N,r]
+ *   Y  : device bf16 [M,N] (out)    XA: device bf16 [M,r] (out; pass it to the backward)
+ *   workspace: device, ws_bytes >= lora_workspace_bytes(M, N, K, r, W->fmt).
+ * Y and XA must not overlap any input.  M == 0 enqueues nothing.
+ */
+lora_status_t lora_linear_fwd(const void* X, int64_t M, const lora_weight_t* W,
+                              const void* A, const void* B, int32_t r, float s,
+                              void* Y, void* XA,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Backward with W frozen.  Computes
+ *   dX = dY·W + s·(dY·B)·A   (skipped when dX == NULL, e.g. for a first layer)
+ *   dB = s·dYᵀ·XA            dA = s·(dY·B)ᵀ·X
+ *   dY : device bf16 [M,N]   X : device bf16 [M,K]   XA : device bf16 [M,r] (from the forward)
+ *   dX : device bf16 [M,K] (out, or NULL)   dA : device bf16 [r,K] (out)   dB : device bf16 [N,r] (out)
+ * With M == 0, dA and dB are set to zero.  Outputs must not overlap inputs.
+ */
+lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int64_t M,
+                              const lora_weight_t* W, const void* A, const void* B,
+                              int32_t r, float s,
+                              void* dX, void* dA, void* dB,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Standalone dequantization of a LORA_W_BLOCK4 weight to bf16 [N,K] (device, out),
+ * element by element as defined for lora_weight_t.  Bit-exact.  Not used by the
+ * forward/backward, which dequantize tiles in shared memory and never write a
+ * dequantized weight to device memory.
+ */
+lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* stream);
+
+/*
+ * Merge the adapter into the weight: W_out = W + s·B·A, bf16 [N,K] (device, out),
+ * accumulated in fp32 ("Rev vs unsloth", GGUF export paragraph: merging LoRA adapters
+ * into base weights; "Unsloth vs The Stack v2", merge paragraph).  W may be bf16
+ * (W_out may then alias W->data exactly) or 4-bit (dequantized first, element by
+ * element as in dequant_blockwise4).  A: device bf16 [r,K]; B: device bf16 [N,r].
+ */
+lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, int32_t r,
+                         float s, void* W_out, void* stream);
+
+/*
+ * Reads and clears the device status word in `workspace` (synchronizes `stream`).
+ * Returns LORA_OK, or LORA_ERR_DEVICE_TIMEOUT if a kernel of an earlier call gave up a
+ * bounded wait (its outputs are then undefined), or LORA_ERR_CUDA.
+ */
+lora_status_t lora_device_status(void* workspace, void* stream);
+
+/* Static message for a status code (never NULL). */
+const char* lora_status_string(int32_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t lora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_LINEAR_H */

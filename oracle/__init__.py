@@ -16,4 +16,5 @@ from .lora_oracle import (  # noqa: F401
     nearest_codes,
     lora_merge,
     weight_f64,
+    lora_adapter_grads_sampled,
 )

@@ -207,3 +207,29 @@ def lora_merge(W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndar
     """Merged weight ``W' = W + s·B·A`` (fp64, ``[N, K]``)."""
     W, A, B = (np.asarray(t, dtype=np.float64) for t in (W, A, B))
     return W + s * (B @ A)
+
+
+def lora_adapter_grads_sampled(dY_bits: np.ndarray, X_bits: np.ndarray, A: np.ndarray, B: np.ndarray, s: float,
+                               n_idx: np.ndarray, k_idx: np.ndarray, chunk_rows: int = 2048):
+    """Selected rows of ``dB = s·dYᵀ·XA`` and columns of ``dA = s·dYBᵀ·X`` for large
+    problems, accumulating over the tokens in chunks of ``chunk_rows`` so that only a
+    chunk of ``X``/``dY`` is held in fp64 at a time.
+
+    ``dY_bits`` [M,N] and ``X_bits`` [M,K] are bf16 bit patterns; ``A`` [r,K] and ``B``
+    [N,r] are fp64.  Returns ``(dB[n_idx, :], dA[:, k_idx])``.  Each output element is
+    the same sum over m as in :func:`lora_backward`, split into consecutive chunks.
+    """
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    M = dY_bits.shape[0]
+    r = A.shape[0]
+    dB = np.zeros((len(n_idx), r))
+    dA = np.zeros((r, len(k_idx)))
+    for m0 in range(0, M, chunk_rows):
+        Xc = bf16_to_f64(X_bits[m0:m0 + chunk_rows])
+        dYc = bf16_to_f64(dY_bits[m0:m0 + chunk_rows])
+        XAc = Xc @ A.T
+        dYBc = dYc @ B
+        dB += dYc[:, n_idx].T @ XAc
+        dA += dYBc.T @ Xc[:, k_idx]
+    return s * dB, s * dA

@@ -1,0 +1,207 @@
+"""ctypes binding of liblora_linear.so (include/lora_linear.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (plumbing for device memory and streams);
+their ``data_ptr()`` is passed straight through.  There is no CPU fallback: if the
+library is missing this module raises on import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora_linear.so")
+
+LORA_OK = 0
+LORA_ERR_INVALID_ARG = 1
+LORA_ERR_ALIGNMENT = 2
+LORA_ERR_UNSUPPORTED = 3
+LORA_ERR_WORKSPACE = 4
+LORA_ERR_CUDA = 5
+LORA_ERR_DEVICE_TIMEOUT = 6
+
+LORA_W_BF16 = 0
+LORA_W_BLOCK4 = 1
+
+EXPORTED = (
+    "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
+    "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
+    "lora_testing_bounded_wait", "lora_timing_enable", "lora_timing_read", "lora_launch_count",
+)
+
+
+class LoraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status}: {status_string(status)}")
+
+
+class lora_weight_t(ctypes.Structure):
+    _fields_ = [
+        ("fmt", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("data", ctypes.c_void_p),
+        ("absmax", ctypes.c_void_p),
+        ("codebook", ctypes.c_void_p),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python qlora_linear_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    W = ctypes.POINTER(lora_weight_t)
+    lib.lora_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
+    lib.lora_workspace_bytes.restype = sz
+    lib.lora_linear_fwd.argtypes = [vp, i64, W, vp, vp, i32, f32, vp, vp, vp, sz, vp]
+    lib.lora_linear_fwd.restype = i32
+    lib.lora_linear_bwd.argtypes = [vp, vp, vp, i64, W, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
+    lib.lora_linear_bwd.restype = i32
+    lib.dequant_blockwise4.argtypes = [W, vp, vp]
+    lib.dequant_blockwise4.restype = i32
+    lib.lora_merge.argtypes = [W, vp, vp, i32, f32, vp, vp]
+    lib.lora_merge.restype = i32
+    lib.lora_device_status.argtypes = [vp, vp]
+    lib.lora_device_status.restype = i32
+    lib.lora_status_string.argtypes = [i32]
+    lib.lora_status_string.restype = ctypes.c_char_p
+    lib.lora_version.argtypes = []
+    lib.lora_version.restype = i32
+    lib.lora_testing_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
+    lib.lora_testing_bounded_wait.restype = i32
+    lib.lora_timing_enable.argtypes = [i32]
+    lib.lora_timing_enable.restype = i32
+    lib.lora_timing_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+    lib.lora_timing_read.restype = i32
+    lib.lora_launch_count.argtypes = []
+    lib.lora_launch_count.restype = i64
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.lora_status_string(int(status)).decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != LORA_OK:
+        raise LoraError(st, where)
+
+
+class LoraWeight:
+    """A frozen weight [N, K]: bf16 tensor, or the 4-bit blockwise triple
+    (codes uint8 [N, K/2], absmax fp16 [N*K/64], codebook float32 [16])."""
+
+    def __init__(self, N: int, K: int, data, absmax=None, codebook=None):
+        self.N, self.K = int(N), int(K)
+        self.data, self.absmax, self.codebook = data, absmax, codebook
+        self.fmt = LORA_W_BF16 if absmax is None else LORA_W_BLOCK4
+
+    @classmethod
+    def bf16(cls, w: torch.Tensor) -> "LoraWeight":
+        return cls(w.shape[0], w.shape[1], w)
+
+    @classmethod
+    def block4(cls, codes: torch.Tensor, absmax: torch.Tensor, codebook: torch.Tensor, K: int) -> "LoraWeight":
+        return cls(codes.shape[0], K, codes, absmax, codebook)
+
+    def c_struct(self) -> lora_weight_t:
+        return lora_weight_t(self.fmt, 0, self.N, self.K, _ptr(self.data), _ptr(self.absmax), _ptr(self.codebook))
+
+
+def workspace_bytes(M: int, N: int, K: int, r: int, fmt: int = LORA_W_BF16) -> int:
+    return int(_lib.lora_workspace_bytes(int(M), int(N), int(K), int(r), int(fmt)))
+
+
+def alloc_workspace(M: int, N: int, K: int, r: int, fmt: int = LORA_W_BF16, device=None) -> torch.Tensor:
+    """Zero-filled workspace (the status word at its head must start at zero)."""
+    n = workspace_bytes(M, N, K, r, fmt)
+    if n == 0:
+        raise LoraError(LORA_ERR_UNSUPPORTED, "workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def lora_linear_fwd(X, M: int, W: LoraWeight, A, B, r: int, s: float, Y, XA, workspace, ws_bytes=None,
+                    stream=None) -> None:
+    w = W.c_struct()
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_linear_fwd(_ptr(X), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r), float(s), _ptr(Y),
+                                _ptr(XA), _ptr(workspace), int(nb), _stream(stream)), "lora_linear_fwd")
+
+
+def lora_linear_bwd(dY, X, XA, M: int, W: LoraWeight, A, B, r: int, s: float, dX, dA, dB, workspace, ws_bytes=None,
+                    stream=None) -> None:
+    w = W.c_struct()
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_linear_bwd(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r),
+                                float(s), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), int(nb), _stream(stream)),
+           "lora_linear_bwd")
+
+
+def dequant_blockwise4(Wq: LoraWeight, W_out, stream=None) -> None:
+    w = Wq.c_struct()
+    _check(_lib.dequant_blockwise4(ctypes.byref(w), _ptr(W_out), _stream(stream)), "dequant_blockwise4")
+
+
+def lora_merge(W: LoraWeight, A, B, r: int, s: float, W_out, stream=None) -> None:
+    w = W.c_struct()
+    _check(_lib.lora_merge(ctypes.byref(w), _ptr(A), _ptr(B), int(r), float(s), _ptr(W_out), _stream(stream)),
+           "lora_merge")
+
+
+def lora_device_status(workspace, stream=None) -> int:
+    return int(_lib.lora_device_status(_ptr(workspace), _stream(stream)))
+
+
+def lora_testing_bounded_wait(workspace, limit_ns: int, stream=None) -> int:
+    return int(_lib.lora_testing_bounded_wait(_ptr(workspace), int(limit_ns), _stream(stream)))
+
+
+
+
+LORA_KERNEL_FWD_GEMM = 0
+LORA_KERNEL_BWD_GEMM = 1
+
+
+def lora_timing_enable(on: bool) -> None:
+    _check(_lib.lora_timing_enable(1 if on else 0), "lora_timing_enable")
+
+
+def lora_timing_read(kernel: int) -> tuple[float, int]:
+    """(summed device milliseconds, launches) of one GEMM kind since the last read."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int64(0)
+    _check(_lib.lora_timing_read(int(kernel), ctypes.byref(ms), ctypes.byref(n)), "lora_timing_read")
+    return ms.value, n.value
+
+
+def lora_launch_count() -> int:
+    return int(_lib.lora_launch_count())

@@ -1,0 +1,564 @@
+// lora_api.cu — host side of liblora_linear.so: argument validation, workspace layout,
+// TMA descriptors, kernel launches and the exported C ABI (include/lora_linear.h).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "lora_linear.h"
+#include "lora_linear_profiling.h"
+#include "lora_linear_testing.h"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+#include "skinny.cuh"
+
+namespace lora {
+namespace {
+
+constexpr int kTargetCtas = 296;          // skinny passes: about two waves of 148 SMs
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s bound for every device wait
+constexpr size_t kStatusBytes = 256;      // workspace head: device status word
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("LORA_WAIT_LIMIT_NS");
+    if (e && *e) {
+      const unsigned long long x = std::strtoull(e, nullptr, 10);
+      if (x > 0) return static_cast<uint64_t>(x);
+    }
+    return kDefaultWaitNs;
+  }();
+  return v;
+}
+
+// ---------------------------------------------------------------- measurement hooks
+std::atomic<long long> g_launches{0};
+std::atomic<bool> g_timing_on{false};
+std::mutex g_timing_mu;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_timing[LORA_KERNEL_COUNT];
+
+inline void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+struct TimedRegion {
+  cudaEvent_t a = nullptr, b = nullptr;
+  cudaStream_t st;
+  int kind;
+  TimedRegion(int k, cudaStream_t s) : st(s), kind(k) {
+    if (!g_timing_on.load(std::memory_order_relaxed)) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+      a = b = nullptr;
+      return;
+    }
+    cudaEventRecord(a, st);
+  }
+  ~TimedRegion() {
+    if (!a) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timing[kind].emplace_back(a, b);
+  }
+};
+
+// ---------------------------------------------------------------- split heuristics
+// Pure functions of the sizes, so the workspace size and the summation order are
+// fixed by the problem alone.
+struct Split {
+  int splits;
+  int tiles_per_split;
+};
+Split make_split(int blocks, int tiles) {
+  if (tiles <= 0) return Split{1, 1};
+  int want = cdiv(kTargetCtas, blocks > 0 ? blocks : 1);
+  int cap = tiles / 2 > 1 ? tiles / 2 : 1;
+  int s = want < cap ? want : cap;
+  if (s < 1) s = 1;
+  const int per = cdiv(tiles, s);
+  return Split{cdiv(tiles, per), per};
+}
+Split rowproj_split(long long M, long long Kred) {
+  return make_split(cdiv(M, SK_BM), cdiv(Kred, SK_BK));
+}
+Split colproj_split(long long M, long long Kout) {
+  return make_split(cdiv(Kout, SK_BM), cdiv(M, SK_BK));
+}
+
+struct WsLayout {
+  size_t skinny_off, part_off, total;
+};
+WsLayout ws_layout(long long M, long long N, long long K, int r) {
+  WsLayout w;
+  w.skinny_off = kStatusBytes;
+  const size_t skinny = align256(static_cast<size_t>(M) * r * 2);
+  w.part_off = w.skinny_off + skinny;
+  size_t part = 0;
+  auto upd = [&](size_t b) { part = b > part ? b : part; };
+  upd(static_cast<size_t>(rowproj_split(M, K).splits) * M * r * 4);  // XA
+  upd(static_cast<size_t>(rowproj_split(M, N).splits) * M * r * 4);  // dY·B
+  upd(static_cast<size_t>(colproj_split(M, N).splits) * N * r * 4);  // dB
+  upd(static_cast<size_t>(colproj_split(M, K).splits) * K * r * 4);  // dA
+  w.total = w.part_off + align256(part);
+  return w;
+}
+
+// ---------------------------------------------------------------- device info
+struct DevInfo {
+  int sms = 0;
+  bool attrs_set = false;
+};
+std::mutex g_mu;
+DevInfo g_dev[64];
+
+lora_status_t dev_info(DevInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LORA_ERR_CUDA;
+  }
+  if (!d.attrs_set) {
+    bool ok = true;
+#define SET_SMEM(fn, bytes) ok &= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+    SET_SMEM((lora_gemm_kernel<false, false>), (GemmCfg<false, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_kernel<true, false>), (GemmCfg<true, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_kernel<false, true>), (GemmCfg<false, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_kernel<true, true>), (GemmCfg<true, true>::SMEM_BYTES));
+    SET_SMEM((rowproj_kernel<16, false>), (rowproj_smem_bytes<16, false>()));
+    SET_SMEM((rowproj_kernel<32, false>), (rowproj_smem_bytes<32, false>()));
+    SET_SMEM((rowproj_kernel<64, false>), (rowproj_smem_bytes<64, false>()));
+    SET_SMEM((rowproj_kernel<128, false>), (rowproj_smem_bytes<128, false>()));
+    SET_SMEM((rowproj_kernel<16, true>), (rowproj_smem_bytes<16, true>()));
+    SET_SMEM((rowproj_kernel<32, true>), (rowproj_smem_bytes<32, true>()));
+    SET_SMEM((rowproj_kernel<64, true>), (rowproj_smem_bytes<64, true>()));
+    SET_SMEM((rowproj_kernel<128, true>), (rowproj_smem_bytes<128, true>()));
+    SET_SMEM((colproj_kernel<16>), (colproj_smem_bytes<16>()));
+    SET_SMEM((colproj_kernel<32>), (colproj_smem_bytes<32>()));
+    SET_SMEM((colproj_kernel<64>), (colproj_smem_bytes<64>()));
+    SET_SMEM((colproj_kernel<128>), (colproj_smem_bytes<128>()));
+#undef SET_SMEM
+    if (!ok) return LORA_ERR_CUDA;
+    d.attrs_set = true;
+  }
+  *out = &d;
+  return LORA_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+lora_status_t get_encode() {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && fn) {
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      ok = true;
+    }
+  });
+  return ok ? LORA_OK : LORA_ERR_CUDA;
+}
+
+// Row-major [rows][inner] matrix with row pitch = inner * elem bytes.
+lora_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
+                      uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LORA_OK : LORA_ERR_CUDA;
+}
+lora_status_t tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t bi, uint32_t br) {
+  return tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, rows, bi, br, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+lora_status_t tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t bi, uint32_t br) {
+  return tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, inner, rows, bi, br, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// ---------------------------------------------------------------- validation
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lora_status_t check_weight(const lora_weight_t* W) {
+  if (!W) return LORA_ERR_INVALID_ARG;
+  if (W->fmt != LORA_W_BF16 && W->fmt != LORA_W_BLOCK4) return LORA_ERR_INVALID_ARG;
+  if (W->reserved != 0) return LORA_ERR_INVALID_ARG;
+  if (W->N <= 0 || W->K <= 0) return LORA_ERR_INVALID_ARG;
+  if (W->N > (1LL << 30) || W->K > (1LL << 30)) return LORA_ERR_UNSUPPORTED;
+  if (!W->data) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(W->data)) return LORA_ERR_ALIGNMENT;
+  if (W->N % 8 != 0) return LORA_ERR_UNSUPPORTED;
+  if (W->fmt == LORA_W_BF16) {
+    if (W->K % 8 != 0) return LORA_ERR_UNSUPPORTED;
+  } else {
+    if (W->K % 64 != 0) return LORA_ERR_UNSUPPORTED;
+    if (!W->absmax || !W->codebook) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(W->absmax) || !aligned16(W->codebook)) return LORA_ERR_ALIGNMENT;
+  }
+  return LORA_OK;
+}
+
+lora_status_t check_rank(int r, float s) {
+  if (!std::isfinite(s)) return LORA_ERR_INVALID_ARG;
+  if (r < 8 || r > 128 || r % 8 != 0) return LORA_ERR_UNSUPPORTED;
+  return LORA_OK;
+}
+
+lora_status_t check_ptr(const void* p) {
+  if (!p) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(p)) return LORA_ERR_ALIGNMENT;
+  return LORA_OK;
+}
+
+#define TRY(x)                              \
+  do {                                      \
+    const lora_status_t _st = (x);          \
+    if (_st != LORA_OK) return _st;         \
+  } while (0)
+
+lora_status_t last_launch() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
+
+int finalize_grid(size_t n) {
+  const size_t g = (n + 255) / 256;
+  return static_cast<int>(g < 4096 ? (g > 0 ? g : 1) : 4096);
+}
+
+// ---------------------------------------------------------------- skinny launches
+template <bool Q_T>
+lora_status_t launch_rowproj(const __nv_bfloat16* P, const __nv_bfloat16* Q, float* part, int M, int Kred, int r,
+                             Split sp, cudaStream_t st) {
+  dim3 grid(cdiv(M, SK_BM), sp.splits);
+  if (r <= 16)
+    rowproj_kernel<16, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<16, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+  else if (r <= 32)
+    rowproj_kernel<32, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<32, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+  else if (r <= 64)
+    rowproj_kernel<64, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<64, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+  else
+    rowproj_kernel<128, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<128, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+  count_launch();
+  return last_launch();
+}
+
+lora_status_t launch_colproj(const __nv_bfloat16* P, const __nv_bfloat16* R, float* part, int M, int Kout, int r,
+                             Split sp, cudaStream_t st) {
+  dim3 grid(cdiv(Kout, SK_BM), sp.splits);
+  if (r <= 16)
+    colproj_kernel<16><<<grid, SK_THREADS, colproj_smem_bytes<16>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+  else if (r <= 32)
+    colproj_kernel<32><<<grid, SK_THREADS, colproj_smem_bytes<32>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+  else if (r <= 64)
+    colproj_kernel<64><<<grid, SK_THREADS, colproj_smem_bytes<64>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+  else
+    colproj_kernel<128><<<grid, SK_THREADS, colproj_smem_bytes<128>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+  count_launch();
+  return last_launch();
+}
+
+// ---------------------------------------------------------------- GEMM launch
+template <bool B_MN, bool W4>
+lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
+                          const GemmParams& p, int sms, cudaStream_t st) {
+  using C = GemmCfg<B_MN, W4>;
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, C::BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  {
+    TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
+    lora_gemm_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+  }
+  count_launch();
+  return last_launch();
+}
+
+}  // namespace
+}  // namespace lora
+
+using namespace lora;
+
+extern "C" {
+
+const char* lora_status_string(int32_t status) {
+  switch (status) {
+    case LORA_OK: return "ok";
+    case LORA_ERR_INVALID_ARG: return "invalid argument (null pointer, bad size, non-finite scale or bad enum)";
+    case LORA_ERR_ALIGNMENT: return "a device pointer is not 16-byte aligned";
+    case LORA_ERR_UNSUPPORTED: return "unsupported sizes (need 8<=r<=128, r%8==0, N%8==0, K%8==0; K%64==0 for 4-bit)";
+    case LORA_ERR_WORKSPACE: return "workspace missing or smaller than lora_workspace_bytes()";
+    case LORA_ERR_CUDA: return "a CUDA call failed";
+    case LORA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait; outputs of that call are undefined";
+    default: return "unknown status";
+  }
+}
+
+int32_t lora_version(void) { return 100; }
+
+size_t lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int32_t fmt) {
+  if (M < 0 || N <= 0 || K <= 0 || r < 8 || r > 128 || r % 8) return 0;
+  if (fmt != LORA_W_BF16 && fmt != LORA_W_BLOCK4) return 0;
+  if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 30)) return 0;
+  return ws_layout(M, N, K, r).total;
+}
+
+lora_status_t lora_linear_fwd(const void* X, int64_t M, const lora_weight_t* W, const void* A, const void* B, int32_t r,
+                              float s, void* Y, void* XA, void* workspace, size_t ws_bytes, void* stream) {
+  TRY(check_weight(W));
+  TRY(check_rank(r, s));
+  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
+  TRY(check_ptr(A));
+  TRY(check_ptr(B));
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(X));
+  TRY(check_ptr(Y));
+  TRY(check_ptr(XA));
+  const long long N = W->N, K = W->K;
+  const WsLayout wl = ws_layout(M, N, K, r);
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* sXA = reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off);
+  float* part = reinterpret_cast<float*>(ws + wl.part_off);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+
+  // XA = X·Aᵀ (saved for the backward) and s·XA (the LoRA K block of the GEMM)
+  const Split sp = rowproj_split(M, K);
+  TRY(launch_rowproj<false>(Xb, static_cast<const __nv_bfloat16*>(A), part, static_cast<int>(M), static_cast<int>(K), r,
+                            sp, st));
+  const size_t n = static_cast<size_t>(M) * r;
+  finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, sp.splits, n, s, static_cast<__nv_bfloat16*>(XA), sXA);
+  count_launch();
+  TRY(last_launch());
+
+  // Y = X·Wᵀ + (s·XA)·Bᵀ
+  CUtensorMap ta, tb, te, tf;
+  TRY(tmap_bf16(&ta, X, K, M, 64, 128));
+  TRY(tmap_bf16(&te, sXA, r, M, 64, 128));
+  TRY(tmap_bf16(&tf, B, r, N, 64, 256));
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.Nout = static_cast<int>(N);
+  p.Kred = static_cast<int>(K);
+  p.r = r;
+  p.out = static_cast<__nv_bfloat16*>(Y);
+  p.status = reinterpret_cast<uint32_t*>(ws);
+  p.wait_ns = wait_limit_ns();
+  p.Nw = static_cast<int>(N);
+  p.Kw = static_cast<int>(K);
+  if (W->fmt == LORA_W_BF16) {
+    TRY(tmap_bf16(&tb, W->data, K, N, 64, 256));
+    return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
+  }
+  TRY(tmap_u8(&tb, W->data, K / 2, N, 32, 256));
+  p.absmax = static_cast<const __half*>(W->absmax);
+  p.codebook = W->codebook;
+  return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
+}
+
+lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
+                              const void* A, const void* B, int32_t r, float s, void* dX, void* dA, void* dB,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  TRY(check_weight(W));
+  TRY(check_rank(r, s));
+  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
+  TRY(check_ptr(A));
+  TRY(check_ptr(B));
+  TRY(check_ptr(dA));
+  TRY(check_ptr(dB));
+  const long long N = W->N, K = W->K;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
+    return LORA_OK;
+  }
+  TRY(check_ptr(dY));
+  TRY(check_ptr(X));
+  TRY(check_ptr(XA));
+  if (dX && !aligned16(dX)) return LORA_ERR_ALIGNMENT;
+  const WsLayout wl = ws_layout(M, N, K, r);
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* sdYB = reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off);
+  float* part = reinterpret_cast<float*>(ws + wl.part_off);
+  const auto* dYb = static_cast<const __nv_bfloat16*>(dY);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+
+  // s·(dY·B)  [M, r]
+  {
+    const Split sp = rowproj_split(M, N);
+    TRY(launch_rowproj<true>(dYb, static_cast<const __nv_bfloat16*>(B), part, Mi, Ni, r, sp, st));
+    const size_t n = static_cast<size_t>(M) * r;
+    finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, sp.splits, n, s, nullptr, sdYB);
+    count_launch();
+    TRY(last_launch());
+  }
+  // dB = s·dYᵀ·XA  [N, r]
+  {
+    const Split sp = colproj_split(M, N);
+    TRY(launch_colproj(dYb, static_cast<const __nv_bfloat16*>(XA), part, Mi, Ni, r, sp, st));
+    const size_t n = static_cast<size_t>(N) * r;
+    finalize_cols_kernel<<<finalize_grid(n), 256, 0, st>>>(part, sp.splits, Ni, r, s, 0, static_cast<__nv_bfloat16*>(dB));
+    count_launch();
+    TRY(last_launch());
+  }
+  // dX = dY·W + (s·dY·B)·A
+  if (dX) {
+    CUtensorMap ta, tb, te, tf;
+    TRY(tmap_bf16(&ta, dY, N, M, 64, 128));
+    TRY(tmap_bf16(&te, sdYB, r, M, 64, 128));
+    TRY(tmap_bf16(&tf, A, K, r, 64, 64));
+    GemmParams p{};
+    p.M = Mi;
+    p.Nout = Ki;
+    p.Kred = Ni;
+    p.r = r;
+    p.out = static_cast<__nv_bfloat16*>(dX);
+    p.status = reinterpret_cast<uint32_t*>(ws);
+    p.wait_ns = wait_limit_ns();
+    p.Nw = Ni;
+    p.Kw = Ki;
+    if (W->fmt == LORA_W_BF16) {
+      TRY(tmap_bf16(&tb, W->data, K, N, 64, 64));
+      TRY((launch_gemm<true, false>(ta, tb, te, tf, p, dev->sms, st)));
+    } else {
+      TRY(tmap_u8(&tb, W->data, K / 2, N, 128, 64));
+      p.absmax = static_cast<const __half*>(W->absmax);
+      p.codebook = W->codebook;
+      TRY((launch_gemm<true, true>(ta, tb, te, tf, p, dev->sms, st)));
+    }
+  }
+  // dA = (s·dY·B)ᵀ·X  [r, K], computed as Xᵀ·(s·dY·B) and written transposed
+  {
+    const Split sp = colproj_split(M, K);
+    TRY(launch_colproj(Xb, sdYB, part, Mi, Ki, r, sp, st));
+    const size_t n = static_cast<size_t>(K) * r;
+    finalize_cols_kernel<<<finalize_grid(n), 256, 0, st>>>(part, sp.splits, Ki, r, 1.0f, 1, static_cast<__nv_bfloat16*>(dA));
+    count_launch();
+    TRY(last_launch());
+  }
+  return LORA_OK;
+}
+
+lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* stream) {
+  TRY(check_weight(Wq));
+  if (Wq->fmt != LORA_W_BLOCK4) return LORA_ERR_INVALID_ARG;
+  TRY(check_ptr(W_out));
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  const size_t total = static_cast<size_t>(Wq->N) * Wq->K;
+  const size_t groups = total / 16;
+  size_t grid = (groups + 255) / 256;
+  const size_t cap = static_cast<size_t>(dev->sms) * 8;
+  if (grid > cap) grid = cap;
+  dequant4_kernel<<<static_cast<int>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(Wq->data), static_cast<const __half*>(Wq->absmax), Wq->codebook,
+      static_cast<__nv_bfloat16*>(W_out), total);
+  count_launch();
+  return last_launch();
+}
+
+lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, int32_t r, float s, void* W_out,
+                         void* stream) {
+  TRY(check_weight(W));
+  TRY(check_rank(r, s));
+  TRY(check_ptr(A));
+  TRY(check_ptr(B));
+  TRY(check_ptr(W_out));
+  const bool bf = W->fmt == LORA_W_BF16;
+  if (!bf) {
+    // an output overlapping the packed codes would be read after it is written
+    const uint8_t* c0 = static_cast<const uint8_t*>(W->data);
+    const uint8_t* c1 = c0 + static_cast<size_t>(W->N) * W->K / 2;
+    const uint8_t* o0 = static_cast<const uint8_t*>(W_out);
+    const uint8_t* o1 = o0 + static_cast<size_t>(W->N) * W->K * 2;
+    if (o0 < c1 && c0 < o1) return LORA_ERR_INVALID_ARG;
+  }
+  const size_t smem = static_cast<size_t>(MG_TN * r + r * MG_TK) * sizeof(float);
+  if (cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return LORA_ERR_CUDA;
+  dim3 grid(cdiv(W->K, MG_TK), cdiv(W->N, MG_TN));
+  merge_kernel<<<grid, MG_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+      bf ? static_cast<const __nv_bfloat16*>(W->data) : nullptr, bf ? nullptr : static_cast<const uint8_t*>(W->data),
+      bf ? nullptr : static_cast<const __half*>(W->absmax), bf ? nullptr : W->codebook,
+      static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), static_cast<int>(W->N),
+      static_cast<int>(W->K), r, s, static_cast<__nv_bfloat16*>(W_out));
+  count_launch();
+  return last_launch();
+}
+
+lora_status_t lora_device_status(void* workspace, void* stream) {
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return LORA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LORA_ERR_CUDA;
+  if (word == 0) return LORA_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return LORA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LORA_ERR_CUDA;
+  return (word & kDevErrTimeout) ? LORA_ERR_DEVICE_TIMEOUT : LORA_ERR_CUDA;
+}
+
+lora_status_t lora_testing_bounded_wait(void* workspace, uint64_t limit_ns, void* stream) {
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return LORA_ERR_INVALID_ARG;
+  bounded_wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(workspace), limit_ns);
+  count_launch();
+  return last_launch();
+}
+
+lora_status_t lora_timing_enable(int32_t on) {
+  g_timing_on.store(on != 0);
+  return LORA_OK;
+}
+
+lora_status_t lora_timing_read(int32_t kernel, double* total_ms, int64_t* launches) {
+  if (kernel < 0 || kernel >= LORA_KERNEL_COUNT || !total_ms || !launches) return LORA_ERR_INVALID_ARG;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev;
+  {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    ev.swap(g_timing[kernel]);
+  }
+  double tot = 0.0;
+  bool ok = true;
+  for (auto& pr : ev) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(pr.second) != cudaSuccess || cudaEventElapsedTime(&ms, pr.first, pr.second) != cudaSuccess)
+      ok = false;
+    tot += ms;
+    cudaEventDestroy(pr.first);
+    cudaEventDestroy(pr.second);
+  }
+  *total_ms = tot;
+  *launches = static_cast<int64_t>(ev.size());
+  return ok ? LORA_OK : LORA_ERR_CUDA;
+}
+
+int64_t lora_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

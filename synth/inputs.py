@@ -65,8 +65,9 @@ class LoraCase:
     r: int
     alpha: float
     fmt: str  # "bf16" or "block4"
-    seed: int
-    x_seed: int | None = None  # lets two projections share one activation tensor
+    seed: int                  # stream of A and B (and of X, W, dY unless set below)
+    x_seed: int | None = None  # X stream: lets two projections share one activation tensor
+    data_seed: int | None = None  # W and dY stream (and X if x_seed is None)
 
     @property
     def s(self) -> float:
@@ -88,14 +89,15 @@ def _cases() -> dict[str, list[LoraCase]]:
     ]
     c["c3"] = [LoraCase("c3_qlora", 8192, 14336, 4096, 16, 32.0, "block4", b + 3)]
     sweep = []
-    i = 0
+    g = 0
     for fmt in ("bf16", "block4"):
         for (K, N) in ((8192, 8192), (8192, 28672)):
             for M in (512, 4096, 16384):
+                g += 1
                 for r in (8, 16, 64, 128):
+                    # X, W and dY are shared by the four ranks of one shape and format
                     sweep.append(LoraCase(f"c4_{fmt}_K{K}_N{N}_M{M}_r{r}", M, N, K, r, 2.0 * r, fmt,
-                                          b + 4 + 1000 * (i + 1)))
-                    i += 1
+                                          b + 4 + 1000 * g + r, data_seed=b + 4 + 1000 * g))
     c["c4"] = sweep
     return c
 
@@ -156,17 +158,18 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
     """Draw the inputs of ``case``.  ``want`` limits which tensors are drawn."""
     M, N, K, r = case.M, case.N, case.K, case.r
     out: dict = {"case": case}
-    xs = case.x_seed if case.x_seed is not None else case.seed
+    ds = case.data_seed if case.data_seed is not None else case.seed
+    xs = case.x_seed if case.x_seed is not None else ds
     if "X" in want:
         out["X"] = _fill((M, K), xs, _TID["X"], _normal_bf16(1.0))
     if "W" in want:
         if case.fmt == "bf16":
-            out["W"] = _fill((N, K), case.seed, _TID["W"], _normal_bf16(1.0 / np.sqrt(K)))
+            out["W"] = _fill((N, K), ds, _TID["W"], _normal_bf16(1.0 / np.sqrt(K)))
         else:
             assert K % 64 == 0
-            g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([case.seed, _TID["codes"]])))
+            g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([ds, _TID["codes"]])))
             out["codes"] = g.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
-            g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([case.seed, _TID["absmax"]])))
+            g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([ds, _TID["absmax"]])))
             u = g.random(N * K // 64)
             out["absmax"] = ((1.2 + 0.8 * u) / np.sqrt(K)).astype(np.float16).view(np.uint16)
             out["codebook"] = codebook_levels()
@@ -176,5 +179,5 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
     if "B" in want:
         out["B"] = _fill((N, r), case.seed, _TID["B"], _normal_bf16(0.1))
     if "dY" in want:
-        out["dY"] = _fill((M, N), case.seed, _TID["dY"], _normal_bf16(1.0))
+        out["dY"] = _fill((M, N), ds, _TID["dY"], _normal_bf16(1.0))
     return out

@@ -1,0 +1,122 @@
+"""The C-ABI library loads, exports every symbol the headers declare, and validates
+arguments on the host before touching the GPU (no device needed for these)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import qlora_linear_b200 as q
+from qlora_linear_b200.binding import lora_weight_t
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# fake, never dereferenced device addresses (validation runs before any CUDA call)
+P = 0x10000
+P2 = 0x20000
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M):
+            if m.group(1) not in ("if", "defined"):
+                names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert {"lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4", "lora_merge",
+            "lora_workspace_bytes", "lora_device_status", "lora_status_string"} <= declared
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    assert set(q.EXPORTED) == declared
+
+
+def test_status_strings_and_version():
+    for code in range(7):
+        assert q.status_string(code)
+    assert q.status_string(99) == "unknown status"
+    assert q.lib().lora_version() >= 100
+
+
+def _w(fmt=0, N=512, K=512, data=P, absmax=P, cb=P):
+    return lora_weight_t(fmt, 0, N, K, data, absmax, cb)
+
+
+def fwd(W, M=256, r=8, s=2.0, X=P, A=P, B=P, Y=P, XA=P, ws=P2, nb=1 << 30):
+    return q.lib().lora_linear_fwd(X, M, ctypes.byref(W) if W is not None else None, A, B, r, s, Y, XA, ws, nb, None)
+
+
+def bwd(W, M=256, r=8, s=2.0, dY=P, X=P, XA=P, A=P, B=P, dX=P, dA=P, dB=P, ws=P2, nb=1 << 30):
+    return q.lib().lora_linear_bwd(dY, X, XA, M, ctypes.byref(W) if W is not None else None, A, B, r, s, dX, dA, dB,
+                                   ws, nb, None)
+
+
+@pytest.mark.parametrize("call", [fwd, bwd])
+def test_host_validation_errors(call):
+    assert call(None) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(fmt=7)) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(N=0)) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(K=-8)) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(data=0)) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(data=P + 8)) == q.LORA_ERR_ALIGNMENT
+    assert call(_w(N=513)) == q.LORA_ERR_UNSUPPORTED
+    assert call(_w(K=516)) == q.LORA_ERR_UNSUPPORTED
+    assert call(_w(fmt=1, K=520)) == q.LORA_ERR_UNSUPPORTED       # 4-bit needs K % 64
+    assert call(_w(fmt=1, absmax=0)) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(fmt=1, cb=P + 4)) == q.LORA_ERR_ALIGNMENT
+    for r in (0, 4, 12, 136, 256):
+        assert call(_w(), r=r) == q.LORA_ERR_UNSUPPORTED, r
+    assert call(_w(), s=float("nan")) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(), s=float("inf")) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(), M=-1) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(), A=0) == q.LORA_ERR_INVALID_ARG
+    assert call(_w(), B=P + 2) == q.LORA_ERR_ALIGNMENT
+    assert call(_w(), ws=0) == q.LORA_ERR_WORKSPACE
+    assert call(_w(), ws=P2 + 4) == q.LORA_ERR_ALIGNMENT
+    assert call(_w(), nb=q.workspace_bytes(256, 512, 512, 8) - 1) == q.LORA_ERR_WORKSPACE
+
+
+def test_forward_specific_validation():
+    assert fwd(_w(), X=0) == q.LORA_ERR_INVALID_ARG
+    assert fwd(_w(), Y=P + 6) == q.LORA_ERR_ALIGNMENT
+    assert fwd(_w(), XA=0) == q.LORA_ERR_INVALID_ARG
+    # an empty batch is valid and enqueues nothing
+    assert fwd(_w(), M=0, X=0, Y=0, XA=0, ws=0, nb=0) == q.LORA_OK
+
+
+def test_backward_specific_validation():
+    assert bwd(_w(), dY=0) == q.LORA_ERR_INVALID_ARG
+    assert bwd(_w(), dA=0) == q.LORA_ERR_INVALID_ARG
+    assert bwd(_w(), dB=P + 2) == q.LORA_ERR_ALIGNMENT
+    assert bwd(_w(), dX=P + 2) == q.LORA_ERR_ALIGNMENT
+
+
+def test_dequant_and_merge_validation():
+    lib = q.lib()
+    assert lib.dequant_blockwise4(ctypes.byref(_w(fmt=0)), P, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.dequant_blockwise4(ctypes.byref(_w(fmt=1)), 0, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.dequant_blockwise4(ctypes.byref(_w(fmt=1)), P + 2, None) == q.LORA_ERR_ALIGNMENT
+    assert lib.lora_merge(ctypes.byref(_w()), P, P, 12, 2.0, P, None) == q.LORA_ERR_UNSUPPORTED
+    assert lib.lora_merge(ctypes.byref(_w()), P, P, 8, float("nan"), P, None) == q.LORA_ERR_INVALID_ARG
+    # a 4-bit merge whose output overlaps the packed codes is rejected
+    assert lib.lora_merge(ctypes.byref(_w(fmt=1, data=P)), P2, P2, 8, 2.0, P, None) == q.LORA_ERR_INVALID_ARG
+
+
+def test_workspace_bytes_is_a_pure_function_of_sizes():
+    a = q.workspace_bytes(16384, 14336, 4096, 16)
+    assert a == q.workspace_bytes(16384, 14336, 4096, 16, q.LORA_W_BLOCK4)
+    assert a >= 256 + 16384 * 16 * 2
+    assert q.workspace_bytes(0, 512, 512, 8) >= 256
+    assert q.workspace_bytes(256, 512, 512, 7) == 0
+    assert q.workspace_bytes(256, 0, 512, 8) == 0
+    assert q.workspace_bytes(256, 512, 512, 8, 5) == 0
+    # grows with M and r
+    assert q.workspace_bytes(512, 4096, 4096, 16) < q.workspace_bytes(4096, 4096, 4096, 16)
+    assert q.workspace_bytes(4096, 4096, 4096, 16) < q.workspace_bytes(4096, 4096, 4096, 128)

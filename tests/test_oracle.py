@@ -314,3 +314,22 @@ def test_zero_block_takes_code_seven():
     # level -1/15 times a zero scale is IEEE negative zero
     d = O.dequant_blockwise4(q, s, cb, 1, 64)
     assert np.all(O.bf16_to_f64(d) == 0.0) and np.all(d == 0x8000)
+
+
+def test_sampled_adapter_grads_match_full_backward():
+    """The chunked, sampled dA/dB helper agrees with the full backward (chunk size
+    smaller than M and not dividing it)."""
+    rng = np.random.default_rng(14)
+    M, K, N, r = 50, 40, 24, 8
+    X = bf16_bits_from_f32(rng.standard_normal((M, K)).astype(np.float32))
+    dY = bf16_bits_from_f32(rng.standard_normal((M, N)).astype(np.float32))
+    W = rng.standard_normal((N, K))
+    A = rng.uniform(-0.2, 0.2, (r, K))
+    B = rng.standard_normal((N, r)) * 0.1
+    s = 3.0
+    g = O.lora_backward(O.bf16_to_f64(dY), O.bf16_to_f64(X), W, A, B, s)
+    n_idx = np.array([0, 3, 23])
+    k_idx = np.array([1, 39, 7])
+    dB_s, dA_s = O.lora_adapter_grads_sampled(dY, X, A, B, s, n_idx, k_idx, chunk_rows=7)
+    assert _rel(dB_s, g["dB"][n_idx]) <= 1e-13
+    assert _rel(dA_s, g["dA"][:, k_idx]) <= 1e-13
