@@ -52,7 +52,8 @@ typedef enum {
   LORA_ERR_UNSUPPORTED = 3,     /* sizes outside the limits above */
   LORA_ERR_WORKSPACE = 4,       /* workspace NULL or smaller than lora_workspace_bytes() */
   LORA_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed (launch error etc.) */
-  LORA_ERR_DEVICE_TIMEOUT = 6   /* a kernel gave up a bounded wait (read with lora_device_status) */
+  LORA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up a bounded wait (read with lora_device_status) */
+  LORA_ERR_SCRATCH_LIMIT = 7    /* lora_linear_fwd_noalloc: problem too large for its fixed scratch */
 } lora_status_t;
 
 typedef enum {
@@ -134,6 +135,45 @@ lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* str
  */
 lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, int32_t r,
                          float s, void* W_out, void* stream);
+
+/*
+ * Forward without any memory allocation and without a caller-provided workspace.
+ * (The pages describe no such call; it exists for callers of this library.)
+ *
+ * Who needs it: callers that are handed only their input and output buffers and may
+ * not obtain any other device memory — for example a plugin running inside a host
+ * framework whose memory is entirely owned by that framework's pool allocator, or
+ * latency-critical code that must not call cudaMalloc/cudaFree because those calls
+ * can synchronize the whole device and may fail under a fixed memory budget.
+ *
+ * Computes exactly what lora_linear_fwd computes (same kernels, same arguments apart
+ * from the workspace), but keeps its scratch (s·XA and the split partial sums of X·Aᵀ)
+ * in one fixed array of LORA_NOALLOC_SCRATCH_BYTES bytes that is part of the library
+ * image: every GPU that loads the library holds that array until the process exits.
+ * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *
+ *   - Size limit: the scratch a problem needs is 2·M·r bytes for s·XA plus 4·S·M·r
+ *     bytes of partial sums (S = number of K splits, which shrinks as M grows), each
+ *     rounded up to 256 bytes.  It fits in LORA_NOALLOC_SCRATCH_BYTES = 16 MiB whenever
+ *     6·M·r + 76000·r <= 16 MiB, e.g. up to about 160 000 tokens at r = 16 and about
+ *     9 000 tokens at r = 128.  A larger problem gets LORA_ERR_SCRATCH_LIMIT and
+ *     nothing is enqueued.  Other arguments are validated as for lora_linear_fwd.
+ *   - First call on each device: it looks up the device address of the array on that
+ *     device (the current device) once and caches it.  Make this first call before
+ *     any stream capture begins on that device.
+ *   - Shared state: all calls in the process share the one array per device, and the
+ *     array keeps whatever the last call left in it.  Every scratch byte a call reads
+ *     is written earlier by the same call, so nothing needs clearing between calls.
+ *     Calls whose work overlaps on the GPU (different streams, or different host
+ *     threads without ordering) race on the array and corrupt each other's results:
+ *     order them on one stream or synchronize between them.
+ *   - A device-side wait that runs out ends the kernels (no hang) but is not reported:
+ *     there is no workspace to hold the status word.
+ */
+#define LORA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weight_t* W,
+                                      const void* A, const void* B, int32_t r, float s,
+                                      void* Y, void* XA, void* stream);
 
 /*
  * Reads and clears the device status word in `workspace` (synchronizes `stream`).

@@ -25,6 +25,9 @@ from .binding import (  # noqa: F401
     lora_device_status,
     lora_linear_bwd,
     lora_linear_fwd,
+    lora_linear_fwd_noalloc,
+    LORA_ERR_SCRATCH_LIMIT,
+    LORA_NOALLOC_SCRATCH_BYTES,
     lora_merge,
     lora_testing_bounded_wait,
     LORA_KERNEL_BWD_GEMM,

@@ -22,6 +22,8 @@ LORA_ERR_UNSUPPORTED = 3
 LORA_ERR_WORKSPACE = 4
 LORA_ERR_CUDA = 5
 LORA_ERR_DEVICE_TIMEOUT = 6
+LORA_ERR_SCRATCH_LIMIT = 7
+LORA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 LORA_W_BF16 = 0
 LORA_W_BLOCK4 = 1
@@ -30,6 +32,7 @@ EXPORTED = (
     "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
     "lora_testing_bounded_wait", "lora_timing_enable", "lora_timing_read", "lora_launch_count",
+    "lora_linear_fwd_noalloc",
 )
 
 
@@ -81,6 +84,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_timing_read.restype = i32
     lib.lora_launch_count.argtypes = []
     lib.lora_launch_count.restype = i64
+    lib.lora_linear_fwd_noalloc.argtypes = [vp, i64, W, vp, vp, i32, f32, vp, vp, vp]
+    lib.lora_linear_fwd_noalloc.restype = i32
     return lib
 
 
@@ -205,3 +210,13 @@ def lora_timing_read(kernel: int) -> tuple[float, int]:
 
 def lora_launch_count() -> int:
     return int(_lib.lora_launch_count())
+
+
+def lora_linear_fwd_noalloc(X, M: int, W: LoraWeight, A, B, r: int, s: float, Y, XA, stream=None) -> None:
+    """Forward that allocates nothing and takes no workspace: for callers that are given
+    only their input and output buffers and may not obtain other device memory.  Its
+    scratch is a fixed 16 MiB array inside the library, shared by every call on a
+    device, so calls must not overlap on the GPU (keep them on one stream)."""
+    w = W.c_struct()
+    _check(_lib.lora_linear_fwd_noalloc(_ptr(X), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r), float(s),
+                                        _ptr(Y), _ptr(XA), _stream(stream)), "lora_linear_fwd_noalloc")

@@ -299,6 +299,8 @@ const char* lora_status_string(int32_t status) {
     case LORA_ERR_WORKSPACE: return "workspace missing or smaller than lora_workspace_bytes()";
     case LORA_ERR_CUDA: return "a CUDA call failed";
     case LORA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait; outputs of that call are undefined";
+    case LORA_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the fixed LORA_NOALLOC_SCRATCH_BYTES of lora_linear_fwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -560,5 +562,107 @@ lora_status_t lora_timing_read(int32_t kernel, double* total_ms, int64_t* launch
 }
 
 int64_t lora_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- forward without allocation
+// The fixed scratch of lora_linear_fwd_noalloc.  In host code this name is only a
+// stand-in for the symbol; its device address is looked up per device with
+// cudaGetSymbolAddress and only that address is handed to kernels.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LORA_NOALLOC_SCRATCH_BYTES];
+
+namespace lora {
+namespace {
+
+struct NoAllocLayout {
+  size_t sxa_off, part_off, total;
+};
+NoAllocLayout noalloc_layout(long long M, long long K, int r) {
+  NoAllocLayout l;
+  l.sxa_off = 0;
+  l.part_off = align256(static_cast<size_t>(M) * r * 2);
+  l.total = l.part_off + align256(static_cast<size_t>(rowproj_split(M, K).splits) * M * r * 4);
+  return l;
+}
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of the fixed scratch on the current device, looked up on first use.
+lora_status_t noalloc_scratch(uint8_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LORA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_addr[dev]);
+  return LORA_OK;
+}
+
+}  // namespace
+}  // namespace lora
+
+extern "C" {
+
+lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weight_t* W, const void* A, const void* B,
+                                      int32_t r, float s, void* Y, void* XA, void* stream) {
+  TRY(check_weight(W));
+  TRY(check_rank(r, s));
+  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
+  TRY(check_ptr(A));
+  TRY(check_ptr(B));
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(X));
+  TRY(check_ptr(Y));
+  TRY(check_ptr(XA));
+  const long long N = W->N, K = W->K;
+  const NoAllocLayout nl = noalloc_layout(M, K, r);
+  if (nl.total > LORA_NOALLOC_SCRATCH_BYTES) return LORA_ERR_SCRATCH_LIMIT;
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  uint8_t* scratch = nullptr;
+  TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* sXA = reinterpret_cast<__nv_bfloat16*>(scratch + nl.sxa_off);
+  float* part = reinterpret_cast<float*>(scratch + nl.part_off);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+
+  // XA = X·Aᵀ and s·XA; every partial the finalize reads is written by rowproj first
+  const Split sp = rowproj_split(M, K);
+  TRY(launch_rowproj<false>(Xb, static_cast<const __nv_bfloat16*>(A), part, static_cast<int>(M), static_cast<int>(K), r,
+                            sp, st));
+  const size_t n = static_cast<size_t>(M) * r;
+  finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, sp.splits, n, s, static_cast<__nv_bfloat16*>(XA), sXA);
+  count_launch();
+  TRY(last_launch());
+
+  // Y = X·Wᵀ + (s·XA)·Bᵀ; no status word (status = null): an expired wait ends the kernel silently
+  CUtensorMap ta, tb, te, tf;
+  TRY(tmap_bf16(&ta, X, K, M, 64, 128));
+  TRY(tmap_bf16(&te, sXA, r, M, 64, 128));
+  TRY(tmap_bf16(&tf, B, r, N, 64, 256));
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.Nout = static_cast<int>(N);
+  p.Kred = static_cast<int>(K);
+  p.r = r;
+  p.out = static_cast<__nv_bfloat16*>(Y);
+  p.status = nullptr;
+  p.wait_ns = wait_limit_ns();
+  p.Nw = static_cast<int>(N);
+  p.Kw = static_cast<int>(K);
+  if (W->fmt == LORA_W_BF16) {
+    TRY(tmap_bf16(&tb, W->data, K, N, 64, 256));
+    return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
+  }
+  TRY(tmap_u8(&tb, W->data, K / 2, N, 32, 256));
+  p.absmax = static_cast<const __half*>(W->absmax);
+  p.codebook = W->codebook;
+  return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
+}
 
 }  // extern "C"
