@@ -13,7 +13,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblora_linear.so")
+# LORA_LIB_PATH selects another build of the library (e.g. one compiled with different flags).
+LIB_PATH = os.environ.get("LORA_LIB_PATH") or os.path.join(_HERE, "liblora_linear.so")
 
 LORA_OK = 0
 LORA_ERR_INVALID_ARG = 1

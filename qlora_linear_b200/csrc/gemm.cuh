@@ -71,6 +71,8 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int gro
 // the block's 16 dequantized levels held as byte planes (lo bytes in L0..L3, hi bytes
 // in H0..H3, entry e in byte e%4 of register e/4).  Element 2j sits in the low
 // nibble of byte j, so the low 16 bits of `w` are the selectors of elements 0..3.
+#ifndef LORA_EXPAND8_DEFINED
+#define LORA_EXPAND8_DEFINED
 __device__ __forceinline__ uint4 expand8(uint32_t w, const uint32_t (&L)[4], const uint32_t (&H)[4]) {
   uint4 o;
   {
@@ -105,6 +107,7 @@ __device__ __forceinline__ void block_levels(const float (&cb)[16], float scale,
     H[i] = prmt(v[2 * i], v[2 * i + 1], 0x7531u);
   }
 }
+#endif
 
 template <bool B_MN, bool W4>
 __global__ void __launch_bounds__(GemmCfg<B_MN, W4>::NUM_THREADS, 1)

@@ -1,0 +1,424 @@
+// gemm_pair.cuh — the Y / dX GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+//     out[M, Nout] = Aop[M, Kred] · Bop[Nout, Kred]ᵀ  +  E[M, r] · F[Nout, r]ᵀ
+//
+// Forward  (B_MN = false): Aop = X, Bop = W (K-major), E = s·XA, F = B      -> Y
+// Backward (B_MN = true) : Aop = dY, Bop[k, n] = W[n, k] (MN-major), E = s·dY·B,
+//                          F[k, j] = A[j, k] (MN-major)                      -> dX
+//
+// The LoRA term is one extra K fill after the main loop — possible because the
+// adapter product is bracketed skinny-first ("Unsloth vs PyTorch: The ONLY Video You
+// Need to Understand the Difference", transcript 1:35-2:00), so the N×K matrix B·A is
+// never formed.  With W4 the frozen weight arrives as packed 4-bit codes ("Rev vs
+// unsloth", fused quantized-LoRA paragraph) and each CTA's dequant warps expand them in
+// shared memory into the bf16 tile the tensor core reads; no dequantized weight ever
+// reaches HBM.
+//
+// A cluster of two CTAs computes a 256×256 tile.  Each CTA loads its own 128 rows of A
+// and its own 128 rows of the B tile (no multicast); the even CTA ("leader") issues
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which reads both CTAs' shared memory
+// and accumulates into both CTAs' TMEM (each CTA holds its 128 rows × 256 fp32 columns,
+// double-buffered).  Per CTA this halves the operand bytes per MMA compared with a
+// 128×256 single-CTA tile, and for W4 halves the dequant work per MMA.
+//
+// Synchronisation.  TMA completions of both CTAs count on the leader's `full` barrier;
+// the leader's MMA commits arrive on both CTAs' `empty` / `tfull` barriers (CTA mask
+// 0b11); both CTAs' epilogue and dequant warps arrive on the leader's `tempty` / `deq`
+// barriers through cluster addresses.  W4 code tiles complete on a CTA-local `cfull`
+// barrier so each CTA's dequant warps can wait locally.  Every wait is bounded.
+//
+// Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
+// warps 2-5 epilogue, warps 6-9 dequant (W4 only).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace lora {
+
+struct PairParams {
+  int M;               // rows of Aop / out
+  int Nout;            // columns of out
+  int Kred;            // reduction length (K forward, N backward)
+  int r;               // adapter rank (<= 128): one extra K fill
+  __nv_bfloat16* out;  // [M, Nout] row-major
+  uint32_t* status;    // device status word, may be null
+  uint64_t wait_ns;    // bound of every mbarrier wait
+  // 4-bit weight only
+  const __half* absmax;   // [Nw*Kw/64]
+  const float* codebook;  // [16]
+  int Nw, Kw;             // logical weight shape [Nw, Kw]
+};
+
+template <bool B_MN, bool W4>
+struct PairCfg {
+  static constexpr int BM = 256, BN = 256, BK = 128;  // pair tile, K per pipeline fill
+  static constexpr int HM = 128, HN = 128;            // per-CTA halves of A rows / B rows
+  static constexpr int STAGES = 3;
+  static constexpr int ATOM = 64;                       // 128-byte swizzle atom width (bf16)
+  static constexpr int A_BYTES = HM * BK * 2;           // 32 KB (two 64-wide K atoms)
+  static constexpr int B_BYTES = HN * BK * 2;           // 32 KB
+  static constexpr int C_BYTES = W4 ? HN * BK / 2 : 0;  // 8 KB of codes
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+  static constexpr int NUM_EPI_WARPS = 4;
+  static constexpr int NUM_DEQ_WARPS = W4 ? 4 : 0;
+  static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS + NUM_DEQ_WARPS);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int NUM_BARS = 4 * STAGES + 5;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+  static constexpr int GROUP_M = 8;  // 256-row tiles per raster group (L2 reuse of W)
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void pair_tile_coords(int t, int num_m, int num_n, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * num_n;
+  const int g = t / per_group;
+  const int first_m = g * group_m;
+  const int gm = min(group_m, num_m - first_m);
+  const int within = t - first_m * num_n;
+  mb = first_m + within % gm;
+  nb = within / gm;
+}
+
+// Expands 8 codes (one 32-bit word) of one 64-element scale block to 8 bf16, using the
+// block's 16 dequantized levels held as byte planes: low bytes of level e in byte e%4
+// of L[e/4], high bytes likewise in H.  Element 2j sits in the low nibble of byte j,
+// so the low 16 bits of `w` select elements 0..3.  Each prmt picks four bytes by
+// 3-bit selectors; the selector's bit 3 (code >= 8) picks between the two halves.
+#ifndef LORA_EXPAND8_DEFINED
+#define LORA_EXPAND8_DEFINED
+__device__ __forceinline__ uint4 expand8(uint32_t w, const uint32_t (&L)[4], const uint32_t (&H)[4]) {
+  uint4 o;
+  {
+    const uint32_t sel = w & 0x7777u;
+    const uint32_t sel2 = ((w >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t lo = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), sel2);
+    const uint32_t hi = prmt(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), sel2);
+    o.x = prmt(lo, hi, 0x5140u);
+    o.y = prmt(lo, hi, 0x7362u);
+  }
+  {
+    const uint32_t w2 = w >> 16;
+    const uint32_t sel = w2 & 0x7777u;
+    const uint32_t sel2 = ((w2 >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t lo = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), sel2);
+    const uint32_t hi = prmt(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), sel2);
+    o.z = prmt(lo, hi, 0x5140u);
+    o.w = prmt(lo, hi, 0x7362u);
+  }
+  return o;
+}
+
+// The 16 levels of one scale block, bf16_rn(fp32_rn(codebook[c] * scale)), as byte
+// planes for expand8().  __fmul_rn keeps the product from being fused with anything.
+__device__ __forceinline__ void block_levels(const float (&cb)[16], float scale, uint32_t (&L)[4], uint32_t (&H)[4]) {
+  uint32_t v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = pack_bf16x2(__fmul_rn(cb[2 * i], scale), __fmul_rn(cb[2 * i + 1], scale));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    L[i] = prmt(v[2 * i], v[2 * i + 1], 0x6420u);
+    H[i] = prmt(v[2 * i], v[2 * i + 1], 0x7531u);
+  }
+}
+#endif
+
+template <bool B_MN, bool W4>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::NUM_THREADS, 1)
+    lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
+                          const PairParams p) {
+  using C = PairCfg<B_MN, W4>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
+  uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
+  uint64_t* cfull = bars + 2 * C::STAGES;   // both (W4): this CTA's code tile landed
+  uint64_t* deq = bars + 3 * C::STAGES;     // leader (W4): both CTAs' dequantized tiles written
+  uint64_t* tfull = bars + 4 * C::STAGES;   // both: accumulator ready for the epilogue
+  uint64_t* tempty = tfull + 2;             // leader: both CTAs drained the accumulator
+  uint64_t* drain = tempty + 2;             // leader: final commit before TMEM release
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* never_flag = tmem_slot + 2;  // stays 0: drain waits ignore the abort
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int num_m = (p.M + C::BM - 1) / C::BM;
+  const int num_n = (p.Nout + C::BN - 1) / C::BN;
+  const int ntiles = num_m * num_n;
+  const int nkb = (p.Kred + C::BK - 1) / C::BK;
+  const int n_ext = p.r > 0 ? 1 : 0;         // one fill holds the whole LoRA block (r <= 128)
+  const int ext_atoms = p.r > 64 ? 2 : 1;   // 64-wide rank atoms actually loaded
+  const WaitCtl wc{abort_flag, p.status, p.wait_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+      mbar_init(smem_u32(&cfull[s]), 1);
+      mbar_init(smem_u32(&deq[s]), 2 * (C::NUM_DEQ_WARPS > 0 ? C::NUM_DEQ_WARPS : 1));
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 2 * C::NUM_EPI_WARPS);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    *never_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmE);
+    tma_prefetch_desc(&tmF);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or TMA
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long fills = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        int mb, nb;
+        pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+        const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A
+        const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;  // this CTA's rows of the B tile
+        for (int kb = 0; kb < nkb + n_ext; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
+          const bool ext = kb >= nkb;
+          const int e = kb - nkb;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sC = sB + C::B_BYTES;
+          const uint32_t full_l = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) {
+            uint32_t per_cta;
+            if (!ext) per_cta = C::A_BYTES + (W4 ? 0 : C::B_BYTES);
+            else per_cta = ext_atoms * (C::A_BYTES / 2) + (B_MN ? C::B_BYTES : ext_atoms * (C::B_BYTES / 2));
+            mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * per_cta);
+          }
+          // every box is 64 wide × 128 rows; a K-major operand takes one box per
+          // 64-wide K atom, an MN-major one (backward weight) one box per 64-wide MN chunk
+          if (!ext) {
+            tma_load_2d_pair(sA, &tmA, full_l, kb * C::BK, arow);
+            tma_load_2d_pair(sA + C::A_BYTES / 2, &tmA, full_l, kb * C::BK + C::ATOM, arow);
+            if (W4) {
+              mbar_arrive_expect_tx(smem_u32(&cfull[stage]), C::C_BYTES);
+              if (!B_MN) tma_load_2d(sC, &tmB, smem_u32(&cfull[stage]), kb * (C::BK / 2), brow);
+              else tma_load_2d(sC, &tmB, smem_u32(&cfull[stage]), brow / 2, kb * C::BK);
+            } else if (!B_MN) {
+              tma_load_2d_pair(sB, &tmB, full_l, kb * C::BK, brow);
+              tma_load_2d_pair(sB + C::B_BYTES / 2, &tmB, full_l, kb * C::BK + C::ATOM, brow);
+            } else {
+              tma_load_2d_pair(sB, &tmB, full_l, brow, kb * C::BK);
+              tma_load_2d_pair(sB + C::B_BYTES / 2, &tmB, full_l, brow + C::ATOM, kb * C::BK);
+            }
+          } else {
+            for (int h = 0; h < ext_atoms; ++h) tma_load_2d_pair(sA + h * (C::A_BYTES / 2), &tmE, full_l, h * C::ATOM, arow);
+            if (!B_MN) {
+              for (int h = 0; h < ext_atoms; ++h)
+                tma_load_2d_pair(sB + h * (C::B_BYTES / 2), &tmF, full_l, h * C::ATOM, brow);
+            } else {
+              tma_load_2d_pair(sB, &tmF, full_l, brow, 0);
+              tma_load_2d_pair(sB + C::B_BYTES / 2, &tmF, full_l, brow + C::ATOM, 0);
+            }
+            if (W4) mbar_arrive(smem_u32(&cfull[stage]));  // nothing to dequantize in this fill
+          }
+          ++fills;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // let this CTA's loads that are still in flight land before shared memory goes away
+        const long long first = fills > C::STAGES ? fills - C::STAGES : 0;
+        const WaitCtl drain_wc{never_flag, nullptr, p.wait_ns};
+        for (long long f = first; f < fills; ++f) {
+          const int s = static_cast<int>(f % C::STAGES);
+          const uint32_t ph = static_cast<uint32_t>((f / C::STAGES) & 1);
+          if (leader) mbar_wait(smem_u32(&full[s]), ph, drain_wc);
+          if (W4) mbar_wait(smem_u32(&cfull[s]), ph, drain_wc);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        if (!mbar_wait<true>(smem_u32(&tempty[acc]), acc_phase ^ 1u, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::BN);
+        for (int kb = 0; kb < nkb + n_ext; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
+          if (W4 && !mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
+          tc_fence_after();
+          const bool ext = kb >= nkb;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const int nk = ext ? (p.r + 15) / 16 : C::BK / 16;
+          for (int k = 0; k < nk; ++k) {
+            // K step k: atom k/4, 32-byte column (k%4) inside the K-major atom; for the
+            // MN-major operand 16 K rows (2 KB) further down its 128-row chunks
+            const uint32_t koff = (k >> 2) * (C::A_BYTES / 2) + (k & 3) * 32;
+            const uint64_t ad = sdesc_sw128(sA + koff, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(sB + k * 2048, C::B_BYTES / 2, 1024) : sdesc_sw128(sB + koff, 16, 1024);
+            tc_mma_bf16_pair(d, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(smem_u32(&tfull[acc]), 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // every pair MMA issued so far must finish before TMEM is released
+      tc_commit_pair(smem_u32(drain));
+      const WaitCtl drain_wc{never_flag, nullptr, p.wait_ns};
+      mbar_wait(smem_u32(drain), 0, drain_wc);
+    }
+  } else if (warp < 2 + C::NUM_EPI_WARPS) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < ntiles; t += npairs) {
+      int mb, nb;
+      pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+      if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, wc)) break;
+      tc_fence_after();
+      const int row = mb * C::BM + static_cast<int>(rank) * C::HM + quarter * 32 + lane;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+      __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
+#pragma unroll 1
+      for (int c = 0; c < C::BN / 32; ++c) {
+        const int col0 = nb * C::BN + c * 32;
+        if (col0 >= p.Nout) break;  // warp-uniform
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, v);
+        tmem_ld_wait();
+        if (row < p.M) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (col0 + q * 8 < p.Nout) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]));
+              o.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]), __uint_as_float(v[q * 8 + 3]));
+              o.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]));
+              o.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]), __uint_as_float(v[q * 8 + 7]));
+              *reinterpret_cast<uint4*>(orow + col0 + q * 8) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  } else if (W4) {
+    // ------------------------------------------------------------ dequant (W4, both CTAs)
+    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..127
+    float cb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
+    const int kblocks_w = p.Kw / 64;  // scale blocks per weight row
+    // Each thread expands two 64-element scale blocks per fill, one per 64-wide atom h:
+    // forward, weight row `dt` of the CTA's 128 rows at K atoms h = 0, 1;
+    // backward, weight row kb*128 + dt (reduction) at output chunks h = 0, 1.
+    auto scale_at = [&](int t, int kb, int h) -> float {
+      int mb, nb;
+      pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+      const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
+      int n, kblk;
+      if (!B_MN) {
+        n = brow + dt;
+        kblk = kb * 2 + h;
+      } else {
+        n = kb * C::BK + dt;
+        kblk = brow / 64 + h;
+      }
+      if (n >= p.Nw || kblk >= kblocks_w) return 0.f;
+      return __half2float(p.absmax[static_cast<size_t>(n) * kblocks_w + kblk]);
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    float sc0 = 0.f, sc1 = 0.f;
+    if (pair < ntiles && nkb > 0) {
+      sc0 = scale_at(pair, 0, 0);
+      sc1 = scale_at(pair, 0, 1);
+    }
+    for (int t = pair; t < ntiles; t += npairs) {
+      bool ok = true;
+      for (int kb = 0; kb < nkb + n_ext; ++kb) {
+        // prefetch the scales of the next fill that has codes
+        float nx0 = 0.f, nx1 = 0.f;
+        if (kb + 1 < nkb) {
+          nx0 = scale_at(t, kb + 1, 0);
+          nx1 = scale_at(t, kb + 1, 1);
+        } else if (kb + 1 == nkb && t + npairs < ntiles) {
+          nx0 = scale_at(t + npairs, 0, 0);
+          nx1 = scale_at(t + npairs, 0, 1);
+        }
+        if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
+        if (kb < nkb) {
+          uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+          const uint8_t* crow = sB + C::B_BYTES + dt * 64;  // 64 code bytes of this thread's row
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t L[4], H[4];
+            block_levels(cb, h ? sc1 : sc0, L, H);
+            const uint4 c0 = *reinterpret_cast<const uint4*>(crow + h * 32);
+            const uint4 c1 = *reinterpret_cast<const uint4*>(crow + h * 32 + 16);
+            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint8_t* rowp = sB + h * (C::B_BYTES / 2) + dt * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(rowp + ((u ^ (dt & 7)) << 4)) = expand8(cw[u], L, H);
+          }
+          fence_proxy_async_smem();
+          sc0 = nx0;
+          sc1 = nx1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // the peer's TMEM and shared memory stay valid until the pair is done
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace lora

@@ -17,6 +17,7 @@
 #include "lora_linear_testing.h"
 #include "elementwise.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "skinny.cuh"
 
 namespace lora {
@@ -133,6 +134,10 @@ lora_status_t dev_info(DevInfo** out) {
     SET_SMEM((lora_gemm_kernel<true, false>), (GemmCfg<true, false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_kernel<false, true>), (GemmCfg<false, true>::SMEM_BYTES));
     SET_SMEM((lora_gemm_kernel<true, true>), (GemmCfg<true, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, false>), (PairCfg<false, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, false>), (PairCfg<true, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, true>), (PairCfg<false, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, true>), (PairCfg<true, true>::SMEM_BYTES));
     SET_SMEM((rowproj_kernel<16, false>), (rowproj_smem_bytes<16, false>()));
     SET_SMEM((rowproj_kernel<32, false>), (rowproj_smem_bytes<32, false>()));
     SET_SMEM((rowproj_kernel<64, false>), (rowproj_smem_bytes<64, false>()));
@@ -269,15 +274,61 @@ lora_status_t launch_colproj(const __nv_bfloat16* P, const __nv_bfloat16* R, flo
 }
 
 // ---------------------------------------------------------------- GEMM launch
+// GEMM kernel family: CTA pairs (default) or single CTAs (LORA_GEMM_1SM=1, kept for
+// comparison measurements).
+bool use_single_cta_gemm() {
+  static const bool v = [] {
+    const char* e = std::getenv("LORA_GEMM_1SM");
+    return e && e[0] == '1';
+  }();
+  return v;
+}
+
+// Tensor-map boxes of the four GEMM operands (x = inner extent, y = rows).
+struct GemmBoxes {
+  uint32_t a_y, b_x, b_y, c_x, c_y, f_x, f_y;
+};
+GemmBoxes gemm_boxes(bool b_mn) {
+  if (use_single_cta_gemm()) {
+    return b_mn ? GemmBoxes{128, 64, 64, 128, 64, 64, 64} : GemmBoxes{128, 64, 256, 32, 256, 64, 256};
+  }
+  // CTA pairs: every box is 64 elements (or 64 code bytes) wide and 128 rows high
+  return GemmBoxes{128, 64, 128, 64, 128, 64, 128};
+}
+
 template <bool B_MN, bool W4>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
                           const GemmParams& p, int sms, cudaStream_t st) {
-  using C = GemmCfg<B_MN, W4>;
+  if (use_single_cta_gemm()) {
+    using C = GemmCfg<B_MN, W4>;
+    const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, C::BN);
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    {
+      TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
+      lora_gemm_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    }
+    count_launch();
+    return last_launch();
+  }
+  using C = PairCfg<B_MN, W4>;
+  PairParams q;
+  q.M = p.M;
+  q.Nout = p.Nout;
+  q.Kred = p.Kred;
+  q.r = p.r;
+  q.out = p.out;
+  q.status = p.status;
+  q.wait_ns = p.wait_ns;
+  q.absmax = p.absmax;
+  q.codebook = p.codebook;
+  q.Nw = p.Nw;
+  q.Kw = p.Kw;
   const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, C::BN);
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+  const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    lora_gemm_pair_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, q);
   }
   count_launch();
   return last_launch();
@@ -350,9 +401,10 @@ lora_status_t lora_linear_fwd(const void* X, int64_t M, const lora_weight_t* W, 
 
   // Y = X·Wᵀ + (s·XA)·Bᵀ
   CUtensorMap ta, tb, te, tf;
-  TRY(tmap_bf16(&ta, X, K, M, 64, 128));
-  TRY(tmap_bf16(&te, sXA, r, M, 64, 128));
-  TRY(tmap_bf16(&tf, B, r, N, 64, 256));
+  const GemmBoxes bx = gemm_boxes(false);
+  TRY(tmap_bf16(&ta, X, K, M, 64, bx.a_y));
+  TRY(tmap_bf16(&te, sXA, r, M, 64, bx.a_y));
+  TRY(tmap_bf16(&tf, B, r, N, bx.f_x, bx.f_y));
   GemmParams p{};
   p.M = static_cast<int>(M);
   p.Nout = static_cast<int>(N);
@@ -364,10 +416,10 @@ lora_status_t lora_linear_fwd(const void* X, int64_t M, const lora_weight_t* W, 
   p.Nw = static_cast<int>(N);
   p.Kw = static_cast<int>(K);
   if (W->fmt == LORA_W_BF16) {
-    TRY(tmap_bf16(&tb, W->data, K, N, 64, 256));
+    TRY(tmap_bf16(&tb, W->data, K, N, bx.b_x, bx.b_y));
     return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
   }
-  TRY(tmap_u8(&tb, W->data, K / 2, N, 32, 256));
+  TRY(tmap_u8(&tb, W->data, K / 2, N, bx.c_x, bx.c_y));
   p.absmax = static_cast<const __half*>(W->absmax);
   p.codebook = W->codebook;
   return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
@@ -429,9 +481,10 @@ lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int
   // dX = dY·W + (s·dY·B)·A
   if (dX) {
     CUtensorMap ta, tb, te, tf;
-    TRY(tmap_bf16(&ta, dY, N, M, 64, 128));
-    TRY(tmap_bf16(&te, sdYB, r, M, 64, 128));
-    TRY(tmap_bf16(&tf, A, K, r, 64, 64));
+    const GemmBoxes bx = gemm_boxes(true);
+    TRY(tmap_bf16(&ta, dY, N, M, 64, bx.a_y));
+    TRY(tmap_bf16(&te, sdYB, r, M, 64, bx.a_y));
+    TRY(tmap_bf16(&tf, A, K, r, bx.f_x, bx.f_y));
     GemmParams p{};
     p.M = Mi;
     p.Nout = Ki;
@@ -443,10 +496,10 @@ lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int
     p.Nw = Ni;
     p.Kw = Ki;
     if (W->fmt == LORA_W_BF16) {
-      TRY(tmap_bf16(&tb, W->data, K, N, 64, 64));
+      TRY(tmap_bf16(&tb, W->data, K, N, bx.b_x, bx.b_y));
       TRY((launch_gemm<true, false>(ta, tb, te, tf, p, dev->sms, st)));
     } else {
-      TRY(tmap_u8(&tb, W->data, K / 2, N, 128, 64));
+      TRY(tmap_u8(&tb, W->data, K / 2, N, bx.c_x, bx.c_y));
       p.absmax = static_cast<const __half*>(W->absmax);
       p.codebook = W->codebook;
       TRY((launch_gemm<true, true>(ta, tb, te, tf, p, dev->sms, st)));
@@ -642,9 +695,10 @@ lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weigh
 
   // Y = X·Wᵀ + (s·XA)·Bᵀ; no status word (status = null): an expired wait ends the kernel silently
   CUtensorMap ta, tb, te, tf;
-  TRY(tmap_bf16(&ta, X, K, M, 64, 128));
-  TRY(tmap_bf16(&te, sXA, r, M, 64, 128));
-  TRY(tmap_bf16(&tf, B, r, N, 64, 256));
+  const GemmBoxes bx = gemm_boxes(false);
+  TRY(tmap_bf16(&ta, X, K, M, 64, bx.a_y));
+  TRY(tmap_bf16(&te, sXA, r, M, 64, bx.a_y));
+  TRY(tmap_bf16(&tf, B, r, N, bx.f_x, bx.f_y));
   GemmParams p{};
   p.M = static_cast<int>(M);
   p.Nout = static_cast<int>(N);
@@ -656,10 +710,10 @@ lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weigh
   p.Nw = static_cast<int>(N);
   p.Kw = static_cast<int>(K);
   if (W->fmt == LORA_W_BF16) {
-    TRY(tmap_bf16(&tb, W->data, K, N, 64, 256));
+    TRY(tmap_bf16(&tb, W->data, K, N, bx.b_x, bx.b_y));
     return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
   }
-  TRY(tmap_u8(&tb, W->data, K / 2, N, 32, 256));
+  TRY(tmap_u8(&tb, W->data, K / 2, N, bx.c_x, bx.c_y));
   p.absmax = static_cast<const __half*>(W->absmax);
   p.codebook = W->codebook;
   return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
