@@ -28,7 +28,7 @@
 // barrier so each CTA's dequant warps can wait locally.  Every wait is bounded.
 //
 // Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
-// warps 2-5 epilogue, warps 6-9 dequant (W4 only).
+// warps 2-5 epilogue, warps 6-13 dequant (W4 only).
 #pragma once
 
 #include "ptx.cuh"
@@ -60,11 +60,13 @@ struct PairCfg {
   static constexpr int C_BYTES = W4 ? HN * BK / 2 : 0;  // 8 KB of codes
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
   static constexpr int NUM_EPI_WARPS = 4;
-  static constexpr int NUM_DEQ_WARPS = W4 ? 4 : 0;
+  static constexpr int NUM_DEQ_WARPS = W4 ? 8 : 0;  // two per SM sub-partition
   static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS + NUM_DEQ_WARPS);
   static constexpr int TMEM_COLS = 512;
   static constexpr int NUM_BARS = 4 * STAGES + 5;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+  static constexpr int SCALE_RING = 4;  // W4: scale words staged this many code fills ahead (minus one)
+  static constexpr int SCALE_BYTES = W4 ? SCALE_RING * 32 * NUM_DEQ_WARPS * 4 : 0;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SCALE_BYTES + 8 * NUM_BARS + 16;
   static constexpr int GROUP_M = 8;  // 256-row tiles per raster group (L2 reuse of W)
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -131,7 +133,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
   using C = PairCfg<B_MN, W4>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint32_t* scale_ring = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES);  // W4
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::SCALE_BYTES);
   uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
   uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
   uint64_t* cfull = bars + 2 * C::STAGES;   // both (W4): this CTA's code tile landed
@@ -340,67 +343,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
     }
   } else if (W4) {
     // ------------------------------------------------------------ dequant (W4, both CTAs)
-    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..127
+    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
+    const int row = dt & 127;  // weight row of this CTA's 128-row half (forward) / of the K fill (backward)
+    const int h = dt >> 7;     // 64-wide atom: K atom (forward) or output chunk (backward)
     float cb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
-    const int kblocks_w = p.Kw / 64;  // scale blocks per weight row
-    // Each thread expands two 64-element scale blocks per fill, one per 64-wide atom h:
-    // forward, weight row `dt` of the CTA's 128 rows at K atoms h = 0, 1;
-    // backward, weight row kb*128 + dt (reduction) at output chunks h = 0, 1.
-    auto scale_at = [&](int t, int kb, int h) -> float {
+    const long long kblocks_w = p.Kw / 64;  // scale blocks per weight row
+    const long long nscales = static_cast<long long>(p.Nw) * kblocks_w;
+    // Each thread expands one 64-element scale block per code fill.  The fp16 scales
+    // are staged in a per-thread shared-memory ring with cp.async, SCALE_RING-1 code
+    // fills ahead, so no register ever waits on an outstanding global load.
+    const int my_tiles = ntiles > pair ? (ntiles - pair + npairs - 1) / npairs : 0;
+    const int code_fills = my_tiles * nkb;  // fills of this CTA that carry codes
+    auto stage_scale = [&](int i) {           // issue the copy for code fill i (always commits a group)
+      if (i < code_fills) {
+        const int t = pair + (i / nkb) * npairs, kb = i % nkb;
+        int mb, nb;
+        pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+        const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
+        const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
+        const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
+        const uint32_t dst = smem_u32(&scale_ring[(i % C::SCALE_RING) * (32 * C::NUM_DEQ_WARPS) + dt]);
+        if (n < p.Nw && kblk < kblocks_w) {
+          // 4-byte aligned word holding the scale; the half beyond the array end reads as zero
+          const long long idx = n * kblocks_w + kblk;
+          const long long w0 = idx & ~1LL;
+          const uint32_t nbytes = (w0 + 1 < nscales) ? 4u : 2u;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(p.absmax + w0), "r"(nbytes)
+                       : "memory");
+        } else {
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, 0;" ::"r"(dst), "l"(p.absmax) : "memory");
+        }
+      }
+      cp_async_commit();
+    };
+    auto scale_of = [&](int i) -> float {
+      int kb = i % nkb, t = pair + (i / nkb) * npairs;
       int mb, nb;
       pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
       const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
-      int n, kblk;
-      if (!B_MN) {
-        n = brow + dt;
-        kblk = kb * 2 + h;
-      } else {
-        n = kb * C::BK + dt;
-        kblk = brow / 64 + h;
-      }
-      if (n >= p.Nw || kblk >= kblocks_w) return 0.f;
-      return __half2float(p.absmax[static_cast<size_t>(n) * kblocks_w + kblk]);
+      const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
+      const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
+      const uint32_t wv = scale_ring[(i % C::SCALE_RING) * (32 * C::NUM_DEQ_WARPS) + dt];
+      const uint16_t hb = ((n * kblocks_w + kblk) & 1) ? static_cast<uint16_t>(wv >> 16) : static_cast<uint16_t>(wv);
+      return __half2float(__ushort_as_half(hb));
     };
+#pragma unroll 1
+    for (int i = 0; i < C::SCALE_RING - 1; ++i) stage_scale(i);
     int stage = 0;
     uint32_t phase = 0;
-    float sc0 = 0.f, sc1 = 0.f;
-    if (pair < ntiles && nkb > 0) {
-      sc0 = scale_at(pair, 0, 0);
-      sc1 = scale_at(pair, 0, 1);
-    }
+    int ci = 0;  // index of the next code fill
     for (int t = pair; t < ntiles; t += npairs) {
       bool ok = true;
       for (int kb = 0; kb < nkb + n_ext; ++kb) {
-        // prefetch the scales of the next fill that has codes
-        float nx0 = 0.f, nx1 = 0.f;
-        if (kb + 1 < nkb) {
-          nx0 = scale_at(t, kb + 1, 0);
-          nx1 = scale_at(t, kb + 1, 1);
-        } else if (kb + 1 == nkb && t + npairs < ntiles) {
-          nx0 = scale_at(t + npairs, 0, 0);
-          nx1 = scale_at(t + npairs, 0, 1);
-        }
+        if (kb < nkb) stage_scale(ci + C::SCALE_RING - 1);
         if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
         if (kb < nkb) {
+          cp_async_wait<C::SCALE_RING - 1>();  // this fill's scale word has landed
+          const float sc = scale_of(ci);
+          ++ci;
           uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-          const uint8_t* crow = sB + C::B_BYTES + dt * 64;  // 64 code bytes of this thread's row
+          const uint8_t* crow = sB + C::B_BYTES + row * 64 + h * 32;  // 32 code bytes = 64 codes
+          uint32_t L[4], H[4];
+          block_levels(cb, sc, L, H);
+          const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint8_t* rowp = sB + h * (C::B_BYTES / 2) + row * 128;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t L[4], H[4];
-            block_levels(cb, h ? sc1 : sc0, L, H);
-            const uint4 c0 = *reinterpret_cast<const uint4*>(crow + h * 32);
-            const uint4 c1 = *reinterpret_cast<const uint4*>(crow + h * 32 + 16);
-            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            uint8_t* rowp = sB + h * (C::B_BYTES / 2) + dt * 128;
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<uint4*>(rowp + ((u ^ (dt & 7)) << 4)) = expand8(cw[u], L, H);
-          }
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) = expand8(cw[u], L, H);
           fence_proxy_async_smem();
-          sc0 = nx0;
-          sc1 = nx1;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
@@ -408,6 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       }
       if (!ok) break;
     }
+    cp_async_wait<0>();  // no copy may still target shared memory at exit
   }
 
   // ------------------------------------------------------------ teardown
