@@ -39,3 +39,4 @@ from .binding import (  # noqa: F401
     workspace_bytes,
 )
 from .layer import LoraLinear  # noqa: F401
+from .dp import allreduce_adapter_grads, token_shard  # noqa: F401
