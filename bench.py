@@ -91,7 +91,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
@@ -100,7 +100,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which: str):
+        setattr(self, which, time.time())
 
     def stop(self):
         if self.proc is None:
@@ -114,7 +117,12 @@ class ClockSampler:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0 = getattr(self, "t_start", 0.0)
+        t1 = getattr(self, "t_end", float("inf"))
+        window = [ln for ts, ln in self.lines if t0 <= ts <= t1 + 0.1]
+        if not window:  # timed region shorter than the sampling period: nearest samples
+            window = [ln for ts, ln in self.lines if ts >= t0][:2] or [ln for _, ln in self.lines[-2:]]
+        for ln in window:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -278,11 +286,13 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark("t_start")
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark("t_end")
     barrier()
     launches = q.lora_launch_count() - launches0
     q.lora_timing_enable(False)
@@ -435,10 +445,11 @@ def run_e2e(args, cases, layers, data, step, world, dev):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3"])
+    ap.add_argument("--only", default=None, help="run a single projection of the workload (e.g. c2_gate)")
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -450,6 +461,11 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cases, desc = workload(args.workload)
+    if args.only:
+        cases = [c for c in cases if c.name == args.only]
+        if not cases:
+            raise SystemExit(f"no projection named {args.only} in {args.workload}")
+        desc = f"{desc}; only {args.only}"
 
     if args.impl == "reference":
         return run_reference(args, cases, desc, rank, world)
