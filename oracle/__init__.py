@@ -17,4 +17,6 @@ from .lora_oracle import (  # noqa: F401
     lora_merge,
     weight_f64,
     lora_adapter_grads_sampled,
+    lora_grouped_forward,
+    lora_grouped_backward,
 )

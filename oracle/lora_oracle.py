@@ -233,3 +233,34 @@ def lora_adapter_grads_sampled(dY_bits: np.ndarray, X_bits: np.ndarray, A: np.nd
         dB += dYc[:, n_idx].T @ XAc
         dA += dYBc.T @ Xc[:, k_idx]
     return s * dB, s * dA
+
+
+# ----------------------------------------------------------------------------
+# several LoRA linears sharing one input (e.g. the q, k, v projections)
+# ----------------------------------------------------------------------------
+
+
+def lora_grouped_forward(X: np.ndarray, Ws: list, As: list, Bs: list, s: float):
+    """G LoRA linears that read the same X (the attention block's q, k and v projections,
+    whose six adapter derivatives "Unsloth vs PyTorch: The ONLY Video You Need to
+    Understand the Difference" counts at transcript 1:14-1:24).  Returns
+    ``(Y, XA)``: Y is the G outputs side by side ``[M, ΣN_g]``, XA the G skinny products
+    side by side ``[M, G·r]``; each part is :func:`lora_forward` of its projection."""
+    outs = [lora_forward(X, W, A, B, s) for W, A, B in zip(Ws, As, Bs)]
+    return np.concatenate([y for y, _ in outs], axis=1), np.concatenate([xa for _, xa in outs], axis=1)
+
+
+def lora_grouped_backward(dY: np.ndarray, X: np.ndarray, Ws: list, As: list, Bs: list, s: float) -> dict:
+    """Backward of :func:`lora_grouped_forward`: ``dY`` is ``[M, ΣN_g]``.  dX is the sum
+    of the G projections' dX (X feeds all of them); dA and dB are per projection,
+    stacked: dA ``[G·r, K]``, dB ``[ΣN_g, r]``; dYB ``[M, G·r]``."""
+    dY = np.asarray(dY, dtype=np.float64)
+    offs = np.cumsum([0] + [np.asarray(W).shape[0] for W in Ws])
+    parts = [lora_backward(dY[:, offs[g]:offs[g + 1]], X, Ws[g], As[g], Bs[g], s) for g in range(len(Ws))]
+    dX = parts[0]["dX"].copy()
+    for q in parts[1:]:
+        dX += q["dX"]
+    return {"dX": dX, "dA": np.concatenate([q["dA"] for q in parts], axis=0),
+            "dB": np.concatenate([q["dB"] for q in parts], axis=0),
+            "dYB": np.concatenate([q["dYB"] for q in parts], axis=1),
+            "XA": np.concatenate([q["XA"] for q in parts], axis=1)}

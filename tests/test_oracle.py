@@ -333,3 +333,80 @@ def test_sampled_adapter_grads_match_full_backward():
     dB_s, dA_s = O.lora_adapter_grads_sampled(dY, X, A, B, s, n_idx, k_idx, chunk_rows=7)
     assert _rel(dB_s, g["dB"][n_idx]) <= 1e-13
     assert _rel(dA_s, g["dA"][:, k_idx]) <= 1e-13
+
+
+# ---------------------------------------------------------------------------
+# grouped projections sharing X (fused q/k/v)
+# ---------------------------------------------------------------------------
+
+def _grouped(rng, M=9, K=12, Ns=(8, 4, 4), r=3):
+    X = rng.standard_normal((M, K))
+    Ws = [rng.standard_normal((n, K)) / np.sqrt(K) for n in Ns]
+    As = [rng.uniform(-1, 1, (r, K)) / np.sqrt(K) for _ in Ns]
+    Bs = [rng.standard_normal((n, r)) * 0.1 for n in Ns]
+    dY = rng.standard_normal((M, sum(Ns)))
+    return X, Ws, As, Bs, dY
+
+
+def test_grouped_equals_one_layer_with_block_diagonal_adapter():
+    """Stacking the weights and the A's and putting the B's on the diagonal of one
+    [ΣN, G·r] matrix turns the G projections into one LoRA linear of rank G·r: same Y,
+    same dX, and the diagonal blocks of its dB / the stacked dA are the per-projection
+    gradients."""
+    rng = np.random.default_rng(21)
+    X, Ws, As, Bs, dY = _grouped(rng)
+    s = 1.5
+    Wall, Aall = np.concatenate(Ws), np.concatenate(As)
+    r, Ns = As[0].shape[0], [W.shape[0] for W in Ws]
+    Bbd = np.zeros((sum(Ns), r * len(Ns)))
+    o = 0
+    for g, B in enumerate(Bs):
+        Bbd[o:o + Ns[g], g * r:(g + 1) * r] = B
+        o += Ns[g]
+    Y, XA = O.lora_grouped_forward(X, Ws, As, Bs, s)
+    Y1, XA1 = O.lora_forward(X, Wall, Aall, Bbd, s)
+    assert _rel(Y, Y1) <= 1e-13 and _rel(XA, XA1) <= 1e-13
+    g = O.lora_grouped_backward(dY, X, Ws, As, Bs, s)
+    g1 = O.lora_backward(dY, X, Wall, Aall, Bbd, s)
+    assert _rel(g["dX"], g1["dX"]) <= 1e-13
+    assert _rel(g["dA"], g1["dA"]) <= 1e-13
+    o = 0
+    for q in range(len(Ns)):
+        assert _rel(g["dB"][o:o + Ns[q]], g1["dB"][o:o + Ns[q], q * r:(q + 1) * r]) <= 1e-13
+        o += Ns[q]
+
+
+def test_grouped_finite_differences():
+    rng = np.random.default_rng(22)
+    X, Ws, As, Bs, dY = _grouped(rng, M=3, K=4, Ns=(2, 3), r=2)
+    s = 0.7
+    g = O.lora_grouped_backward(dY, X, Ws, As, Bs, s)
+
+    def L(X_, As_, Bs_):
+        return float(np.sum(dY * O.lora_grouped_forward(X_, Ws, As_, Bs_, s)[0]))
+
+    h = 1e-3
+    fd = np.zeros_like(X)
+    for idx in np.ndindex(X.shape):
+        Xp, Xm = X.copy(), X.copy()
+        Xp[idx] += h
+        Xm[idx] -= h
+        fd[idx] = (L(Xp, As, Bs) - L(Xm, As, Bs)) / (2 * h)
+    assert _rel(fd, g["dX"]) <= 1e-9
+    for q in range(2):
+        for name, T in (("A", As[q]), ("B", Bs[q])):
+            fdT = np.zeros_like(T)
+            for idx in np.ndindex(T.shape):
+                Tp, Tm = T.copy(), T.copy()
+                Tp[idx] += h
+                Tm[idx] -= h
+                Ap, Am = list(As), list(As)
+                Bp, Bm = list(Bs), list(Bs)
+                if name == "A":
+                    Ap[q], Am[q] = Tp, Tm
+                else:
+                    Bp[q], Bm[q] = Tp, Tm
+                fdT[idx] = (L(X, Ap, Bp) - L(X, Am, Bm)) / (2 * h)
+            r = As[0].shape[0]
+            want = g["dA"][q * r:(q + 1) * r] if name == "A" else g["dB"][sum(W.shape[0] for W in Ws[:q]):][:Ws[q].shape[0]]
+            assert _rel(fdT, want) <= 1e-9, (name, q)
