@@ -119,6 +119,48 @@ lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int
                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Grouped projections sharing one input — e.g. the q, k and v projections of an
+ * attention block, whose six adapter derivatives (dA and dB of each) "Unsloth vs
+ * PyTorch: The ONLY Video You Need to Understand the Difference" counts at transcript
+ * 1:14-1:24.  G projections g = 0..G-1 with weights W_g:[N_g,K], adapters A_g:[r,K],
+ * B_g:[N_g,r] and a common scale s read the same X:
+ *
+ *     Y_g = X·W_gᵀ + s·(X·A_gᵀ)·B_gᵀ
+ *     dX  = Σ_g (dY_g·W_g + s·(dY_g·B_g)·A_g)     dB_g = s·dY_gᵀ·(X·A_gᵀ)     dA_g = s·(dY_g·B_g)ᵀ·X
+ *
+ * computed as one layer: X is read once for all X·A_gᵀ, one GEMM produces every Y_g, and
+ * one GEMM produces dX with the G adapter terms summed inside it.  The caller stacks the
+ * projections along rows: W (lora_weight_t) = [W_0; W_1; ...] of N = ΣN_g rows;
+ * A = [A_0; A_1; ...] bf16 [G·r, K]; B = [B_0; B_1; ...] bf16 [N, r]; Y, dY: [M, N]
+ * (projection g in columns [N_0+...+N_{g-1}, +N_g)); XA: bf16 [M, G·r] (X·A_gᵀ in
+ * columns [g·r, g·r+r)); dA: [G·r, K]; dB: [N, r].
+ * Limits: 1 <= G <= LORA_MAX_SEGMENTS, G·r <= 128, N_g % 8 == 0, and every projection
+ * but the last starts and ends on a multiple of 256 rows (LORA_ERR_UNSUPPORTED
+ * otherwise); ΣN_g must equal W->N (LORA_ERR_INVALID_ARG).  The workspace is
+ * lora_grouped_workspace_bytes(M, N, K, r, G, fmt).  G = 1 is exactly lora_linear_fwd /
+ * lora_linear_bwd.
+ */
+#define LORA_MAX_SEGMENTS 8
+typedef struct {
+  int32_t count;                       /* G */
+  int32_t reserved;                    /* must be 0 */
+  int64_t rows[LORA_MAX_SEGMENTS];     /* N_g; entries past count are ignored */
+} lora_segments_t;
+
+size_t lora_grouped_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int32_t nseg, int32_t fmt);
+
+lora_status_t lora_grouped_fwd(const void* X, int64_t M, const lora_weight_t* W, const lora_segments_t* segs,
+                               const void* A, const void* B, int32_t r, float s,
+                               void* Y, void* XA,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, int64_t M,
+                               const lora_weight_t* W, const lora_segments_t* segs,
+                               const void* A, const void* B, int32_t r, float s,
+                               void* dX, void* dA, void* dB,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Standalone dequantization of a LORA_W_BLOCK4 weight to bf16 [N,K] (device, out),
  * element by element as defined for lora_weight_t.  Bit-exact.  Not used by the
  * forward/backward, which dequantize tiles in shared memory and never write a

@@ -26,6 +26,10 @@ from .binding import (  # noqa: F401
     lora_linear_bwd,
     lora_linear_fwd,
     lora_linear_fwd_noalloc,
+    lora_grouped_fwd,
+    lora_grouped_bwd,
+    grouped_workspace_bytes,
+    segments,
     LORA_ERR_SCRATCH_LIMIT,
     LORA_NOALLOC_SCRATCH_BYTES,
     lora_merge,
@@ -38,5 +42,5 @@ from .binding import (  # noqa: F401
     status_string,
     workspace_bytes,
 )
-from .layer import LoraLinear  # noqa: F401
+from .layer import LoraGroupedLinear, LoraLinear  # noqa: F401
 from .dp import allreduce_adapter_grads, token_shard  # noqa: F401

@@ -33,8 +33,10 @@ EXPORTED = (
     "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
     "lora_testing_bounded_wait", "lora_timing_enable", "lora_timing_read", "lora_launch_count",
-    "lora_linear_fwd_noalloc",
+    "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
 )
+
+LORA_MAX_SEGMENTS = 8
 
 
 class LoraError(RuntimeError):
@@ -53,6 +55,26 @@ class lora_weight_t(ctypes.Structure):
         ("absmax", ctypes.c_void_p),
         ("codebook", ctypes.c_void_p),
     ]
+
+
+class lora_segments_t(ctypes.Structure):
+    _fields_ = [
+        ("count", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("rows", ctypes.c_int64 * 8),
+    ]
+
+
+def segments(rows) -> lora_segments_t:
+    rows = [int(x) for x in rows]
+    if not 1 <= len(rows) <= LORA_MAX_SEGMENTS:
+        raise ValueError("between 1 and 8 projections")
+    seg = lora_segments_t()
+    seg.count = len(rows)
+    seg.reserved = 0
+    for i, n in enumerate(rows):
+        seg.rows[i] = n
+    return seg
 
 
 def _load() -> ctypes.CDLL:
@@ -87,6 +109,13 @@ def _load() -> ctypes.CDLL:
     lib.lora_launch_count.restype = i64
     lib.lora_linear_fwd_noalloc.argtypes = [vp, i64, W, vp, vp, i32, f32, vp, vp, vp]
     lib.lora_linear_fwd_noalloc.restype = i32
+    S = ctypes.POINTER(lora_segments_t)
+    lib.lora_grouped_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
+    lib.lora_grouped_workspace_bytes.restype = sz
+    lib.lora_grouped_fwd.argtypes = [vp, i64, W, S, vp, vp, i32, f32, vp, vp, vp, sz, vp]
+    lib.lora_grouped_fwd.restype = i32
+    lib.lora_grouped_bwd.argtypes = [vp, vp, vp, i64, W, S, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
+    lib.lora_grouped_bwd.restype = i32
     return lib
 
 
@@ -221,3 +250,28 @@ def lora_linear_fwd_noalloc(X, M: int, W: LoraWeight, A, B, r: int, s: float, Y,
     w = W.c_struct()
     _check(_lib.lora_linear_fwd_noalloc(_ptr(X), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r), float(s),
                                         _ptr(Y), _ptr(XA), _stream(stream)), "lora_linear_fwd_noalloc")
+
+
+def grouped_workspace_bytes(M: int, N: int, K: int, r: int, nseg: int, fmt: int = LORA_W_BF16) -> int:
+    return int(_lib.lora_grouped_workspace_bytes(int(M), int(N), int(K), int(r), int(nseg), int(fmt)))
+
+
+def lora_grouped_fwd(X, M: int, W: LoraWeight, rows, A, B, r: int, s: float, Y, XA, workspace, ws_bytes=None,
+                     stream=None) -> None:
+    """Forward of G projections sharing X (weights stacked along rows, see lora_linear.h)."""
+    w = W.c_struct()
+    seg = segments(rows)
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_grouped_fwd(_ptr(X), int(M), ctypes.byref(w), ctypes.byref(seg), _ptr(A), _ptr(B), int(r),
+                                 float(s), _ptr(Y), _ptr(XA), _ptr(workspace), int(nb), _stream(stream)),
+           "lora_grouped_fwd")
+
+
+def lora_grouped_bwd(dY, X, XA, M: int, W: LoraWeight, rows, A, B, r: int, s: float, dX, dA, dB, workspace,
+                     ws_bytes=None, stream=None) -> None:
+    w = W.c_struct()
+    seg = segments(rows)
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_grouped_bwd(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), ctypes.byref(seg), _ptr(A),
+                                 _ptr(B), int(r), float(s), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), int(nb),
+                                 _stream(stream)), "lora_grouped_bwd")

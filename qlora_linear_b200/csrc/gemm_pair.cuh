@@ -39,7 +39,12 @@ struct PairParams {
   int M;               // rows of Aop / out
   int Nout;            // columns of out
   int Kred;            // reduction length (K forward, N backward)
-  int r;               // adapter rank (<= 128): one extra K fill
+  int r;               // rank of the LoRA fill (<= 128): one extra K fill
+  // Grouped projections (forward): output tile columns [seg_end[g-1], seg_end[g]) (in
+  // 256-column tiles) belong to segment g, whose E columns start at g * e_seg_stride.
+  int nseg;            // 1 for a single projection
+  int e_seg_stride;
+  int seg_end_tile[8];
   __nv_bfloat16* out;  // [M, Nout] row-major
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
@@ -206,7 +211,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
         for (int kb = 0; kb < nkb + n_ext; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
           const bool ext = kb >= nkb;
-          const int e = kb - nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const uint32_t sC = sB + C::B_BYTES;
@@ -234,7 +238,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmB, full_l, brow + C::ATOM, kb * C::BK);
             }
           } else {
-            for (int h = 0; h < ext_atoms; ++h) tma_load_2d_pair(sA + h * (C::A_BYTES / 2), &tmE, full_l, h * C::ATOM, arow);
+            int seg = 0;
+            while (seg + 1 < p.nseg && nb >= p.seg_end_tile[seg]) ++seg;
+            const int e0 = seg * p.e_seg_stride;  // this tile's columns of E
+            for (int h = 0; h < ext_atoms; ++h)
+              tma_load_2d_pair(sA + h * (C::A_BYTES / 2), &tmE, full_l, e0 + h * C::ATOM, arow);
             if (!B_MN) {
               for (int h = 0; h < ext_atoms; ++h)
                 tma_load_2d_pair(sB + h * (C::B_BYTES / 2), &tmF, full_l, h * C::ATOM, brow);

@@ -16,7 +16,6 @@
 #include "lora_linear_profiling.h"
 #include "lora_linear_testing.h"
 #include "elementwise.cuh"
-#include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "skinny.cuh"
 
@@ -130,10 +129,6 @@ lora_status_t dev_info(DevInfo** out) {
   if (!d.attrs_set) {
     bool ok = true;
 #define SET_SMEM(fn, bytes) ok &= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-    SET_SMEM((lora_gemm_kernel<false, false>), (GemmCfg<false, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_kernel<true, false>), (GemmCfg<true, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_kernel<false, true>), (GemmCfg<false, true>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_kernel<true, true>), (GemmCfg<true, true>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<false, false>), (PairCfg<false, false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<true, false>), (PairCfg<true, false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<false, true>), (PairCfg<false, true>::SMEM_BYTES));
@@ -243,95 +238,295 @@ int finalize_grid(size_t n) {
 
 // ---------------------------------------------------------------- skinny launches
 template <bool Q_T>
-lora_status_t launch_rowproj(const __nv_bfloat16* P, const __nv_bfloat16* Q, float* part, int M, int Kred, int r,
-                             Split sp, cudaStream_t st) {
+lora_status_t launch_rowproj(const __nv_bfloat16* P, int ldp, const __nv_bfloat16* Q, float* part, int M, int Kred,
+                             int r, Split sp, cudaStream_t st) {
   dim3 grid(cdiv(M, SK_BM), sp.splits);
   if (r <= 16)
-    rowproj_kernel<16, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<16, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+    rowproj_kernel<16, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<16, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
+                                                                                     sp.tiles_per_split);
   else if (r <= 32)
-    rowproj_kernel<32, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<32, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+    rowproj_kernel<32, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<32, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
+                                                                                     sp.tiles_per_split);
   else if (r <= 64)
-    rowproj_kernel<64, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<64, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+    rowproj_kernel<64, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<64, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
+                                                                                     sp.tiles_per_split);
   else
-    rowproj_kernel<128, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<128, Q_T>(), st>>>(P, Q, part, M, Kred, r, sp.tiles_per_split);
+    rowproj_kernel<128, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<128, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
+                                                                                       sp.tiles_per_split);
   count_launch();
   return last_launch();
 }
 
-lora_status_t launch_colproj(const __nv_bfloat16* P, const __nv_bfloat16* R, float* part, int M, int Kout, int r,
-                             Split sp, cudaStream_t st) {
+lora_status_t launch_colproj(const __nv_bfloat16* P, int ldp, const __nv_bfloat16* R, int ldr, float* part, int M,
+                             int Kout, int r, Split sp, cudaStream_t st) {
   dim3 grid(cdiv(Kout, SK_BM), sp.splits);
   if (r <= 16)
-    colproj_kernel<16><<<grid, SK_THREADS, colproj_smem_bytes<16>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+    colproj_kernel<16><<<grid, SK_THREADS, colproj_smem_bytes<16>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
+                                                                           sp.tiles_per_split);
   else if (r <= 32)
-    colproj_kernel<32><<<grid, SK_THREADS, colproj_smem_bytes<32>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+    colproj_kernel<32><<<grid, SK_THREADS, colproj_smem_bytes<32>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
+                                                                           sp.tiles_per_split);
   else if (r <= 64)
-    colproj_kernel<64><<<grid, SK_THREADS, colproj_smem_bytes<64>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+    colproj_kernel<64><<<grid, SK_THREADS, colproj_smem_bytes<64>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
+                                                                           sp.tiles_per_split);
   else
-    colproj_kernel<128><<<grid, SK_THREADS, colproj_smem_bytes<128>(), st>>>(P, R, part, M, Kout, r, sp.tiles_per_split);
+    colproj_kernel<128><<<grid, SK_THREADS, colproj_smem_bytes<128>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
+                                                                             sp.tiles_per_split);
+  count_launch();
+  return last_launch();
+}
+
+// Σ of the split partials [splits][rows][r] -> out1 (plain) and/or out2 (times scale),
+// row i written at out + i*opitch.
+lora_status_t finalize_rows(const float* part, int splits, long long rows, int r, int opitch, float scale,
+                            __nv_bfloat16* out1, __nv_bfloat16* out2, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(rows) * r;
+  finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, splits, n, r, opitch, scale, out1, out2);
+  count_launch();
+  return last_launch();
+}
+
+// scale · Σ of the split partials [splits][C][r] -> out [C][r], or [r][C] if transpose.
+lora_status_t finalize_cols(const float* part, int splits, int C, int r, float scale, bool transpose,
+                            __nv_bfloat16* out, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(C) * r;
+  finalize_cols_kernel<<<finalize_grid(n), 256, 0, st>>>(part, splits, C, r, scale, transpose ? 1 : 0, out);
   count_launch();
   return last_launch();
 }
 
 // ---------------------------------------------------------------- GEMM launch
-// GEMM kernel family: CTA pairs (default) or single CTAs (LORA_GEMM_1SM=1, kept for
-// comparison measurements).
-bool use_single_cta_gemm() {
-  static const bool v = [] {
-    const char* e = std::getenv("LORA_GEMM_1SM");
-    return e && e[0] == '1';
-  }();
-  return v;
-}
-
-// Tensor-map boxes of the four GEMM operands (x = inner extent, y = rows).
-struct GemmBoxes {
-  uint32_t a_y, b_x, b_y, c_x, c_y, f_x, f_y;
-};
-GemmBoxes gemm_boxes(bool b_mn) {
-  if (use_single_cta_gemm()) {
-    return b_mn ? GemmBoxes{128, 64, 64, 128, 64, 64, 64} : GemmBoxes{128, 64, 256, 32, 256, 64, 256};
-  }
-  // CTA pairs: every box is 64 elements (or 64 code bytes) wide and 128 rows high
-  return GemmBoxes{128, 64, 128, 64, 128, 64, 128};
-}
-
 template <bool B_MN, bool W4>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
-                          const GemmParams& p, int sms, cudaStream_t st) {
-  if (use_single_cta_gemm()) {
-    using C = GemmCfg<B_MN, W4>;
-    const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, C::BN);
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    {
-      TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-      lora_gemm_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
-    }
-    count_launch();
-    return last_launch();
-  }
+                          const PairParams& p, int sms, cudaStream_t st) {
   using C = PairCfg<B_MN, W4>;
-  PairParams q;
-  q.M = p.M;
-  q.Nout = p.Nout;
-  q.Kred = p.Kred;
-  q.r = p.r;
-  q.out = p.out;
-  q.status = p.status;
-  q.wait_ns = p.wait_ns;
-  q.absmax = p.absmax;
-  q.codebook = p.codebook;
-  q.Nw = p.Nw;
-  q.Kw = p.Kw;
   const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, C::BN);
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_pair_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, q);
+    lora_gemm_pair_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
   }
   count_launch();
   return last_launch();
+}
+
+// Every tensor-map box of the pair GEMM is 64 elements (or 64 code bytes) wide, 128 rows high.
+constexpr uint32_t kBoxX = 64, kBoxY = 128;
+
+// ---------------------------------------------------------------- output segments
+// Grouped projections share X: W, A and B stack the projections' weights, adapters
+// A_g [r, K] and B_g [N_g, r] along rows.  A single projection is one segment.
+struct Segs {
+  int n = 1;
+  long long rows[LORA_MAX_SEGMENTS] = {};
+  long long off[LORA_MAX_SEGMENTS + 1] = {};
+};
+
+lora_status_t make_segs(const lora_segments_t* sg, long long N, Segs* out) {
+  Segs s;
+  if (!sg) {
+    s.n = 1;
+    s.rows[0] = N;
+    s.off[1] = N;
+    *out = s;
+    return LORA_OK;
+  }
+  if (sg->count < 1 || sg->count > LORA_MAX_SEGMENTS || sg->reserved != 0) return LORA_ERR_INVALID_ARG;
+  s.n = sg->count;
+  for (int g = 0; g < s.n; ++g) {
+    if (sg->rows[g] <= 0) return LORA_ERR_INVALID_ARG;
+    if (sg->rows[g] % 8 != 0) return LORA_ERR_UNSUPPORTED;
+    s.rows[g] = sg->rows[g];
+    s.off[g + 1] = s.off[g] + sg->rows[g];
+    // a 256-column output tile must not straddle two projections
+    if (g + 1 < s.n && s.off[g + 1] % 256 != 0) return LORA_ERR_UNSUPPORTED;
+  }
+  if (s.off[s.n] != N) return LORA_ERR_INVALID_ARG;
+  *out = s;
+  return LORA_OK;
+}
+
+void set_segments(PairParams& p, const Segs& sg, int e_stride) {
+  p.nseg = sg.n;
+  p.e_seg_stride = e_stride;
+  for (int g = 0; g < LORA_MAX_SEGMENTS; ++g)
+    p.seg_end_tile[g] = g < sg.n ? static_cast<int>(sg.off[g + 1] / 256) : 0x7fffffff;
+}
+
+PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void* out, uint32_t* status,
+                       const lora_weight_t* W) {
+  PairParams p{};
+  p.M = static_cast<int>(M);
+  p.Nout = static_cast<int>(Nout);
+  p.Kred = static_cast<int>(Kred);
+  p.r = r;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = status;
+  p.wait_ns = wait_limit_ns();
+  p.nseg = 1;
+  p.e_seg_stride = 0;
+  for (int g = 0; g < LORA_MAX_SEGMENTS; ++g) p.seg_end_tile[g] = 0x7fffffff;
+  p.Nw = static_cast<int>(W->N);
+  p.Kw = static_cast<int>(W->K);
+  if (W->fmt == LORA_W_BLOCK4) {
+    p.absmax = static_cast<const __half*>(W->absmax);
+    p.codebook = W->codebook;
+  }
+  return p;
+}
+
+// ---------------------------------------------------------------- forward core
+// XA = X·Aᵀ for all segments at once (rank G·r), then Y = X·Wᵀ + s·XA_g·B_gᵀ with the
+// LoRA fill of each output tile taking its segment's columns of s·XA.
+lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, const Segs& sg, const void* A,
+                           const void* B, int r, float s, void* Y, void* XA, __nv_bfloat16* sXA, float* part,
+                           uint32_t* status, cudaStream_t st) {
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  const long long N = W->N, K = W->K;
+  const int rt = sg.n * r;
+  const int Mi = static_cast<int>(M), Ki = static_cast<int>(K);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+
+  const Split sp = rowproj_split(M, K);
+  TRY(launch_rowproj<false>(Xb, Ki, static_cast<const __nv_bfloat16*>(A), part, Mi, Ki, rt, sp, st));
+  TRY(finalize_rows(part, sp.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
+
+  CUtensorMap ta, tb, te, tf;
+  TRY(tmap_bf16(&ta, X, K, M, kBoxX, kBoxY));
+  TRY(tmap_bf16(&te, sXA, rt, M, kBoxX, kBoxY));
+  TRY(tmap_bf16(&tf, B, r, N, kBoxX, kBoxY));
+  PairParams p = gemm_params(M, N, K, r, Y, status, W);
+  set_segments(p, sg, r);
+  if (W->fmt == LORA_W_BF16) {
+    TRY(tmap_bf16(&tb, W->data, K, N, kBoxX, kBoxY));
+    return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
+  }
+  TRY(tmap_u8(&tb, W->data, K / 2, N, kBoxX, kBoxY));
+  return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
+}
+
+// ---------------------------------------------------------------- backward core
+lora_status_t backward_core(const void* dY, const void* X, const void* XA, long long M, const lora_weight_t* W,
+                            const Segs& sg, const void* A, const void* B, int r, float s, void* dX, void* dA,
+                            void* dB, __nv_bfloat16* sdYB, float* part, uint32_t* status, cudaStream_t st) {
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  const long long N = W->N, K = W->K;
+  const int rt = sg.n * r;
+  const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+  const auto* dYb = static_cast<const __nv_bfloat16*>(dY);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  const auto* Bb = static_cast<const __nv_bfloat16*>(B);
+  const auto* XAb = static_cast<const __nv_bfloat16*>(XA);
+
+  for (int g = 0; g < sg.n; ++g) {
+    const int rows = static_cast<int>(sg.rows[g]);
+    const long long o = sg.off[g];
+    // s·dY_g·B_g -> columns [g·r, g·r + r) of s·dY·B
+    const Split sp = rowproj_split(M, rows);
+    TRY(launch_rowproj<true>(dYb + o, Ni, Bb + o * r, part, Mi, rows, r, sp, st));
+    TRY(finalize_rows(part, sp.splits, M, r, rt, s, nullptr, sdYB + g * r, st));
+  }
+  for (int g = 0; g < sg.n; ++g) {
+    const int rows = static_cast<int>(sg.rows[g]);
+    const long long o = sg.off[g];
+    // dB_g = s·dY_gᵀ·XA_g
+    const Split sp = colproj_split(M, rows);
+    TRY(launch_colproj(dYb + o, Ni, XAb + g * r, rt, part, Mi, rows, r, sp, st));
+    TRY(finalize_cols(part, sp.splits, rows, r, s, false, static_cast<__nv_bfloat16*>(dB) + o * r, st));
+  }
+  if (dX) {
+    // dX = dY·W + (s·dY·B)·A with the LoRA fill over all G·r ranks
+    CUtensorMap ta, tb, te, tf;
+    TRY(tmap_bf16(&ta, dY, N, M, kBoxX, kBoxY));
+    TRY(tmap_bf16(&te, sdYB, rt, M, kBoxX, kBoxY));
+    TRY(tmap_bf16(&tf, A, K, rt, kBoxX, kBoxY));
+    PairParams p = gemm_params(M, K, N, rt, dX, status, W);
+    if (W->fmt == LORA_W_BF16) {
+      TRY(tmap_bf16(&tb, W->data, K, N, kBoxX, kBoxY));
+      TRY((launch_gemm<true, false>(ta, tb, te, tf, p, dev->sms, st)));
+    } else {
+      TRY(tmap_u8(&tb, W->data, K / 2, N, kBoxX, kBoxY));
+      TRY((launch_gemm<true, true>(ta, tb, te, tf, p, dev->sms, st)));
+    }
+  }
+  // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
+  const Split sp = colproj_split(M, K);
+  TRY(launch_colproj(Xb, Ki, sdYB, rt, part, Mi, Ki, rt, sp, st));
+  return finalize_cols(part, sp.splits, Ki, rt, 1.0f, true, static_cast<__nv_bfloat16*>(dA), st);
+}
+
+// ---------------------------------------------------------------- argument checks shared by the entries
+lora_status_t check_common(const lora_weight_t* W, const lora_segments_t* segs, int r, float s, long long M,
+                           const void* A, const void* B, Segs* sg) {
+  TRY(check_weight(W));
+  TRY(check_rank(r, s));
+  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
+  TRY(make_segs(segs, W->N, sg));
+  if (sg->n * r > 128) return LORA_ERR_UNSUPPORTED;
+  TRY(check_ptr(A));
+  TRY(check_ptr(B));
+  return LORA_OK;
+}
+
+lora_status_t fwd_entry(const void* X, int64_t M, const lora_weight_t* W, const lora_segments_t* segs, const void* A,
+                        const void* B, int32_t r, float s, void* Y, void* XA, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  Segs sg;
+  TRY(check_common(W, segs, r, s, M, A, B, &sg));
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(X));
+  TRY(check_ptr(Y));
+  TRY(check_ptr(XA));
+  const WsLayout wl = ws_layout(M, W->N, W->K, sg.n * r);
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return forward_core(X, M, W, sg, A, B, r, s, Y, XA, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
+                      reinterpret_cast<float*>(ws + wl.part_off), reinterpret_cast<uint32_t*>(ws),
+                      static_cast<cudaStream_t>(stream));
+}
+
+lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
+                        const lora_segments_t* segs, const void* A, const void* B, int32_t r, float s, void* dX,
+                        void* dA, void* dB, void* workspace, size_t ws_bytes, void* stream) {
+  Segs sg;
+  TRY(check_common(W, segs, r, s, M, A, B, &sg));
+  TRY(check_ptr(dA));
+  TRY(check_ptr(dB));
+  const long long N = W->N, K = W->K;
+  const int rt = sg.n * r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(rt) * K * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
+    return LORA_OK;
+  }
+  TRY(check_ptr(dY));
+  TRY(check_ptr(X));
+  TRY(check_ptr(XA));
+  if (dX && !aligned16(dX)) return LORA_ERR_ALIGNMENT;
+  const WsLayout wl = ws_layout(M, N, K, rt);
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return backward_core(dY, X, XA, M, W, sg, A, B, r, s, dX, dA, dB,
+                       reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off), reinterpret_cast<float*>(ws + wl.part_off),
+                       reinterpret_cast<uint32_t*>(ws), st);
+}
+
+size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K, int32_t r, int32_t nseg, int32_t fmt) {
+  if (M < 0 || N <= 0 || K <= 0 || r < 8 || r > 128 || r % 8) return 0;
+  if (nseg < 1 || nseg > LORA_MAX_SEGMENTS || nseg * r > 128) return 0;
+  if (fmt != LORA_W_BF16 && fmt != LORA_W_BLOCK4) return 0;
+  if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 30)) return 0;
+  return ws_layout(M, N, K, nseg * r).total;
 }
 
 }  // namespace
@@ -346,7 +541,9 @@ const char* lora_status_string(int32_t status) {
     case LORA_OK: return "ok";
     case LORA_ERR_INVALID_ARG: return "invalid argument (null pointer, bad size, non-finite scale or bad enum)";
     case LORA_ERR_ALIGNMENT: return "a device pointer is not 16-byte aligned";
-    case LORA_ERR_UNSUPPORTED: return "unsupported sizes (need 8<=r<=128, r%8==0, N%8==0, K%8==0; K%64==0 for 4-bit)";
+    case LORA_ERR_UNSUPPORTED:
+      return "unsupported sizes (need 8<=r<=128, r%8==0, N%8==0, K%8==0; K%64==0 for 4-bit; "
+             "projections of a group start at multiples of 256 rows and G*r<=128)";
     case LORA_ERR_WORKSPACE: return "workspace missing or smaller than lora_workspace_bytes()";
     case LORA_ERR_CUDA: return "a CUDA call failed";
     case LORA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait; outputs of that call are undefined";
@@ -356,165 +553,39 @@ const char* lora_status_string(int32_t status) {
   }
 }
 
-int32_t lora_version(void) { return 100; }
+int32_t lora_version(void) { return 200; }
 
 size_t lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int32_t fmt) {
-  if (M < 0 || N <= 0 || K <= 0 || r < 8 || r > 128 || r % 8) return 0;
-  if (fmt != LORA_W_BF16 && fmt != LORA_W_BLOCK4) return 0;
-  if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 30)) return 0;
-  return ws_layout(M, N, K, r).total;
+  return workspace_bytes_for(M, N, K, r, 1, fmt);
+}
+
+size_t lora_grouped_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int32_t nseg, int32_t fmt) {
+  return workspace_bytes_for(M, N, K, r, nseg, fmt);
 }
 
 lora_status_t lora_linear_fwd(const void* X, int64_t M, const lora_weight_t* W, const void* A, const void* B, int32_t r,
                               float s, void* Y, void* XA, void* workspace, size_t ws_bytes, void* stream) {
-  TRY(check_weight(W));
-  TRY(check_rank(r, s));
-  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
-  TRY(check_ptr(A));
-  TRY(check_ptr(B));
-  if (M == 0) return LORA_OK;
-  TRY(check_ptr(X));
-  TRY(check_ptr(Y));
-  TRY(check_ptr(XA));
-  const long long N = W->N, K = W->K;
-  const WsLayout wl = ws_layout(M, N, K, r);
-  if (!workspace) return LORA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
-  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
-  DevInfo* dev = nullptr;
-  TRY(dev_info(&dev));
-  TRY(get_encode());
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  __nv_bfloat16* sXA = reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off);
-  float* part = reinterpret_cast<float*>(ws + wl.part_off);
-  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
-
-  // XA = X·Aᵀ (saved for the backward) and s·XA (the LoRA K block of the GEMM)
-  const Split sp = rowproj_split(M, K);
-  TRY(launch_rowproj<false>(Xb, static_cast<const __nv_bfloat16*>(A), part, static_cast<int>(M), static_cast<int>(K), r,
-                            sp, st));
-  const size_t n = static_cast<size_t>(M) * r;
-  finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, sp.splits, n, s, static_cast<__nv_bfloat16*>(XA), sXA);
-  count_launch();
-  TRY(last_launch());
-
-  // Y = X·Wᵀ + (s·XA)·Bᵀ
-  CUtensorMap ta, tb, te, tf;
-  const GemmBoxes bx = gemm_boxes(false);
-  TRY(tmap_bf16(&ta, X, K, M, 64, bx.a_y));
-  TRY(tmap_bf16(&te, sXA, r, M, 64, bx.a_y));
-  TRY(tmap_bf16(&tf, B, r, N, bx.f_x, bx.f_y));
-  GemmParams p{};
-  p.M = static_cast<int>(M);
-  p.Nout = static_cast<int>(N);
-  p.Kred = static_cast<int>(K);
-  p.r = r;
-  p.out = static_cast<__nv_bfloat16*>(Y);
-  p.status = reinterpret_cast<uint32_t*>(ws);
-  p.wait_ns = wait_limit_ns();
-  p.Nw = static_cast<int>(N);
-  p.Kw = static_cast<int>(K);
-  if (W->fmt == LORA_W_BF16) {
-    TRY(tmap_bf16(&tb, W->data, K, N, bx.b_x, bx.b_y));
-    return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
-  }
-  TRY(tmap_u8(&tb, W->data, K / 2, N, bx.c_x, bx.c_y));
-  p.absmax = static_cast<const __half*>(W->absmax);
-  p.codebook = W->codebook;
-  return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
+  return fwd_entry(X, M, W, nullptr, A, B, r, s, Y, XA, workspace, ws_bytes, stream);
 }
 
 lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
                               const void* A, const void* B, int32_t r, float s, void* dX, void* dA, void* dB,
                               void* workspace, size_t ws_bytes, void* stream) {
-  TRY(check_weight(W));
-  TRY(check_rank(r, s));
-  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
-  TRY(check_ptr(A));
-  TRY(check_ptr(B));
-  TRY(check_ptr(dA));
-  TRY(check_ptr(dB));
-  const long long N = W->N, K = W->K;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (M == 0) {
-    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
-    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
-    return LORA_OK;
-  }
-  TRY(check_ptr(dY));
-  TRY(check_ptr(X));
-  TRY(check_ptr(XA));
-  if (dX && !aligned16(dX)) return LORA_ERR_ALIGNMENT;
-  const WsLayout wl = ws_layout(M, N, K, r);
-  if (!workspace) return LORA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
-  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
-  DevInfo* dev = nullptr;
-  TRY(dev_info(&dev));
-  TRY(get_encode());
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  __nv_bfloat16* sdYB = reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off);
-  float* part = reinterpret_cast<float*>(ws + wl.part_off);
-  const auto* dYb = static_cast<const __nv_bfloat16*>(dY);
-  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
-  const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+  return bwd_entry(dY, X, XA, M, W, nullptr, A, B, r, s, dX, dA, dB, workspace, ws_bytes, stream);
+}
 
-  // s·(dY·B)  [M, r]
-  {
-    const Split sp = rowproj_split(M, N);
-    TRY(launch_rowproj<true>(dYb, static_cast<const __nv_bfloat16*>(B), part, Mi, Ni, r, sp, st));
-    const size_t n = static_cast<size_t>(M) * r;
-    finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, sp.splits, n, s, nullptr, sdYB);
-    count_launch();
-    TRY(last_launch());
-  }
-  // dB = s·dYᵀ·XA  [N, r]
-  {
-    const Split sp = colproj_split(M, N);
-    TRY(launch_colproj(dYb, static_cast<const __nv_bfloat16*>(XA), part, Mi, Ni, r, sp, st));
-    const size_t n = static_cast<size_t>(N) * r;
-    finalize_cols_kernel<<<finalize_grid(n), 256, 0, st>>>(part, sp.splits, Ni, r, s, 0, static_cast<__nv_bfloat16*>(dB));
-    count_launch();
-    TRY(last_launch());
-  }
-  // dX = dY·W + (s·dY·B)·A
-  if (dX) {
-    CUtensorMap ta, tb, te, tf;
-    const GemmBoxes bx = gemm_boxes(true);
-    TRY(tmap_bf16(&ta, dY, N, M, 64, bx.a_y));
-    TRY(tmap_bf16(&te, sdYB, r, M, 64, bx.a_y));
-    TRY(tmap_bf16(&tf, A, K, r, bx.f_x, bx.f_y));
-    GemmParams p{};
-    p.M = Mi;
-    p.Nout = Ki;
-    p.Kred = Ni;
-    p.r = r;
-    p.out = static_cast<__nv_bfloat16*>(dX);
-    p.status = reinterpret_cast<uint32_t*>(ws);
-    p.wait_ns = wait_limit_ns();
-    p.Nw = Ni;
-    p.Kw = Ki;
-    if (W->fmt == LORA_W_BF16) {
-      TRY(tmap_bf16(&tb, W->data, K, N, bx.b_x, bx.b_y));
-      TRY((launch_gemm<true, false>(ta, tb, te, tf, p, dev->sms, st)));
-    } else {
-      TRY(tmap_u8(&tb, W->data, K / 2, N, bx.c_x, bx.c_y));
-      p.absmax = static_cast<const __half*>(W->absmax);
-      p.codebook = W->codebook;
-      TRY((launch_gemm<true, true>(ta, tb, te, tf, p, dev->sms, st)));
-    }
-  }
-  // dA = (s·dY·B)ᵀ·X  [r, K], computed as Xᵀ·(s·dY·B) and written transposed
-  {
-    const Split sp = colproj_split(M, K);
-    TRY(launch_colproj(Xb, sdYB, part, Mi, Ki, r, sp, st));
-    const size_t n = static_cast<size_t>(K) * r;
-    finalize_cols_kernel<<<finalize_grid(n), 256, 0, st>>>(part, sp.splits, Ki, r, 1.0f, 1, static_cast<__nv_bfloat16*>(dA));
-    count_launch();
-    TRY(last_launch());
-  }
-  return LORA_OK;
+lora_status_t lora_grouped_fwd(const void* X, int64_t M, const lora_weight_t* W, const lora_segments_t* segs,
+                               const void* A, const void* B, int32_t r, float s, void* Y, void* XA, void* workspace,
+                               size_t ws_bytes, void* stream) {
+  if (!segs) return LORA_ERR_INVALID_ARG;
+  return fwd_entry(X, M, W, segs, A, B, r, s, Y, XA, workspace, ws_bytes, stream);
+}
+
+lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
+                               const lora_segments_t* segs, const void* A, const void* B, int32_t r, float s,
+                               void* dX, void* dA, void* dB, void* workspace, size_t ws_bytes, void* stream) {
+  if (!segs) return LORA_ERR_INVALID_ARG;
+  return bwd_entry(dY, X, XA, M, W, segs, A, B, r, s, dX, dA, dB, workspace, ws_bytes, stream);
 }
 
 lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* stream) {
@@ -662,61 +733,22 @@ extern "C" {
 
 lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weight_t* W, const void* A, const void* B,
                                       int32_t r, float s, void* Y, void* XA, void* stream) {
-  TRY(check_weight(W));
-  TRY(check_rank(r, s));
-  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
-  TRY(check_ptr(A));
-  TRY(check_ptr(B));
+  Segs sg;
+  TRY(check_common(W, nullptr, r, s, M, A, B, &sg));
   if (M == 0) return LORA_OK;
   TRY(check_ptr(X));
   TRY(check_ptr(Y));
   TRY(check_ptr(XA));
-  const long long N = W->N, K = W->K;
-  const NoAllocLayout nl = noalloc_layout(M, K, r);
+  const NoAllocLayout nl = noalloc_layout(M, W->K, r);
   if (nl.total > LORA_NOALLOC_SCRATCH_BYTES) return LORA_ERR_SCRATCH_LIMIT;
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
-  TRY(get_encode());
   uint8_t* scratch = nullptr;
   TRY(noalloc_scratch(&scratch));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  __nv_bfloat16* sXA = reinterpret_cast<__nv_bfloat16*>(scratch + nl.sxa_off);
-  float* part = reinterpret_cast<float*>(scratch + nl.part_off);
-  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
-
-  // XA = X·Aᵀ and s·XA; every partial the finalize reads is written by rowproj first
-  const Split sp = rowproj_split(M, K);
-  TRY(launch_rowproj<false>(Xb, static_cast<const __nv_bfloat16*>(A), part, static_cast<int>(M), static_cast<int>(K), r,
-                            sp, st));
-  const size_t n = static_cast<size_t>(M) * r;
-  finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, sp.splits, n, s, static_cast<__nv_bfloat16*>(XA), sXA);
-  count_launch();
-  TRY(last_launch());
-
-  // Y = X·Wᵀ + (s·XA)·Bᵀ; no status word (status = null): an expired wait ends the kernel silently
-  CUtensorMap ta, tb, te, tf;
-  const GemmBoxes bx = gemm_boxes(false);
-  TRY(tmap_bf16(&ta, X, K, M, 64, bx.a_y));
-  TRY(tmap_bf16(&te, sXA, r, M, 64, bx.a_y));
-  TRY(tmap_bf16(&tf, B, r, N, bx.f_x, bx.f_y));
-  GemmParams p{};
-  p.M = static_cast<int>(M);
-  p.Nout = static_cast<int>(N);
-  p.Kred = static_cast<int>(K);
-  p.r = r;
-  p.out = static_cast<__nv_bfloat16*>(Y);
-  p.status = nullptr;
-  p.wait_ns = wait_limit_ns();
-  p.Nw = static_cast<int>(N);
-  p.Kw = static_cast<int>(K);
-  if (W->fmt == LORA_W_BF16) {
-    TRY(tmap_bf16(&tb, W->data, K, N, bx.b_x, bx.b_y));
-    return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
-  }
-  TRY(tmap_u8(&tb, W->data, K / 2, N, bx.c_x, bx.c_y));
-  p.absmax = static_cast<const __half*>(W->absmax);
-  p.codebook = W->codebook;
-  return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
+  // every scratch byte read below (the split partials, then s·XA) is written earlier in
+  // the same call; no status word: an expired device wait ends the kernel silently
+  return forward_core(X, M, W, sg, A, B, r, s, Y, XA, reinterpret_cast<__nv_bfloat16*>(scratch + nl.sxa_off),
+                      reinterpret_cast<float*>(scratch + nl.part_off), nullptr, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

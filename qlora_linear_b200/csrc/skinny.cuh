@@ -55,16 +55,17 @@ __device__ __forceinline__ void load_tile_rows64(uint32_t sdst, int pitch, const
     cp_async_16(sdst + (rr * pitch + cc * 8) * 2, src, in ? 16u : 0u);
   }
 }
-// [64 rows × RPAD cols] tile of a row-major [nrows × r] matrix (r % 8 == 0), zero-filled
-// beyond nrows / r.
+// [64 rows × RPAD cols] tile of the first r columns of a row-major matrix with row pitch
+// ldg (r % 8 == 0), zero-filled beyond nrows / r.
 template <int RPAD>
-__device__ __forceinline__ void load_tile_rpad(uint32_t sdst, const __nv_bfloat16* g, int r, int row0, int nrows) {
+__device__ __forceinline__ void load_tile_rpad(uint32_t sdst, const __nv_bfloat16* g, int ldg, int r, int row0,
+                                               int nrows) {
   constexpr int CPR = RPAD / 8;  // 16-byte chunks per row
   for (int c = threadIdx.x; c < SK_BK * CPR; c += SK_THREADS) {
     const int rr = c / CPR, cc = c % CPR;
     const int gr = row0 + rr, gc = cc * 8;
     const bool in = gr < nrows && gc < r;
-    const __nv_bfloat16* src = in ? g + static_cast<size_t>(gr) * r + gc : g;
+    const __nv_bfloat16* src = in ? g + static_cast<size_t>(gr) * ldg + gc : g;
     cp_async_16(sdst + (rr * SkinnyCfg<RPAD>::QPITCH_T + cc * 8) * 2, src, in ? 16u : 0u);
   }
 }
@@ -72,8 +73,8 @@ __device__ __forceinline__ void load_tile_rpad(uint32_t sdst, const __nv_bfloat1
 // part[split][m][j] (fp32, row pitch r) over k-tiles [kt0, kt1) of split blockIdx.y.
 template <int RPAD, bool Q_T>
 __global__ void __launch_bounds__(SK_THREADS)
-    rowproj_kernel(const __nv_bfloat16* __restrict__ P, const __nv_bfloat16* __restrict__ Q, float* __restrict__ part,
-                   int M, int Kred, int r, int ktiles_per_split) {
+    rowproj_kernel(const __nv_bfloat16* __restrict__ P, int ldp, const __nv_bfloat16* __restrict__ Q,
+                   float* __restrict__ part, int M, int Kred, int r, int ktiles_per_split) {
   using S = SkinnyCfg<RPAD>;
   constexpr int QE = Q_T ? S::QT_ELEMS : S::QN_ELEMS;
   extern __shared__ __align__(16) uint8_t sk_smem[];
@@ -91,10 +92,10 @@ __global__ void __launch_bounds__(SK_THREADS)
   auto issue = [&](int i) {
     const int st = i % SK_STAGES;
     const int k0 = (kt0 + i) * SK_BK;
-    load_tile_rows64(sP(st), SK_PITCH, P, Kred, m0, M, k0, Kred, SK_BM);
+    load_tile_rows64(sP(st), SK_PITCH, P, ldp, m0, M, k0, Kred, SK_BM);
     if (Q_T) {
       // Q stored [Kred][r]: rows k0..k0+63
-      load_tile_rpad<RPAD>(sQ(st), Q, r, k0, Kred);
+      load_tile_rpad<RPAD>(sQ(st), Q, r, r, k0, Kred);
     } else {
       // Q stored [r][Kred]: RPAD rows j, columns k0..k0+63
       load_tile_rows64(sQ(st), SK_PITCH, Q, Kred, 0, r, k0, Kred, RPAD);
@@ -158,8 +159,8 @@ __global__ void __launch_bounds__(SK_THREADS)
 // part[split][c][j] (fp32, row pitch r) = Σ over m-tiles [mt0, mt1) of P[m][c]·R[m][j].
 template <int RPAD>
 __global__ void __launch_bounds__(SK_THREADS)
-    colproj_kernel(const __nv_bfloat16* __restrict__ P, const __nv_bfloat16* __restrict__ R, float* __restrict__ part,
-                   int M, int Kout, int r, int mtiles_per_split) {
+    colproj_kernel(const __nv_bfloat16* __restrict__ P, int ldp, const __nv_bfloat16* __restrict__ R, int ldr,
+                   float* __restrict__ part, int M, int Kout, int r, int mtiles_per_split) {
   using S = SkinnyCfg<RPAD>;
   extern __shared__ __align__(16) uint8_t sk_smem[];
   const uint32_t sbase = smem_u32(sk_smem);
@@ -176,8 +177,8 @@ __global__ void __launch_bounds__(SK_THREADS)
   auto issue = [&](int i) {
     const int st = i % SK_STAGES;
     const int mrow = (mt0 + i) * SK_BK;
-    load_tile_rows64(sP(st), SK_PITCH, P, Kout, mrow, M, c0, Kout, SK_BK);
-    load_tile_rpad<RPAD>(sR(st), R, r, mrow, M);
+    load_tile_rows64(sP(st), SK_PITCH, P, ldp, mrow, M, c0, Kout, SK_BK);
+    load_tile_rpad<RPAD>(sR(st), R, ldr, r, mrow, M);
   };
 
   float acc[RPAD / 8][4];
@@ -235,19 +236,22 @@ __global__ void __launch_bounds__(SK_THREADS)
 }
 
 // out1 = bf16(Σ_s part[s]), out2 = bf16(scale · Σ_s part[s]); either may be null.
-// part is [splits][rows*r]; summed in split order.
-__global__ void finalize_rows_kernel(const float* __restrict__ part, int splits, size_t n, float scale,
-                                     __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2) {
+// part is [splits][rows][r]; summed in split order.  Row i of the result goes to
+// out[i*opitch .. i*opitch + r) (opitch >= r lets a result fill one column block of a
+// wider matrix).
+__global__ void finalize_rows_kernel(const float* __restrict__ part, int splits, size_t n, int r, int opitch,
+                                     float scale, __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2) {
   for (size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x * 2) {
+    const size_t o = (opitch == r) ? i : (i / r) * opitch + i % r;
     float2 acc = *reinterpret_cast<const float2*>(part + i);
     for (int s = 1; s < splits; ++s) {
       const float2 v = *reinterpret_cast<const float2*>(part + static_cast<size_t>(s) * n + i);
       acc.x += v.x;
       acc.y += v.y;
     }
-    if (out1) *reinterpret_cast<uint32_t*>(out1 + i) = pack_bf16x2(acc.x, acc.y);
-    if (out2) *reinterpret_cast<uint32_t*>(out2 + i) = pack_bf16x2(scale * acc.x, scale * acc.y);
+    if (out1) *reinterpret_cast<uint32_t*>(out1 + o) = pack_bf16x2(acc.x, acc.y);
+    if (out2) *reinterpret_cast<uint32_t*>(out2 + o) = pack_bf16x2(scale * acc.x, scale * acc.y);
   }
 }
 

@@ -10,5 +10,6 @@ from .inputs import (  # noqa: F401
     bf16_bits_from_f32,
     f32_from_bf16_bits,
     make_case,
+    make_grouped_case,
     config_cases,
 )

@@ -181,3 +181,18 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
     if "dY" in want:
         out["dY"] = _fill((M, N), ds, _TID["dY"], _normal_bf16(1.0))
     return out
+
+
+def make_grouped_case(case: LoraCase, rows, want=("X", "W", "A", "B", "dY")) -> dict:
+    """Inputs of G projections sharing X: ``case.N`` must equal ``sum(rows)``; W, B and dY
+    are drawn for the stacked ``[ΣN_g, ...]`` shapes and A for ``[G·r, K]`` (same
+    distributions as :func:`make_case`)."""
+    rows = [int(n) for n in rows]
+    assert sum(rows) == case.N
+    G = len(rows)
+    out = make_case(case, want=tuple(w for w in want if w != "A"))
+    if "A" in want:
+        a = 1.0 / np.sqrt(case.K)
+        out["A"] = _fill((G * case.r, case.K), case.seed, _TID["A"], _uniform_bf16(-a, a))
+    out["rows"] = rows
+    return out

@@ -120,3 +120,28 @@ def test_workspace_bytes_is_a_pure_function_of_sizes():
     # grows with M and r
     assert q.workspace_bytes(512, 4096, 4096, 16) < q.workspace_bytes(4096, 4096, 4096, 16)
     assert q.workspace_bytes(4096, 4096, 4096, 16) < q.workspace_bytes(4096, 4096, 4096, 128)
+
+
+def test_grouped_validation():
+    from qlora_linear_b200.binding import segments
+    lib = q.lib()
+    W = _w(N=6144, K=512)
+
+    def gf(rows, r=16, nseg_ptr=True):
+        seg = segments(rows) if nseg_ptr else None
+        return lib.lora_grouped_fwd(P, 256, ctypes.byref(W), ctypes.byref(seg) if seg else None, P, P, r, 2.0, P, P,
+                                    P2, 1 << 30, None)
+
+    assert gf([4096, 1024, 1024], nseg_ptr=False) == q.LORA_ERR_INVALID_ARG
+    assert gf([4096, 1024, 1000]) == q.LORA_ERR_INVALID_ARG          # rows do not add up to N
+    assert gf([4000, 1024, 1120]) == q.LORA_ERR_UNSUPPORTED          # boundary not on 256 rows
+    assert gf([4096, 1024, 1024], r=48) == q.LORA_ERR_UNSUPPORTED    # G·r > 128
+    assert gf([6144, 0]) == q.LORA_ERR_INVALID_ARG
+    seg = segments([4096, 1024, 1024])
+    seg.reserved = 1
+    assert lib.lora_grouped_fwd(P, 256, ctypes.byref(W), ctypes.byref(seg), P, P, 16, 2.0, P, P, P2, 1 << 30,
+                                None) == q.LORA_ERR_INVALID_ARG
+    # the workspace grows with the number of projections and is zero when G·r > 128
+    assert q.grouped_workspace_bytes(4096, 6144, 4096, 16, 3) > q.workspace_bytes(4096, 6144, 4096, 16)
+    assert q.grouped_workspace_bytes(4096, 6144, 4096, 16, 1) == q.workspace_bytes(4096, 6144, 4096, 16)
+    assert q.grouped_workspace_bytes(4096, 6144, 4096, 48, 3) == 0
