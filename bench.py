@@ -4,7 +4,7 @@ One step = forward and backward of every projection of the workload (default: th
 Llama-8B MLP projections gate, up and down at M = 16384 tokens, r = 16, bf16 weight),
 with inputs resident in device memory.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|qkv] [--impl ours|reference]
 
 Multi-GPU (one process per GPU under torch.distributed.run): data parallel over tokens,
 every rank runs the full per-rank workload (weak scaling) and the adapter gradients dA
@@ -39,18 +39,21 @@ def workload(name: str):
               "M=16384, r=16, alpha=32, bf16 weight",
         "c3": "QLoRA 4-bit blockwise weight K=4096 N=14336 (16-level codebook, fp16 absmax per 64), "
               "M=8192, r=16, alpha=32",
+        "qkv": "Llama-8B attention q/k/v as one grouped layer (q 4096, k 1024, v 1024 rows, K=4096), "
+               "M=8192, r=16 per projection, alpha=32, bf16 weight",
     }[name]
     return cases, desc
 
 
 def case_flops(c) -> float:
-    """Algorithmic FLOPs of one forward + backward: 4MNK + 6Mr(N+K)."""
-    return 4.0 * c.M * c.N * c.K + 6.0 * c.M * c.r * (c.N + c.K)
+    """Algorithmic FLOPs of one forward + backward: 4MNK + 6Mr(N+K) per projection
+    (a grouped case sums this over its projections: 4MNK + 6Mr(N + G·K))."""
+    return 4.0 * c.M * c.N * c.K + 6.0 * c.M * c.r * (c.N + c.G * c.K)
 
 
 def gemm_flops(c) -> tuple[float, float]:
-    """Algorithmic FLOPs of the Y GEMM (2MNK + 2MNr) and of the dX GEMM (2MNK + 2MKr)."""
-    return 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.N * c.r, 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.K * c.r
+    """Algorithmic FLOPs of the Y GEMM (2MNK + 2MNr) and of the dX GEMM (2MNK + 2MK·Gr)."""
+    return 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.N * c.r, 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.K * c.G * c.r
 
 
 def load_peaks():
@@ -161,8 +164,18 @@ def oracle_sample(cases, tokens: int):
         c = inp["case"]
         W = O.weight_f64(inp)
         X, A, B, dY = (O.bf16_to_f64(inp[k]) for k in ("X", "A", "B", "dY"))
-        O.lora_forward(X, W, A, B, c.s)
-        O.lora_backward(dY, X, W, A, B, c.s)
+        if c.rows is None:
+            O.lora_forward(X, W, A, B, c.s)
+            O.lora_backward(dY, X, W, A, B, c.s)
+        else:
+            offs = [0]
+            for n in c.rows:
+                offs.append(offs[-1] + n)
+            Ws = [W[offs[g]:offs[g + 1]] for g in range(c.G)]
+            As = [A[g * c.r:(g + 1) * c.r] for g in range(c.G)]
+            Bs = [B[offs[g]:offs[g + 1]] for g in range(c.G)]
+            O.lora_grouped_forward(X, Ws, As, Bs, c.s)
+            O.lora_grouped_backward(dY, X, Ws, As, Bs, c.s)
         flops += case_flops(c)
     return time.perf_counter() - t0, flops
 
@@ -242,13 +255,16 @@ def run_ours(args, cases, desc, rank, world, local_rank):
             W = q.LoraWeight(c.N, c.K, d["W"])
         else:
             W = q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
-        layer = q.LoraLinear(W, d["A"], d["B"], c.alpha)
+        if c.rows is None:
+            layer = q.LoraLinear(W, d["A"], d["B"], c.alpha)
+        else:
+            layer = q.LoraGroupedLinear(W, c.rows, d["A"], d["B"], c.alpha)
         layer.workspace(c.M)
         out = {
             "Y": torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev),
-            "XA": torch.empty((c.M, c.r), dtype=torch.bfloat16, device=dev),
+            "XA": torch.empty((c.M, c.G * c.r), dtype=torch.bfloat16, device=dev),
             "dX": torch.empty((c.M, c.K), dtype=torch.bfloat16, device=dev),
-            "dA": torch.empty((c.r, c.K), dtype=torch.bfloat16, device=dev),
+            "dA": torch.empty((c.G * c.r, c.K), dtype=torch.bfloat16, device=dev),
             "dB": torch.empty((c.N, c.r), dtype=torch.bfloat16, device=dev),
         }
         layers.append(layer)
@@ -341,6 +357,11 @@ def run_ours(args, cases, desc, rank, world, local_rank):
         "gemm_share_of_step": g_ms / (ms * args.steps) if ms > 0 else None,
     }
 
+    # ---- grouped workloads: the same projections as separate layers, for comparison
+    separate = None
+    if any(c.rows is not None for c in cases) and world == 1:
+        separate = time_separate(args, cases, data, dev)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -370,7 +391,53 @@ def run_ours(args, cases, desc, rank, world, local_rank):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk,
         }
+        if separate is not None:
+            line["separate_layers"] = separate
         print(json.dumps(line), flush=True)
+
+
+def time_separate(args, cases, data, dev):
+    """Device time per step of a grouped workload run as G separate single-projection
+    layers (each with its own dY and outputs, as an unfused model would hold them)."""
+    import torch
+
+    import qlora_linear_b200 as q
+
+    stream = torch.cuda.current_stream()
+    parts = []
+    for c, (d, _) in zip(cases, data):
+        off = 0
+        for g, n in enumerate(c.rows):
+            W = q.LoraWeight(n, c.K, d["W"][off:off + n])
+            layer = q.LoraLinear(W, d["A"][g * c.r:(g + 1) * c.r], d["B"][off:off + n], c.alpha)
+            layer.workspace(c.M)
+            dY = d["dY"][:, off:off + n].contiguous()
+            o = (torch.empty((c.M, n), dtype=torch.bfloat16, device=dev),
+                 torch.empty((c.M, c.r), dtype=torch.bfloat16, device=dev),
+                 torch.empty((c.M, c.K), dtype=torch.bfloat16, device=dev),
+                 torch.empty((c.r, c.K), dtype=torch.bfloat16, device=dev),
+                 torch.empty((n, c.r), dtype=torch.bfloat16, device=dev))
+            parts.append((layer, d["X"], dY, o))
+            off += n
+
+    def step():
+        for layer, X, dY, (Y, XA, dX, dA, dB) in parts:
+            layer.forward(X, Y=Y, XA=XA)
+            layer.backward(dY, X, XA, out=(dX, dA, dB))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops_step = sum(case_flops(c) for c in cases)
+    return {"ms_per_step": ms, "value": flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "note": "the same projections as separate layers (dX of each written separately, not summed)"}
 
 
 def run_e2e(args, cases, layers, data, step, world, dev):
@@ -448,7 +515,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "qkv"])
     ap.add_argument("--only", default=None, help="run a single projection of the workload (e.g. c2_gate)")
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -45,6 +45,7 @@ struct PairParams {
   int nseg;            // 1 for a single projection
   int e_seg_stride;
   int seg_end_tile[8];
+  int group_m;         // 256-row tiles per raster group (L2 reuse of the B operand)
   __nv_bfloat16* out;  // [M, Nout] row-major
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
@@ -72,7 +73,6 @@ struct PairCfg {
   static constexpr int SCALE_RING = 4;  // W4: scale words staged this many code fills ahead (minus one)
   static constexpr int SCALE_BYTES = W4 ? SCALE_RING * 32 * NUM_DEQ_WARPS * 4 : 0;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SCALE_BYTES + 8 * NUM_BARS + 16;
-  static constexpr int GROUP_M = 8;  // 256-row tiles per raster group (L2 reuse of W)
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -205,7 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       bool ok = true;
       for (int t = pair; t < ntiles && ok; t += npairs) {
         int mb, nb;
-        pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+        pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
         const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A
         const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;  // this CTA's rows of the B tile
         for (int kb = 0; kb < nkb + n_ext; ++kb) {
@@ -316,7 +316,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
     uint32_t acc_phase = 0;
     for (int t = pair; t < ntiles; t += npairs) {
       int mb, nb;
-      pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
       if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, wc)) break;
       tc_fence_after();
       const int row = mb * C::BM + static_cast<int>(rank) * C::HM + quarter * 32 + lane;
@@ -368,7 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       if (i < code_fills) {
         const int t = pair + (i / nkb) * npairs, kb = i % nkb;
         int mb, nb;
-        pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+        pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
         const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
         const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
         const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
@@ -389,7 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
     auto scale_of = [&](int i) -> float {
       int kb = i % nkb, t = pair + (i / nkb) * npairs;
       int mb, nb;
-      pair_tile_coords(t, num_m, num_n, C::GROUP_M, mb, nb);
+      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
       const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
       const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
       const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;

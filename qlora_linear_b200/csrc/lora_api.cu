@@ -41,6 +41,19 @@ uint64_t wait_limit_ns() {
   return v;
 }
 
+// 256-row output tiles per raster group of the GEMMs; LORA_GROUP_M overrides (1..64).
+int group_m_default() {
+  static int v = [] {
+    const char* e = std::getenv("LORA_GROUP_M");
+    if (e && *e) {
+      const long x = std::strtol(e, nullptr, 10);
+      if (x >= 1 && x <= 64) return static_cast<int>(x);
+    }
+    return 8;
+  }();
+  return v;
+}
+
 // ---------------------------------------------------------------- measurement hooks
 std::atomic<long long> g_launches{0};
 std::atomic<bool> g_timing_on{false};
@@ -364,6 +377,7 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = status;
   p.wait_ns = wait_limit_ns();
+  p.group_m = group_m_default();
   p.nseg = 1;
   p.e_seg_stride = 0;
   for (int g = 0; g < LORA_MAX_SEGMENTS; ++g) p.seg_end_tile[g] = 0x7fffffff;

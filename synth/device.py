@@ -47,7 +47,7 @@ def make_case_device(case: LoraCase, device, rank: int = 0, want=("X", "W", "A",
     if "A" in want:
         a = 1.0 / math.sqrt(K)
         g = _gen(device, case.seed, _TID["A"], rank)
-        out["A"] = (torch.rand((r, K), generator=g, device=device, dtype=torch.float32) * (2 * a) - a).to(torch.bfloat16)
+        out["A"] = (torch.rand((case.G * r, K), generator=g, device=device, dtype=torch.float32) * (2 * a) - a).to(torch.bfloat16)
     if "B" in want:
         out["B"] = _normal_bf16((N, r), 0.1, device, _gen(device, case.seed, _TID["B"], rank))
     if "dY" in want:

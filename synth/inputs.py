@@ -68,10 +68,16 @@ class LoraCase:
     seed: int                  # stream of A and B (and of X, W, dY unless set below)
     x_seed: int | None = None  # X stream: lets two projections share one activation tensor
     data_seed: int | None = None  # W and dY stream (and X if x_seed is None)
+    rows: tuple | None = None  # several projections sharing X, stacked along N (rows sum to N)
 
     @property
     def s(self) -> float:
         return float(self.alpha) / float(self.r)
+
+    @property
+    def G(self) -> int:
+        """Number of projections (1 unless ``rows`` is set); A is ``[G·r, K]``."""
+        return 1 if self.rows is None else len(self.rows)
 
     def with_M(self, M: int) -> "LoraCase":
         return dataclasses.replace(self, M=M, name=f"{self.name}_M{M}")
@@ -99,6 +105,8 @@ def _cases() -> dict[str, list[LoraCase]]:
                     sweep.append(LoraCase(f"c4_{fmt}_K{K}_N{N}_M{M}_r{r}", M, N, K, r, 2.0 * r, fmt,
                                           b + 4 + 1000 * g + r, data_seed=b + 4 + 1000 * g))
     c["c4"] = sweep
+    # Llama-8B attention q/k/v (grouped-query: 32 query heads, 8 key/value heads of 128)
+    c["qkv"] = [LoraCase("qkv_llama8b", 8192, 6144, 4096, 16, 32.0, "bf16", b + 5, rows=(4096, 1024, 1024))]
     return c
 
 
@@ -175,24 +183,18 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
             out["codebook"] = codebook_levels()
     if "A" in want:
         a = 1.0 / np.sqrt(K)
-        out["A"] = _fill((r, K), case.seed, _TID["A"], _uniform_bf16(-a, a))
+        out["A"] = _fill((case.G * r, K), case.seed, _TID["A"], _uniform_bf16(-a, a))
     if "B" in want:
         out["B"] = _fill((N, r), case.seed, _TID["B"], _normal_bf16(0.1))
+    if case.rows is not None:
+        out["rows"] = [int(n) for n in case.rows]
     if "dY" in want:
         out["dY"] = _fill((M, N), ds, _TID["dY"], _normal_bf16(1.0))
     return out
 
 
 def make_grouped_case(case: LoraCase, rows, want=("X", "W", "A", "B", "dY")) -> dict:
-    """Inputs of G projections sharing X: ``case.N`` must equal ``sum(rows)``; W, B and dY
-    are drawn for the stacked ``[ΣN_g, ...]`` shapes and A for ``[G·r, K]`` (same
-    distributions as :func:`make_case`)."""
-    rows = [int(n) for n in rows]
-    assert sum(rows) == case.N
-    G = len(rows)
-    out = make_case(case, want=tuple(w for w in want if w != "A"))
-    if "A" in want:
-        a = 1.0 / np.sqrt(case.K)
-        out["A"] = _fill((G * case.r, case.K), case.seed, _TID["A"], _uniform_bf16(-a, a))
-    out["rows"] = rows
-    return out
+    """Inputs of G projections sharing X (``rows`` sum to ``case.N``): W, B and dY are
+    drawn for the stacked ``[ΣN_g, ...]`` shapes and A for ``[G·r, K]``."""
+    assert sum(int(n) for n in rows) == case.N
+    return make_case(dataclasses.replace(case, rows=tuple(int(n) for n in rows)), want=want)
