@@ -19,4 +19,9 @@ from .lora_oracle import (  # noqa: F401
     lora_adapter_grads_sampled,
     lora_grouped_forward,
     lora_grouped_backward,
+    sigmoid,
+    swiglu_forward,
+    swiglu_backward,
+    lora_mlp_forward,
+    lora_mlp_backward,
 )

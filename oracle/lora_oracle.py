@@ -30,6 +30,8 @@ What it computes (the method is exact, so the oracle is the plain definition):
   one fp16 absmax per 64 contiguous elements of the row-major weight and a
   16-entry float32 codebook.  One element dequantizes to
   ``bf16_rn(fp32_rn(codebook[code] * absmax))``.
+* The feed-forward block (gate and up LoRA linears, ``H = silu(G)·U``, down LoRA
+  linear) and its chain-rule backward, see :func:`lora_mlp_forward`.
 * Merge of the adapter into the weight ("Rev vs unsloth", GGUF export paragraph;
   "Unsloth vs The Stack v2", merge paragraph): ``W' = W + s·B·A``.
 
@@ -264,3 +266,73 @@ def lora_grouped_backward(dY: np.ndarray, X: np.ndarray, Ws: list, As: list, Bs:
             "dB": np.concatenate([q["dB"] for q in parts], axis=0),
             "dYB": np.concatenate([q["dYB"] for q in parts], axis=1),
             "XA": np.concatenate([q["XA"] for q in parts], axis=1)}
+
+
+# ----------------------------------------------------------------------------
+# the feed-forward block: gate and up LoRA linears, SwiGLU, down LoRA linear
+# ----------------------------------------------------------------------------
+
+
+def sigmoid(g: np.ndarray) -> np.ndarray:
+    """The logistic function 1/(1+e^-g), evaluated without overflow on either side."""
+    g = np.asarray(g, dtype=np.float64)
+    e = np.exp(-np.abs(g))
+    return np.where(g >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def swiglu_forward(G: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """SwiGLU gating of the feed-forward block: ``H = silu(G)·U`` element by element,
+    with ``silu(g) = g·sigmoid(g)`` (the "SwiGLU block" that the "Unsloth" wiki entry,
+    Theory, first bullet, lists among the fused kernels; Llama's feed-forward)."""
+    G = np.asarray(G, dtype=np.float64)
+    return G * sigmoid(G) * np.asarray(U, dtype=np.float64)
+
+
+def swiglu_backward(dH: np.ndarray, G: np.ndarray, U: np.ndarray):
+    """Hand-derived derivatives of ``H = silu(G)·U``: with ``σ = sigmoid(G)``,
+    ``silu'(g) = σ·(1 + g·(1-σ))``, so ``dG = dH·U·σ·(1 + G·(1-σ))`` and
+    ``dU = dH·G·σ``."""
+    G = np.asarray(G, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
+    dH = np.asarray(dH, dtype=np.float64)
+    sg = sigmoid(G)
+    return dH * U * sg * (1.0 + G * (1.0 - sg)), dH * G * sg
+
+
+def lora_mlp_forward(X: np.ndarray, W_gu: np.ndarray, A_gu: np.ndarray, B_gu: np.ndarray,
+                     W_d: np.ndarray, A_d: np.ndarray, B_d: np.ndarray, s: float) -> dict:
+    """Feed-forward block with LoRA on all three projections ("Unsloth" wiki entry, Theory:
+    fused SwiGLU block and hand-derived LoRA backward; "Unsloth vs PyTorch: The ONLY Video
+    You Need to Understand the Difference", transcript 2:11-2:22, the feed-forward blocks).
+
+    ``W_gu:[2I,D]`` is the gate weight stacked over the up weight, ``A_gu:[2r,D]`` and
+    ``B_gu:[2I,r]`` their adapters stacked the same way; ``W_d:[D,I]``, ``A_d:[r,I]``,
+    ``B_d:[D,r]`` the down projection.  ``G`` and ``U`` are the gate and up LoRA
+    linears of X, ``H = silu(G)·U`` and ``Z`` the down LoRA linear of H."""
+    I2 = np.asarray(W_gu).shape[0]
+    I = I2 // 2
+    r = np.asarray(A_gu).shape[0] // 2
+    G, XA_g = lora_forward(X, W_gu[:I], A_gu[:r], B_gu[:I], s)
+    U, XA_u = lora_forward(X, W_gu[I:], A_gu[r:], B_gu[I:], s)
+    H = swiglu_forward(G, U)
+    Z, XA_d = lora_forward(H, W_d, A_d, B_d, s)
+    return {"Z": Z, "H": H, "G": G, "U": U, "XA_gu": np.concatenate([XA_g, XA_u], axis=1), "XA_d": XA_d}
+
+
+def lora_mlp_backward(dZ: np.ndarray, X: np.ndarray, W_gu: np.ndarray, A_gu: np.ndarray, B_gu: np.ndarray,
+                      W_d: np.ndarray, A_d: np.ndarray, B_d: np.ndarray, s: float) -> dict:
+    """Backward of :func:`lora_mlp_forward` by the chain rule, one step at a time: the down
+    projection's backward gives ``dH`` (its dX) and the down adapter's gradients; SwiGLU's
+    derivative gives ``dG``, ``dU``; the gate and up projections' backward gives their
+    adapter gradients (stacked like the forward's) and ``dX = dX_gate + dX_up``."""
+    I = np.asarray(W_gu).shape[0] // 2
+    r = np.asarray(A_gu).shape[0] // 2
+    f = lora_mlp_forward(X, W_gu, A_gu, B_gu, W_d, A_d, B_d, s)
+    gd = lora_backward(dZ, f["H"], W_d, A_d, B_d, s)
+    dH = gd["dX"]
+    dG, dU = swiglu_backward(dH, f["G"], f["U"])
+    gg = lora_backward(dG, X, W_gu[:I], A_gu[:r], B_gu[:I], s)
+    gu = lora_backward(dU, X, W_gu[I:], A_gu[r:], B_gu[I:], s)
+    return {"dX": gg["dX"] + gu["dX"], "dA_gu": np.concatenate([gg["dA"], gu["dA"]], axis=0),
+            "dB_gu": np.concatenate([gg["dB"], gu["dB"]], axis=0), "dA_d": gd["dA"], "dB_d": gd["dB"],
+            "dH": dH, "dG": dG, "dU": dU, "fwd": f}

@@ -410,3 +410,113 @@ def test_grouped_finite_differences():
             r = As[0].shape[0]
             want = g["dA"][q * r:(q + 1) * r] if name == "A" else g["dB"][sum(W.shape[0] for W in Ws[:q]):][:Ws[q].shape[0]]
             assert _rel(fdT, want) <= 1e-9, (name, q)
+
+
+# ---------------------------------------------------------------- feed-forward block
+
+
+def test_sigmoid_closed_forms_and_symmetry():
+    """sigmoid(0) = 1/2, sigmoid(±ln 3) = 3/4 and 1/4 exactly (1/(1+1/3)); no overflow at
+    ±800; sigmoid(x) + sigmoid(-x) = 1; silu(g) = g·sigmoid(g) follows."""
+    ln3 = np.log(3.0)
+    got = O.sigmoid(np.array([0.0, ln3, -ln3, 800.0, -800.0]))
+    assert got[0] == 0.5
+    assert abs(got[1] - 0.75) <= 2e-16 and abs(got[2] - 0.25) <= 2e-16
+    assert got[3] == 1.0 and 0.0 <= got[4] < 1e-300
+    x = np.linspace(-30, 30, 1001)
+    assert np.max(np.abs(O.sigmoid(x) + O.sigmoid(-x) - 1.0)) <= np.finfo(np.float64).eps  # one ulp of 1
+    H = O.swiglu_forward(np.array([ln3, 0.0, -ln3]), np.array([2.0, 5.0, 4.0]))
+    assert np.allclose(H, [0.75 * ln3 * 2.0, 0.0, -0.25 * ln3 * 4.0], rtol=0, atol=1e-15)
+
+
+def test_swiglu_backward_against_torch_autograd():
+    """The hand-derived dG, dU equal torch's autograd of F.silu(G)·U in float64."""
+    rng = np.random.default_rng(31)
+    G = rng.standard_normal((7, 11)) * 3
+    U = rng.standard_normal((7, 11))
+    dH = rng.standard_normal((7, 11))
+    tg = torch.tensor(G, requires_grad=True)
+    tu = torch.tensor(U, requires_grad=True)
+    th = torch.nn.functional.silu(tg) * tu
+    th.backward(torch.tensor(dH))
+    assert _rel(O.swiglu_forward(G, U), th.detach().numpy()) <= 1e-15
+    dG, dU = O.swiglu_backward(dH, G, U)
+    assert _rel(dG, tg.grad.numpy()) <= 1e-14
+    assert _rel(dU, tu.grad.numpy()) <= 1e-14
+
+
+def _mlp(rng, M=6, D=10, I=7, r=3):
+    X = rng.standard_normal((M, D))
+    W_gu = rng.standard_normal((2 * I, D)) / np.sqrt(D)
+    A_gu = rng.uniform(-1, 1, (2 * r, D)) / np.sqrt(D)
+    B_gu = rng.standard_normal((2 * I, r)) * 0.3
+    W_d = rng.standard_normal((D, I)) / np.sqrt(I)
+    A_d = rng.uniform(-1, 1, (r, I)) / np.sqrt(I)
+    B_d = rng.standard_normal((D, r)) * 0.3
+    dZ = rng.standard_normal((M, D))
+    return X, W_gu, A_gu, B_gu, W_d, A_d, B_d, dZ
+
+
+def test_mlp_block_against_torch_autograd():
+    """Forward against the block written with torch's own linear and silu; every gradient
+    against torch's autograd of it (float64), so the chain rule is checked by a
+    derivation other than the oracle's."""
+    rng = np.random.default_rng(32)
+    X, W_gu, A_gu, B_gu, W_d, A_d, B_d, dZ = _mlp(rng)
+    s = 1.25
+    I, r = W_d.shape[1], A_d.shape[0]
+    t = {k: torch.tensor(v, requires_grad=True) for k, v in
+         dict(X=X, A_gu=A_gu, B_gu=B_gu, A_d=A_d, B_d=B_d).items()}
+    F = torch.nn.functional
+
+    def lin(x, W, A, B):
+        return F.linear(x, torch.tensor(W)) + s * F.linear(F.linear(x, A), B)
+
+    G = lin(t["X"], W_gu[:I], t["A_gu"][:r], t["B_gu"][:I])
+    U = lin(t["X"], W_gu[I:], t["A_gu"][r:], t["B_gu"][I:])
+    Z = lin(F.silu(G) * U, W_d, t["A_d"], t["B_d"])
+    Z.backward(torch.tensor(dZ))
+    f = O.lora_mlp_forward(X, W_gu, A_gu, B_gu, W_d, A_d, B_d, s)
+    assert _rel(f["Z"], Z.detach().numpy()) <= 1e-14
+    g = O.lora_mlp_backward(dZ, X, W_gu, A_gu, B_gu, W_d, A_d, B_d, s)
+    for k in ("X", "A_gu", "B_gu", "A_d", "B_d"):
+        assert _rel(g["d" + k], t[k].grad.numpy()) <= 1e-13, k
+
+
+def test_mlp_finite_differences():
+    rng = np.random.default_rng(33)
+    X, W_gu, A_gu, B_gu, W_d, A_d, B_d, dZ = _mlp(rng, M=3, D=4, I=3, r=2)
+    s = 0.8
+    g = O.lora_mlp_backward(dZ, X, W_gu, A_gu, B_gu, W_d, A_d, B_d, s)
+    args = dict(X=X, A_gu=A_gu, B_gu=B_gu, A_d=A_d, B_d=B_d)
+
+    def L(**kw):
+        a = dict(args, **kw)
+        return float(np.sum(dZ * O.lora_mlp_forward(a["X"], W_gu, a["A_gu"], a["B_gu"], W_d, a["A_d"], a["B_d"],
+                                                      s)["Z"]))
+
+    h = 1e-4
+    for name, T in args.items():
+        fd = np.zeros_like(T)
+        for idx in np.ndindex(T.shape):
+            Tp, Tm = T.copy(), T.copy()
+            Tp[idx] += h
+            Tm[idx] -= h
+            fd[idx] = (L(**{name: Tp}) - L(**{name: Tm})) / (2 * h)
+        assert _rel(fd, g["d" + name]) <= 1e-7, name
+
+
+def test_mlp_zero_adapters_give_the_plain_block():
+    """With every B zero (the adapter's initial state) the block is the plain SwiGLU
+    feed-forward, silu from torch; the A gradients are exactly zero."""
+    rng = np.random.default_rng(34)
+    X, W_gu, A_gu, B_gu, W_d, A_d, B_d, dZ = _mlp(rng)
+    B_gu, B_d = np.zeros_like(B_gu), np.zeros_like(B_d)
+    I = W_d.shape[1]
+    f = O.lora_mlp_forward(X, W_gu, A_gu, B_gu, W_d, A_d, B_d, 2.0)
+    G, U = X @ W_gu[:I].T, X @ W_gu[I:].T
+    H = torch.nn.functional.silu(torch.tensor(G)).numpy() * U
+    assert _rel(f["Z"], H @ W_d.T) <= 1e-14
+    g = O.lora_mlp_backward(dZ, X, W_gu, A_gu, B_gu, W_d, A_d, B_d, 2.0)
+    assert np.all(g["dA_gu"] == 0) and np.all(g["dA_d"] == 0)
+    assert np.any(g["dB_gu"] != 0) and np.any(g["dB_d"] != 0)
