@@ -161,6 +161,60 @@ lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, in
                                void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Feed-forward block with LoRA on all three projections and SwiGLU gating ("Unsloth"
+ * wiki entry, Theory: the fused SwiGLU block and the hand-derived LoRA backward; "Unsloth
+ * vs PyTorch: The ONLY Video You Need to Understand the Difference", transcript
+ * 2:11-2:22, the feed-forward blocks).  With model width D, hidden width I, rank r and
+ * scale s:
+ *
+ *     G = X·W_gᵀ + s·(X·A_gᵀ)·B_gᵀ      U = X·W_uᵀ + s·(X·A_uᵀ)·B_uᵀ        [M, I]
+ *     H = silu(G)·U,  silu(g) = g/(1+e^-g)                                   [M, I]
+ *     Z = H·W_dᵀ + s·(H·A_dᵀ)·B_dᵀ                                           [M, D]
+ *
+ * Backward, by hand: dH = dZ·W_d + s·(dZ·B_d)·A_d; with σ = sigmoid(G),
+ * dG = dH·U·σ·(1 + G·(1-σ)) and dU = dH·G·σ; then each of gate and up as a LoRA linear
+ * of X with dX = dX_gate + dX_up.
+ *
+ * The forward's gate and up GEMMs run as one GEMM whose epilogue applies SwiGLU (each
+ * output tile holds matching gate and up columns), writing H and the saved G, U; the
+ * backward's dH GEMM applies SwiGLU's derivative in its epilogue, turning the saved
+ * G, U into dG, dU in place, so dH is never written.
+ *
+ * Layout: gate_up is the gate weight stacked over the up weight, [2I, D] (a 4-bit
+ * gate_up stacks codes and absmax the same way); down is [D, I].  A_gate_up bf16
+ * [2r, D] = [A_g; A_u]; B_gate_up bf16 [2I, r] = [B_g; B_u]; A_down bf16 [r, I];
+ * B_down bf16 [D, r].  GU bf16 [M, 2I] holds G in columns [0, I) and U in [I, 2I);
+ * XA_gate_up bf16 [M, 2r] = [X·A_gᵀ | X·A_uᵀ]; XA_down bf16 [M, r] = H·A_dᵀ.
+ * Both weights have the same format.  Limits: D % 8 == 0 and I % 8 == 0 (% 64 for
+ * 4-bit), 8 <= r <= 64 with r % 8 == 0 (else LORA_ERR_UNSUPPORTED).  The workspace is
+ * lora_mlp_workspace_bytes(M, D, I, r, fmt).
+ */
+typedef struct {
+  lora_weight_t gate_up;   /* [2I, D] */
+  lora_weight_t down;      /* [D, I] */
+  const void* A_gate_up;   /* bf16 [2r, D] */
+  const void* B_gate_up;   /* bf16 [2I, r] */
+  const void* A_down;      /* bf16 [r, I] */
+  const void* B_down;      /* bf16 [D, r] */
+} lora_mlp_t;
+
+size_t lora_mlp_workspace_bytes(int64_t M, int64_t D, int64_t I, int32_t r, int32_t fmt);
+
+/* Forward.  Writes Z [M, D] and, for the backward, GU [M, 2I], H [M, I], XA_gate_up
+ * [M, 2r] and XA_down [M, r] (all bf16, device). */
+lora_status_t lora_mlp_fwd(const void* X, int64_t M, const lora_mlp_t* mlp, int32_t r, float s,
+                           void* Z, void* GU, void* H, void* XA_gate_up, void* XA_down,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward.  GU holds the forward's G and U on entry and dG, dU (same columns) on
+ * return.  Writes dX [M, D] (skipped when NULL), dA_gate_up [2r, D], dB_gate_up [2I, r],
+ * dA_down [r, I], dB_down [D, r] (bf16, device).  M = 0 zeroes the adapter gradients. */
+lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
+                           const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s,
+                           void* dX, void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Standalone dequantization of a LORA_W_BLOCK4 weight to bf16 [N,K] (device, out),
  * element by element as defined for lora_weight_t.  Bit-exact.  Not used by the
  * forward/backward, which dequantize tiles in shared memory and never write a

@@ -29,6 +29,11 @@ from .binding import (  # noqa: F401
     lora_grouped_fwd,
     lora_grouped_bwd,
     grouped_workspace_bytes,
+    lora_mlp_fwd,
+    lora_mlp_bwd,
+    lora_mlp_t,
+    mlp_struct,
+    mlp_workspace_bytes,
     segments,
     LORA_ERR_SCRATCH_LIMIT,
     LORA_NOALLOC_SCRATCH_BYTES,
@@ -42,5 +47,5 @@ from .binding import (  # noqa: F401
     status_string,
     workspace_bytes,
 )
-from .layer import LoraGroupedLinear, LoraLinear  # noqa: F401
+from .layer import LoraGroupedLinear, LoraLinear, LoraMLP  # noqa: F401
 from .dp import allreduce_adapter_grads, token_shard  # noqa: F401

@@ -34,6 +34,7 @@ EXPORTED = (
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
     "lora_testing_bounded_wait", "lora_timing_enable", "lora_timing_read", "lora_launch_count",
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
+    "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd",
 )
 
 LORA_MAX_SEGMENTS = 8
@@ -62,6 +63,17 @@ class lora_segments_t(ctypes.Structure):
         ("count", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
         ("rows", ctypes.c_int64 * 8),
+    ]
+
+
+class lora_mlp_t(ctypes.Structure):
+    _fields_ = [
+        ("gate_up", lora_weight_t),
+        ("down", lora_weight_t),
+        ("A_gate_up", ctypes.c_void_p),
+        ("B_gate_up", ctypes.c_void_p),
+        ("A_down", ctypes.c_void_p),
+        ("B_down", ctypes.c_void_p),
     ]
 
 
@@ -116,6 +128,13 @@ def _load() -> ctypes.CDLL:
     lib.lora_grouped_fwd.restype = i32
     lib.lora_grouped_bwd.argtypes = [vp, vp, vp, i64, W, S, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
     lib.lora_grouped_bwd.restype = i32
+    P = ctypes.POINTER(lora_mlp_t)
+    lib.lora_mlp_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
+    lib.lora_mlp_workspace_bytes.restype = sz
+    lib.lora_mlp_fwd.argtypes = [vp, i64, P, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.lora_mlp_fwd.restype = i32
+    lib.lora_mlp_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, P, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.lora_mlp_bwd.restype = i32
     return lib
 
 
@@ -275,3 +294,31 @@ def lora_grouped_bwd(dY, X, XA, M: int, W: LoraWeight, rows, A, B, r: int, s: fl
     _check(_lib.lora_grouped_bwd(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), ctypes.byref(seg), _ptr(A),
                                  _ptr(B), int(r), float(s), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), int(nb),
                                  _stream(stream)), "lora_grouped_bwd")
+
+
+def mlp_workspace_bytes(M: int, D: int, I: int, r: int, fmt: int = LORA_W_BF16) -> int:
+    return int(_lib.lora_mlp_workspace_bytes(int(M), int(D), int(I), int(r), int(fmt)))
+
+
+def mlp_struct(gate_up: LoraWeight, down: LoraWeight, A_gate_up, B_gate_up, A_down, B_down) -> lora_mlp_t:
+    return lora_mlp_t(gate_up.c_struct(), down.c_struct(), _ptr(A_gate_up), _ptr(B_gate_up), _ptr(A_down),
+                      _ptr(B_down))
+
+
+def lora_mlp_fwd(X, M: int, mlp: lora_mlp_t, r: int, s: float, Z, GU, H, XA_gate_up, XA_down, workspace,
+                 ws_bytes=None, stream=None) -> None:
+    """Forward of the SwiGLU feed-forward block with LoRA on gate, up and down (see lora_linear.h)."""
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_mlp_fwd(_ptr(X), int(M), ctypes.byref(mlp), int(r), float(s), _ptr(Z), _ptr(GU), _ptr(H),
+                             _ptr(XA_gate_up), _ptr(XA_down), _ptr(workspace), int(nb), _stream(stream)),
+           "lora_mlp_fwd")
+
+
+def lora_mlp_bwd(dZ, X, GU, H, XA_gate_up, XA_down, M: int, mlp: lora_mlp_t, r: int, s: float, dX, dA_gate_up,
+                 dB_gate_up, dA_down, dB_down, workspace, ws_bytes=None, stream=None) -> None:
+    """Backward of the block; GU (the forward's G | U) is overwritten with dG | dU."""
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_mlp_bwd(_ptr(dZ), _ptr(X), _ptr(GU), _ptr(H), _ptr(XA_gate_up), _ptr(XA_down), int(M),
+                             ctypes.byref(mlp), int(r), float(s), _ptr(dX), _ptr(dA_gate_up), _ptr(dB_gate_up),
+                             _ptr(dA_down), _ptr(dB_down), _ptr(workspace), int(nb), _stream(stream)),
+           "lora_mlp_bwd")

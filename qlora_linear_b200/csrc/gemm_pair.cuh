@@ -46,6 +46,14 @@ struct PairParams {
   int e_seg_stride;
   int seg_end_tile[8];
   int group_m;         // 256-row tiles per raster group (L2 reuse of the B operand)
+  // SwiGLU epilogues (feed-forward block).  Forward: the even CTA of a pair takes gate
+  // rows nb*128.., the odd CTA the up rows half_rows further on, and the odd CTA's LoRA
+  // F tile starts f_shift columns to the left, so it meets the up half of E.
+  int half_rows;
+  int f_shift;
+  __nv_bfloat16* aux;  // [M, ld_aux]: gate pre-activations, up pre-activations aux_off columns on
+  int ld_aux;
+  int aux_off;
   __nv_bfloat16* out;  // [M, Nout] row-major
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
@@ -76,6 +84,31 @@ struct PairCfg {
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
+
+// Epilogue of the pair GEMM.
+enum : int {
+  EPI_STORE = 0,       // out = accumulator (bf16)
+  EPI_SWIGLU_FWD = 1,  // accumulator columns [0,128) gate g, [128,256) up u of the same 128
+                       // output columns: aux <- g, u; out <- silu(g)·u
+  EPI_SWIGLU_BWD = 2,  // accumulator = dH; aux holds g, u and is overwritten in place with
+                       // dG = dH·u·silu'(g), dU = dH·silu(g); out is not written
+};
+
+template <int EPI>
+struct EpiTile {
+  static constexpr int COLS = EPI == EPI_SWIGLU_FWD ? 128 : 256;  // output columns per pair tile
+};
+
+// First row of this CTA's half of the B tile (and of its LoRA F tile).
+template <int EPI>
+__device__ __forceinline__ int pair_brow(int nb, uint32_t rank, const PairParams& p) {
+  if (EPI == EPI_SWIGLU_FWD) return nb * 128 + static_cast<int>(rank) * p.half_rows;
+  return nb * 256 + static_cast<int>(rank) * 128;
+}
+
+// silu(g) = g·sigmoid(g); sigmoid from the exponential intrinsic and a rounded reciprocal
+// (1/(1+e^-g) is 0, not NaN, when e^-g overflows).
+__device__ __forceinline__ float sigmoid_f(float g) { return __frcp_rn(1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void pair_tile_coords(int t, int num_m, int num_n, int group_m, int& mb, int& nb) {
   const int per_group = group_m * num_n;
@@ -130,7 +163,7 @@ __device__ __forceinline__ void block_levels(const float (&cb)[16], float scale,
 }
 #endif
 
-template <bool B_MN, bool W4>
+template <bool B_MN, bool W4, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::NUM_THREADS, 1)
     lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
@@ -158,7 +191,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
   const int num_m = (p.M + C::BM - 1) / C::BM;
-  const int num_n = (p.Nout + C::BN - 1) / C::BN;
+  const int num_n = (p.Nout + EpiTile<EPI>::COLS - 1) / EpiTile<EPI>::COLS;
   const int ntiles = num_m * num_n;
   const int nkb = (p.Kred + C::BK - 1) / C::BK;
   const int n_ext = p.r > 0 ? 1 : 0;         // one fill holds the whole LoRA block (r <= 128)
@@ -207,7 +240,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
         int mb, nb;
         pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
         const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A
-        const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;  // this CTA's rows of the B tile
+        const int brow = pair_brow<EPI>(nb, rank, p);  // this CTA's rows of the B tile
         for (int kb = 0; kb < nkb + n_ext; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
           const bool ext = kb >= nkb;
@@ -244,8 +277,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
             for (int h = 0; h < ext_atoms; ++h)
               tma_load_2d_pair(sA + h * (C::A_BYTES / 2), &tmE, full_l, e0 + h * C::ATOM, arow);
             if (!B_MN) {
+              // the SwiGLU forward's odd CTA reads F from x = -f_shift: its first f_shift
+              // columns are the zero fill, so the gate half of E meets zeros
+              const int fx = EPI == EPI_SWIGLU_FWD ? -static_cast<int>(rank) * p.f_shift : 0;
               for (int h = 0; h < ext_atoms; ++h)
-                tma_load_2d_pair(sB + h * (C::B_BYTES / 2), &tmF, full_l, h * C::ATOM, brow);
+                tma_load_2d_pair(sB + h * (C::B_BYTES / 2), &tmF, full_l, fx + h * C::ATOM, brow);
             } else {
               tma_load_2d_pair(sB, &tmF, full_l, brow, 0);
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmF, full_l, brow + C::ATOM, 0);
@@ -322,24 +358,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       const int row = mb * C::BM + static_cast<int>(rank) * C::HM + quarter * 32 + lane;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
-      __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
+      if constexpr (EPI == EPI_STORE) {
+        __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; ++c) {
-        const int col0 = nb * C::BN + c * 32;
-        if (col0 >= p.Nout) break;  // warp-uniform
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, v);
-        tmem_ld_wait();
-        if (row < p.M) {
+        for (int c = 0; c < C::BN / 32; ++c) {
+          const int col0 = nb * C::BN + c * 32;
+          if (col0 >= p.Nout) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (row < p.M) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (col0 + q * 8 < p.Nout) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]));
-              o.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]), __uint_as_float(v[q * 8 + 3]));
-              o.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]));
-              o.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]), __uint_as_float(v[q * 8 + 7]));
-              *reinterpret_cast<uint4*>(orow + col0 + q * 8) = o;
+            for (int q = 0; q < 4; ++q) {
+              if (col0 + q * 8 < p.Nout) {
+                uint4 o;
+                o.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]));
+                o.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]), __uint_as_float(v[q * 8 + 3]));
+                o.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]));
+                o.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]), __uint_as_float(v[q * 8 + 7]));
+                *reinterpret_cast<uint4*>(orow + col0 + q * 8) = o;
+              }
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+        __nv_bfloat16* hrow = p.out + static_cast<size_t>(row) * p.Nout;
+        __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const int col0 = nb * 128 + c * 32;
+          if (col0 >= p.Nout) break;  // warp-uniform
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, g);
+          tmem_ld_32x32b_x32(tbase + 128 + c * 32, u);
+          tmem_ld_wait();
+          if (row < p.M) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col0 + q * 8 < p.Nout) {
+                uint32_t og[4], ou[4], oh[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float g0 = __uint_as_float(g[q * 8 + 2 * e]), g1 = __uint_as_float(g[q * 8 + 2 * e + 1]);
+                  const float u0 = __uint_as_float(u[q * 8 + 2 * e]), u1 = __uint_as_float(u[q * 8 + 2 * e + 1]);
+                  og[e] = pack_bf16x2(g0, g1);
+                  ou[e] = pack_bf16x2(u0, u1);
+                  oh[e] = pack_bf16x2(g0 * sigmoid_f(g0) * u0, g1 * sigmoid_f(g1) * u1);
+                }
+                *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(og[0], og[1], og[2], og[3]);
+                *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+                *reinterpret_cast<uint4*>(hrow + col0 + q * 8) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+              }
+            }
+          }
+        }
+      } else {
+        __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll 1
+        for (int c = 0; c < C::BN / 32; ++c) {
+          const int col0 = nb * C::BN + c * 32;
+          if (col0 >= p.Nout) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          uint4 gq[4], uq[4];
+          if (row < p.M) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col0 + q * 8 < p.Nout) {
+                gq[q] = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
+                uq[q] = *reinterpret_cast<const uint4*>(grow + p.aux_off + col0 + q * 8);
+              }
+            }
+          }
+          tmem_ld_wait();
+          if (row < p.M) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col0 + q * 8 < p.Nout) {
+                const uint32_t gw[4] = {gq[q].x, gq[q].y, gq[q].z, gq[q].w};
+                const uint32_t uw[4] = {uq[q].x, uq[q].y, uq[q].z, uq[q].w};
+                uint32_t odg[4], odu[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  float dg[2], du[2];
+#pragma unroll
+                  for (int h2 = 0; h2 < 2; ++h2) {
+                    const float gv = __uint_as_float(h2 ? (gw[e] & 0xffff0000u) : (gw[e] << 16));
+                    const float uv = __uint_as_float(h2 ? (uw[e] & 0xffff0000u) : (uw[e] << 16));
+                    const float dh = __uint_as_float(v[q * 8 + 2 * e + h2]);
+                    const float sg = sigmoid_f(gv);
+                    du[h2] = dh * gv * sg;
+                    dg[h2] = dh * uv * sg * (1.0f + gv * (1.0f - sg));
+                  }
+                  odg[e] = pack_bf16x2(dg[0], dg[1]);
+                  odu[e] = pack_bf16x2(du[0], du[1]);
+                }
+                *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(odg[0], odg[1], odg[2], odg[3]);
+                *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(odu[0], odu[1], odu[2], odu[3]);
+              }
             }
           }
         }
@@ -369,7 +485,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
         const int t = pair + (i / nkb) * npairs, kb = i % nkb;
         int mb, nb;
         pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
-        const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
+        const int brow = pair_brow<EPI>(nb, rank, p);
         const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
         const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
         const uint32_t dst = smem_u32(&scale_ring[(i % C::SCALE_RING) * (32 * C::NUM_DEQ_WARPS) + dt]);
@@ -390,7 +506,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       int kb = i % nkb, t = pair + (i / nkb) * npairs;
       int mb, nb;
       pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
-      const int brow = nb * C::BN + static_cast<int>(rank) * C::HN;
+      const int brow = pair_brow<EPI>(nb, rank, p);
       const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
       const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
       const uint32_t wv = scale_ring[(i % C::SCALE_RING) * (32 * C::NUM_DEQ_WARPS) + dt];

@@ -142,10 +142,14 @@ lora_status_t dev_info(DevInfo** out) {
   if (!d.attrs_set) {
     bool ok = true;
 #define SET_SMEM(fn, bytes) ok &= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-    SET_SMEM((lora_gemm_pair_kernel<false, false>), (PairCfg<false, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, false>), (PairCfg<true, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<false, true>), (PairCfg<false, true>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, true>), (PairCfg<true, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, false, EPI_STORE>), (PairCfg<false, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, false, EPI_STORE>), (PairCfg<true, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, true, EPI_STORE>), (PairCfg<false, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, true, EPI_STORE>), (PairCfg<true, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, false, EPI_SWIGLU_FWD>), (PairCfg<false, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, true, EPI_SWIGLU_FWD>), (PairCfg<false, true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, false, EPI_SWIGLU_BWD>), (PairCfg<true, false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, true, EPI_SWIGLU_BWD>), (PairCfg<true, true>::SMEM_BYTES));
     SET_SMEM((rowproj_kernel<16, false>), (rowproj_smem_bytes<16, false>()));
     SET_SMEM((rowproj_kernel<32, false>), (rowproj_smem_bytes<32, false>()));
     SET_SMEM((rowproj_kernel<64, false>), (rowproj_smem_bytes<64, false>()));
@@ -309,16 +313,16 @@ lora_status_t finalize_cols(const float* part, int splits, int C, int r, float s
 }
 
 // ---------------------------------------------------------------- GEMM launch
-template <bool B_MN, bool W4>
+template <bool B_MN, bool W4, int EPI = EPI_STORE>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
                           const PairParams& p, int sms, cudaStream_t st) {
   using C = PairCfg<B_MN, W4>;
-  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, C::BN);
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_pair_kernel<B_MN, W4><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    lora_gemm_pair_kernel<B_MN, W4, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
   }
   count_launch();
   return last_launch();
@@ -535,6 +539,144 @@ lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M
                        reinterpret_cast<uint32_t*>(ws), st);
 }
 
+// ---------------------------------------------------------------- feed-forward block
+// Workspace of the block: the status head, one bf16 skinny operand of rank 2r and the
+// largest set of fp32 split partials any of its skinny passes needs.
+WsLayout mlp_ws_layout(long long M, long long D, long long I, int r) {
+  WsLayout w;
+  w.skinny_off = kStatusBytes;
+  w.part_off = w.skinny_off + align256(static_cast<size_t>(M) * 2 * r * 2);
+  size_t part = 0;
+  auto upd = [&](size_t b) { part = b > part ? b : part; };
+  upd(static_cast<size_t>(rowproj_split(M, D).splits) * M * 2 * r * 4);  // [X·A_gᵀ | X·A_uᵀ]
+  upd(static_cast<size_t>(rowproj_split(M, I).splits) * M * r * 4);      // H·A_dᵀ, dG·B_g, dU·B_u
+  upd(static_cast<size_t>(rowproj_split(M, D).splits) * M * r * 4);      // dZ·B_d
+  upd(static_cast<size_t>(colproj_split(M, D).splits) * D * r * 4);      // dB_d
+  upd(static_cast<size_t>(colproj_split(M, I).splits) * I * r * 4);      // dA_d, dB_g, dB_u
+  upd(static_cast<size_t>(colproj_split(M, D).splits) * D * 2 * r * 4);  // [dA_g; dA_u]
+  w.total = w.part_off + align256(part);
+  return w;
+}
+
+lora_status_t mlp_check(const lora_mlp_t* m, int r, float s, long long M) {
+  if (!m) return LORA_ERR_INVALID_ARG;
+  TRY(check_weight(&m->gate_up));
+  TRY(check_weight(&m->down));
+  if (m->gate_up.fmt != m->down.fmt) return LORA_ERR_INVALID_ARG;
+  TRY(check_rank(r, s));
+  if (2 * r > 128) return LORA_ERR_UNSUPPORTED;
+  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
+  const long long D = m->gate_up.K, I = m->down.K;
+  if (m->gate_up.N != 2 * I || m->down.N != D) return LORA_ERR_INVALID_ARG;
+  TRY(check_ptr(m->A_gate_up));
+  TRY(check_ptr(m->B_gate_up));
+  TRY(check_ptr(m->A_down));
+  TRY(check_ptr(m->B_down));
+  return LORA_OK;
+}
+
+Segs gate_up_segs(long long I) {
+  Segs g;
+  g.n = 2;
+  g.rows[0] = g.rows[1] = I;
+  g.off[1] = I;
+  g.off[2] = 2 * I;
+  return g;
+}
+
+// [X·A_gᵀ | X·A_uᵀ] in one pass over X; one GEMM for gate and up whose epilogue writes
+// G, U and H = silu(G)·U; then the down projection as a LoRA linear of H.
+lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, int r, float s, void* Z, void* GU,
+                               void* H, void* XAgu, void* XAd, __nv_bfloat16* skinny, float* part, uint32_t* status,
+                               cudaStream_t st) {
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  const long long D = m->gate_up.K, I = m->down.K;
+  const int r2 = 2 * r;
+  const int Mi = static_cast<int>(M), Di = static_cast<int>(D);
+  const Split sp = rowproj_split(M, D);
+  TRY(launch_rowproj<false>(static_cast<const __nv_bfloat16*>(X), Di,
+                            static_cast<const __nv_bfloat16*>(m->A_gate_up), part, Mi, Di, r2, sp, st));
+  TRY(finalize_rows(part, sp.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
+
+  CUtensorMap ta, tb, te, tf;
+  TRY(tmap_bf16(&ta, X, D, M, kBoxX, kBoxY));
+  TRY(tmap_bf16(&te, skinny, r2, M, kBoxX, kBoxY));
+  TRY(tmap_bf16(&tf, m->B_gate_up, r, 2 * I, kBoxX, kBoxY));
+  PairParams p = gemm_params(M, I, D, r2, H, status, &m->gate_up);
+  p.half_rows = static_cast<int>(I);
+  p.f_shift = r;
+  p.aux = static_cast<__nv_bfloat16*>(GU);
+  p.ld_aux = static_cast<int>(2 * I);
+  p.aux_off = static_cast<int>(I);
+  if (m->gate_up.fmt == LORA_W_BF16) {
+    TRY(tmap_bf16(&tb, m->gate_up.data, D, 2 * I, kBoxX, kBoxY));
+    TRY((launch_gemm<false, false, EPI_SWIGLU_FWD>(ta, tb, te, tf, p, dev->sms, st)));
+  } else {
+    TRY(tmap_u8(&tb, m->gate_up.data, D / 2, 2 * I, kBoxX, kBoxY));
+    TRY((launch_gemm<false, true, EPI_SWIGLU_FWD>(ta, tb, te, tf, p, dev->sms, st)));
+  }
+  Segs one;
+  one.rows[0] = D;
+  one.off[1] = D;
+  return forward_core(H, M, &m->down, one, m->A_down, m->B_down, r, s, Z, XAd, skinny, part, status, st);
+}
+
+// Down projection's backward with SwiGLU's derivative in the dH GEMM's epilogue (GU
+// becomes [dG | dU]), then gate and up as two projections of X with dY = [dG | dU].
+lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const void* H, const void* XAgu,
+                                const void* XAd, long long M, const lora_mlp_t* m, int r, float s, void* dX,
+                                void* dAgu, void* dBgu, void* dAd, void* dBd, __nv_bfloat16* skinny, float* part,
+                                uint32_t* status, cudaStream_t st) {
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  const long long D = m->gate_up.K, I = m->down.K;
+  const int Mi = static_cast<int>(M), Di = static_cast<int>(D), Ii = static_cast<int>(I);
+  const auto* dZb = static_cast<const __nv_bfloat16*>(dZ);
+  // s·dZ·B_d
+  Split sp = rowproj_split(M, D);
+  TRY(launch_rowproj<true>(dZb, Di, static_cast<const __nv_bfloat16*>(m->B_down), part, Mi, Di, r, sp, st));
+  TRY(finalize_rows(part, sp.splits, M, r, r, s, nullptr, skinny, st));
+  // dB_d = s·dZᵀ·(H·A_dᵀ)
+  sp = colproj_split(M, D);
+  TRY(launch_colproj(dZb, Di, static_cast<const __nv_bfloat16*>(XAd), r, part, Mi, Di, r, sp, st));
+  TRY(finalize_cols(part, sp.splits, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
+  // dH = dZ·W_d + (s·dZ·B_d)·A_d, consumed by the epilogue: GU <- [dG | dU]
+  {
+    CUtensorMap ta, tb, te, tf;
+    TRY(tmap_bf16(&ta, dZ, D, M, kBoxX, kBoxY));
+    TRY(tmap_bf16(&te, skinny, r, M, kBoxX, kBoxY));
+    TRY(tmap_bf16(&tf, m->A_down, I, r, kBoxX, kBoxY));
+    PairParams p = gemm_params(M, I, D, r, nullptr, status, &m->down);
+    p.aux = static_cast<__nv_bfloat16*>(GU);
+    p.ld_aux = static_cast<int>(2 * I);
+    p.aux_off = static_cast<int>(I);
+    if (m->down.fmt == LORA_W_BF16) {
+      TRY(tmap_bf16(&tb, m->down.data, I, D, kBoxX, kBoxY));
+      TRY((launch_gemm<true, false, EPI_SWIGLU_BWD>(ta, tb, te, tf, p, dev->sms, st)));
+    } else {
+      TRY(tmap_u8(&tb, m->down.data, I / 2, D, kBoxX, kBoxY));
+      TRY((launch_gemm<true, true, EPI_SWIGLU_BWD>(ta, tb, te, tf, p, dev->sms, st)));
+    }
+  }
+  // dA_d = (s·dZ·B_d)ᵀ·H
+  sp = colproj_split(M, I);
+  TRY(launch_colproj(static_cast<const __nv_bfloat16*>(H), Ii, skinny, r, part, Mi, Ii, r, sp, st));
+  TRY(finalize_cols(part, sp.splits, Ii, r, 1.0f, true, static_cast<__nv_bfloat16*>(dAd), st));
+  return backward_core(GU, X, XAgu, M, &m->gate_up, gate_up_segs(I), m->A_gate_up, m->B_gate_up, r, s, dX, dAgu,
+                       dBgu, skinny, part, status, st);
+}
+
+lora_status_t mlp_ws_check(long long M, const lora_mlp_t* m, int r, void* workspace, size_t ws_bytes) {
+  const WsLayout wl = mlp_ws_layout(M, m->gate_up.K, m->down.K, r);
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
+  return LORA_OK;
+}
+
 size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K, int32_t r, int32_t nseg, int32_t fmt) {
   if (M < 0 || N <= 0 || K <= 0 || r < 8 || r > 128 || r % 8) return 0;
   if (nseg < 1 || nseg > LORA_MAX_SEGMENTS || nseg * r > 128) return 0;
@@ -600,6 +742,65 @@ lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, in
                                void* dX, void* dA, void* dB, void* workspace, size_t ws_bytes, void* stream) {
   if (!segs) return LORA_ERR_INVALID_ARG;
   return bwd_entry(dY, X, XA, M, W, segs, A, B, r, s, dX, dA, dB, workspace, ws_bytes, stream);
+}
+
+size_t lora_mlp_workspace_bytes(int64_t M, int64_t D, int64_t I, int32_t r, int32_t fmt) {
+  if (M < 0 || D <= 0 || I <= 0 || r < 8 || 2 * r > 128 || r % 8) return 0;
+  if (fmt != LORA_W_BF16 && fmt != LORA_W_BLOCK4) return 0;
+  if (M > (1LL << 31) - 256 || D > (1LL << 30) || I > (1LL << 29)) return 0;
+  return mlp_ws_layout(M, D, I, r).total;
+}
+
+lora_status_t lora_mlp_fwd(const void* X, int64_t M, const lora_mlp_t* mlp, int32_t r, float s, void* Z, void* GU,
+                           void* H, void* XA_gate_up, void* XA_down, void* workspace, size_t ws_bytes, void* stream) {
+  TRY(mlp_check(mlp, r, s, M));
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(X));
+  TRY(check_ptr(Z));
+  TRY(check_ptr(GU));
+  TRY(check_ptr(H));
+  TRY(check_ptr(XA_gate_up));
+  TRY(check_ptr(XA_down));
+  TRY(mlp_ws_check(M, mlp, r, workspace, ws_bytes));
+  const WsLayout wl = mlp_ws_layout(M, mlp->gate_up.K, mlp->down.K, r);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return mlp_forward_core(X, M, mlp, r, s, Z, GU, H, XA_gate_up, XA_down,
+                          reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off), reinterpret_cast<float*>(ws + wl.part_off),
+                          reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
+                           const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s, void* dX,
+                           void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  TRY(mlp_check(mlp, r, s, M));
+  TRY(check_ptr(dA_gate_up));
+  TRY(check_ptr(dB_gate_up));
+  TRY(check_ptr(dA_down));
+  TRY(check_ptr(dB_down));
+  const long long D = mlp->gate_up.K, I = mlp->down.K;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    const size_t z[4] = {static_cast<size_t>(2 * r) * D * 2, static_cast<size_t>(2 * I) * r * 2,
+                         static_cast<size_t>(r) * I * 2, static_cast<size_t>(D) * r * 2};
+    void* ptrs[4] = {dA_gate_up, dB_gate_up, dA_down, dB_down};
+    for (int i = 0; i < 4; ++i)
+      if (cudaMemsetAsync(ptrs[i], 0, z[i], st) != cudaSuccess) return LORA_ERR_CUDA;
+    return LORA_OK;
+  }
+  TRY(check_ptr(dZ));
+  TRY(check_ptr(X));
+  TRY(check_ptr(GU));
+  TRY(check_ptr(H));
+  TRY(check_ptr(XA_gate_up));
+  TRY(check_ptr(XA_down));
+  if (dX) TRY(check_ptr(dX));
+  TRY(mlp_ws_check(M, mlp, r, workspace, ws_bytes));
+  const WsLayout wl = mlp_ws_layout(M, D, I, r);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return mlp_backward_core(dZ, X, GU, H, XA_gate_up, XA_down, M, mlp, r, s, dX, dA_gate_up, dB_gate_up, dA_down,
+                           dB_down, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
+                           reinterpret_cast<float*>(ws + wl.part_off), reinterpret_cast<uint32_t*>(ws), st);
 }
 
 lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* stream) {

@@ -101,3 +101,69 @@ class LoraGroupedLinear:
         _b.lora_grouped_bwd(dY, X, XA, M, self.W, self.rows, self.A, self.B, self.r, self.s, dX, dA, dB,
                             self.workspace(M), stream=stream)
         return dX, dA, dB
+
+
+class LoraMLP:
+    """SwiGLU feed-forward block with LoRA on gate, up and down projections.
+
+    ``gate_up`` is a :class:`LoraWeight` of shape ``[2I, D]`` (gate rows over up rows),
+    ``down`` one of ``[D, I]``; ``A_gate_up [2r, D]``, ``B_gate_up [2I, r]``,
+    ``A_down [r, I]``, ``B_down [D, r]`` are bf16 tensors.  ``forward`` returns ``Z`` and
+    the tensors ``backward`` needs (``saved``: GU, H, XA_gate_up, XA_down); ``backward``
+    overwrites ``saved["GU"]`` with ``[dG | dU]`` and returns
+    ``(dX, dA_gate_up, dB_gate_up, dA_down, dB_down)``.
+    """
+
+    def __init__(self, gate_up: "_b.LoraWeight", down: "_b.LoraWeight", A_gate_up: torch.Tensor,
+                 B_gate_up: torch.Tensor, A_down: torch.Tensor, B_down: torch.Tensor, alpha: float):
+        self.gate_up, self.down = gate_up, down
+        self.A_gate_up, self.B_gate_up, self.A_down, self.B_down = A_gate_up, B_gate_up, A_down, B_down
+        self.D, self.I = gate_up.K, down.K
+        self.r = int(A_down.shape[0])
+        self.s = float(alpha) / float(self.r)
+        self._ws = None
+        self._ws_M = -1
+
+    def c_struct(self):
+        return _b.mlp_struct(self.gate_up, self.down, self.A_gate_up, self.B_gate_up, self.A_down, self.B_down)
+
+    def workspace(self, M: int) -> torch.Tensor:
+        if self._ws is None or self._ws_M < M:
+            n = _b.mlp_workspace_bytes(M, self.D, self.I, self.r, self.gate_up.fmt)
+            if n == 0:
+                raise _b.LoraError(_b.LORA_ERR_UNSUPPORTED, "mlp_workspace_bytes")
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.A_down.device)
+            self._ws_M = M
+        return self._ws
+
+    def alloc_saved(self, M: int, device) -> dict:
+        bf = torch.bfloat16
+        return {"GU": torch.empty((M, 2 * self.I), dtype=bf, device=device),
+                "H": torch.empty((M, self.I), dtype=bf, device=device),
+                "XA_gate_up": torch.empty((M, 2 * self.r), dtype=bf, device=device),
+                "XA_down": torch.empty((M, self.r), dtype=bf, device=device)}
+
+    def forward(self, X: torch.Tensor, Z=None, saved=None, stream=None):
+        M = X.shape[0]
+        if Z is None:
+            Z = torch.empty((M, self.D), dtype=torch.bfloat16, device=X.device)
+        if saved is None:
+            saved = self.alloc_saved(M, X.device)
+        _b.lora_mlp_fwd(X, M, self.c_struct(), self.r, self.s, Z, saved["GU"], saved["H"], saved["XA_gate_up"],
+                        saved["XA_down"], self.workspace(M), stream=stream)
+        return Z, saved
+
+    def backward(self, dZ: torch.Tensor, X: torch.Tensor, saved: dict, need_dX: bool = True, out=None, stream=None):
+        M = dZ.shape[0]
+        dev = dZ.device
+        bf = torch.bfloat16
+        if out is None:
+            out = (torch.empty((M, self.D), dtype=bf, device=dev) if need_dX else None,
+                   torch.empty((2 * self.r, self.D), dtype=bf, device=dev),
+                   torch.empty((2 * self.I, self.r), dtype=bf, device=dev),
+                   torch.empty((self.r, self.I), dtype=bf, device=dev),
+                   torch.empty((self.D, self.r), dtype=bf, device=dev))
+        dX, dAgu, dBgu, dAd, dBd = out
+        _b.lora_mlp_bwd(dZ, X, saved["GU"], saved["H"], saved["XA_gate_up"], saved["XA_down"], M, self.c_struct(),
+                        self.r, self.s, dX, dAgu, dBgu, dAd, dBd, self.workspace(M), stream=stream)
+        return out

@@ -11,5 +11,7 @@ from .inputs import (  # noqa: F401
     f32_from_bf16_bits,
     make_case,
     make_grouped_case,
+    MlpCase,
+    make_mlp_case,
     config_cases,
 )

@@ -198,3 +198,39 @@ def make_grouped_case(case: LoraCase, rows, want=("X", "W", "A", "B", "dY")) -> 
     drawn for the stacked ``[ΣN_g, ...]`` shapes and A for ``[G·r, K]``."""
     assert sum(int(n) for n in rows) == case.N
     return make_case(dataclasses.replace(case, rows=tuple(int(n) for n in rows)), want=want)
+
+
+@dataclasses.dataclass(frozen=True)
+class MlpCase:
+    """One feed-forward block: tokens M, model width D, hidden width I, rank r."""
+
+    name: str
+    M: int
+    D: int
+    I: int  # noqa: E741
+    r: int
+    alpha: float
+    fmt: str
+    seed: int
+
+    @property
+    def s(self) -> float:
+        return float(self.alpha) / float(self.r)
+
+    def gate_up_case(self) -> LoraCase:
+        """The gate and up projections as two projections of X stacked along rows."""
+        return LoraCase(self.name + "_gate_up", self.M, 2 * self.I, self.D, self.r, self.alpha, self.fmt, self.seed,
+                        rows=(self.I, self.I))
+
+    def down_case(self) -> LoraCase:
+        return LoraCase(self.name + "_down", self.M, self.D, self.I, self.r, self.alpha, self.fmt, self.seed + 7919)
+
+
+def make_mlp_case(case: MlpCase) -> dict:
+    """Inputs of a feed-forward block: X and the gate/up weight and adapters from the
+    gate/up case (W ~ N(0, 1/D)), the down weight and adapters and dZ (the down case's dY)
+    from the down case (W ~ N(0, 1/I)); same distributions as :func:`make_case`."""
+    gu = make_case(case.gate_up_case(), want=("X", "W", "A", "B"))
+    dn = make_case(case.down_case(), want=("W", "A", "B", "dY"))
+    return {"case": case, "X": gu["X"], "A_gu": gu["A"], "B_gu": gu["B"], "A_d": dn["A"], "B_d": dn["B"],
+            "dZ": dn["dY"], "gate_up": gu, "down": dn}

@@ -60,7 +60,11 @@ def run_layer(q, inp, need_dX=True):
             "X": X, "dY": dY}
 
 
-def check(name: str, got: np.ndarray, ref: np.ndarray):
+def check(name: str, got: np.ndarray, ref: np.ndarray, rel_elem: float = 0.0):
+    """Parity bar.  ``rel_elem`` adds ``rel_elem·|ref|`` to the per-element bound for
+    outputs whose own bf16 storage rounding (2^-8 relative) and that of the bf16 values
+    they are computed from are not covered by ``ELEM_RMS·rms``: heavy-tailed products
+    such as SwiGLU's derivatives, whose largest elements lie over 12·rms."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -71,5 +75,10 @@ def check(name: str, got: np.ndarray, ref: np.ndarray):
     rms = nref / np.sqrt(ref.size) if ref.size else 0.0
     emax = np.max(np.abs(err)) if err.size else 0.0
     assert rel <= REL_FRO, f"{name}: relative Frobenius error {rel:.3e} > {REL_FRO}"
-    assert emax <= ELEM_RMS * rms + 1e-30, f"{name}: max |err| {emax:.3e} > {ELEM_RMS}*rms {rms:.3e}"
+    if rel_elem == 0.0:
+        assert emax <= ELEM_RMS * rms + 1e-30, f"{name}: max |err| {emax:.3e} > {ELEM_RMS}*rms {rms:.3e}"
+    else:
+        excess = np.abs(err) - (ELEM_RMS * rms + rel_elem * np.abs(ref))
+        worst = float(np.max(excess)) if excess.size else 0.0
+        assert worst <= 1e-30, f"{name}: an element exceeds {ELEM_RMS}*rms + {rel_elem:.4f}*|ref| by {worst:.3e}"
     return rel, emax / rms if rms > 0 else 0.0

@@ -145,3 +145,33 @@ def test_grouped_validation():
     assert q.grouped_workspace_bytes(4096, 6144, 4096, 16, 3) > q.workspace_bytes(4096, 6144, 4096, 16)
     assert q.grouped_workspace_bytes(4096, 6144, 4096, 16, 1) == q.workspace_bytes(4096, 6144, 4096, 16)
     assert q.grouped_workspace_bytes(4096, 6144, 4096, 48, 3) == 0
+
+
+def test_mlp_validation():
+    lib = q.lib()
+    D, I, r = 512, 1024, 16
+
+    def mlp(**kw):
+        gu = _w(N=2 * I, K=D)
+        dn = _w(N=D, K=I)
+        m = q.lora_mlp_t(gu, dn, P, P, P, P)
+        for k, v in kw.items():
+            setattr(m, k, v)
+        return m
+
+    def fwd(m, r=r, M=256, X=P):
+        return lib.lora_mlp_fwd(X, M, ctypes.byref(m), r, 2.0, P, P, P, P, P, P2, 1 << 30, None)
+
+    assert lib.lora_mlp_fwd(P, 256, None, r, 2.0, P, P, P, P, P, P2, 1 << 30, None) == q.LORA_ERR_INVALID_ARG
+    assert fwd(mlp(down=_w(N=D + 8, K=I))) == q.LORA_ERR_INVALID_ARG      # down rows != D
+    assert fwd(mlp(down=_w(N=D, K=I - 8))) == q.LORA_ERR_INVALID_ARG      # gate_up rows != 2I
+    assert fwd(mlp(), r=72) == q.LORA_ERR_UNSUPPORTED                     # 2r > 128
+    assert fwd(mlp(), r=12) == q.LORA_ERR_UNSUPPORTED
+    assert fwd(mlp(A_down=None)) == q.LORA_ERR_INVALID_ARG
+    assert fwd(mlp(B_gate_up=P + 2)) == q.LORA_ERR_ALIGNMENT
+    assert fwd(mlp(), M=0, X=None) == q.LORA_OK                            # empty batch: nothing to do
+    assert fwd(mlp(), X=None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_mlp_fwd(P, 256, ctypes.byref(mlp()), r, 2.0, P, P, P, P, P, P2, 1000, None) == \
+        q.LORA_ERR_WORKSPACE
+    assert q.mlp_workspace_bytes(4096, D, I, r) > 0
+    assert q.mlp_workspace_bytes(4096, D, I, 72) == 0
