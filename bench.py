@@ -4,7 +4,7 @@ One step = forward and backward of every projection of the workload (default: th
 Llama-8B MLP projections gate, up and down at M = 16384 tokens, r = 16, bf16 weight),
 with inputs resident in device memory.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|qkv] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|qkv|mlp] [--impl ours|reference]
 
 Multi-GPU (one process per GPU under torch.distributed.run): data parallel over tokens,
 every rank runs the full per-rank workload (weak scaling) and the adapter gradients dA
@@ -31,14 +31,20 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 
 
 def workload(name: str):
-    from synth import CONFIGS
-    cases = CONFIGS[name]
+    from synth import CONFIGS, MlpCase
+    if name == "mlp":
+        blk = MlpCase("mlp_llama8b", 16384, 4096, 14336, 16, 32.0, "bf16", 7000)
+        cases = [blk.gate_up_case(), blk.down_case()]
+    else:
+        cases = CONFIGS[name]
     desc = {
         "c1": "Llama-8B attention projection, M=8192, K=N=4096, r=16, alpha=32, bf16 weight",
         "c2": "Llama-8B MLP projections gate+up (K=4096,N=14336) and down (K=14336,N=4096), "
               "M=16384, r=16, alpha=32, bf16 weight",
         "c3": "QLoRA 4-bit blockwise weight K=4096 N=14336 (16-level codebook, fp16 absmax per 64), "
               "M=8192, r=16, alpha=32",
+        "mlp": "Llama-8B feed-forward block (D=4096, I=14336) with LoRA on gate, up and down and SwiGLU, "
+               "M=16384, r=16, alpha=32, bf16 weights",
         "qkv": "Llama-8B attention q/k/v as one grouped layer (q 4096, k 1024, v 1024 rows, K=4096), "
                "M=8192, r=16 per projection, alpha=32, bf16 weight",
     }[name]
@@ -152,11 +158,21 @@ def gpu_uuid(dev) -> str:
 
 
 # ---------------------------------------------------------------------------- oracle leg
-def oracle_sample(cases, tokens: int):
+def oracle_sample(cases, tokens: int, mlp: bool = False):
     """Runs the fp64 oracle (as it stands) on the first `tokens` tokens of every
-    projection; returns (seconds, algorithmic flops of the sample)."""
+    projection (of the feed-forward block when `mlp`); returns (seconds, algorithmic
+    flops of the sample)."""
     import oracle as O
     from synth import make_case
+    if mlp:
+        gu_c, dn_c = (c.with_M(tokens) for c in cases)
+        gu = make_case(gu_c, want=("X", "W", "A", "B"))
+        dn = make_case(dn_c, want=("W", "A", "B", "dY"))
+        t0 = time.perf_counter()
+        args = (O.bf16_to_f64(gu["X"]), O.weight_f64(gu), O.bf16_to_f64(gu["A"]), O.bf16_to_f64(gu["B"]),
+                O.weight_f64(dn), O.bf16_to_f64(dn["A"]), O.bf16_to_f64(dn["B"]))
+        O.lora_mlp_backward(O.bf16_to_f64(dn["dY"]), *args, gu_c.s)  # runs the forward too
+        return time.perf_counter() - t0, case_flops(gu_c) + case_flops(dn_c)
     inputs = [make_case(c.with_M(tokens)) for c in cases]
     t0 = time.perf_counter()
     flops = 0.0
@@ -185,10 +201,10 @@ def run_reference(args, cases, desc, rank, world):
         return 0
     tokens = args.cpu_tokens
     for _ in range(args.warmup):
-        oracle_sample(cases, tokens)
+        oracle_sample(cases, tokens, mlp=args.workload == "mlp")
     times, flops = [], 0.0
     for _ in range(args.steps):
-        t, flops = oracle_sample(cases, tokens)
+        t, flops = oracle_sample(cases, tokens, mlp=args.workload == "mlp")
         times.append(t)
     total = sum(times)
     val = args.steps * flops / total / 1e12
@@ -227,6 +243,223 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+class LinearSet:
+    """The projections of a layer workload with their resident inputs and outputs."""
+
+    def __init__(self, cases, dev, rank, world):
+        import torch
+
+        import qlora_linear_b200 as q
+        from synth.device import make_case_device
+
+        self.cases, self.world = cases, world
+        self.layers, self.data = [], []
+        x_cache = {}
+        for c in cases:
+            want = ["W", "A", "B", "dY"]
+            xkey = c.x_seed if c.x_seed is not None else (c.data_seed if c.data_seed is not None else c.seed)
+            xkey = (xkey, c.M, c.K)
+            if xkey not in x_cache:
+                want.append("X")
+            d = make_case_device(c, dev, rank=rank, want=tuple(want))
+            if "X" in d:
+                x_cache[xkey] = d["X"]
+            d["X"] = x_cache[xkey]
+            if c.fmt == "bf16":
+                W = q.LoraWeight(c.N, c.K, d["W"])
+            else:
+                W = q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
+            if c.rows is None:
+                layer = q.LoraLinear(W, d["A"], d["B"], c.alpha)
+            else:
+                layer = q.LoraGroupedLinear(W, c.rows, d["A"], d["B"], c.alpha)
+            layer.workspace(c.M)
+            out = {
+                "Y": torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev),
+                "XA": torch.empty((c.M, c.G * c.r), dtype=torch.bfloat16, device=dev),
+                "dX": torch.empty((c.M, c.K), dtype=torch.bfloat16, device=dev),
+                "dA": torch.empty((c.G * c.r, c.K), dtype=torch.bfloat16, device=dev),
+                "dB": torch.empty((c.N, c.r), dtype=torch.bfloat16, device=dev),
+            }
+            self.layers.append(layer)
+            self.data.append((d, out))
+
+    def step(self, inputs=None):
+        import qlora_linear_b200 as q
+        for i, (layer, (d, o)) in enumerate(zip(self.layers, self.data)):
+            X = d["X"] if inputs is None else inputs[i]["X"]
+            dY = d["dY"] if inputs is None else inputs[i]["dY"]
+            layer.forward(X, Y=o["Y"], XA=o["XA"])
+            layer.backward(dY, X, o["XA"], out=(o["dX"], o["dA"], o["dB"]))
+            if self.world > 1:
+                q.allreduce_adapter_grads(o["dA"], o["dB"])
+
+    def statuses(self):
+        import qlora_linear_b200 as q
+        return [q.lora_device_status(layer.workspace(c.M)) for layer, c in zip(self.layers, self.cases)]
+
+
+class MlpSet:
+    """The feed-forward block workload: one LoraMLP (cases = its gate/up and down
+    projections, for the FLOP count) with resident inputs, saved tensors and outputs."""
+
+    def __init__(self, cases, dev, rank, world):
+        import torch
+
+        import qlora_linear_b200 as q
+        from synth.device import make_case_device
+
+        gu_c, dn_c = cases
+        self.cases, self.world, self.dev = cases, world, dev
+        self.M, self.D, self.I, self.r = gu_c.M, gu_c.K, dn_c.K, gu_c.r
+        gu = make_case_device(gu_c, dev, rank=rank, want=("X", "W", "A", "B"))
+        dn = make_case_device(dn_c, dev, rank=rank, want=("W", "A", "B", "dY"))
+
+        def weight(c, d):
+            if c.fmt == "bf16":
+                return q.LoraWeight(c.N, c.K, d["W"])
+            return q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
+
+        self.mlp = q.LoraMLP(weight(gu_c, gu), weight(dn_c, dn), gu["A"], gu["B"], dn["A"], dn["B"], gu_c.alpha)
+        self.inputs = {"X": gu["X"], "dZ": dn["dY"], "gu": gu, "dn": dn}
+        self.mlp.workspace(self.M)
+        bf = torch.bfloat16
+        self.saved = self.mlp.alloc_saved(self.M, dev)
+        self.Z = torch.empty((self.M, self.D), dtype=bf, device=dev)
+        self.grads = (torch.empty((self.M, self.D), dtype=bf, device=dev),
+                      torch.empty((2 * self.r, self.D), dtype=bf, device=dev),
+                      torch.empty((2 * self.I, self.r), dtype=bf, device=dev),
+                      torch.empty((self.r, self.I), dtype=bf, device=dev),
+                      torch.empty((self.D, self.r), dtype=bf, device=dev))
+        self.layers = [self.mlp]
+        self.data = []
+
+    def step(self, inputs=None):
+        import qlora_linear_b200 as q
+        X = self.inputs["X"] if inputs is None else inputs["X"]
+        dZ = self.inputs["dZ"] if inputs is None else inputs["dZ"]
+        self.mlp.forward(X, Z=self.Z, saved=self.saved)
+        self.mlp.backward(dZ, X, self.saved, out=self.grads)
+        if self.world > 1:
+            q.allreduce_adapter_grads(self.grads[1], self.grads[2])
+            q.allreduce_adapter_grads(self.grads[3], self.grads[4])
+
+    def statuses(self):
+        import qlora_linear_b200 as q
+        return [q.lora_device_status(self.mlp.workspace(self.M))]
+
+    def e2e(self, args, step):
+        """End to end with host buffers: X, dZ and the four adapters in, Z, dX and the four
+        adapter gradients out, every step; the frozen weights stay resident."""
+        import torch
+        import torch.distributed as dist
+
+        stream = torch.cuda.current_stream()
+        m = self.mlp
+        h_in = {k: t.cpu().pin_memory() for k, t in (("X", self.inputs["X"]), ("dZ", self.inputs["dZ"]),
+                                                       ("A_gate_up", m.A_gate_up), ("B_gate_up", m.B_gate_up),
+                                                       ("A_down", m.A_down), ("B_down", m.B_down))}
+        d_in = {"X": torch.empty_like(self.inputs["X"]), "dZ": torch.empty_like(self.inputs["dZ"])}
+        outs = (self.Z,) + tuple(self.grads)
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+        h2d = sum(t.numel() * 2 for t in h_in.values())
+        d2h = sum(t.numel() * 2 for t in h_out)
+
+        def e2e_step():
+            d_in["X"].copy_(h_in["X"], non_blocking=True)
+            d_in["dZ"].copy_(h_in["dZ"], non_blocking=True)
+            for k in ("A_gate_up", "B_gate_up", "A_down", "B_down"):
+                getattr(m, k).copy_(h_in[k], non_blocking=True)
+            step(inputs=d_in)
+            for h, t in zip(h_out, outs):
+                h.copy_(t, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        steps = max(3, args.steps // 2)
+        if self.world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        if self.world > 1:
+            t = torch.tensor([ms], device=self.dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        flops_step = sum(case_flops(c) for c in self.cases)
+        return {"value": self.world * flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+                "note": "X, dZ and the four adapters copied from pinned host memory and Z, dX and the four adapter "
+                        "gradients read back every step; the frozen weights stay resident"}
+
+
+def time_separate_mlp(args, cases, ws, dev):
+    """The same block unfused: gate, up and down as three separate layers, SwiGLU and its
+    derivative as torch elementwise ops between them (what a model without the fused
+    block runs)."""
+    import torch
+
+    import qlora_linear_b200 as q
+
+    stream = torch.cuda.current_stream()
+    m, M, D, I, r = ws.mlp, ws.M, ws.D, ws.I, ws.r
+    gu = ws.inputs["gu"]
+    bf = torch.bfloat16
+    Wg = q.LoraWeight(I, D, m.gate_up.data[:I]) if m.gate_up.fmt == q.LORA_W_BF16 else None
+    if Wg is None:
+        return None
+    Wu = q.LoraWeight(I, D, m.gate_up.data[I:])
+    gate = q.LoraLinear(Wg, m.A_gate_up[:r], m.B_gate_up[:I], r * m.s)
+    up = q.LoraLinear(Wu, m.A_gate_up[r:], m.B_gate_up[I:], r * m.s)
+    down = q.LoraLinear(m.down, m.A_down, m.B_down, r * m.s)
+    for L in (gate, up, down):
+        L.workspace(M)
+    X, dZ = gu["X"], ws.inputs["dZ"]
+    G, U, H = (torch.empty((M, I), dtype=bf, device=dev) for _ in range(3))
+    XAg, XAu, XAd = (torch.empty((M, r), dtype=bf, device=dev) for _ in range(3))
+    Z = torch.empty((M, D), dtype=bf, device=dev)
+    dH = torch.empty((M, I), dtype=bf, device=dev)
+    gbufs = [(torch.empty((M, D), dtype=bf, device=dev), torch.empty((r, D), dtype=bf, device=dev),
+              torch.empty((I, r), dtype=bf, device=dev)) for _ in range(2)]
+    dgd = (dH, torch.empty((r, I), dtype=bf, device=dev), torch.empty((D, r), dtype=bf, device=dev))
+
+    def step():
+        gate.forward(X, Y=G, XA=XAg)
+        up.forward(X, Y=U, XA=XAu)
+        g32 = G.float()
+        H.copy_(g32 * torch.sigmoid(g32) * U.float())
+        down.forward(H, Y=Z, XA=XAd)
+        down.backward(dZ, H, XAd, out=dgd)
+        g32, u32, dh32 = G.float(), U.float(), dH.float()
+        sg = torch.sigmoid(g32)
+        dG = (dh32 * u32 * sg * (1 + g32 * (1 - sg))).to(bf)
+        dU = (dh32 * g32 * sg).to(bf)
+        gate.backward(dG, X, XAg, out=gbufs[0])
+        up.backward(dU, X, XAu, out=gbufs[1])
+        gbufs[0][0].add_(gbufs[1][0])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops_step = sum(case_flops(c) for c in cases)
+    return {"ms_per_step": ms, "value": flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "note": "gate, up, down as three separate layers of this library, SwiGLU forward and backward as "
+                    "torch elementwise ops in fp32, dX of gate and up summed by torch"}
+
+
 def run_ours(args, cases, desc, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -239,46 +472,12 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     # ---- inputs resident in HBM (drawn on the device)
-    layers, data = [], []
-    x_cache = {}
-    for c in cases:
-        want = ["W", "A", "B", "dY"]
-        xkey = c.x_seed if c.x_seed is not None else (c.data_seed if c.data_seed is not None else c.seed)
-        xkey = (xkey, c.M, c.K)
-        if xkey not in x_cache:
-            want.append("X")
-        d = make_case_device(c, dev, rank=rank, want=tuple(want))
-        if "X" in d:
-            x_cache[xkey] = d["X"]
-        d["X"] = x_cache[xkey]
-        if c.fmt == "bf16":
-            W = q.LoraWeight(c.N, c.K, d["W"])
-        else:
-            W = q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
-        if c.rows is None:
-            layer = q.LoraLinear(W, d["A"], d["B"], c.alpha)
-        else:
-            layer = q.LoraGroupedLinear(W, c.rows, d["A"], d["B"], c.alpha)
-        layer.workspace(c.M)
-        out = {
-            "Y": torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev),
-            "XA": torch.empty((c.M, c.G * c.r), dtype=torch.bfloat16, device=dev),
-            "dX": torch.empty((c.M, c.K), dtype=torch.bfloat16, device=dev),
-            "dA": torch.empty((c.G * c.r, c.K), dtype=torch.bfloat16, device=dev),
-            "dB": torch.empty((c.N, c.r), dtype=torch.bfloat16, device=dev),
-        }
-        layers.append(layer)
-        data.append((d, out))
+    if args.workload == "mlp":
+        ws = MlpSet(cases, dev, rank, world)
+    else:
+        ws = LinearSet(cases, dev, rank, world)
+    layers, data, step = ws.layers, ws.data, ws.step
     torch.cuda.synchronize()
-
-    def step(inputs=None):
-        for i, (layer, (d, o)) in enumerate(zip(layers, data)):
-            X = d["X"] if inputs is None else inputs[i]["X"]
-            dY = d["dY"] if inputs is None else inputs[i]["dY"]
-            layer.forward(X, Y=o["Y"], XA=o["XA"])
-            layer.backward(dY, X, o["XA"], out=(o["dX"], o["dA"], o["dB"]))
-            if world > 1:
-                q.allreduce_adapter_grads(o["dA"], o["dB"])
 
     def barrier():
         if world > 1:
@@ -287,9 +486,9 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    st = q.lora_device_status(layers[0].workspace(cases[0].M))
-    if st != q.LORA_OK:
-        raise RuntimeError("device status after warm-up: " + q.status_string(st))
+    for st in ws.statuses():
+        if st != q.LORA_OK:
+            raise RuntimeError("device status after warm-up: " + q.status_string(st))
 
     # ---- timed region: K steps, device time (CUDA events), max over ranks
     clocks = ClockSampler(gpu_uuid(dev))
@@ -320,8 +519,7 @@ def run_ours(args, cases, desc, rank, world, local_rank):
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    for layer, c in zip(layers, cases):
-        st = q.lora_device_status(layer.workspace(c.M))
+    for st in ws.statuses():
         if st != q.LORA_OK:
             raise RuntimeError("device status after timing: " + q.status_string(st))
 
@@ -359,18 +557,22 @@ def run_ours(args, cases, desc, rank, world, local_rank):
 
     # ---- grouped workloads: the same projections as separate layers, for comparison
     separate = None
-    if any(c.rows is not None for c in cases) and world == 1:
+    if args.no_separate:
+        pass
+    elif world == 1 and args.workload == "mlp":
+        separate = time_separate_mlp(args, cases, ws, dev)
+    elif world == 1 and any(c.rows is not None for c in cases):
         separate = time_separate(args, cases, data, dev)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, cases, layers, data, step, world, dev)
+        e2e = ws.e2e(args, step) if args.workload == "mlp" else run_e2e(args, cases, layers, data, step, world, dev)
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, fl = oracle_sample(cases, args.cpu_tokens)
+        t, fl = oracle_sample(cases, args.cpu_tokens, mlp=args.workload == "mlp")
         cpu = {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"first {args.cpu_tokens} tokens of each projection (full K and N), fp64 numpy oracle, "
                          f"{t:.1f} s", "tokens_per_s": args.cpu_tokens / t}
@@ -515,11 +717,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "qkv"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "qkv", "mlp"])
     ap.add_argument("--only", default=None, help="run a single projection of the workload (e.g. c2_gate)")
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-separate", action="store_true", help="skip the unfused comparison of qkv / mlp")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
