@@ -24,4 +24,9 @@ from .lora_oracle import (  # noqa: F401
     swiglu_backward,
     lora_mlp_forward,
     lora_mlp_backward,
+    int8_value,
+    e4m3_value,
+    dequant_rowwise8,
+    e4m3_nearest,
+    quantize_rowwise8,
 )

@@ -32,6 +32,10 @@ What it computes (the method is exact, so the oracle is the plain definition):
   ``bf16_rn(fp32_rn(codebook[code] * absmax))``.
 * The feed-forward block (gate and up LoRA linears, ``H = silu(G)·U``, down LoRA
   linear) and its chain-rule backward, see :func:`lora_mlp_forward`.
+* The 8-bit weights ("Rev vs unsloth", fused quantized-LoRA paragraph: int8 and fp8;
+  "Unsloth vs The Stack v2", quantized fine-tuning paragraph: 8-bit): one int8 or fp8
+  e4m3 byte per element and one fp32 scale per weight row; an element dequantizes to
+  ``bf16_rn(fp32_rn(value(code) * scale[row]))``.
 * Merge of the adapter into the weight ("Rev vs unsloth", GGUF export paragraph;
   "Unsloth vs The Stack v2", merge paragraph): ``W' = W + s·B·A``.
 
@@ -156,11 +160,92 @@ def quantize_blockwise4(W: np.ndarray, codebook: np.ndarray):
     return packed, scale16.view(np.uint16)
 
 
+# ----------------------------------------------------------------------------
+# 8-bit formats: int8 or fp8 e4m3 codes, one fp32 scale per weight row
+# ----------------------------------------------------------------------------
+
+
+def int8_value(codes: np.ndarray) -> np.ndarray:
+    """Two's-complement value of each byte."""
+    return np.asarray(codes, dtype=np.uint8).view(np.int8).astype(np.float64)
+
+
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    """Value of each fp8 e4m3 byte: sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+    exponent field 0 is subnormal (``m/8 · 2^-6``); exponent 15 with mantissa 7 is NaN
+    and there are no infinities, so the largest finite value is ``1.75 · 2^8 = 448``."""
+    b = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & ((b & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def code8_value(codes: np.ndarray, fmt: str) -> np.ndarray:
+    return int8_value(codes) if fmt == "int8" else e4m3_value(codes)
+
+
+def dequant_rowwise8(codes: np.ndarray, row_scale: np.ndarray, fmt: str) -> np.ndarray:
+    """Dequantize 8-bit codes ``[N, K]`` with fp32 row scales ``[N]`` to bf16 bit patterns:
+    element ``(n, k)`` is ``bf16_rn(fp32_rn(value(code) · scale[n]))``.  value(code) has at
+    most 8 significant bits and the scale 24, so the fp64 product is exact and its
+    float32 cast is the correctly rounded fp32 product."""
+    v = code8_value(codes, fmt)
+    sc = np.asarray(row_scale, dtype=np.float32).astype(np.float64)
+    return bf16_round_bits((v * sc[:, None]).astype(np.float32))
+
+
+def e4m3_finite_values() -> np.ndarray:
+    """The 254 finite e4m3 values by code (codes 0x7F and 0xFF left out)."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    return codes, e4m3_value(codes)
+
+
+def e4m3_nearest(x: np.ndarray) -> np.ndarray:
+    """Code of the e4m3 value nearest to each x (|x| <= 448), ties to the code with an even
+    mantissa; the sign of zero follows x."""
+    x = np.asarray(x, dtype=np.float64)
+    codes, vals = e4m3_finite_values()
+    pos = vals >= 0
+    pc, pv = codes[pos & (codes < 0x80)], vals[pos & (codes < 0x80)]  # +0 .. 448
+    a = np.abs(x)
+    d = np.abs(a[..., None] - pv)
+    best = d.min(axis=-1, keepdims=True)
+    tie = d == best
+    # among equally near codes take the even one (at most two candidates)
+    even = tie & ((pc & 1) == 0)
+    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(tie, axis=-1))
+    c = pc[pick].astype(np.uint8)
+    return np.where(np.signbit(x), c | 0x80, c).astype(np.uint8)
+
+
+def quantize_rowwise8(W: np.ndarray, fmt: str):
+    """Quantize ``[N, K]`` to 8-bit codes with one fp32 scale per row:
+    int8: ``scale = fp32(max|w| / 127)``, ``code = clip(rint(w/scale), -127, 127)``;
+    fp8:  ``scale = fp32(max|w| / 448)``, ``code = e4m3_nearest(w/scale)``.
+    A zero row takes scale 0 and code 0.  Returns ``(codes uint8 [N, K], scale float32 [N])``."""
+    W = np.asarray(W, dtype=np.float64)
+    top = 127.0 if fmt == "int8" else 448.0
+    scale = (np.max(np.abs(W), axis=1) / top).astype(np.float32)
+    safe = np.where(scale > 0, scale.astype(np.float64), 1.0)
+    q = W / safe[:, None]
+    if fmt == "int8":
+        codes = np.clip(np.rint(q), -127, 127).astype(np.int8).view(np.uint8)
+    else:
+        codes = e4m3_nearest(np.clip(q, -448.0, 448.0))
+    codes[scale == 0] = 0
+    return codes, scale
+
+
 def weight_f64(inputs: dict) -> np.ndarray:
-    """The frozen weight of an input dict as fp64 ``[N, K]`` (dequantized if 4-bit)."""
+    """The frozen weight of an input dict as fp64 ``[N, K]`` (dequantized if 4- or 8-bit)."""
     if inputs.get("W") is not None:
         return bf16_to_f64(inputs["W"])
     case = inputs["case"]
+    if case.fmt in ("int8", "fp8"):
+        return bf16_to_f64(dequant_rowwise8(inputs["codes"], inputs["row_scale"], case.fmt))
     bits = dequant_blockwise4(inputs["codes"], inputs["absmax"], inputs["codebook"], case.N, case.K)
     return bf16_to_f64(bits)
 

@@ -64,7 +64,7 @@ class LoraCase:
     K: int
     r: int
     alpha: float
-    fmt: str  # "bf16" or "block4"
+    fmt: str  # "bf16", "block4", "int8" or "fp8"
     seed: int                  # stream of A and B (and of X, W, dY unless set below)
     x_seed: int | None = None  # X stream: lets two projections share one activation tensor
     data_seed: int | None = None  # W and dY stream (and X if x_seed is None)
@@ -173,7 +173,7 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
     if "W" in want:
         if case.fmt == "bf16":
             out["W"] = _fill((N, K), ds, _TID["W"], _normal_bf16(1.0 / np.sqrt(K)))
-        else:
+        elif case.fmt == "block4":
             assert K % 64 == 0
             g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([ds, _TID["codes"]])))
             out["codes"] = g.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
@@ -181,6 +181,8 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
             u = g.random(N * K // 64)
             out["absmax"] = ((1.2 + 0.8 * u) / np.sqrt(K)).astype(np.float16).view(np.uint16)
             out["codebook"] = codebook_levels()
+        if case.fmt in ("int8", "fp8"):
+            out.update(_codes8(case, ds))
     if "A" in want:
         a = 1.0 / np.sqrt(K)
         out["A"] = _fill((case.G * r, K), case.seed, _TID["A"], _uniform_bf16(-a, a))
@@ -191,6 +193,34 @@ def make_case(case: LoraCase, want=("X", "W", "A", "B", "dY")) -> dict:
     if "dY" in want:
         out["dY"] = _fill((M, N), ds, _TID["dY"], _normal_bf16(1.0))
     return out
+
+
+# rms of the decoded codes drawn below: int8 uniform on [-127, 127] has mean square
+# 127·128/3; fp8 with exponent field uniform on 1..14 and mantissa uniform on 0..7 has
+# mean square (4^14 - 1)/(3·4^6)/14 · 2.1484375
+RMS_INT8 = float(np.sqrt(127 * 128 / 3))
+RMS_FP8 = float(np.sqrt((4 ** 14 - 1) / (3 * 4 ** 6) / 14 * 2.1484375))
+
+
+def _codes8(case: LoraCase, ds: int) -> dict:
+    """8-bit weight codes [N, K] and fp32 row scales [N]: int8 codes uniform on
+    [-127, 127]; fp8 e4m3 codes with sign uniform, exponent field uniform on 1..14 and
+    mantissa uniform on 0..7 (never NaN); scale of row n ``(0.8 + 0.4 u_n)/(rms·sqrt(K))``
+    so that the weight's rms is about 1/sqrt(K), as for the bf16 weights."""
+    N, K = case.N, case.K
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([ds, _TID["codes"]])))
+    if case.fmt == "int8":
+        codes = g.integers(-127, 128, size=(N, K), dtype=np.int16).astype(np.int8).view(np.uint8)
+        rms = RMS_INT8
+    else:
+        sign = g.integers(0, 2, size=(N, K), dtype=np.uint8)
+        expo = g.integers(1, 15, size=(N, K), dtype=np.uint8)
+        mant = g.integers(0, 8, size=(N, K), dtype=np.uint8)
+        codes = ((sign << 7) | (expo << 3) | mant).astype(np.uint8)
+        rms = RMS_FP8
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([ds, _TID["absmax"]])))
+    u = g.random(N)
+    return {"codes": codes, "row_scale": ((0.8 + 0.4 * u) / (rms * np.sqrt(K))).astype(np.float32)}
 
 
 def make_grouped_case(case: LoraCase, rows, want=("X", "W", "A", "B", "dY")) -> dict:

@@ -520,3 +520,89 @@ def test_mlp_zero_adapters_give_the_plain_block():
     g = O.lora_mlp_backward(dZ, X, W_gu, A_gu, B_gu, W_d, A_d, B_d, 2.0)
     assert np.all(g["dA_gu"] == 0) and np.all(g["dA_d"] == 0)
     assert np.any(g["dB_gu"] != 0) and np.any(g["dB_d"] != 0)
+
+
+# ---------------------------------------------------------------- 8-bit formats
+
+
+def test_e4m3_decode_against_torch_and_closed_forms():
+    c = np.arange(256, dtype=np.uint8)
+    v = O.e4m3_value(c)
+    t = torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(v), np.isnan(t))
+    assert np.array_equal(v[~np.isnan(v)], t[~np.isnan(t)])
+    assert v[0x38] == 1.0 and v[0x7E] == 448.0 and v[0x01] == 2.0 ** -9 and v[0x08] == 2.0 ** -6
+    assert v[0x80] == 0.0 and np.signbit(v[0x80]) and v[0xB8] == -1.0
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and np.sum(np.isnan(v)) == 2
+
+
+def test_int8_decode_closed_forms():
+    v = O.int8_value(np.array([0x00, 0x01, 0x7F, 0x80, 0xFF, 0xFE], dtype=np.uint8))
+    assert list(v) == [0.0, 1.0, 127.0, -128.0, -1.0, -2.0]
+
+
+def test_dequant_rowwise8_hand_example():
+    """int8 codes [[1, -2], [127, 0]] with row scales [0.5, 3]: 0.5, -1, 381 -> 380 (a tie
+    between the bf16 neighbours 380 and 382 goes to the even mantissa), 0."""
+    codes = np.array([[1, 0xFE], [127, 0]], dtype=np.uint8)
+    got = O.bf16_to_f64(O.dequant_rowwise8(codes, np.array([0.5, 3.0], dtype=np.float32), "int8"))
+    assert got.tolist() == [[0.5, -1.0], [380.0, 0.0]]
+    # fp8: 0x38 = 1.0 and 0xC4 = -(1 + 4/8)·2^1 = -3.0 at scale 0.25
+    got = O.bf16_to_f64(O.dequant_rowwise8(np.array([[0x38, 0xC4]], dtype=np.uint8),
+                                           np.array([0.25], dtype=np.float32), "fp8"))
+    assert got.tolist() == [[0.25, -0.75]]
+
+
+@pytest.mark.parametrize("fmt", ["int8", "fp8"])
+def test_dequant_rowwise8_against_torch(fmt):
+    """Bit-exact against torch: decode (int8 / float8_e4m3fn dtype), float32 multiply by
+    the row scale, bf16 cast."""
+    rng = np.random.default_rng(41)
+    N, K = 37, 96
+    codes = rng.integers(0, 256, (N, K), dtype=np.uint8)
+    if fmt == "fp8":
+        codes[(codes & 0x7F) == 0x7F] = 0x10  # no NaN codes
+    scale = (rng.random(N) * 0.01 + 1e-4).astype(np.float32)
+    tc = torch.from_numpy(codes.copy())
+    val = (tc.view(torch.int8) if fmt == "int8" else tc.view(torch.float8_e4m3fn)).to(torch.float32)
+    ref = (val * torch.from_numpy(scale)[:, None]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.dequant_rowwise8(codes, scale, fmt), ref)
+
+
+def test_e4m3_nearest_round_trip_ties_and_torch():
+    finite = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    v = O.e4m3_value(np.array(finite, dtype=np.uint8))
+    assert np.array_equal(O.e4m3_nearest(v), np.array(finite, dtype=np.uint8))  # every code back, -0 included
+    # midpoints go to the even mantissa
+    assert O.e4m3_nearest(np.array([1.0625, 1.1875, -1.0625]))[:].tolist() == [0x38, 0x3A, 0xB8]
+    x = np.linspace(-448, 448, 20001)
+    t = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_nearest(x), t)
+
+
+@pytest.mark.parametrize("fmt", ["int8", "fp8"])
+def test_quantize_rowwise8_round_trip_and_bound(fmt):
+    """Rows that hold the extreme code (127 or 448) quantize back to the same codes and
+    scales exactly; a random weight dequantizes within half a step of the format."""
+    rng = np.random.default_rng(42)
+    N, K = 16, 64
+    if fmt == "int8":
+        codes = rng.integers(-127, 128, (N, K)).astype(np.int8).view(np.uint8)
+        codes[:, 3] = 127
+    else:
+        codes = rng.integers(0, 256, (N, K), dtype=np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0x33
+        codes[:, 3] = 0x7E
+    scale = (rng.random(N) + 0.5).astype(np.float32)
+    from oracle.lora_oracle import code8_value
+    W = code8_value(codes, fmt) * scale.astype(np.float64)[:, None]
+    c2, s2 = O.quantize_rowwise8(W, fmt)
+    assert np.array_equal(s2, scale)
+    assert np.array_equal(code8_value(c2, fmt), code8_value(codes, fmt))
+    Wr = rng.standard_normal((N, K))
+    c3, s3 = O.quantize_rowwise8(Wr, fmt)
+    err = np.abs(code8_value(c3, fmt) * s3.astype(np.float64)[:, None] - Wr)
+    if fmt == "int8":
+        assert np.all(err <= 0.5 * s3[:, None] * (1 + 1e-6))
+    else:  # half a spacing of e4m3 at the value's binade, 2^-4 relative, plus the subnormal step
+        assert np.all(err <= np.abs(Wr) * 2.0 ** -4 + s3[:, None] * 2.0 ** -10)
