@@ -1,7 +1,7 @@
 /*
  * lora_linear.h — C ABI of liblora_linear.so: forward and hand-derived backward of a
- * LoRA-adapted linear layer over a frozen weight (bf16 or 4-bit blockwise), for NVIDIA
- * B200 (sm_100a).
+ * LoRA-adapted linear layer over a frozen weight (bf16, 4-bit blockwise, or 8-bit int8 /
+ * fp8 e4m3 with per-row scales), for NVIDIA B200 (sm_100a).
  *
  * The operation.  A linear layer with frozen weight W:[N,K] and a trainable rank-r
  * adapter A:[r,K], B:[N,r] scaled by s = alpha/r:
@@ -30,8 +30,8 @@
  *     anything is enqueued; on a validation error nothing is enqueued.
  *   - Device pointers must be 16-byte aligned (LORA_ERR_ALIGNMENT otherwise).
  *   - Results are deterministic: the same inputs give the same bits on every call.
- *   - Limits: 8 <= r <= 128 with r % 8 == 0; K % 8 == 0 and N % 8 == 0 (bf16 weight)
- *     or K % 64 == 0 and N % 8 == 0 (4-bit weight); M >= 0 (M == 0 is an empty batch);
+ *   - Limits: 8 <= r <= 128 with r % 8 == 0; N % 8 == 0 and K % 8 == 0 (bf16 weight),
+ *     K % 64 == 0 (4-bit weight) or K % 16 == 0 (8-bit weights); M >= 0 (M == 0 is an empty batch);
  *     s finite.  Sizes outside these give LORA_ERR_UNSUPPORTED (r, alignment of sizes)
  *     or LORA_ERR_INVALID_ARG (negative or zero N/K, non-finite s, NULL pointers).
  */
@@ -57,8 +57,10 @@ typedef enum {
 } lora_status_t;
 
 typedef enum {
-  LORA_W_BF16 = 0,    /* data: bf16 [N,K] */
-  LORA_W_BLOCK4 = 1   /* data: uint8 [N,K/2] codes; absmax: fp16 [N*K/64]; codebook: fp32 [16] */
+  LORA_W_BF16 = 0,     /* data: bf16 [N,K] */
+  LORA_W_BLOCK4 = 1,   /* data: uint8 [N,K/2] codes; absmax: fp16 [N*K/64]; codebook: fp32 [16] */
+  LORA_W_INT8 = 2,     /* data: int8 [N,K]; absmax: fp32 [N] row scales */
+  LORA_W_FP8_E4M3 = 3  /* data: fp8 e4m3 [N,K]; absmax: fp32 [N] row scales */
 } lora_wfmt_t;
 
 /*
@@ -74,6 +76,14 @@ typedef enum {
  *   levels.  Element value = bf16_rn(fp32_rn(codebook[code] * float(absmax[block]))),
  *   computed as an fp32 multiply (never fused into an FMA) followed by a
  *   round-to-nearest-even conversion to bf16.
+ * LORA_W_INT8 / LORA_W_FP8_E4M3: the 8-bit frozen weights ("Rev vs unsloth", fused
+ *   quantized-LoRA paragraph: int4, int8 and fp8 weights; "Unsloth vs The Stack v2",
+ *   quantized fine-tuning paragraph: 4-bit and 8-bit).  data = one byte per element,
+ *   [N,K] row-major: a two's-complement int8, or an fp8 e4m3 (1 sign, 4 exponent bits
+ *   with bias 7, 3 mantissa bits, no infinities; 0x7F and 0xFF are NaN).  absmax = fp32
+ *   [N]: the scale of weight row n.  Element value =
+ *   bf16_rn(fp32_rn(value(code) * absmax[n])), the multiply never fused into an FMA.
+ *   codebook is ignored (may be NULL).
  */
 typedef struct {
   int32_t fmt;            /* lora_wfmt_t */
@@ -215,6 +225,13 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
                            void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Standalone dequantization of a weight of any format to bf16 [N,K] (device, out),
+ * element by element as defined for lora_weight_t (bit-exact; a bf16 weight is copied).
+ * W_out must not overlap the weight's arrays.
+ */
+lora_status_t lora_dequant(const lora_weight_t* W, void* W_out, void* stream);
+
+/*
  * Standalone dequantization of a LORA_W_BLOCK4 weight to bf16 [N,K] (device, out),
  * element by element as defined for lora_weight_t.  Bit-exact.  Not used by the
  * forward/backward, which dequantize tiles in shared memory and never write a
@@ -226,8 +243,8 @@ lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* str
  * Merge the adapter into the weight: W_out = W + s·B·A, bf16 [N,K] (device, out),
  * accumulated in fp32 ("Rev vs unsloth", GGUF export paragraph: merging LoRA adapters
  * into base weights; "Unsloth vs The Stack v2", merge paragraph).  W may be bf16
- * (W_out may then alias W->data exactly) or 4-bit (dequantized first, element by
- * element as in dequant_blockwise4).  A: device bf16 [r,K]; B: device bf16 [N,r].
+ * (W_out may then alias W->data exactly) or 4-bit / 8-bit (dequantized first, element by
+ * element as in lora_dequant).  A: device bf16 [r,K]; B: device bf16 [N,r].
  */
 lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, int32_t r,
                          float s, void* W_out, void* stream);

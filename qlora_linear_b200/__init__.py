@@ -17,6 +17,9 @@ from .binding import (  # noqa: F401
     LORA_OK,
     LORA_W_BF16,
     LORA_W_BLOCK4,
+    LORA_W_INT8,
+    LORA_W_FP8_E4M3,
+    lora_dequant,
     LoraError,
     LoraWeight,
     alloc_workspace,

@@ -28,13 +28,15 @@ LORA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 LORA_W_BF16 = 0
 LORA_W_BLOCK4 = 1
+LORA_W_INT8 = 2
+LORA_W_FP8_E4M3 = 3
 
 EXPORTED = (
     "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
     "lora_testing_bounded_wait", "lora_timing_enable", "lora_timing_read", "lora_launch_count",
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
-    "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd",
+    "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
 )
 
 LORA_MAX_SEGMENTS = 8
@@ -103,6 +105,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_linear_bwd.restype = i32
     lib.dequant_blockwise4.argtypes = [W, vp, vp]
     lib.dequant_blockwise4.restype = i32
+    lib.lora_dequant.argtypes = [W, vp, vp]
+    lib.lora_dequant.restype = i32
     lib.lora_merge.argtypes = [W, vp, vp, i32, f32, vp, vp]
     lib.lora_merge.restype = i32
     lib.lora_device_status.argtypes = [vp, vp]
@@ -171,13 +175,24 @@ def _check(st: int, where: str):
 
 
 class LoraWeight:
-    """A frozen weight [N, K]: bf16 tensor, or the 4-bit blockwise triple
-    (codes uint8 [N, K/2], absmax fp16 [N*K/64], codebook float32 [16])."""
+    """A frozen weight [N, K]: bf16 tensor, the 4-bit blockwise triple (codes uint8
+    [N, K/2], absmax fp16 [N*K/64], codebook float32 [16]), or 8-bit codes [N, K]
+    (int8 or fp8 e4m3, one byte each) with float32 row scales [N] (``fmt`` given)."""
 
-    def __init__(self, N: int, K: int, data, absmax=None, codebook=None):
+    def __init__(self, N: int, K: int, data, absmax=None, codebook=None, fmt=None):
         self.N, self.K = int(N), int(K)
         self.data, self.absmax, self.codebook = data, absmax, codebook
-        self.fmt = LORA_W_BF16 if absmax is None else LORA_W_BLOCK4
+        if fmt is None:
+            fmt = LORA_W_BF16 if absmax is None else LORA_W_BLOCK4
+        self.fmt = int(fmt)
+
+    @classmethod
+    def int8(cls, codes: torch.Tensor, row_scale: torch.Tensor) -> "LoraWeight":
+        return cls(codes.shape[0], codes.shape[1], codes, row_scale, None, LORA_W_INT8)
+
+    @classmethod
+    def fp8(cls, codes: torch.Tensor, row_scale: torch.Tensor) -> "LoraWeight":
+        return cls(codes.shape[0], codes.shape[1], codes, row_scale, None, LORA_W_FP8_E4M3)
 
     @classmethod
     def bf16(cls, w: torch.Tensor) -> "LoraWeight":
@@ -218,6 +233,12 @@ def lora_linear_bwd(dY, X, XA, M: int, W: LoraWeight, A, B, r: int, s: float, dX
     _check(_lib.lora_linear_bwd(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r),
                                 float(s), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), int(nb), _stream(stream)),
            "lora_linear_bwd")
+
+
+def lora_dequant(W: LoraWeight, W_out, stream=None) -> None:
+    """bf16 [N, K] copy of a weight of any format (bit-exact)."""
+    w = W.c_struct()
+    _check(_lib.lora_dequant(ctypes.byref(w), _ptr(W_out), _stream(stream)), "lora_dequant")
 
 
 def dequant_blockwise4(Wq: LoraWeight, W_out, stream=None) -> None:

@@ -1,4 +1,4 @@
-// elementwise.cuh — standalone 4-bit dequantization and the adapter merge.
+// elementwise.cuh — standalone dequantization (4-bit and 8-bit) and the adapter merge.
 //
 // Both are HBM-bound and sit outside the forward/backward: the forward and backward
 // dequantize tiles in shared memory and never write a dequantized weight to HBM.
@@ -42,22 +42,59 @@ __global__ void dequant4_kernel(const uint8_t* __restrict__ codes, const __half*
   }
 }
 
+// Value of one 8-bit code: the signed byte (int8) or the e4m3 number (fp8), exact in fp32.
+template <int WF8>
+__device__ __forceinline__ float w8_value(uint32_t byte) {
+  if constexpr (WF8 == 2) {
+    return static_cast<float>(static_cast<int8_t>(static_cast<uint8_t>(byte)));
+  } else {
+    uint32_t h2;
+    asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "r"(byte & 0xFFu));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  }
+}
+
+// W_out[N*K] (bf16) from 8-bit codes [N, K] and fp32 row scales [N]: each thread expands
+// 16 elements (16 code bytes -> 32 output bytes) per grid-stride step (K % 16 == 0).
+template <int WF8>
+__global__ void dequant8_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scale,
+                                __nv_bfloat16* __restrict__ out, size_t total, long long K) {
+  const size_t groups = total / 16;
+  for (size_t g = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
+       g += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 c = *reinterpret_cast<const uint4*>(codes + g * 16);
+    const float sc = scale[static_cast<long long>(g * 16) / K];
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = pack_bf16x2(__fmul_rn(w8_value<WF8>(w[i]), sc), __fmul_rn(w8_value<WF8>(w[i] >> 8), sc));
+      o[2 * i + 1] = pack_bf16x2(__fmul_rn(w8_value<WF8>(w[i] >> 16), sc), __fmul_rn(w8_value<WF8>(w[i] >> 24), sc));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + g * 16);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 // W_out = W + s·B·A over a tile of 32 rows × 256 columns per CTA (256 threads, each
-// 8 rows × 4 columns), fp32 accumulation.  W is bf16 [N,K] (w16 != null) or the 4-bit
-// format (codes/absmax/codebook).  W_out may alias w16: every element is read and then
+// 8 rows × 4 columns), fp32 accumulation.  W is bf16 [N,K] (fmt 0, w16), the 4-bit
+// format (fmt 1, codes/absmax/codebook) or 8-bit codes with row scales (fmt 2 int8, 3
+// fp8 e4m3; codes/row_scale).  W_out may alias w16: every element is read and then
 // written by the same thread.
 constexpr int MG_TN = 32, MG_TK = 256, MG_THREADS = 256;
 
 __global__ void __launch_bounds__(MG_THREADS)
-    merge_kernel(const __nv_bfloat16* w16, const uint8_t* __restrict__ codes, const __half* __restrict__ absmax,
-                 const float* __restrict__ codebook, const __nv_bfloat16* __restrict__ A,
+    merge_kernel(int fmt, const __nv_bfloat16* w16, const uint8_t* __restrict__ codes,
+                 const __half* __restrict__ absmax, const float* __restrict__ codebook,
+                 const float* __restrict__ row_scale, const __nv_bfloat16* __restrict__ A,
                  const __nv_bfloat16* __restrict__ B, int N, int K, int r, float s, __nv_bfloat16* out) {
   extern __shared__ __align__(16) float mg_smem[];
   float* sB = mg_smem;                 // [MG_TN][r]
   float* sA = mg_smem + MG_TN * r;     // [r][MG_TK]
   __shared__ float lut[16];
   const int n0 = blockIdx.y * MG_TN, k0 = blockIdx.x * MG_TK;
-  if (codes && threadIdx.x < 16) lut[threadIdx.x] = codebook[threadIdx.x];
+  if (fmt == 1 && threadIdx.x < 16) lut[threadIdx.x] = codebook[threadIdx.x];
   for (int i = threadIdx.x; i < MG_TN * r; i += MG_THREADS) {
     const int n = n0 + i / r, j = i % r;
     sB[i] = n < N ? __bfloat162float(B[static_cast<size_t>(n) * r + j]) : 0.f;
@@ -94,12 +131,15 @@ __global__ void __launch_bounds__(MG_THREADS)
       if (k >= K) continue;
       const size_t idx = static_cast<size_t>(n) * K + k;
       float w;
-      if (w16) {
+      if (fmt == 0) {
         w = __bfloat162float(w16[idx]);
-      } else {
+      } else if (fmt == 1) {
         const uint8_t byte = codes[idx >> 1];
         const uint32_t code = (idx & 1) ? (byte >> 4) : (byte & 0xFu);
         w = __bfloat162float(__float2bfloat16_rn(dq_level(lut, code, __half2float(absmax[idx / 64]))));
+      } else {
+        const float v = fmt == 2 ? w8_value<2>(codes[idx]) : w8_value<3>(codes[idx]);
+        w = __bfloat162float(__float2bfloat16_rn(__fmul_rn(v, row_scale[n])));
       }
       out[idx] = __float2bfloat16_rn(w + s * acc[a][b]);
     }

@@ -57,14 +57,21 @@ struct PairParams {
   __nv_bfloat16* out;  // [M, Nout] row-major
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
-  // 4-bit weight only
-  const __half* absmax;   // [Nw*Kw/64]
-  const float* codebook;  // [16]
-  int Nw, Kw;             // logical weight shape [Nw, Kw]
+  // quantized weights only
+  const __half* absmax;      // 4-bit: fp16 [Nw*Kw/64]
+  const float* codebook;     // 4-bit: [16]
+  const float* row_scale;    // 8-bit: fp32 [Nw]
+  int Nw, Kw;                // logical weight shape [Nw, Kw]
 };
 
-template <bool B_MN, bool W4>
+// Storage format of the frozen weight (the values of lora_wfmt_t).
+enum : int { WF_BF16 = 0, WF_BLOCK4 = 1, WF_INT8 = 2, WF_FP8 = 3 };
+
+template <bool B_MN, int WF>
 struct PairCfg {
+  static constexpr bool W4 = WF == WF_BLOCK4;
+  static constexpr bool W8 = WF == WF_INT8 || WF == WF_FP8;
+  static constexpr bool DEQ = W4 || W8;  // the B tile is expanded in shared memory
   static constexpr int BM = 256, BN = 256, BK = 128;  // pair tile, K per pipeline fill
   static constexpr int HM = 128, HN = 128;            // per-CTA halves of A rows / B rows
   static constexpr int STAGES = 3;
@@ -74,7 +81,7 @@ struct PairCfg {
   static constexpr int C_BYTES = W4 ? HN * BK / 2 : 0;  // 8 KB of codes
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
   static constexpr int NUM_EPI_WARPS = 4;
-  static constexpr int NUM_DEQ_WARPS = W4 ? 8 : 0;  // two per SM sub-partition
+  static constexpr int NUM_DEQ_WARPS = DEQ ? 8 : 0;  // two per SM sub-partition
   static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS + NUM_DEQ_WARPS);
   static constexpr int TMEM_COLS = 512;
   static constexpr int NUM_BARS = 4 * STAGES + 5;
@@ -163,20 +170,54 @@ __device__ __forceinline__ void block_levels(const float (&cb)[16], float scale,
 }
 #endif
 
-template <bool B_MN, bool W4, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::NUM_THREADS, 1)
+// Eight 8-bit codes (two words, element 4i+j in byte j of word i) to eight bf16
+// bf16_rn(fp32_rn(value(code) * scale)).  int8: value = the signed byte, made exact in
+// fp32 by placing the biased byte in the mantissa of 2^23; fp8: e4m3 decoded exactly
+// through f16 by the hardware conversion.
+template <int WF>
+__device__ __forceinline__ uint4 expand8_w8(uint32_t w0, uint32_t w1, float sc) {
+  float f[8];
+  if constexpr (WF == WF_INT8) {
+    const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;  // byte + 128, unsigned
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[j] = __uint_as_float(prmt(u0, 0x4B000000u, 0x7540u | j)) - 8388736.0f;  // 2^23 + 128
+      f[4 + j] = __uint_as_float(prmt(u1, 0x4B000000u, 0x7540u | j)) - 8388736.0f;
+    }
+  } else {
+    const uint32_t hw[4] = {w0 & 0xffffu, w0 >> 16, w1 & 0xffffu, w1 >> 16};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t h2;
+      asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "r"(hw[j]));
+      const __half2 hv = *reinterpret_cast<const __half2*>(&h2);
+      f[2 * j] = __low2float(hv);
+      f[2 * j + 1] = __high2float(hv);
+    }
+  }
+  uint4 o;
+  o.x = pack_bf16x2(__fmul_rn(f[0], sc), __fmul_rn(f[1], sc));
+  o.y = pack_bf16x2(__fmul_rn(f[2], sc), __fmul_rn(f[3], sc));
+  o.z = pack_bf16x2(__fmul_rn(f[4], sc), __fmul_rn(f[5], sc));
+  o.w = pack_bf16x2(__fmul_rn(f[6], sc), __fmul_rn(f[7], sc));
+  return o;
+}
+
+template <bool B_MN, int WF, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::NUM_THREADS, 1)
     lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
                           const PairParams p) {
-  using C = PairCfg<B_MN, W4>;
+  using C = PairCfg<B_MN, WF>;
+  constexpr bool W4 = C::W4, W8 = C::W8, DEQ = C::DEQ;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* scale_ring = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES);  // W4
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::SCALE_BYTES);
   uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
   uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
-  uint64_t* cfull = bars + 2 * C::STAGES;   // both (W4): this CTA's code tile landed
-  uint64_t* deq = bars + 3 * C::STAGES;     // leader (W4): both CTAs' dequantized tiles written
+  uint64_t* cfull = bars + 2 * C::STAGES;   // both (4-/8-bit): this CTA's code tile landed
+  uint64_t* deq = bars + 3 * C::STAGES;     // leader (4-/8-bit): both CTAs' dequantized tiles written
   uint64_t* tfull = bars + 4 * C::STAGES;   // both: accumulator ready for the epilogue
   uint64_t* tempty = tfull + 2;             // leader: both CTAs drained the accumulator
   uint64_t* drain = tempty + 2;             // leader: final commit before TMEM release
@@ -250,7 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
           const uint32_t full_l = mapa_shared(smem_u32(&full[stage]), 0);
           if (leader) {
             uint32_t per_cta;
-            if (!ext) per_cta = C::A_BYTES + (W4 ? 0 : C::B_BYTES);
+            if (!ext) per_cta = C::A_BYTES + (DEQ ? 0 : C::B_BYTES);
             else per_cta = ext_atoms * (C::A_BYTES / 2) + (B_MN ? C::B_BYTES : ext_atoms * (C::B_BYTES / 2));
             mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * per_cta);
           }
@@ -263,6 +304,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
               mbar_arrive_expect_tx(smem_u32(&cfull[stage]), C::C_BYTES);
               if (!B_MN) tma_load_2d(sC, &tmB, smem_u32(&cfull[stage]), kb * (C::BK / 2), brow);
               else tma_load_2d(sC, &tmB, smem_u32(&cfull[stage]), brow / 2, kb * C::BK);
+            } else if (W8) {
+              // 8-bit codes, one 32-row × 64-byte box per dequant warp, placed in the upper
+              // half of the 4 KB of the B buffer that warp will write, so each warp reads its
+              // codes and expands them in place with no other warp involved
+              mbar_arrive_expect_tx(smem_u32(&cfull[stage]), C::B_BYTES / 2);
+              for (int w = 0; w < 8; ++w) {
+                const int hh = w >> 2, rq = (w & 3) * 32;
+                const uint32_t dst = sB + hh * (C::B_BYTES / 2) + rq * 128 + 2048;
+                if (!B_MN) tma_load_2d(dst, &tmB, smem_u32(&cfull[stage]), kb * C::BK + hh * C::ATOM, brow + rq);
+                else tma_load_2d(dst, &tmB, smem_u32(&cfull[stage]), brow + hh * C::ATOM, kb * C::BK + rq);
+              }
             } else if (!B_MN) {
               tma_load_2d_pair(sB, &tmB, full_l, kb * C::BK, brow);
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmB, full_l, kb * C::BK + C::ATOM, brow);
@@ -286,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
               tma_load_2d_pair(sB, &tmF, full_l, brow, 0);
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmF, full_l, brow + C::ATOM, 0);
             }
-            if (W4) mbar_arrive(smem_u32(&cfull[stage]));  // nothing to dequantize in this fill
+            if (DEQ) mbar_arrive(smem_u32(&cfull[stage]));  // nothing to dequantize in this fill
           }
           ++fills;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -300,7 +352,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
           const int s = static_cast<int>(f % C::STAGES);
           const uint32_t ph = static_cast<uint32_t>((f / C::STAGES) & 1);
           if (leader) mbar_wait(smem_u32(&full[s]), ph, drain_wc);
-          if (W4) mbar_wait(smem_u32(&cfull[s]), ph, drain_wc);
+          if (DEQ) mbar_wait(smem_u32(&cfull[s]), ph, drain_wc);
         }
       }
     }
@@ -319,7 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < nkb + n_ext; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
-          if (W4 && !mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
+          if (DEQ && !mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
           tc_fence_after();
           const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
@@ -465,8 +517,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-  } else if (W4) {
-    // ------------------------------------------------------------ dequant (W4, both CTAs)
+  } else if constexpr (W4) {
+    // ------------------------------------------------------------ dequant (4-bit, both CTAs)
     const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
     const int row = dt & 127;  // weight row of this CTA's 128-row half (forward) / of the K fill (backward)
     const int h = dt >> 7;     // 64-wide atom: K atom (forward) or output chunk (backward)
@@ -547,6 +599,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, W4>::N
       if (!ok) break;
     }
     cp_async_wait<0>();  // no copy may still target shared memory at exit
+  } else if constexpr (W8) {
+    // ------------------------------------------------------------ dequant (8-bit, both CTAs)
+    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
+    const int row = dt & 127;  // weight row of this CTA's half (forward) / of the K fill (backward)
+    const int h = dt >> 7;     // 64-wide atom: K atom (forward) or output chunk (backward)
+    // fp32 scale of the weight row this thread expands in code fill (t, kb)
+    auto scale_at = [&](int t, int kb) -> float {
+      int mb, nb;
+      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+      const long long n = !B_MN ? static_cast<long long>(pair_brow<EPI>(nb, rank, p)) + row
+                                : static_cast<long long>(kb) * C::BK + row;
+      return n < p.Nw ? __ldg(p.row_scale + n) : 0.0f;
+    };
+    float sc_next = (pair < ntiles && nkb > 0) ? scale_at(pair, 0) : 0.0f;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = pair; t < ntiles; t += npairs) {
+      bool ok = true;
+      for (int kb = 0; kb < nkb + n_ext; ++kb) {
+        float sc = 0.0f;
+        if (kb < nkb) {
+          sc = sc_next;  // the next code fill's scale is loaded one fill ahead
+          const int tn = kb + 1 < nkb ? t : t + npairs;
+          if (tn < ntiles) sc_next = scale_at(tn, kb + 1 < nkb ? kb + 1 : 0);
+        }
+        if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
+        if (kb < nkb) {
+          uint8_t* rowp = smem + stage * C::STAGE_BYTES + C::A_BYTES + h * (C::B_BYTES / 2) + row * 128;
+          const uint8_t* crow = rowp - (row & 31) * 128 + 2048 + (row & 31) * 64;  // this warp's code box
+          uint32_t cw[16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 c = *reinterpret_cast<const uint4*>(crow + 16 * u);
+            cw[4 * u] = c.x;
+            cw[4 * u + 1] = c.y;
+            cw[4 * u + 2] = c.z;
+            cw[4 * u + 3] = c.w;
+          }
+          __syncwarp();  // the warp's codes are all in registers before its rows are overwritten
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) = expand8_w8<WF>(cw[2 * u], cw[2 * u + 1], sc);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
   }
 
   // ------------------------------------------------------------ teardown

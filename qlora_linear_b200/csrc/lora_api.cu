@@ -142,14 +142,16 @@ lora_status_t dev_info(DevInfo** out) {
   if (!d.attrs_set) {
     bool ok = true;
 #define SET_SMEM(fn, bytes) ok &= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-    SET_SMEM((lora_gemm_pair_kernel<false, false, EPI_STORE>), (PairCfg<false, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, false, EPI_STORE>), (PairCfg<true, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<false, true, EPI_STORE>), (PairCfg<false, true>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, true, EPI_STORE>), (PairCfg<true, true>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<false, false, EPI_SWIGLU_FWD>), (PairCfg<false, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<false, true, EPI_SWIGLU_FWD>), (PairCfg<false, true>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, false, EPI_SWIGLU_BWD>), (PairCfg<true, false>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, true, EPI_SWIGLU_BWD>), (PairCfg<true, true>::SMEM_BYTES));
+#define SET_GEMM(WF)                                                                                    \
+  SET_SMEM((lora_gemm_pair_kernel<false, WF, EPI_STORE>), (PairCfg<false, WF>::SMEM_BYTES));           \
+  SET_SMEM((lora_gemm_pair_kernel<true, WF, EPI_STORE>), (PairCfg<true, WF>::SMEM_BYTES));             \
+  SET_SMEM((lora_gemm_pair_kernel<false, WF, EPI_SWIGLU_FWD>), (PairCfg<false, WF>::SMEM_BYTES));      \
+  SET_SMEM((lora_gemm_pair_kernel<true, WF, EPI_SWIGLU_BWD>), (PairCfg<true, WF>::SMEM_BYTES));
+    SET_GEMM(WF_BF16)
+    SET_GEMM(WF_BLOCK4)
+    SET_GEMM(WF_INT8)
+    SET_GEMM(WF_FP8)
+#undef SET_GEMM
     SET_SMEM((rowproj_kernel<16, false>), (rowproj_smem_bytes<16, false>()));
     SET_SMEM((rowproj_kernel<32, false>), (rowproj_smem_bytes<32, false>()));
     SET_SMEM((rowproj_kernel<64, false>), (rowproj_smem_bytes<64, false>()));
@@ -211,7 +213,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 lora_status_t check_weight(const lora_weight_t* W) {
   if (!W) return LORA_ERR_INVALID_ARG;
-  if (W->fmt != LORA_W_BF16 && W->fmt != LORA_W_BLOCK4) return LORA_ERR_INVALID_ARG;
+  if (W->fmt < LORA_W_BF16 || W->fmt > LORA_W_FP8_E4M3) return LORA_ERR_INVALID_ARG;
   if (W->reserved != 0) return LORA_ERR_INVALID_ARG;
   if (W->N <= 0 || W->K <= 0) return LORA_ERR_INVALID_ARG;
   if (W->N > (1LL << 30) || W->K > (1LL << 30)) return LORA_ERR_UNSUPPORTED;
@@ -220,10 +222,14 @@ lora_status_t check_weight(const lora_weight_t* W) {
   if (W->N % 8 != 0) return LORA_ERR_UNSUPPORTED;
   if (W->fmt == LORA_W_BF16) {
     if (W->K % 8 != 0) return LORA_ERR_UNSUPPORTED;
-  } else {
+  } else if (W->fmt == LORA_W_BLOCK4) {
     if (W->K % 64 != 0) return LORA_ERR_UNSUPPORTED;
     if (!W->absmax || !W->codebook) return LORA_ERR_INVALID_ARG;
     if (!aligned16(W->absmax) || !aligned16(W->codebook)) return LORA_ERR_ALIGNMENT;
+  } else {
+    if (W->K % 16 != 0) return LORA_ERR_UNSUPPORTED;
+    if (!W->absmax) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(W->absmax)) return LORA_ERR_ALIGNMENT;
   }
   return LORA_OK;
 }
@@ -313,23 +319,46 @@ lora_status_t finalize_cols(const float* part, int splits, int C, int r, float s
 }
 
 // ---------------------------------------------------------------- GEMM launch
-template <bool B_MN, bool W4, int EPI = EPI_STORE>
+template <bool B_MN, int WF, int EPI>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
                           const PairParams& p, int sms, cudaStream_t st) {
-  using C = PairCfg<B_MN, W4>;
+  using C = PairCfg<B_MN, WF>;
   const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_pair_kernel<B_MN, W4, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    lora_gemm_pair_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
   }
   count_launch();
   return last_launch();
 }
 
-// Every tensor-map box of the pair GEMM is 64 elements (or 64 code bytes) wide, 128 rows high.
-constexpr uint32_t kBoxX = 64, kBoxY = 128;
+// Every tensor-map box of the pair GEMM is 64 elements (or 64 code bytes) wide and 128
+// rows high, except the 8-bit code boxes: 64 bytes × 32 rows, one per dequant warp.
+constexpr uint32_t kBoxX = 64, kBoxY = 128, kBoxY8 = 32;
+
+// The weight operand's tensor map (over the stored [N, K] array, for either direction)
+// and the launch of the GEMM instantiation for the weight's format.
+template <bool B_MN, int EPI>
+lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const CUtensorMap& e, const CUtensorMap& f,
+                            const PairParams& p, int sms, cudaStream_t st) {
+  CUtensorMap b;
+  switch (W->fmt) {
+    case LORA_W_BF16:
+      TRY(tmap_bf16(&b, W->data, W->K, W->N, kBoxX, kBoxY));
+      return launch_gemm<B_MN, WF_BF16, EPI>(a, b, e, f, p, sms, st);
+    case LORA_W_BLOCK4:
+      TRY(tmap_u8(&b, W->data, W->K / 2, W->N, kBoxX, kBoxY));
+      return launch_gemm<B_MN, WF_BLOCK4, EPI>(a, b, e, f, p, sms, st);
+    case LORA_W_INT8:
+      TRY(tmap_u8(&b, W->data, W->K, W->N, kBoxX, kBoxY8));
+      return launch_gemm<B_MN, WF_INT8, EPI>(a, b, e, f, p, sms, st);
+    default:
+      TRY(tmap_u8(&b, W->data, W->K, W->N, kBoxX, kBoxY8));
+      return launch_gemm<B_MN, WF_FP8, EPI>(a, b, e, f, p, sms, st);
+  }
+}
 
 // ---------------------------------------------------------------- output segments
 // Grouped projections share X: W, A and B stack the projections' weights, adapters
@@ -390,6 +419,8 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   if (W->fmt == LORA_W_BLOCK4) {
     p.absmax = static_cast<const __half*>(W->absmax);
     p.codebook = W->codebook;
+  } else if (W->fmt != LORA_W_BF16) {
+    p.row_scale = static_cast<const float*>(W->absmax);
   }
   return p;
 }
@@ -412,18 +443,13 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   TRY(launch_rowproj<false>(Xb, Ki, static_cast<const __nv_bfloat16*>(A), part, Mi, Ki, rt, sp, st));
   TRY(finalize_rows(part, sp.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
 
-  CUtensorMap ta, tb, te, tf;
+  CUtensorMap ta, te, tf;
   TRY(tmap_bf16(&ta, X, K, M, kBoxX, kBoxY));
   TRY(tmap_bf16(&te, sXA, rt, M, kBoxX, kBoxY));
   TRY(tmap_bf16(&tf, B, r, N, kBoxX, kBoxY));
   PairParams p = gemm_params(M, N, K, r, Y, status, W);
   set_segments(p, sg, r);
-  if (W->fmt == LORA_W_BF16) {
-    TRY(tmap_bf16(&tb, W->data, K, N, kBoxX, kBoxY));
-    return launch_gemm<false, false>(ta, tb, te, tf, p, dev->sms, st);
-  }
-  TRY(tmap_u8(&tb, W->data, K / 2, N, kBoxX, kBoxY));
-  return launch_gemm<false, true>(ta, tb, te, tf, p, dev->sms, st);
+  return launch_gemm_w<false, EPI_STORE>(W, ta, te, tf, p, dev->sms, st);
 }
 
 // ---------------------------------------------------------------- backward core
@@ -459,18 +485,12 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
   }
   if (dX) {
     // dX = dY·W + (s·dY·B)·A with the LoRA fill over all G·r ranks
-    CUtensorMap ta, tb, te, tf;
+    CUtensorMap ta, te, tf;
     TRY(tmap_bf16(&ta, dY, N, M, kBoxX, kBoxY));
     TRY(tmap_bf16(&te, sdYB, rt, M, kBoxX, kBoxY));
     TRY(tmap_bf16(&tf, A, K, rt, kBoxX, kBoxY));
     PairParams p = gemm_params(M, K, N, rt, dX, status, W);
-    if (W->fmt == LORA_W_BF16) {
-      TRY(tmap_bf16(&tb, W->data, K, N, kBoxX, kBoxY));
-      TRY((launch_gemm<true, false>(ta, tb, te, tf, p, dev->sms, st)));
-    } else {
-      TRY(tmap_u8(&tb, W->data, K / 2, N, kBoxX, kBoxY));
-      TRY((launch_gemm<true, true>(ta, tb, te, tf, p, dev->sms, st)));
-    }
+    TRY((launch_gemm_w<true, EPI_STORE>(W, ta, te, tf, p, dev->sms, st)));
   }
   // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
   const Split sp = colproj_split(M, K);
@@ -600,7 +620,7 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
                             static_cast<const __nv_bfloat16*>(m->A_gate_up), part, Mi, Di, r2, sp, st));
   TRY(finalize_rows(part, sp.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
 
-  CUtensorMap ta, tb, te, tf;
+  CUtensorMap ta, te, tf;
   TRY(tmap_bf16(&ta, X, D, M, kBoxX, kBoxY));
   TRY(tmap_bf16(&te, skinny, r2, M, kBoxX, kBoxY));
   TRY(tmap_bf16(&tf, m->B_gate_up, r, 2 * I, kBoxX, kBoxY));
@@ -610,13 +630,7 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
   p.aux = static_cast<__nv_bfloat16*>(GU);
   p.ld_aux = static_cast<int>(2 * I);
   p.aux_off = static_cast<int>(I);
-  if (m->gate_up.fmt == LORA_W_BF16) {
-    TRY(tmap_bf16(&tb, m->gate_up.data, D, 2 * I, kBoxX, kBoxY));
-    TRY((launch_gemm<false, false, EPI_SWIGLU_FWD>(ta, tb, te, tf, p, dev->sms, st)));
-  } else {
-    TRY(tmap_u8(&tb, m->gate_up.data, D / 2, 2 * I, kBoxX, kBoxY));
-    TRY((launch_gemm<false, true, EPI_SWIGLU_FWD>(ta, tb, te, tf, p, dev->sms, st)));
-  }
+  TRY((launch_gemm_w<false, EPI_SWIGLU_FWD>(&m->gate_up, ta, te, tf, p, dev->sms, st)));
   Segs one;
   one.rows[0] = D;
   one.off[1] = D;
@@ -645,7 +659,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
   TRY(finalize_cols(part, sp.splits, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
   // dH = dZ·W_d + (s·dZ·B_d)·A_d, consumed by the epilogue: GU <- [dG | dU]
   {
-    CUtensorMap ta, tb, te, tf;
+    CUtensorMap ta, te, tf;
     TRY(tmap_bf16(&ta, dZ, D, M, kBoxX, kBoxY));
     TRY(tmap_bf16(&te, skinny, r, M, kBoxX, kBoxY));
     TRY(tmap_bf16(&tf, m->A_down, I, r, kBoxX, kBoxY));
@@ -653,13 +667,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
     p.aux = static_cast<__nv_bfloat16*>(GU);
     p.ld_aux = static_cast<int>(2 * I);
     p.aux_off = static_cast<int>(I);
-    if (m->down.fmt == LORA_W_BF16) {
-      TRY(tmap_bf16(&tb, m->down.data, I, D, kBoxX, kBoxY));
-      TRY((launch_gemm<true, false, EPI_SWIGLU_BWD>(ta, tb, te, tf, p, dev->sms, st)));
-    } else {
-      TRY(tmap_u8(&tb, m->down.data, I / 2, D, kBoxX, kBoxY));
-      TRY((launch_gemm<true, true, EPI_SWIGLU_BWD>(ta, tb, te, tf, p, dev->sms, st)));
-    }
+    TRY((launch_gemm_w<true, EPI_SWIGLU_BWD>(&m->down, ta, te, tf, p, dev->sms, st)));
   }
   // dA_d = (s·dZ·B_d)ᵀ·H
   sp = colproj_split(M, I);
@@ -680,7 +688,7 @@ lora_status_t mlp_ws_check(long long M, const lora_mlp_t* m, int r, void* worksp
 size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K, int32_t r, int32_t nseg, int32_t fmt) {
   if (M < 0 || N <= 0 || K <= 0 || r < 8 || r > 128 || r % 8) return 0;
   if (nseg < 1 || nseg > LORA_MAX_SEGMENTS || nseg * r > 128) return 0;
-  if (fmt != LORA_W_BF16 && fmt != LORA_W_BLOCK4) return 0;
+  if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3) return 0;
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 30)) return 0;
   return ws_layout(M, N, K, nseg * r).total;
 }
@@ -746,7 +754,7 @@ lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, in
 
 size_t lora_mlp_workspace_bytes(int64_t M, int64_t D, int64_t I, int32_t r, int32_t fmt) {
   if (M < 0 || D <= 0 || I <= 0 || r < 8 || 2 * r > 128 || r % 8) return 0;
-  if (fmt != LORA_W_BF16 && fmt != LORA_W_BLOCK4) return 0;
+  if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3) return 0;
   if (M > (1LL << 31) - 256 || D > (1LL << 30) || I > (1LL << 29)) return 0;
   return mlp_ws_layout(M, D, I, r).total;
 }
@@ -821,6 +829,40 @@ lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* str
   return last_launch();
 }
 
+lora_status_t lora_dequant(const lora_weight_t* W, void* W_out, void* stream) {
+  TRY(check_weight(W));
+  TRY(check_ptr(W_out));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t total = static_cast<size_t>(W->N) * W->K;
+  if (W->fmt == LORA_W_BLOCK4) return dequant_blockwise4(W, W_out, stream);
+  {
+    // the output may not overlap the stored weight
+    const uint8_t* c0 = static_cast<const uint8_t*>(W->data);
+    const uint8_t* c1 = c0 + total * (W->fmt == LORA_W_BF16 ? 2 : 1);
+    const uint8_t* o0 = static_cast<const uint8_t*>(W_out);
+    if (o0 < c1 && c0 < o0 + total * 2) return LORA_ERR_INVALID_ARG;
+  }
+  if (W->fmt == LORA_W_BF16) {
+    if (cudaMemcpyAsync(W_out, W->data, total * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return LORA_ERR_CUDA;
+    return LORA_OK;
+  }
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  const size_t groups = total / 16;
+  size_t grid = (groups + 255) / 256;
+  const size_t cap = static_cast<size_t>(dev->sms) * 8;
+  if (grid > cap) grid = cap;
+  const auto* codes = static_cast<const uint8_t*>(W->data);
+  const auto* scale = static_cast<const float*>(W->absmax);
+  auto* out = static_cast<__nv_bfloat16*>(W_out);
+  if (W->fmt == LORA_W_INT8)
+    dequant8_kernel<2><<<static_cast<int>(grid), 256, 0, st>>>(codes, scale, out, total, W->K);
+  else
+    dequant8_kernel<3><<<static_cast<int>(grid), 256, 0, st>>>(codes, scale, out, total, W->K);
+  count_launch();
+  return last_launch();
+}
+
 lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, int32_t r, float s, void* W_out,
                          void* stream) {
   TRY(check_weight(W));
@@ -830,9 +872,9 @@ lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, i
   TRY(check_ptr(W_out));
   const bool bf = W->fmt == LORA_W_BF16;
   if (!bf) {
-    // an output overlapping the packed codes would be read after it is written
+    // an output overlapping the codes would be read after it is written
     const uint8_t* c0 = static_cast<const uint8_t*>(W->data);
-    const uint8_t* c1 = c0 + static_cast<size_t>(W->N) * W->K / 2;
+    const uint8_t* c1 = c0 + static_cast<size_t>(W->N) * W->K / (W->fmt == LORA_W_BLOCK4 ? 2 : 1);
     const uint8_t* o0 = static_cast<const uint8_t*>(W_out);
     const uint8_t* o1 = o0 + static_cast<size_t>(W->N) * W->K * 2;
     if (o0 < c1 && c0 < o1) return LORA_ERR_INVALID_ARG;
@@ -842,9 +884,11 @@ lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, i
       cudaSuccess)
     return LORA_ERR_CUDA;
   dim3 grid(cdiv(W->K, MG_TK), cdiv(W->N, MG_TN));
+  const bool w4 = W->fmt == LORA_W_BLOCK4;
   merge_kernel<<<grid, MG_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
-      bf ? static_cast<const __nv_bfloat16*>(W->data) : nullptr, bf ? nullptr : static_cast<const uint8_t*>(W->data),
-      bf ? nullptr : static_cast<const __half*>(W->absmax), bf ? nullptr : W->codebook,
+      W->fmt, bf ? static_cast<const __nv_bfloat16*>(W->data) : nullptr,
+      bf ? nullptr : static_cast<const uint8_t*>(W->data), w4 ? static_cast<const __half*>(W->absmax) : nullptr,
+      w4 ? W->codebook : nullptr, (!bf && !w4) ? static_cast<const float*>(W->absmax) : nullptr,
       static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), static_cast<int>(W->N),
       static_cast<int>(W->K), r, s, static_cast<__nv_bfloat16*>(W_out));
   count_launch();

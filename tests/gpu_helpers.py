@@ -39,6 +39,11 @@ def make_weight(q, inp):
     if case.fmt == "bf16":
         w = dev_bf16(inp["W"])
         return q.LoraWeight(case.N, case.K, w), (w,)
+    if case.fmt in ("int8", "fp8"):
+        codes = dev_u8(inp["codes"])
+        sc = torch.from_numpy(inp["row_scale"]).cuda()
+        fmt = q.LORA_W_INT8 if case.fmt == "int8" else q.LORA_W_FP8_E4M3
+        return q.LoraWeight(case.N, case.K, codes, sc, None, fmt), (codes, sc)
     codes = dev_u8(inp["codes"])
     absmax = dev_f16_bits(inp["absmax"])
     cb = torch.from_numpy(inp["codebook"]).cuda()

@@ -71,6 +71,11 @@ def test_host_validation_errors(call):
     assert call(_w(fmt=1, K=520)) == q.LORA_ERR_UNSUPPORTED       # 4-bit needs K % 64
     assert call(_w(fmt=1, absmax=0)) == q.LORA_ERR_INVALID_ARG
     assert call(_w(fmt=1, cb=P + 4)) == q.LORA_ERR_ALIGNMENT
+    for f8 in (2, 3):                                               # 8-bit: K % 16, fp32 row scales
+        assert call(_w(fmt=f8, K=520)) == q.LORA_ERR_UNSUPPORTED
+        assert call(_w(fmt=f8, absmax=0)) == q.LORA_ERR_INVALID_ARG
+        assert call(_w(fmt=f8, absmax=P + 4)) == q.LORA_ERR_ALIGNMENT
+    assert call(_w(fmt=4)) == q.LORA_ERR_INVALID_ARG
     for r in (0, 4, 12, 136, 256):
         assert call(_w(), r=r) == q.LORA_ERR_UNSUPPORTED, r
     assert call(_w(), s=float("nan")) == q.LORA_ERR_INVALID_ARG
@@ -175,3 +180,15 @@ def test_mlp_validation():
         q.LORA_ERR_WORKSPACE
     assert q.mlp_workspace_bytes(4096, D, I, r) > 0
     assert q.mlp_workspace_bytes(4096, D, I, 72) == 0
+
+
+def test_dequant_validation():
+    lib = q.lib()
+    assert lib.lora_dequant(None, P2, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_dequant(ctypes.byref(_w(fmt=2)), 0, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_dequant(ctypes.byref(_w(fmt=3)), P2 + 2, None) == q.LORA_ERR_ALIGNMENT
+    # the output may not overlap the stored codes
+    assert lib.lora_dequant(ctypes.byref(_w(fmt=2, data=P)), P + 256, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_dequant(ctypes.byref(_w(fmt=0, data=P)), P, None) == q.LORA_ERR_INVALID_ARG
+    assert q.workspace_bytes(4096, 4096, 4096, 16, q.LORA_W_INT8) == q.workspace_bytes(4096, 4096, 4096, 16)
+    assert q.workspace_bytes(4096, 4096, 4096, 16, 4) == 0
