@@ -243,6 +243,16 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def make_weight_dev(q, c, d):
+    """LoraWeight over the device-drawn arrays of case c."""
+    if c.fmt == "bf16":
+        return q.LoraWeight(c.N, c.K, d["W"])
+    if c.fmt == "block4":
+        return q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
+    fmt = q.LORA_W_INT8 if c.fmt == "int8" else q.LORA_W_FP8_E4M3
+    return q.LoraWeight(c.N, c.K, d["codes"], d["row_scale"], None, fmt)
+
+
 class LinearSet:
     """The projections of a layer workload with their resident inputs and outputs."""
 
@@ -265,10 +275,7 @@ class LinearSet:
             if "X" in d:
                 x_cache[xkey] = d["X"]
             d["X"] = x_cache[xkey]
-            if c.fmt == "bf16":
-                W = q.LoraWeight(c.N, c.K, d["W"])
-            else:
-                W = q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
+            W = make_weight_dev(q, c, d)
             if c.rows is None:
                 layer = q.LoraLinear(W, d["A"], d["B"], c.alpha)
             else:
@@ -315,12 +322,7 @@ class MlpSet:
         gu = make_case_device(gu_c, dev, rank=rank, want=("X", "W", "A", "B"))
         dn = make_case_device(dn_c, dev, rank=rank, want=("W", "A", "B", "dY"))
 
-        def weight(c, d):
-            if c.fmt == "bf16":
-                return q.LoraWeight(c.N, c.K, d["W"])
-            return q.LoraWeight(c.N, c.K, d["codes"], d["absmax"], d["codebook"])
-
-        self.mlp = q.LoraMLP(weight(gu_c, gu), weight(dn_c, dn), gu["A"], gu["B"], dn["A"], dn["B"], gu_c.alpha)
+        self.mlp = q.LoraMLP(make_weight_dev(q, gu_c, gu), make_weight_dev(q, dn_c, dn), gu["A"], gu["B"], dn["A"], dn["B"], gu_c.alpha)
         self.inputs = {"X": gu["X"], "dZ": dn["dY"], "gu": gu, "dn": dn}
         self.mlp.workspace(self.M)
         bf = torch.bfloat16
@@ -723,6 +725,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-separate", action="store_true", help="skip the unfused comparison of qkv / mlp")
+    ap.add_argument("--weight", default=None, choices=["bf16", "block4", "int8", "fp8"],
+                    help="store every frozen weight of the workload in this format")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -731,6 +735,10 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cases, desc = workload(args.workload)
+    if args.weight:
+        import dataclasses
+        cases = [dataclasses.replace(c, fmt=args.weight) for c in cases]
+        desc = f"{desc}; frozen weights stored as {args.weight}"
     if args.only:
         cases = [c for c in cases if c.name == args.only]
         if not cases:

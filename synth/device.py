@@ -9,7 +9,7 @@ import math
 
 import torch
 
-from .inputs import LoraCase, codebook_levels
+from .inputs import RMS_FP8, RMS_INT8, LoraCase, codebook_levels
 
 _TID = {"X": 1, "W": 2, "A": 3, "B": 4, "dY": 5, "codes": 6, "absmax": 7}
 
@@ -37,6 +37,21 @@ def make_case_device(case: LoraCase, device, rank: int = 0, want=("X", "W", "A",
     if "W" in want:
         if case.fmt == "bf16":
             out["W"] = _normal_bf16((N, K), 1.0 / math.sqrt(K), device, _gen(device, ds, _TID["W"], rank))
+        elif case.fmt in ("int8", "fp8"):
+            g = _gen(device, ds, _TID["codes"], rank)
+            if case.fmt == "int8":
+                out["codes"] = torch.randint(-127, 128, (N, K), generator=g, device=device,
+                                             dtype=torch.int16).to(torch.int8).view(torch.uint8)
+                rms = RMS_INT8
+            else:
+                sign = torch.randint(0, 2, (N, K), generator=g, device=device, dtype=torch.uint8)
+                expo = torch.randint(1, 15, (N, K), generator=g, device=device, dtype=torch.uint8)
+                mant = torch.randint(0, 8, (N, K), generator=g, device=device, dtype=torch.uint8)
+                out["codes"] = (sign << 7) | (expo << 3) | mant
+                rms = RMS_FP8
+            g = _gen(device, ds, _TID["absmax"], rank)
+            u = torch.rand(N, generator=g, device=device, dtype=torch.float32)
+            out["row_scale"] = (0.8 + 0.4 * u) / (rms * math.sqrt(K))
         else:
             g = _gen(device, ds, _TID["codes"], rank)
             out["codes"] = torch.randint(0, 256, (N, K // 2), generator=g, device=device, dtype=torch.uint8)
