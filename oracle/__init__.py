@@ -29,4 +29,6 @@ from .lora_oracle import (  # noqa: F401
     dequant_rowwise8,
     e4m3_nearest,
     quantize_rowwise8,
+    cross_entropy,
+    cross_entropy_rows_bits,
 )

@@ -36,6 +36,8 @@ What it computes (the method is exact, so the oracle is the plain definition):
   "Unsloth vs The Stack v2", quantized fine-tuning paragraph: 8-bit): one int8 or fp8
   e4m3 byte per element and one fp32 scale per weight row; an element dequantizes to
   ``bf16_rn(fp32_rn(value(code) * scale[row]))``.
+* Cross-entropy over a frozen LM head and its gradient in the hidden states, see
+  :func:`cross_entropy`.
 * Merge of the adapter into the weight ("Rev vs unsloth", GGUF export paragraph;
   "Unsloth vs The Stack v2", merge paragraph): ``W' = W + s·B·A``.
 
@@ -421,3 +423,61 @@ def lora_mlp_backward(dZ: np.ndarray, X: np.ndarray, W_gu: np.ndarray, A_gu: np.
     return {"dX": gg["dX"] + gu["dX"], "dA_gu": np.concatenate([gg["dA"], gu["dA"]], axis=0),
             "dB_gu": np.concatenate([gg["dB"], gu["dB"]], axis=0), "dA_d": gd["dA"], "dB_d": gd["dB"],
             "dH": dH, "dG": dG, "dU": dU, "fwd": f}
+
+
+# ----------------------------------------------------------------------------
+# cross-entropy over a frozen LM head
+# ----------------------------------------------------------------------------
+
+
+def cross_entropy(X: np.ndarray, W: np.ndarray, labels: np.ndarray, ignore_index: int, dloss=None):
+    """Cross-entropy of the logits ``z = X·Wᵀ`` ("Unsloth" wiki entry, Theory: chunked
+    cross-entropy; "Unsloth vs PyTorch: The ONLY Video You Need to Understand the
+    Difference", transcript 3:06-3:51), the plain definition on the full logits:
+    ``lse_m = log Σ_v exp(z_mv)`` (evaluated as ``max + log Σ exp(z - max)``),
+    ``loss_m = lse_m - z_{m,y_m}`` and, when ``dloss`` is given,
+    ``dX = (softmax(z) - onehot(y))·diag(dloss)·W``.  Rows whose label is ``ignore_index``
+    have loss 0 and zero gradient.  Returns ``(loss, lse, dX or None)``."""
+    X = np.asarray(X, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    y = np.asarray(labels, dtype=np.int64)
+    z = X @ W.T
+    zmax = z.max(axis=1, keepdims=True)
+    lse = (zmax + np.log(np.sum(np.exp(z - zmax), axis=1, keepdims=True)))[:, 0]
+    keep = y != ignore_index
+    ysafe = np.where(keep, y, 0)
+    loss = np.where(keep, lse - z[np.arange(len(y)), ysafe], 0.0)
+    dX = None
+    if dloss is not None:
+        P = np.exp(z - lse[:, None])
+        P[np.arange(len(y)), ysafe] -= 1.0
+        P *= np.where(keep, np.asarray(dloss, dtype=np.float64), 0.0)[:, None]
+        dX = P @ W
+    return loss, lse, dX
+
+
+def cross_entropy_rows_bits(X_rows_bits: np.ndarray, W_bits: np.ndarray, labels: np.ndarray, ignore_index: int,
+                            dloss=None, chunk: int = 8192):
+    """:func:`cross_entropy` for a few rows against a large bf16 head ``W_bits [V, D]``:
+    the logits of the rows are built in full (fp64), converting the head to fp64
+    ``chunk`` vocabulary rows at a time for the matrix products only."""
+    X = bf16_to_f64(X_rows_bits)
+    V = W_bits.shape[0]
+    z = np.empty((X.shape[0], V))
+    for v0 in range(0, V, chunk):
+        z[:, v0:v0 + chunk] = X @ bf16_to_f64(W_bits[v0:v0 + chunk]).T
+    y = np.asarray(labels, dtype=np.int64)
+    zmax = z.max(axis=1, keepdims=True)
+    lse = (zmax + np.log(np.sum(np.exp(z - zmax), axis=1, keepdims=True)))[:, 0]
+    keep = y != ignore_index
+    ysafe = np.where(keep, y, 0)
+    loss = np.where(keep, lse - z[np.arange(len(y)), ysafe], 0.0)
+    dX = None
+    if dloss is not None:
+        P = np.exp(z - lse[:, None])
+        P[np.arange(len(y)), ysafe] -= 1.0
+        P *= np.where(keep, np.asarray(dloss, dtype=np.float64), 0.0)[:, None]
+        dX = np.zeros((X.shape[0], W_bits.shape[1]))
+        for v0 in range(0, V, chunk):
+            dX += P[:, v0:v0 + chunk] @ bf16_to_f64(W_bits[v0:v0 + chunk])
+    return loss, lse, dX

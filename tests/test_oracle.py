@@ -606,3 +606,66 @@ def test_quantize_rowwise8_round_trip_and_bound(fmt):
         assert np.all(err <= 0.5 * s3[:, None] * (1 + 1e-6))
     else:  # half a spacing of e4m3 at the value's binade, 2^-4 relative, plus the subnormal step
         assert np.all(err <= np.abs(Wr) * 2.0 ** -4 + s3[:, None] * 2.0 ** -10)
+
+
+# ---------------------------------------------------------------- cross-entropy over an LM head
+
+
+def _ce_inputs(rng, M=9, D=12, V=37):
+    X = rng.standard_normal((M, D))
+    W = rng.standard_normal((V, D)) / np.sqrt(D) * 2
+    y = rng.integers(0, V, M)
+    y[[1, min(5, M - 1)]] = -100
+    dloss = rng.random(M) + 0.5
+    return X, W, y, dloss
+
+
+def test_cross_entropy_against_torch():
+    """Loss against torch's cross_entropy (float64, no reduction, ignore_index) and dX
+    against torch's autograd of the dloss-weighted sum of the losses."""
+    rng = np.random.default_rng(51)
+    X, W, y, dloss = _ce_inputs(rng)
+    loss, lse, dX = O.cross_entropy(X, W, y, -100, dloss)
+    tX = torch.tensor(X, requires_grad=True)
+    tl = torch.nn.functional.cross_entropy(tX @ torch.tensor(W).T, torch.tensor(y), ignore_index=-100,
+                                           reduction="none")
+    assert _rel(loss, tl.detach().numpy()) <= 1e-14
+    (tl * torch.tensor(dloss)).sum().backward()
+    assert _rel(dX, tX.grad.numpy()) <= 1e-13
+    assert _rel(lse, torch.logsumexp(torch.tensor(X @ W.T), dim=1).numpy()) <= 1e-15
+    assert np.all(loss[[1, 5]] == 0) and np.all(dX[[1, 5]] == 0)
+
+
+def test_cross_entropy_uniform_logits_and_finite_differences():
+    rng = np.random.default_rng(52)
+    X, W, y, dloss = _ce_inputs(rng)
+    loss, lse, dX = O.cross_entropy(X, np.zeros_like(W), y, -100, dloss)
+    V = W.shape[0]
+    assert np.allclose(lse, np.log(V), rtol=0, atol=1e-15)
+    assert np.allclose(loss[y != -100], np.log(V), rtol=0, atol=1e-15)
+    assert np.all(dX == 0)
+    X, W, y, dloss = _ce_inputs(rng, M=4, D=5, V=7)
+    _, _, dX = O.cross_entropy(X, W, y, -100, dloss)
+    h = 1e-5
+    fd = np.zeros_like(X)
+    for idx in np.ndindex(X.shape):
+        Xp, Xm = X.copy(), X.copy()
+        Xp[idx] += h
+        Xm[idx] -= h
+        fd[idx] = (np.sum(dloss * O.cross_entropy(Xp, W, y, -100)[0]) -
+                   np.sum(dloss * O.cross_entropy(Xm, W, y, -100)[0])) / (2 * h)
+    assert _rel(fd, dX) <= 1e-8
+
+
+def test_cross_entropy_rows_helper_matches_full():
+    rng = np.random.default_rng(53)
+    M, D, V = 6, 16, 1000
+    Xb = bf16_bits_from_f32(rng.standard_normal((M, D)).astype(np.float32))
+    Wb = bf16_bits_from_f32((rng.standard_normal((V, D)) / 4).astype(np.float32))
+    y = rng.integers(0, V, M)
+    y[2] = -1
+    dloss = rng.random(M)
+    full = O.cross_entropy(O.bf16_to_f64(Xb), O.bf16_to_f64(Wb), y, -1, dloss)
+    rows = O.cross_entropy_rows_bits(Xb, Wb, y, -1, dloss, chunk=97)
+    for a, b in zip(full, rows):
+        assert _rel(a, b) <= 1e-13
