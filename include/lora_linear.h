@@ -225,6 +225,40 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
                            void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Cross-entropy over a frozen LM head without the [M, V] logits ("Unsloth" wiki entry,
+ * Theory: chunked cross-entropy never materialises the logits; "Unsloth vs PyTorch: The
+ * ONLY Video You Need to Understand the Difference", transcript 3:06-3:51: the loss
+ * computed slice by slice, each slice thrown away, the slice size picked from the memory
+ * left).  With hidden states X [M, D] (bf16), head W [V, D] (LORA_W_BF16 only,
+ * LORA_ERR_UNSUPPORTED otherwise) and labels y [M] (device int32):
+ *
+ *     z = X·Wᵀ          lse_m = log Σ_v exp(z_mv)          loss_m = lse_m - z_{m,y_m}
+ *     dX = (softmax(z) - onehot(y))·diag(dloss)·W  (row m scaled by dloss_m)
+ *
+ * Rows with y_m == ignore_index have loss 0 and no gradient; a label outside [0, V) that
+ * is not ignore_index gives a NaN loss (its gradient is unspecified).
+ *
+ * lora_ce_fwd writes loss [M] and lse [M] (fp32, device; lse is the backward's input);
+ * it needs lora_ce_workspace_bytes(M, D, V, 0) bytes or more of workspace.
+ * lora_ce_bwd recomputes the logits slice by slice: the slice is the largest multiple
+ * of 256 vocabulary rows whose bf16 dlogits [M, slice] fit in the workspace beside an
+ * fp32 [M, D] running sum of dX, so a larger workspace means fewer, wider slices
+ * (lora_ce_workspace_bytes(M, D, V, slice) gives the size for a chosen slice; fewer
+ * than 256 columns' room is LORA_ERR_WORKSPACE).  dX: bf16 [M, D] (device, out);
+ * dloss: fp32 [M] (device), e.g. 1/(number of rows not ignored) for a mean loss.
+ * W is frozen: there is no dW.  Limits as for the layer: D % 8 == 0, V % 8 == 0.
+ */
+size_t lora_ce_workspace_bytes(int64_t M, int64_t D, int64_t V, int64_t slice);
+
+lora_status_t lora_ce_fwd(const void* X, int64_t M, const lora_weight_t* W, const int32_t* labels,
+                          int32_t ignore_index, float* loss, float* lse,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+lora_status_t lora_ce_bwd(const void* X, int64_t M, const lora_weight_t* W, const int32_t* labels,
+                          int32_t ignore_index, const float* lse, const float* dloss, void* dX,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Standalone dequantization of a weight of any format to bf16 [N,K] (device, out),
  * element by element as defined for lora_weight_t (bit-exact; a bf16 weight is copied).
  * W_out must not overlap the weight's arrays.

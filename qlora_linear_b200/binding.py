@@ -37,6 +37,7 @@ EXPORTED = (
     "lora_testing_bounded_wait", "lora_timing_enable", "lora_timing_read", "lora_launch_count",
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
     "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
+    "lora_ce_workspace_bytes", "lora_ce_fwd", "lora_ce_bwd",
 )
 
 LORA_MAX_SEGMENTS = 8
@@ -107,6 +108,12 @@ def _load() -> ctypes.CDLL:
     lib.dequant_blockwise4.restype = i32
     lib.lora_dequant.argtypes = [W, vp, vp]
     lib.lora_dequant.restype = i32
+    lib.lora_ce_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.lora_ce_workspace_bytes.restype = sz
+    lib.lora_ce_fwd.argtypes = [vp, i64, W, vp, i32, vp, vp, vp, sz, vp]
+    lib.lora_ce_fwd.restype = i32
+    lib.lora_ce_bwd.argtypes = [vp, i64, W, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.lora_ce_bwd.restype = i32
     lib.lora_merge.argtypes = [W, vp, vp, i32, f32, vp, vp]
     lib.lora_merge.restype = i32
     lib.lora_device_status.argtypes = [vp, vp]
@@ -343,3 +350,25 @@ def lora_mlp_bwd(dZ, X, GU, H, XA_gate_up, XA_down, M: int, mlp: lora_mlp_t, r: 
                              ctypes.byref(mlp), int(r), float(s), _ptr(dX), _ptr(dA_gate_up), _ptr(dB_gate_up),
                              _ptr(dA_down), _ptr(dB_down), _ptr(workspace), int(nb), _stream(stream)),
            "lora_mlp_bwd")
+
+
+def ce_workspace_bytes(M: int, D: int, V: int, slice_: int = 0) -> int:
+    return int(_lib.lora_ce_workspace_bytes(int(M), int(D), int(V), int(slice_)))
+
+
+def lora_ce_fwd(X, M: int, W: LoraWeight, labels, ignore_index: int, loss, lse, workspace, ws_bytes=None,
+                stream=None) -> None:
+    """Per-row cross-entropy of X·Wᵀ against labels, without the logits (see lora_linear.h)."""
+    w = W.c_struct()
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_ce_fwd(_ptr(X), int(M), ctypes.byref(w), _ptr(labels), int(ignore_index), _ptr(loss),
+                            _ptr(lse), _ptr(workspace), int(nb), _stream(stream)), "lora_ce_fwd")
+
+
+def lora_ce_bwd(X, M: int, W: LoraWeight, labels, ignore_index: int, lse, dloss, dX, workspace, ws_bytes=None,
+                stream=None) -> None:
+    """Gradient of Σ dloss·loss in X, vocabulary slice by slice (slice size from the workspace)."""
+    w = W.c_struct()
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_ce_bwd(_ptr(X), int(M), ctypes.byref(w), _ptr(labels), int(ignore_index), _ptr(lse),
+                            _ptr(dloss), _ptr(dX), _ptr(workspace), int(nb), _stream(stream)), "lora_ce_bwd")

@@ -146,6 +146,26 @@ __global__ void __launch_bounds__(MG_THREADS)
   }
 }
 
+// Cross-entropy: one thread per row combines the per-tile (max, Σ exp(z - max)) partials
+// in tile order: lse = m + log Σ_t s_t·exp(m_t - m) with m = max_t m_t, and
+// loss = lse - z_label (0 for an ignored row).
+__global__ void ce_finalize_kernel(const float2* __restrict__ part, int ntiles, int M,
+                                   const float* __restrict__ label_logit, const int32_t* __restrict__ labels,
+                                   int ignore_index, float* __restrict__ loss, float* __restrict__ lse) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= M) return;
+  float m = -INFINITY;
+  for (int t = 0; t < ntiles; ++t) m = fmaxf(m, part[static_cast<size_t>(t) * M + row].x);
+  float sum = 0.0f;
+  for (int t = 0; t < ntiles; ++t) {
+    const float2 q = part[static_cast<size_t>(t) * M + row];
+    if (q.x != -INFINITY) sum += q.y * expf(q.x - m);
+  }
+  const float l = m + logf(sum);
+  lse[row] = l;
+  loss[row] = labels[row] == ignore_index ? 0.0f : l - label_logit[row];
+}
+
 // Test hook: waits on an mbarrier that nothing arrives on, with the library's bounded
 // wait, so the host can check that an expired wait ends the kernel and sets the status.
 __global__ void bounded_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {

@@ -54,6 +54,17 @@ struct PairParams {
   __nv_bfloat16* aux;  // [M, ld_aux]: gate pre-activations, up pre-activations aux_off columns on
   int ld_aux;
   int aux_off;
+  // Cross-entropy over an LM head (logits = the GEMM's output columns, vocabulary index
+  // v0 + column).
+  const int32_t* labels;   // [M]
+  int ignore_index;
+  int v0;
+  float* lse_part;         // EPI_CE_LSE: [num_n][M][2] (max, sum of exp(z - max)) per 256-column tile
+  float* label_logit;      // EPI_CE_LSE: [M], written by the tile holding the row's label
+  const float* lse;        // EPI_CE_DLOGITS: [M]
+  const float* dloss;      // EPI_CE_DLOGITS: [M] upstream gradient of each row's loss
+  float* acc32;            // EPI_ACC_F32: [M, Nout] fp32 running sum
+  int acc_mode;            // EPI_ACC_F32: bit 0 add the running sum, bit 1 write bf16 to out instead
   __nv_bfloat16* out;  // [M, Nout] row-major
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
@@ -99,6 +110,10 @@ enum : int {
                        // output columns: aux <- g, u; out <- silu(g)·u
   EPI_SWIGLU_BWD = 2,  // accumulator = dH; aux holds g, u and is overwritten in place with
                        // dG = dH·u·silu'(g), dU = dH·silu(g); out is not written
+  EPI_CE_LSE = 3,      // accumulator = logits: per row and tile (max, Σ exp(z - max)) and the
+                       // label's logit; no logits are written
+  EPI_CE_DLOGITS = 4,  // accumulator = logits: out <- dloss·(exp(z - lse) - [label == column])
+  EPI_ACC_F32 = 5,     // out/acc32 <- accumulator (+ acc32), see acc_mode
 };
 
 template <int EPI>
@@ -460,6 +475,112 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
                 *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(og[0], og[1], og[2], og[3]);
                 *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
                 *reinterpret_cast<uint4*>(hrow + col0 + q * 8) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+              }
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_CE_LSE) {
+        float m = -INFINITY, sum = 0.0f;
+        const int y = row < p.M ? p.labels[row] : p.ignore_index;
+        const int ylocal = (y == p.ignore_index) ? -1 : y - p.v0 - nb * C::BN;  // column in this tile
+#pragma unroll 1
+        for (int c = 0; c < C::BN / 32; ++c) {
+          const int col0 = nb * C::BN + c * 32;
+          if (col0 >= p.Nout) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          const int nv = min(32, p.Nout - col0);
+          float cm = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nv) cm = fmaxf(cm, __uint_as_float(v[j]));
+          const float nm = fmaxf(m, cm);
+          float cs = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nv) cs += __expf(__uint_as_float(v[j]) - nm);
+          sum = (m == -INFINITY ? 0.0f : sum * __expf(m - nm)) + cs;
+          m = nm;
+          if (ylocal >= c * 32 && ylocal < c * 32 + nv) {
+            float z = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j == ylocal - c * 32) z = __uint_as_float(v[j]);
+            p.label_logit[row] = z;
+          }
+        }
+        if (row < p.M) {
+          float2* part = reinterpret_cast<float2*>(p.lse_part) + static_cast<size_t>(nb) * p.M + row;
+          *part = make_float2(m, sum);
+        }
+      } else if constexpr (EPI == EPI_CE_DLOGITS) {
+        __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
+        int ylocal = -1;
+        float l = 0.0f, g = 0.0f;
+        if (row < p.M) {
+          const int y = p.labels[row];
+          if (y != p.ignore_index) {
+            ylocal = y - p.v0 - nb * C::BN;
+            l = p.lse[row];
+            g = p.dloss[row];
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < C::BN / 32; ++c) {
+          const int col0 = nb * C::BN + c * 32;
+          if (col0 >= p.Nout) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (row < p.M) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col0 + q * 8 < p.Nout) {
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int j0 = q * 8 + 2 * e;
+                  const float d0 = g * (__expf(__uint_as_float(v[j0]) - l) - (c * 32 + j0 == ylocal ? 1.0f : 0.0f));
+                  const float d1 =
+                      g * (__expf(__uint_as_float(v[j0 + 1]) - l) - (c * 32 + j0 + 1 == ylocal ? 1.0f : 0.0f));
+                  o[e] = pack_bf16x2(d0, d1);
+                }
+                *reinterpret_cast<uint4*>(orow + col0 + q * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_ACC_F32) {
+        float* arow = p.acc32 + static_cast<size_t>(row) * p.Nout;
+        __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
+#pragma unroll 1
+        for (int c = 0; c < C::BN / 32; ++c) {
+          const int col0 = nb * C::BN + c * 32;
+          if (col0 >= p.Nout) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (row < p.M) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col0 + q * 8 < p.Nout) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[q * 8 + e]);
+                if (p.acc_mode & 1) {
+                  const float4 a0 = *reinterpret_cast<const float4*>(arow + col0 + q * 8);
+                  const float4 a1 = *reinterpret_cast<const float4*>(arow + col0 + q * 8 + 4);
+                  f[0] += a0.x; f[1] += a0.y; f[2] += a0.z; f[3] += a0.w;
+                  f[4] += a1.x; f[5] += a1.y; f[6] += a1.z; f[7] += a1.w;
+                }
+                if (p.acc_mode & 2) {
+                  *reinterpret_cast<uint4*>(orow + col0 + q * 8) = make_uint4(
+                      pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                } else {
+                  *reinterpret_cast<float4*>(arow + col0 + q * 8) = make_float4(f[0], f[1], f[2], f[3]);
+                  *reinterpret_cast<float4*>(arow + col0 + q * 8 + 4) = make_float4(f[4], f[5], f[6], f[7]);
+                }
               }
             }
           }

@@ -152,6 +152,9 @@ lora_status_t dev_info(DevInfo** out) {
     SET_GEMM(WF_INT8)
     SET_GEMM(WF_FP8)
 #undef SET_GEMM
+    SET_SMEM((lora_gemm_pair_kernel<false, WF_BF16, EPI_CE_LSE>), (PairCfg<false, WF_BF16>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, WF_BF16, EPI_CE_DLOGITS>), (PairCfg<false, WF_BF16>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, WF_BF16, EPI_ACC_F32>), (PairCfg<true, WF_BF16>::SMEM_BYTES));
     SET_SMEM((rowproj_kernel<16, false>), (rowproj_smem_bytes<16, false>()));
     SET_SMEM((rowproj_kernel<32, false>), (rowproj_smem_bytes<32, false>()));
     SET_SMEM((rowproj_kernel<64, false>), (rowproj_smem_bytes<64, false>()));
@@ -344,6 +347,11 @@ template <bool B_MN, int EPI>
 lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const CUtensorMap& e, const CUtensorMap& f,
                             const PairParams& p, int sms, cudaStream_t st) {
   CUtensorMap b;
+  if constexpr (EPI == EPI_CE_LSE || EPI == EPI_CE_DLOGITS || EPI == EPI_ACC_F32) {
+    // the cross-entropy head is bf16 only (checked by the caller)
+    TRY(tmap_bf16(&b, W->data, W->K, W->N, kBoxX, kBoxY));
+    return launch_gemm<B_MN, WF_BF16, EPI>(a, b, e, f, p, sms, st);
+  } else {
   switch (W->fmt) {
     case LORA_W_BF16:
       TRY(tmap_bf16(&b, W->data, W->K, W->N, kBoxX, kBoxY));
@@ -357,6 +365,7 @@ lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const 
     default:
       TRY(tmap_u8(&b, W->data, W->K, W->N, kBoxX, kBoxY8));
       return launch_gemm<B_MN, WF_FP8, EPI>(a, b, e, f, p, sms, st);
+  }
   }
 }
 
@@ -685,6 +694,41 @@ lora_status_t mlp_ws_check(long long M, const lora_mlp_t* m, int r, void* worksp
   return LORA_OK;
 }
 
+// ---------------------------------------------------------------- cross-entropy over an LM head
+// Workspace: status head, then for the forward the per-tile partials [ceil(V/256)][M][2]
+// and the label logits [M]; for the backward (the same bytes, reused) an fp32 dX running
+// sum [M, D] and one bf16 slice of dlogits [M, Vc].
+struct CeLayout {
+  size_t part_off, zy_off, fwd_total, acc_off, dlog_off, bwd_fixed;
+};
+CeLayout ce_layout(long long M, long long D, long long V) {
+  CeLayout c;
+  c.part_off = kStatusBytes;
+  c.zy_off = c.part_off + align256(static_cast<size_t>(cdiv(V, 256)) * M * 8);
+  c.fwd_total = c.zy_off + align256(static_cast<size_t>(M) * 4);
+  c.acc_off = kStatusBytes;
+  c.dlog_off = c.acc_off + align256(static_cast<size_t>(M) * D * 4);
+  c.bwd_fixed = c.dlog_off;
+  return c;
+}
+
+lora_status_t ce_check(const void* X, long long M, const lora_weight_t* W, const int32_t* labels) {
+  TRY(check_weight(W));
+  if (W->fmt != LORA_W_BF16) return LORA_ERR_UNSUPPORTED;
+  if (M < 0 || M > (1LL << 31) - 256) return LORA_ERR_INVALID_ARG;
+  if (W->N > (1LL << 31) - 256) return LORA_ERR_UNSUPPORTED;
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(X));
+  TRY(check_ptr(labels));
+  return LORA_OK;
+}
+
+PairParams ce_params(long long M, long long Nout, long long Kred, void* out, uint32_t* status,
+                     const lora_weight_t* W) {
+  PairParams p = gemm_params(M, Nout, Kred, 0, out, status, W);
+  return p;
+}
+
 size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K, int32_t r, int32_t nseg, int32_t fmt) {
   if (M < 0 || N <= 0 || K <= 0 || r < 8 || r > 128 || r % 8) return 0;
   if (nseg < 1 || nseg > LORA_MAX_SEGMENTS || nseg * r > 128) return 0;
@@ -809,6 +853,103 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
   return mlp_backward_core(dZ, X, GU, H, XA_gate_up, XA_down, M, mlp, r, s, dX, dA_gate_up, dB_gate_up, dA_down,
                            dB_down, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
                            reinterpret_cast<float*>(ws + wl.part_off), reinterpret_cast<uint32_t*>(ws), st);
+}
+
+size_t lora_ce_workspace_bytes(int64_t M, int64_t D, int64_t V, int64_t chunk) {
+  if (M < 0 || D <= 0 || V <= 0 || chunk < 0) return 0;
+  if (M > (1LL << 31) - 256 || D > (1LL << 30) || V > (1LL << 31) - 256) return 0;
+  const CeLayout c = ce_layout(M, D, V);
+  long long vc = chunk == 0 ? V : chunk;
+  vc = (vc + 255) / 256 * 256;
+  const size_t bwd = c.bwd_fixed + align256(static_cast<size_t>(M) * vc * 2);
+  return c.fwd_total > bwd ? c.fwd_total : bwd;
+}
+
+lora_status_t lora_ce_fwd(const void* X, int64_t M, const lora_weight_t* W, const int32_t* labels,
+                          int32_t ignore_index, float* loss, float* lse, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  TRY(ce_check(X, M, W, labels));
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(loss));
+  TRY(check_ptr(lse));
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  const long long V = W->N, D = W->K;
+  const CeLayout c = ce_layout(M, D, V);
+  if (ws_bytes < c.fwd_total) return LORA_ERR_WORKSPACE;
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* zy = reinterpret_cast<float*>(ws + c.zy_off);
+  // a label outside [0, V) finds no tile: its logit stays NaN and so does its loss
+  if (cudaMemsetAsync(zy, 0xFF, static_cast<size_t>(M) * 4, st) != cudaSuccess) return LORA_ERR_CUDA;
+  CUtensorMap ta;
+  TRY(tmap_bf16(&ta, X, D, M, kBoxX, kBoxY));
+  PairParams p = ce_params(M, V, D, nullptr, reinterpret_cast<uint32_t*>(ws), W);
+  p.labels = labels;
+  p.ignore_index = ignore_index;
+  p.lse_part = reinterpret_cast<float*>(ws + c.part_off);
+  p.label_logit = zy;
+  TRY((launch_gemm_w<false, EPI_CE_LSE>(W, ta, ta, ta, p, dev->sms, st)));
+  ce_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(reinterpret_cast<const float2*>(ws + c.part_off),
+                                                   cdiv(V, 256), static_cast<int>(M), zy, labels, ignore_index, loss,
+                                                   lse);
+  count_launch();
+  return last_launch();
+}
+
+lora_status_t lora_ce_bwd(const void* X, int64_t M, const lora_weight_t* W, const int32_t* labels,
+                          int32_t ignore_index, const float* lse, const float* dloss, void* dX, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  TRY(ce_check(X, M, W, labels));
+  if (M == 0) return LORA_OK;
+  TRY(check_ptr(lse));
+  TRY(check_ptr(dloss));
+  TRY(check_ptr(dX));
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  const long long V = W->N, D = W->K;
+  const CeLayout c = ce_layout(M, D, V);
+  // the vocabulary slice: as many 256-column tiles of dlogits as the workspace holds
+  if (ws_bytes < c.bwd_fixed) return LORA_ERR_WORKSPACE;
+  long long vc = static_cast<long long>((ws_bytes - c.bwd_fixed) / (static_cast<size_t>(M) * 2)) / 256 * 256;
+  if (vc < 256) return LORA_ERR_WORKSPACE;
+  if (vc > V) vc = V;
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* acc = reinterpret_cast<float*>(ws + c.acc_off);
+  auto* dlog = reinterpret_cast<__nv_bfloat16*>(ws + c.dlog_off);
+  CUtensorMap tx;
+  TRY(tmap_bf16(&tx, X, D, M, kBoxX, kBoxY));
+  const int nslices = static_cast<int>((V + vc - 1) / vc);
+  for (int i = 0; i < nslices; ++i) {
+    const long long v0 = i * vc, w = (V - v0 < vc) ? V - v0 : vc;
+    lora_weight_t Wc = *W;  // rows [v0, v0 + w) of the head
+    Wc.N = w;
+    Wc.data = static_cast<const uint8_t*>(W->data) + static_cast<size_t>(v0) * D * 2;
+    // dlogits of the slice
+    PairParams p = ce_params(M, w, D, dlog, status, &Wc);
+    p.labels = labels;
+    p.ignore_index = ignore_index;
+    p.v0 = static_cast<int>(v0);
+    p.lse = lse;
+    p.dloss = dloss;
+    TRY((launch_gemm_w<false, EPI_CE_DLOGITS>(&Wc, tx, tx, tx, p, dev->sms, st)));
+    // dX (+)= dlogits_slice · W_slice, summed over slices in fp32
+    CUtensorMap ta;
+    TRY(tmap_bf16(&ta, dlog, w, M, kBoxX, kBoxY));
+    PairParams q = ce_params(M, D, w, dX, status, &Wc);
+    q.acc32 = acc;
+    q.acc_mode = (i > 0 ? 1 : 0) | (i == nslices - 1 ? 2 : 0);
+    TRY((launch_gemm_w<true, EPI_ACC_F32>(&Wc, ta, ta, ta, q, dev->sms, st)));
+  }
+  return LORA_OK;
 }
 
 lora_status_t dequant_blockwise4(const lora_weight_t* Wq, void* W_out, void* stream) {

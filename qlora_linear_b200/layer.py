@@ -167,3 +167,38 @@ class LoraMLP:
         _b.lora_mlp_bwd(dZ, X, saved["GU"], saved["H"], saved["XA_gate_up"], saved["XA_down"], M, self.c_struct(),
                         self.r, self.s, dX, dAgu, dBgu, dAd, dBd, self.workspace(M), stream=stream)
         return out
+
+
+class LoraCrossEntropy:
+    """Cross-entropy over a frozen bf16 LM head ``W [V, D]`` (a :class:`LoraWeight`), per
+    row, without the ``[M, V]`` logits.  ``slice_`` (vocabulary rows per backward slice,
+    0 = all) sizes the workspace; the backward takes the widest slice the workspace holds."""
+
+    def __init__(self, W: "_b.LoraWeight", ignore_index: int = -100, slice_: int = 8192):
+        self.W, self.ignore_index, self.slice = W, int(ignore_index), int(slice_)
+        self._ws = None
+        self._ws_M = -1
+
+    def workspace(self, M: int) -> torch.Tensor:
+        if self._ws is None or self._ws_M < M:
+            n = _b.ce_workspace_bytes(M, self.W.K, self.W.N, self.slice)
+            if n == 0:
+                raise _b.LoraError(_b.LORA_ERR_UNSUPPORTED, "ce_workspace_bytes")
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.W.data.device)
+            self._ws_M = M
+        return self._ws
+
+    def forward(self, X: torch.Tensor, labels: torch.Tensor, stream=None):
+        M = X.shape[0]
+        loss = torch.empty(M, dtype=torch.float32, device=X.device)
+        lse = torch.empty(M, dtype=torch.float32, device=X.device)
+        _b.lora_ce_fwd(X, M, self.W, labels, self.ignore_index, loss, lse, self.workspace(M), stream=stream)
+        return loss, lse
+
+    def backward(self, X: torch.Tensor, labels: torch.Tensor, lse: torch.Tensor, dloss: torch.Tensor, dX=None,
+                 stream=None):
+        M = X.shape[0]
+        if dX is None:
+            dX = torch.empty((M, self.W.K), dtype=torch.bfloat16, device=X.device)
+        _b.lora_ce_bwd(X, M, self.W, labels, self.ignore_index, lse, dloss, dX, self.workspace(M), stream=stream)
+        return dX

@@ -13,5 +13,7 @@ from .inputs import (  # noqa: F401
     make_grouped_case,
     MlpCase,
     make_mlp_case,
+    CeCase,
+    make_ce_case,
     config_cases,
 )

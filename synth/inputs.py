@@ -264,3 +264,30 @@ def make_mlp_case(case: MlpCase) -> dict:
     dn = make_case(case.down_case(), want=("W", "A", "B", "dY"))
     return {"case": case, "X": gu["X"], "A_gu": gu["A"], "B_gu": gu["B"], "A_d": dn["A"], "B_d": dn["B"],
             "dZ": dn["dY"], "gate_up": gu, "down": dn}
+
+
+@dataclasses.dataclass(frozen=True)
+class CeCase:
+    """Cross-entropy over an LM head: M rows of hidden states of width D, vocabulary V."""
+
+    name: str
+    M: int
+    D: int
+    V: int
+    seed: int
+    ignore_index: int = -100
+    ignore_frac: float = 0.05
+
+
+def make_ce_case(case: CeCase) -> dict:
+    """X ~ N(0, 1) [M, D] and head W ~ N(0, 4/D) [V, D] in bf16 (logits of std about 2);
+    labels uniform on [0, V) with a fraction set to ignore_index; dloss uniform on
+    [0.5, 1.5) as fp32."""
+    M, D, V = case.M, case.D, case.V
+    X = _fill((M, D), case.seed, _TID["X"], _normal_bf16(1.0))
+    W = _fill((V, D), case.seed, _TID["W"], _normal_bf16(2.0 / np.sqrt(D)))
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([case.seed, 8])))
+    labels = g.integers(0, V, M).astype(np.int32)
+    labels[g.random(M) < case.ignore_frac] = case.ignore_index
+    dloss = (0.5 + g.random(M)).astype(np.float32)
+    return {"case": case, "X": X, "W": W, "labels": labels, "dloss": dloss}

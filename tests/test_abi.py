@@ -192,3 +192,28 @@ def test_dequant_validation():
     assert lib.lora_dequant(ctypes.byref(_w(fmt=0, data=P)), P, None) == q.LORA_ERR_INVALID_ARG
     assert q.workspace_bytes(4096, 4096, 4096, 16, q.LORA_W_INT8) == q.workspace_bytes(4096, 4096, 4096, 16)
     assert q.workspace_bytes(4096, 4096, 4096, 16, 4) == 0
+
+
+def test_ce_validation():
+    lib = q.lib()
+    W = _w(N=1000, K=256)
+
+    def fwd(W=W, M=64, X=P, labels=P, loss=P, lse=P, ws=P2, nb=1 << 30):
+        return lib.lora_ce_fwd(X, M, ctypes.byref(W) if W is not None else None, labels, -100, loss, lse, ws, nb, None)
+
+    def bwd(W=W, M=64, nb=1 << 30, dX=P):
+        return lib.lora_ce_bwd(P, M, ctypes.byref(W), P, -100, P, P, dX, P2, nb, None)
+
+    assert fwd(W=None) == q.LORA_ERR_INVALID_ARG
+    assert fwd(W=_w(fmt=1, N=1000, K=256)) == q.LORA_ERR_UNSUPPORTED   # the head is bf16
+    assert fwd(labels=0) == q.LORA_ERR_INVALID_ARG
+    assert fwd(loss=P + 4) == q.LORA_ERR_ALIGNMENT
+    assert fwd(M=-1) == q.LORA_ERR_INVALID_ARG
+    assert fwd(M=0, X=0, labels=0) == q.LORA_OK
+    assert fwd(nb=100) == q.LORA_ERR_WORKSPACE
+    assert bwd(dX=0) == q.LORA_ERR_INVALID_ARG
+    # room for fewer than 256 vocabulary columns of dlogits beside the fp32 dX sum
+    fixed = q.ce_workspace_bytes(64, 256, 1000, 256) - 64 * 256 * 2
+    assert bwd(nb=fixed + 64 * 255 * 2) == q.LORA_ERR_WORKSPACE
+    assert q.ce_workspace_bytes(64, 256, 1000, 512) > q.ce_workspace_bytes(64, 256, 1000, 256)
+    assert q.ce_workspace_bytes(64, 256, 1000, 0) == q.ce_workspace_bytes(64, 256, 1000, 1024)
