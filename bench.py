@@ -4,7 +4,7 @@ One step = forward and backward of every projection of the workload (default: th
 Llama-8B MLP projections gate, up and down at M = 16384 tokens, r = 16, bf16 weight),
 with inputs resident in device memory.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|qkv|mlp] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|qkv|mlp|ce] [--impl ours|reference]
 
 Multi-GPU (one process per GPU under torch.distributed.run): data parallel over tokens,
 every rank runs the full per-rank workload (weak scaling) and the adapter gradients dA
@@ -35,6 +35,10 @@ def workload(name: str):
     if name == "mlp":
         blk = MlpCase("mlp_llama8b", 16384, 4096, 14336, 16, 32.0, "bf16", 7000)
         cases = [blk.gate_up_case(), blk.down_case()]
+    elif name == "ce":
+        # the LM head as a projection: M tokens, K = D, N = V (no adapter; r only sizes nothing)
+        from synth import LoraCase
+        cases = [LoraCase("ce_llama3_head", 16384, 128256, 4096, 8, 16.0, "bf16", 7100)]
     else:
         cases = CONFIGS[name]
     desc = {
@@ -43,12 +47,20 @@ def workload(name: str):
               "M=16384, r=16, alpha=32, bf16 weight",
         "c3": "QLoRA 4-bit blockwise weight K=4096 N=14336 (16-level codebook, fp16 absmax per 64), "
               "M=8192, r=16, alpha=32",
+        "ce": "cross-entropy over the Llama-3 LM head (V=128256, D=4096), M=16384 tokens, backward in "
+              "16384-column vocabulary slices, bf16 head, no [M, V] logits",
         "mlp": "Llama-8B feed-forward block (D=4096, I=14336) with LoRA on gate, up and down and SwiGLU, "
                "M=16384, r=16, alpha=32, bf16 weights",
         "qkv": "Llama-8B attention q/k/v as one grouped layer (q 4096, k 1024, v 1024 rows, K=4096), "
                "M=8192, r=16 per projection, alpha=32, bf16 weight",
     }[name]
     return cases, desc
+
+
+def ce_flops(c) -> float:
+    """Cross-entropy step: logits in the forward and again in the backward, and dX:
+    three M×V×D products, 6MVD."""
+    return 6.0 * c.M * c.N * c.K
 
 
 def case_flops(c) -> float:
@@ -158,12 +170,19 @@ def gpu_uuid(dev) -> str:
 
 
 # ---------------------------------------------------------------------------- oracle leg
-def oracle_sample(cases, tokens: int, mlp: bool = False):
+def oracle_sample(cases, tokens: int, mlp: bool = False, ce: bool = False):
     """Runs the fp64 oracle (as it stands) on the first `tokens` tokens of every
-    projection (of the feed-forward block when `mlp`); returns (seconds, algorithmic
-    flops of the sample)."""
+    projection (of the feed-forward block when `mlp`, of the LM-head cross-entropy when
+    `ce`); returns (seconds, algorithmic flops of the sample)."""
     import oracle as O
     from synth import make_case
+    if ce:
+        from synth import CeCase, make_ce_case
+        c = cases[0].with_M(tokens)
+        inp = make_ce_case(CeCase(c.name, tokens, c.K, c.N, c.seed))
+        t0 = time.perf_counter()
+        O.cross_entropy_rows_bits(inp["X"], inp["W"], inp["labels"], -100, inp["dloss"])
+        return time.perf_counter() - t0, ce_flops(c)
     if mlp:
         gu_c, dn_c = (c.with_M(tokens) for c in cases)
         gu = make_case(gu_c, want=("X", "W", "A", "B"))
@@ -201,10 +220,10 @@ def run_reference(args, cases, desc, rank, world):
         return 0
     tokens = args.cpu_tokens
     for _ in range(args.warmup):
-        oracle_sample(cases, tokens, mlp=args.workload == "mlp")
+        oracle_sample(cases, tokens, mlp=args.workload == "mlp", ce=args.workload == "ce")
     times, flops = [], 0.0
     for _ in range(args.steps):
-        t, flops = oracle_sample(cases, tokens, mlp=args.workload == "mlp")
+        t, flops = oracle_sample(cases, tokens, mlp=args.workload == "mlp", ce=args.workload == "ce")
         times.append(t)
     total = sum(times)
     val = args.steps * flops / total / 1e12
@@ -401,6 +420,108 @@ class MlpSet:
                         "gradients read back every step; the frozen weights stay resident"}
 
 
+class CeSet:
+    """The cross-entropy workload: hidden states, head, labels and dloss resident."""
+
+    def __init__(self, cases, dev, rank, world):
+        import torch
+
+        import qlora_linear_b200 as q
+
+        c = cases[0]
+        self.cases, self.world, self.dev = cases, world, dev
+        self.M, self.D, self.V = c.M, c.K, c.N
+        g = torch.Generator(device=dev)
+        g.manual_seed(c.seed * 1_000_003 + rank)
+        self.X = torch.randn((self.M, self.D), generator=g, device=dev).to(torch.bfloat16)
+        self.Wt = (torch.randn((self.V, self.D), generator=g, device=dev) * (2.0 / self.D ** 0.5)).to(torch.bfloat16)
+        self.labels = torch.randint(0, self.V, (self.M,), generator=g, device=dev, dtype=torch.int32)
+        self.labels[torch.rand(self.M, generator=g, device=dev) < 0.05] = -100
+        self.dloss = torch.full((self.M,), 1.0 / self.M, device=dev)
+        self.ce = q.LoraCrossEntropy(q.LoraWeight(self.V, self.D, self.Wt), -100, 16384)
+        self.ce.workspace(self.M)
+        self.dX = torch.empty((self.M, self.D), dtype=torch.bfloat16, device=dev)
+        self.layers, self.data = [self.ce], []
+
+    def step(self, inputs=None):
+        X = self.X if inputs is None else inputs["X"]
+        loss, lse = self.ce.forward(X, self.labels)
+        self.loss = loss
+        self.ce.backward(X, self.labels, lse, self.dloss, dX=self.dX)
+
+    def statuses(self):
+        import qlora_linear_b200 as q
+        return [q.lora_device_status(self.ce.workspace(self.M))]
+
+    def e2e(self, args, step):
+        """X in from pinned host memory and the per-row losses and dX out, every step."""
+        import torch
+
+        stream = torch.cuda.current_stream()
+        hX = self.X.cpu().pin_memory()
+        dXin = torch.empty_like(self.X)
+        hloss = torch.empty(self.M, dtype=torch.float32).pin_memory()
+        hdX = torch.empty(self.dX.shape, dtype=self.dX.dtype).pin_memory()
+
+        def e2e_step():
+            dXin.copy_(hX, non_blocking=True)
+            step(inputs={"X": dXin})
+            hloss.copy_(self.loss, non_blocking=True)
+            hdX.copy_(self.dX, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        steps = max(3, args.steps // 2)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        return {"value": self.world * ce_flops(self.cases[0]) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": hX.numel() * 2, "d2h_bytes_per_step": hloss.numel() * 4 + hdX.numel() * 2,
+                "ms_per_step": ms, "steps": steps,
+                "note": "X copied from pinned host memory and the per-row losses and dX read back every step; "
+                        "head, labels and dloss resident"}
+
+
+def time_separate_ce(args, cases, ws, dev):
+    """The same loss the plain way: full [M, V] logits by torch.matmul, torch's
+    cross_entropy in fp32 and autograd for dX; reports its time and peak memory."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    X = ws.X.clone().requires_grad_(True)
+    labels = ws.labels.long()
+
+    def step():
+        X.grad = None
+        logits = X @ ws.Wt.T
+        loss = torch.nn.functional.cross_entropy(logits.float(), labels, ignore_index=-100, reduction="none")
+        (loss * ws.dloss).sum().backward()
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    steps = max(3, args.steps // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    peak = torch.cuda.max_memory_allocated(dev) - base
+    return {"ms_per_step": ms, "value": ce_flops(cases[0]) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "extra_peak_bytes": int(peak),
+            "note": "full logits (torch.matmul, bf16), fp32 cross_entropy and autograd; extra_peak_bytes is the "
+                    "memory above the resident inputs"}
+
+
 def time_separate_mlp(args, cases, ws, dev):
     """The same block unfused: gate, up and down as three separate layers, SwiGLU and its
     derivative as torch elementwise ops between them (what a model without the fused
@@ -476,6 +597,8 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     # ---- inputs resident in HBM (drawn on the device)
     if args.workload == "mlp":
         ws = MlpSet(cases, dev, rank, world)
+    elif args.workload == "ce":
+        ws = CeSet(cases, dev, rank, world)
     else:
         ws = LinearSet(cases, dev, rank, world)
     layers, data, step = ws.layers, ws.data, ws.step
@@ -525,13 +648,14 @@ def run_ours(args, cases, desc, rank, world, local_rank):
         if st != q.LORA_OK:
             raise RuntimeError("device status after timing: " + q.status_string(st))
 
-    flops_step = sum(case_flops(c) for c in cases)
+    ce = args.workload == "ce"
+    flops_step = ce_flops(cases[0]) if ce else sum(case_flops(c) for c in cases)
     tokens_step = cases[0].M
     value = world * flops_step / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
 
     # ---- roofline of the dominant kernel (the tcgen05 GEMM: Y and dX launches)
-    gflops = sum(sum(gemm_flops(c)) for c in cases) * args.steps
+    gflops = (ce_flops(cases[0]) if ce else sum(sum(gemm_flops(c)) for c in cases)) * args.steps
     g_ms = fwd_ms + bwd_ms
     g_launches = fwd_n + bwd_n
     achieved = gflops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
@@ -563,18 +687,21 @@ def run_ours(args, cases, desc, rank, world, local_rank):
         pass
     elif world == 1 and args.workload == "mlp":
         separate = time_separate_mlp(args, cases, ws, dev)
+    elif world == 1 and args.workload == "ce":
+        separate = time_separate_ce(args, cases, ws, dev)
     elif world == 1 and any(c.rows is not None for c in cases):
         separate = time_separate(args, cases, data, dev)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = ws.e2e(args, step) if args.workload == "mlp" else run_e2e(args, cases, layers, data, step, world, dev)
+        e2e = ws.e2e(args, step) if args.workload in ("mlp", "ce") else run_e2e(args, cases, layers, data, step, world,
+                                                                               dev)
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, fl = oracle_sample(cases, args.cpu_tokens, mlp=args.workload == "mlp")
+        t, fl = oracle_sample(cases, args.cpu_tokens, mlp=args.workload == "mlp", ce=args.workload == "ce")
         cpu = {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"first {args.cpu_tokens} tokens of each projection (full K and N), fp64 numpy oracle, "
                          f"{t:.1f} s", "tokens_per_s": args.cpu_tokens / t}
@@ -719,7 +846,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "qkv", "mlp"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "qkv", "mlp", "ce"])
     ap.add_argument("--only", default=None, help="run a single projection of the workload (e.g. c2_gate)")
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
