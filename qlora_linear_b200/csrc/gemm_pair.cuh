@@ -9,29 +9,26 @@
 // The LoRA term is one extra K fill after the main loop — possible because the
 // adapter product is bracketed skinny-first ("Unsloth vs PyTorch: The ONLY Video You
 // Need to Understand the Difference", transcript 1:35-2:00), so the N×K matrix B·A is
-// never formed.  With W4 the frozen weight arrives as packed 4-bit codes ("Rev vs
-// unsloth", fused quantized-LoRA paragraph) and each CTA's dequant warps expand them in
-// shared memory into the bf16 tile the tensor core reads; no dequantized weight ever
-// reaches HBM.
+// never formed.  This kernel takes a bf16 weight (and, for the LM-head cross-entropy,
+// a bf16 head); quantized weights go to lora_gemm_q_kernel (gemm_q.cuh).
 //
 // A cluster of two CTAs computes a 256×256 tile.  Each CTA loads its own 128 rows of A
 // and its own 128 rows of the B tile (no multicast); the even CTA ("leader") issues
 // tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which reads both CTAs' shared memory
 // and accumulates into both CTAs' TMEM (each CTA holds its 128 rows × 256 fp32 columns,
 // double-buffered).  Per CTA this halves the operand bytes per MMA compared with a
-// 128×256 single-CTA tile, and for W4 halves the dequant work per MMA.
+// 128×256 single-CTA tile.
 //
 // Synchronisation.  TMA completions of both CTAs count on the leader's `full` barrier;
 // the leader's MMA commits arrive on both CTAs' `empty` / `tfull` barriers (CTA mask
-// 0b11); both CTAs' epilogue and dequant warps arrive on the leader's `tempty` / `deq`
-// barriers through cluster addresses.  W4 code tiles complete on a CTA-local `cfull`
-// barrier so each CTA's dequant warps can wait locally.  Every wait is bounded.
+// 0b11); both CTAs' epilogue warps arrive on the leader's `tempty` barriers through
+// cluster addresses.  Every wait is bounded.
 //
 // Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
-// warps 2-5 epilogue, warps 6-13 dequant (W4 only).
+// warps 2-5 epilogue.
 #pragma once
 
-#include "ptx.cuh"
+#include "dequant.cuh"
 
 namespace lora {
 
@@ -75,30 +72,20 @@ struct PairParams {
   int Nw, Kw;                // logical weight shape [Nw, Kw]
 };
 
-// Storage format of the frozen weight (the values of lora_wfmt_t).
-enum : int { WF_BF16 = 0, WF_BLOCK4 = 1, WF_INT8 = 2, WF_FP8 = 3 };
-
-template <bool B_MN, int WF>
+template <bool B_MN>
 struct PairCfg {
-  static constexpr bool W4 = WF == WF_BLOCK4;
-  static constexpr bool W8 = WF == WF_INT8 || WF == WF_FP8;
-  static constexpr bool DEQ = W4 || W8;  // the B tile is expanded in shared memory
   static constexpr int BM = 256, BN = 256, BK = 128;  // pair tile, K per pipeline fill
   static constexpr int HM = 128, HN = 128;            // per-CTA halves of A rows / B rows
   static constexpr int STAGES = 3;
   static constexpr int ATOM = 64;                       // 128-byte swizzle atom width (bf16)
   static constexpr int A_BYTES = HM * BK * 2;           // 32 KB (two 64-wide K atoms)
   static constexpr int B_BYTES = HN * BK * 2;           // 32 KB
-  static constexpr int C_BYTES = W4 ? HN * BK / 2 : 0;  // 8 KB of codes
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NUM_EPI_WARPS = 4;
-  static constexpr int NUM_DEQ_WARPS = DEQ ? 8 : 0;  // two per SM sub-partition
-  static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS + NUM_DEQ_WARPS);
+  static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS);
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NUM_BARS = 4 * STAGES + 5;
-  static constexpr int SCALE_RING = 4;  // W4: scale words staged this many code fills ahead (minus one)
-  static constexpr int SCALE_BYTES = W4 ? SCALE_RING * 32 * NUM_DEQ_WARPS * 4 : 0;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SCALE_BYTES + 8 * NUM_BARS + 16;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -142,98 +129,18 @@ __device__ __forceinline__ void pair_tile_coords(int t, int num_m, int num_n, in
   nb = within / gm;
 }
 
-// Expands 8 codes (one 32-bit word) of one 64-element scale block to 8 bf16, using the
-// block's 16 dequantized levels held as byte planes: low bytes of level e in byte e%4
-// of L[e/4], high bytes likewise in H.  Element 2j sits in the low nibble of byte j,
-// so the low 16 bits of `w` select elements 0..3.  Each prmt picks four bytes by
-// 3-bit selectors; the selector's bit 3 (code >= 8) picks between the two halves.
-#ifndef LORA_EXPAND8_DEFINED
-#define LORA_EXPAND8_DEFINED
-__device__ __forceinline__ uint4 expand8(uint32_t w, const uint32_t (&L)[4], const uint32_t (&H)[4]) {
-  uint4 o;
-  {
-    const uint32_t sel = w & 0x7777u;
-    const uint32_t sel2 = ((w >> 1) & 0x4444u) | 0x3210u;
-    const uint32_t lo = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), sel2);
-    const uint32_t hi = prmt(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), sel2);
-    o.x = prmt(lo, hi, 0x5140u);
-    o.y = prmt(lo, hi, 0x7362u);
-  }
-  {
-    const uint32_t w2 = w >> 16;
-    const uint32_t sel = w2 & 0x7777u;
-    const uint32_t sel2 = ((w2 >> 1) & 0x4444u) | 0x3210u;
-    const uint32_t lo = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), sel2);
-    const uint32_t hi = prmt(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), sel2);
-    o.z = prmt(lo, hi, 0x5140u);
-    o.w = prmt(lo, hi, 0x7362u);
-  }
-  return o;
-}
-
-// The 16 levels of one scale block, bf16_rn(fp32_rn(codebook[c] * scale)), as byte
-// planes for expand8().  __fmul_rn keeps the product from being fused with anything.
-__device__ __forceinline__ void block_levels(const float (&cb)[16], float scale, uint32_t (&L)[4], uint32_t (&H)[4]) {
-  uint32_t v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = pack_bf16x2(__fmul_rn(cb[2 * i], scale), __fmul_rn(cb[2 * i + 1], scale));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    L[i] = prmt(v[2 * i], v[2 * i + 1], 0x6420u);
-    H[i] = prmt(v[2 * i], v[2 * i + 1], 0x7531u);
-  }
-}
-#endif
-
-// Eight 8-bit codes (two words, element 4i+j in byte j of word i) to eight bf16
-// bf16_rn(fp32_rn(value(code) * scale)).  int8: value = the signed byte, made exact in
-// fp32 by placing the biased byte in the mantissa of 2^23; fp8: e4m3 decoded exactly
-// through f16 by the hardware conversion.
-template <int WF>
-__device__ __forceinline__ uint4 expand8_w8(uint32_t w0, uint32_t w1, float sc) {
-  float f[8];
-  if constexpr (WF == WF_INT8) {
-    const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;  // byte + 128, unsigned
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      f[j] = __uint_as_float(prmt(u0, 0x4B000000u, 0x7540u | j)) - 8388736.0f;  // 2^23 + 128
-      f[4 + j] = __uint_as_float(prmt(u1, 0x4B000000u, 0x7540u | j)) - 8388736.0f;
-    }
-  } else {
-    const uint32_t hw[4] = {w0 & 0xffffu, w0 >> 16, w1 & 0xffffu, w1 >> 16};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t h2;
-      asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "r"(hw[j]));
-      const __half2 hv = *reinterpret_cast<const __half2*>(&h2);
-      f[2 * j] = __low2float(hv);
-      f[2 * j + 1] = __high2float(hv);
-    }
-  }
-  uint4 o;
-  o.x = pack_bf16x2(__fmul_rn(f[0], sc), __fmul_rn(f[1], sc));
-  o.y = pack_bf16x2(__fmul_rn(f[2], sc), __fmul_rn(f[3], sc));
-  o.z = pack_bf16x2(__fmul_rn(f[4], sc), __fmul_rn(f[5], sc));
-  o.w = pack_bf16x2(__fmul_rn(f[6], sc), __fmul_rn(f[7], sc));
-  return o;
-}
-
-template <bool B_MN, int WF, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::NUM_THREADS, 1)
+template <bool B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_THREADS, 1)
     lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
                           const PairParams p) {
-  using C = PairCfg<B_MN, WF>;
-  constexpr bool W4 = C::W4, W8 = C::W8, DEQ = C::DEQ;
+  using C = PairCfg<B_MN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* scale_ring = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES);  // W4
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::SCALE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
   uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
-  uint64_t* cfull = bars + 2 * C::STAGES;   // both (4-/8-bit): this CTA's code tile landed
-  uint64_t* deq = bars + 3 * C::STAGES;     // leader (4-/8-bit): both CTAs' dequantized tiles written
-  uint64_t* tfull = bars + 4 * C::STAGES;   // both: accumulator ready for the epilogue
+  uint64_t* tfull = bars + 2 * C::STAGES;   // both: accumulator ready for the epilogue
   uint64_t* tempty = tfull + 2;             // leader: both CTAs drained the accumulator
   uint64_t* drain = tempty + 2;             // leader: final commit before TMEM release
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -258,8 +165,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
-      mbar_init(smem_u32(&cfull[s]), 1);
-      mbar_init(smem_u32(&deq[s]), 2 * (C::NUM_DEQ_WARPS > 0 ? C::NUM_DEQ_WARPS : 1));
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
@@ -302,11 +207,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
           const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
-          const uint32_t sC = sB + C::B_BYTES;
           const uint32_t full_l = mapa_shared(smem_u32(&full[stage]), 0);
           if (leader) {
             uint32_t per_cta;
-            if (!ext) per_cta = C::A_BYTES + (DEQ ? 0 : C::B_BYTES);
+            if (!ext) per_cta = C::A_BYTES + C::B_BYTES;
             else per_cta = ext_atoms * (C::A_BYTES / 2) + (B_MN ? C::B_BYTES : ext_atoms * (C::B_BYTES / 2));
             mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * per_cta);
           }
@@ -315,22 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
           if (!ext) {
             tma_load_2d_pair(sA, &tmA, full_l, kb * C::BK, arow);
             tma_load_2d_pair(sA + C::A_BYTES / 2, &tmA, full_l, kb * C::BK + C::ATOM, arow);
-            if (W4) {
-              mbar_arrive_expect_tx(smem_u32(&cfull[stage]), C::C_BYTES);
-              if (!B_MN) tma_load_2d(sC, &tmB, smem_u32(&cfull[stage]), kb * (C::BK / 2), brow);
-              else tma_load_2d(sC, &tmB, smem_u32(&cfull[stage]), brow / 2, kb * C::BK);
-            } else if (W8) {
-              // 8-bit codes, one 32-row × 64-byte box per dequant warp, placed in the upper
-              // half of the 4 KB of the B buffer that warp will write, so each warp reads its
-              // codes and expands them in place with no other warp involved
-              mbar_arrive_expect_tx(smem_u32(&cfull[stage]), C::B_BYTES / 2);
-              for (int w = 0; w < 8; ++w) {
-                const int hh = w >> 2, rq = (w & 3) * 32;
-                const uint32_t dst = sB + hh * (C::B_BYTES / 2) + rq * 128 + 2048;
-                if (!B_MN) tma_load_2d(dst, &tmB, smem_u32(&cfull[stage]), kb * C::BK + hh * C::ATOM, brow + rq);
-                else tma_load_2d(dst, &tmB, smem_u32(&cfull[stage]), brow + hh * C::ATOM, kb * C::BK + rq);
-              }
-            } else if (!B_MN) {
+            if (!B_MN) {
               tma_load_2d_pair(sB, &tmB, full_l, kb * C::BK, brow);
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmB, full_l, kb * C::BK + C::ATOM, brow);
             } else {
@@ -353,7 +242,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
               tma_load_2d_pair(sB, &tmF, full_l, brow, 0);
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmF, full_l, brow + C::ATOM, 0);
             }
-            if (DEQ) mbar_arrive(smem_u32(&cfull[stage]));  // nothing to dequantize in this fill
           }
           ++fills;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -367,7 +255,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
           const int s = static_cast<int>(f % C::STAGES);
           const uint32_t ph = static_cast<uint32_t>((f / C::STAGES) & 1);
           if (leader) mbar_wait(smem_u32(&full[s]), ph, drain_wc);
-          if (DEQ) mbar_wait(smem_u32(&cfull[s]), ph, drain_wc);
         }
       }
     }
@@ -386,7 +273,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < nkb + n_ext; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
-          if (DEQ && !mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
           tc_fence_after();
           const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
@@ -637,138 +523,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN, WF>::N
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-    }
-  } else if constexpr (W4) {
-    // ------------------------------------------------------------ dequant (4-bit, both CTAs)
-    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
-    const int row = dt & 127;  // weight row of this CTA's 128-row half (forward) / of the K fill (backward)
-    const int h = dt >> 7;     // 64-wide atom: K atom (forward) or output chunk (backward)
-    float cb[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
-    const long long kblocks_w = p.Kw / 64;  // scale blocks per weight row
-    const long long nscales = static_cast<long long>(p.Nw) * kblocks_w;
-    // Each thread expands one 64-element scale block per code fill.  The fp16 scales
-    // are staged in a per-thread shared-memory ring with cp.async, SCALE_RING-1 code
-    // fills ahead, so no register ever waits on an outstanding global load.
-    const int my_tiles = ntiles > pair ? (ntiles - pair + npairs - 1) / npairs : 0;
-    const int code_fills = my_tiles * nkb;  // fills of this CTA that carry codes
-    auto stage_scale = [&](int i) {           // issue the copy for code fill i (always commits a group)
-      if (i < code_fills) {
-        const int t = pair + (i / nkb) * npairs, kb = i % nkb;
-        int mb, nb;
-        pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
-        const int brow = pair_brow<EPI>(nb, rank, p);
-        const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
-        const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
-        const uint32_t dst = smem_u32(&scale_ring[(i % C::SCALE_RING) * (32 * C::NUM_DEQ_WARPS) + dt]);
-        if (n < p.Nw && kblk < kblocks_w) {
-          // 4-byte aligned word holding the scale; the half beyond the array end reads as zero
-          const long long idx = n * kblocks_w + kblk;
-          const long long w0 = idx & ~1LL;
-          const uint32_t nbytes = (w0 + 1 < nscales) ? 4u : 2u;
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(p.absmax + w0), "r"(nbytes)
-                       : "memory");
-        } else {
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, 0;" ::"r"(dst), "l"(p.absmax) : "memory");
-        }
-      }
-      cp_async_commit();
-    };
-    auto scale_of = [&](int i) -> float {
-      int kb = i % nkb, t = pair + (i / nkb) * npairs;
-      int mb, nb;
-      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
-      const int brow = pair_brow<EPI>(nb, rank, p);
-      const long long n = !B_MN ? brow + row : static_cast<long long>(kb) * C::BK + row;
-      const long long kblk = !B_MN ? kb * 2 + h : brow / 64 + h;
-      const uint32_t wv = scale_ring[(i % C::SCALE_RING) * (32 * C::NUM_DEQ_WARPS) + dt];
-      const uint16_t hb = ((n * kblocks_w + kblk) & 1) ? static_cast<uint16_t>(wv >> 16) : static_cast<uint16_t>(wv);
-      return __half2float(__ushort_as_half(hb));
-    };
-#pragma unroll 1
-    for (int i = 0; i < C::SCALE_RING - 1; ++i) stage_scale(i);
-    int stage = 0;
-    uint32_t phase = 0;
-    int ci = 0;  // index of the next code fill
-    for (int t = pair; t < ntiles; t += npairs) {
-      bool ok = true;
-      for (int kb = 0; kb < nkb + n_ext; ++kb) {
-        if (kb < nkb) stage_scale(ci + C::SCALE_RING - 1);
-        if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
-        if (kb < nkb) {
-          cp_async_wait<C::SCALE_RING - 1>();  // this fill's scale word has landed
-          const float sc = scale_of(ci);
-          ++ci;
-          uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-          const uint8_t* crow = sB + C::B_BYTES + row * 64 + h * 32;  // 32 code bytes = 64 codes
-          uint32_t L[4], H[4];
-          block_levels(cb, sc, L, H);
-          const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
-          const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
-          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint8_t* rowp = sB + h * (C::B_BYTES / 2) + row * 128;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) = expand8(cw[u], L, H);
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) break;
-    }
-    cp_async_wait<0>();  // no copy may still target shared memory at exit
-  } else if constexpr (W8) {
-    // ------------------------------------------------------------ dequant (8-bit, both CTAs)
-    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
-    const int row = dt & 127;  // weight row of this CTA's half (forward) / of the K fill (backward)
-    const int h = dt >> 7;     // 64-wide atom: K atom (forward) or output chunk (backward)
-    // fp32 scale of the weight row this thread expands in code fill (t, kb)
-    auto scale_at = [&](int t, int kb) -> float {
-      int mb, nb;
-      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
-      const long long n = !B_MN ? static_cast<long long>(pair_brow<EPI>(nb, rank, p)) + row
-                                : static_cast<long long>(kb) * C::BK + row;
-      return n < p.Nw ? __ldg(p.row_scale + n) : 0.0f;
-    };
-    float sc_next = (pair < ntiles && nkb > 0) ? scale_at(pair, 0) : 0.0f;
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int t = pair; t < ntiles; t += npairs) {
-      bool ok = true;
-      for (int kb = 0; kb < nkb + n_ext; ++kb) {
-        float sc = 0.0f;
-        if (kb < nkb) {
-          sc = sc_next;  // the next code fill's scale is loaded one fill ahead
-          const int tn = kb + 1 < nkb ? t : t + npairs;
-          if (tn < ntiles) sc_next = scale_at(tn, kb + 1 < nkb ? kb + 1 : 0);
-        }
-        if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
-        if (kb < nkb) {
-          uint8_t* rowp = smem + stage * C::STAGE_BYTES + C::A_BYTES + h * (C::B_BYTES / 2) + row * 128;
-          const uint8_t* crow = rowp - (row & 31) * 128 + 2048 + (row & 31) * 64;  // this warp's code box
-          uint32_t cw[16];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 c = *reinterpret_cast<const uint4*>(crow + 16 * u);
-            cw[4 * u] = c.x;
-            cw[4 * u + 1] = c.y;
-            cw[4 * u + 2] = c.z;
-            cw[4 * u + 3] = c.w;
-          }
-          __syncwarp();  // the warp's codes are all in registers before its rows are overwritten
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) = expand8_w8<WF>(cw[2 * u], cw[2 * u + 1], sc);
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) break;
     }
   }
 

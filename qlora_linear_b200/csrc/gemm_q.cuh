@@ -1,0 +1,469 @@
+// gemm_q.cuh — the Y / dX GEMM for quantized frozen weights (4-bit blockwise codes,
+// int8 or fp8 e4m3 with row scales) on CTA pairs, with 512-row pair tiles.
+//
+//     out[M, Nout] = Aop[M, Kred] · Bop[Nout, Kred]ᵀ  +  E[M, r] · F[Nout, r]ᵀ
+//
+// Same operation and operand roles as lora_gemm_pair_kernel (gemm_pair.cuh); the weight
+// arrives as codes and is expanded to bf16 in shared memory by the CTA's dequant warps
+// ("Rev vs unsloth", fused quantized-LoRA paragraph: the quantized weight is never
+// dequantized to device memory).
+//
+// Why a separate kernel.  The expanded B tile is written by ordinary shared-memory
+// stores, which compete with the tensor core's operand reads; measured per 128-deep
+// fill of a 256×256 pair tile, the expansion and its proxy fence took about as long as
+// the fill's MMAs, and the MMAs themselves ran a third slower.  Here every expanded B
+// tile feeds two M = 256 MMAs (a 512-row pair tile with two accumulators), which halves
+// the expanded bytes and the expansion work per MMA FLOP.  To keep three-plus stages
+// within shared memory the fills are 64 deep (16 MMAs of M=256, N=256, K=16 each, the
+// same MMA work per fill as the bf16 kernel's 128-deep fills), four stages, and the two
+// accumulators fill all 512 TMEM columns: instead of double-buffering, each accumulator
+// has its own full/empty barrier pair, so the next tile's MMAs into the first
+// accumulator start while the epilogue still drains the second.
+//
+// Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
+// warps 2-5 epilogue, warps 6-13 dequant, warp 14 forwards the dequant warps' completion
+// of each fill to the leader.  Every wait is bounded.
+#pragma once
+
+#include "gemm_pair.cuh"
+
+namespace lora {
+
+template <bool B_MN, int WF>
+struct QCfg {
+  static constexpr bool W4 = WF == WF_BLOCK4;
+  static constexpr int BM = 512, BN = 256, BK = 64;  // pair tile, K per pipeline fill
+  static constexpr int MB = 2;                        // 256-row M blocks (accumulators) per pair tile
+  static constexpr int HM = 128, HN = 128;            // per-CTA rows of an A block / of the B tile
+  static constexpr int STAGES = 4;
+  static constexpr int ATOM = 64;                       // 128-byte swizzle atom width (bf16)
+  static constexpr int A_BLOCK_BYTES = HM * BK * 2;     // 16 KB
+  static constexpr int A_BYTES = MB * A_BLOCK_BYTES;    // 32 KB
+  static constexpr int B_BYTES = HN * BK * 2;           // 16 KB (two 8 KB MN atoms when B is MN-major)
+  static constexpr int C_BYTES = W4 ? HN * BK / 2 : HN * BK;  // codes: 4 KB (4-bit) or 8 KB (8-bit)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+  static constexpr int NUM_EPI_WARPS = 4;
+  static constexpr int NUM_DEQ_WARPS = 8;
+  static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS + NUM_DEQ_WARPS + 1);  // + the forwarder warp
+  static constexpr int TMEM_COLS = 512;  // MB accumulators of BN fp32 columns
+  static constexpr int NUM_BARS = 5 * STAGES + 2 * MB + 1;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+// ---------------------------------------------------------------- epilogue pieces
+// 32 accumulator columns of one row to bf16 out[row, col0 ..].
+__device__ __forceinline__ void epi_store_chunk(const PairParams& p, const uint32_t (&v)[32], int row, int col0) {
+  __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      uint4 o;
+      o.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]));
+      o.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]), __uint_as_float(v[q * 8 + 3]));
+      o.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]));
+      o.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]), __uint_as_float(v[q * 8 + 7]));
+      *reinterpret_cast<uint4*>(orow + col0 + q * 8) = o;
+    }
+  }
+}
+
+// SwiGLU forward: gate g and up u of 32 output columns -> aux (g, u) and out silu(g)·u.
+__device__ __forceinline__ void epi_swiglu_fwd_chunk(const PairParams& p, const uint32_t (&g)[32],
+                                                     const uint32_t (&u)[32], int row, int col0) {
+  __nv_bfloat16* hrow = p.out + static_cast<size_t>(row) * p.Nout;
+  __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      uint32_t og[4], ou[4], oh[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float g0 = __uint_as_float(g[q * 8 + 2 * e]), g1 = __uint_as_float(g[q * 8 + 2 * e + 1]);
+        const float u0 = __uint_as_float(u[q * 8 + 2 * e]), u1 = __uint_as_float(u[q * 8 + 2 * e + 1]);
+        og[e] = pack_bf16x2(g0, g1);
+        ou[e] = pack_bf16x2(u0, u1);
+        oh[e] = pack_bf16x2(g0 * sigmoid_f(g0) * u0, g1 * sigmoid_f(g1) * u1);
+      }
+      *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(og[0], og[1], og[2], og[3]);
+      *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+      *reinterpret_cast<uint4*>(hrow + col0 + q * 8) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    }
+  }
+}
+
+// SwiGLU backward: dH of 32 columns; aux (g, u) overwritten with dG, dU.
+__device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const uint32_t (&v)[32], int row,
+                                                     int col0) {
+  __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      const uint4 gq = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
+      const uint4 uq = *reinterpret_cast<const uint4*>(grow + p.aux_off + col0 + q * 8);
+      const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+      const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+      uint32_t odg[4], odu[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float dg[2], du[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float gv = __uint_as_float(h2 ? (gw[e] & 0xffff0000u) : (gw[e] << 16));
+          const float uv = __uint_as_float(h2 ? (uw[e] & 0xffff0000u) : (uw[e] << 16));
+          const float dh = __uint_as_float(v[q * 8 + 2 * e + h2]);
+          const float sg = sigmoid_f(gv);
+          du[h2] = dh * gv * sg;
+          dg[h2] = dh * uv * sg * (1.0f + gv * (1.0f - sg));
+        }
+        odg[e] = pack_bf16x2(dg[0], dg[1]);
+        odu[e] = pack_bf16x2(du[0], du[1]);
+      }
+      *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(odg[0], odg[1], odg[2], odg[3]);
+      *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(odu[0], odu[1], odu[2], odu[3]);
+    }
+  }
+}
+
+template <bool B_MN, int WF, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_THREADS, 1)
+    lora_gemm_q_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
+                       const PairParams p) {
+  using C = QCfg<B_MN, WF>;
+  constexpr bool W4 = C::W4;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
+  uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
+  uint64_t* cfull = bars + 2 * C::STAGES;   // both: this CTA's code tile landed
+  uint64_t* deq = bars + 3 * C::STAGES;     // leader: both CTAs' expanded tiles written (one forward each)
+  uint64_t* tfull = bars + 4 * C::STAGES;   // both: accumulator b ready for the epilogue
+  uint64_t* tempty = tfull + C::MB;         // leader: both CTAs drained accumulator b
+  uint64_t* drain = tempty + C::MB;         // leader: final commit before TMEM release
+  uint64_t* deql = drain + 1;               // both: this CTA's dequant warps wrote the stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(deql + C::STAGES);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* never_flag = tmem_slot + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int num_m = (p.M + C::BM - 1) / C::BM;
+  const int num_n = (p.Nout + EpiTile<EPI>::COLS - 1) / EpiTile<EPI>::COLS;
+  const int ntiles = num_m * num_n;
+  const int nkb = (p.Kred + C::BK - 1) / C::BK;
+  const int n_ext = p.r > 0 ? (p.r + C::ATOM - 1) / C::ATOM : 0;  // 64 ranks per LoRA fill
+  const WaitCtl wc{abort_flag, p.status, p.wait_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+      mbar_init(smem_u32(&cfull[s]), 1);
+      mbar_init(smem_u32(&deq[s]), 2);
+      mbar_init(smem_u32(&deql[s]), C::NUM_DEQ_WARPS);
+    }
+    for (int b = 0; b < C::MB; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 2 * C::NUM_EPI_WARPS);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    *never_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmC);
+    tma_prefetch_desc(&tmE);
+    tma_prefetch_desc(&tmF);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long fills = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        int mb, nb;
+        pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+        const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A block 0
+        const int brow = pair_brow<EPI>(nb, rank, p);
+        for (int kb = 0; kb < nkb + n_ext; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
+          const bool ext = kb >= nkb;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sC = sB + C::B_BYTES;
+          const uint32_t full_l = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + (ext ? C::B_BYTES : 0)));
+          if (!ext) {
+            for (int b = 0; b < C::MB; ++b)
+              tma_load_2d_pair(sA + b * C::A_BLOCK_BYTES, &tmA, full_l, kb * C::BK, arow + b * 256);
+            const uint32_t cb = smem_u32(&cfull[stage]);
+            mbar_arrive_expect_tx(cb, C::C_BYTES);
+            if (W4) {
+              if (!B_MN) tma_load_2d(sC, &tmC, cb, kb * (C::BK / 2), brow);  // 32 B × 128 rows
+              else tma_load_2d(sC, &tmC, cb, brow / 2, kb * C::BK);         // 64 B × 64 rows
+            } else {
+              if (!B_MN) tma_load_2d(sC, &tmC, cb, kb * C::BK, brow);       // 64 B × 128 rows
+              else tma_load_2d(sC, &tmC, cb, brow, kb * C::BK);             // 128 B × 64 rows
+            }
+          } else {
+            const int e = kb - nkb;
+            int seg = 0;
+            while (seg + 1 < p.nseg && nb >= p.seg_end_tile[seg]) ++seg;
+            const int e0 = seg * p.e_seg_stride + e * C::ATOM;  // this fill's columns of E
+            for (int b = 0; b < C::MB; ++b)
+              tma_load_2d_pair(sA + b * C::A_BLOCK_BYTES, &tmE, full_l, e0, arow + b * 256);
+            if (!B_MN) {
+              const int fx = EPI == EPI_SWIGLU_FWD ? -static_cast<int>(rank) * p.f_shift : 0;
+              tma_load_2d_pair(sB, &tmF, full_l, fx + e * C::ATOM, brow);  // 64 ranks × 128 rows
+            } else {
+              tma_load_2d_pair(sB, &tmF, full_l, brow, e * C::ATOM);       // 64 columns × 64 ranks
+              tma_load_2d_pair(sB + C::B_BYTES / 2, &tmF, full_l, brow + C::ATOM, e * C::ATOM);
+            }
+            mbar_arrive(smem_u32(&cfull[stage]));  // nothing to expand in this fill
+          }
+          ++fills;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        const long long first = fills > C::STAGES ? fills - C::STAGES : 0;
+        const WaitCtl drain_wc{never_flag, nullptr, p.wait_ns};
+        for (long long f = first; f < fills; ++f) {
+          const int s = static_cast<int>(f % C::STAGES);
+          const uint32_t ph = static_cast<uint32_t>((f / C::STAGES) & 1);
+          if (leader) mbar_wait(smem_u32(&full[s]), ph, drain_wc);
+          mbar_wait(smem_u32(&cfull[s]), ph, drain_wc);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, C::BN, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t tphase = 0;  // parity of the accumulator barriers for this tile
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        for (int kb = 0; kb < nkb + n_ext; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
+          if (!mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
+          tc_fence_after();
+          const bool ext = kb >= nkb;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const int nk = ext ? min(C::BK / 16, (p.r - (kb - nkb) * C::ATOM + 15) / 16) : C::BK / 16;
+          for (int b = 0; b < C::MB; ++b) {
+            if (kb == 0) {
+              // the epilogue must have drained accumulator b of the previous tile
+              if (!mbar_wait<true>(smem_u32(&tempty[b]), tphase ^ 1u, wc)) { ok = false; break; }
+              tc_fence_after();
+            }
+            const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::BN);
+            for (int k = 0; k < nk; ++k) {
+              const uint64_t ad = sdesc_sw128(sA + b * C::A_BLOCK_BYTES + k * 32, 16, 1024);
+              const uint64_t bd = B_MN ? sdesc_sw128(sB + k * 2048, C::B_BYTES / 2, 1024) : sdesc_sw128(sB + k * 32, 16, 1024);
+              tc_mma_bf16_pair(d, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        for (int b = 0; b < C::MB; ++b) tc_commit_pair_mc(smem_u32(&tfull[b]), 0x3);
+        tphase ^= 1u;
+      }
+      tc_commit_pair(smem_u32(drain));
+      const WaitCtl drain_wc{never_flag, nullptr, p.wait_ns};
+      mbar_wait(smem_u32(drain), 0, drain_wc);
+    }
+  } else if (warp < 2 + C::NUM_EPI_WARPS) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t tphase = 0;
+    bool ok = true;
+    for (int t = pair; t < ntiles && ok; t += npairs) {
+      int mb, nb;
+      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+      for (int b = 0; b < C::MB; ++b) {
+        if (!mbar_wait_warp(smem_u32(&tfull[b]), tphase, wc)) { ok = false; break; }
+        tc_fence_after();
+        const int row = mb * C::BM + b * 256 + static_cast<int>(rank) * C::HM + quarter * 32 + lane;
+        const uint32_t tbase =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * C::BN);
+        if constexpr (EPI == EPI_SWIGLU_FWD) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            const int col0 = nb * 128 + c * 32;
+            if (col0 >= p.Nout) break;  // warp-uniform
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(tbase + c * 32, g);
+            tmem_ld_32x32b_x32(tbase + 128 + c * 32, u);
+            tmem_ld_wait();
+            if (row < p.M) epi_swiglu_fwd_chunk(p, g, u, row, col0);
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < C::BN / 32; ++c) {
+            const int col0 = nb * C::BN + c * 32;
+            if (col0 >= p.Nout) break;  // warp-uniform
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + c * 32, v);
+            tmem_ld_wait();
+            if (row < p.M) {
+              if constexpr (EPI == EPI_SWIGLU_BWD) epi_swiglu_bwd_chunk(p, v, row, col0);
+              else epi_store_chunk(p, v, row, col0);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[b]), 0));
+      }
+      tphase ^= 1u;
+    }
+  } else if (warp == 2 + C::NUM_EPI_WARPS + C::NUM_DEQ_WARPS) {
+    // ------------------------------------------------------------ forwarder (both CTAs)
+    // The dequant warps signal a CTA-local barrier (release at CTA scope); this warp turns
+    // each completed fill into the one cluster-scope release arrive the leader's MMA
+    // issuer waits for.  A release at cluster scope costs about a fill's worth of cycles
+    // when every dequant warp issues its own.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        for (int kb = 0; kb < nkb + n_ext; ++kb) {
+          if (!mbar_wait(smem_u32(&deql[stage]), phase, wc)) { ok = false; break; }
+          mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dequant (both CTAs)
+    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
+    // forward: weight row `row` of this CTA's 128, 32-element half `h` of the 64-deep fill;
+    // backward: weight row `krow` of the 64-deep fill, 32-column chunk `c4` of this CTA's 128
+    const int row = !B_MN ? (dt & 127) : (dt >> 2);
+    const int sub = !B_MN ? (dt >> 7) : (dt & 3);
+    float cb[16];
+    if (W4) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
+    }
+    const long long kblocks_w = p.Kw / 64;  // 4-bit scale blocks per weight row
+    // scale for code fill kb of tile t: a fp16 block scale (4-bit) or a fp32 row scale (8-bit)
+    auto scale_at = [&](int t, int kb) -> float {
+      int mb, nb;
+      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+      const int brow = pair_brow<EPI>(nb, rank, p);
+      const long long n = !B_MN ? static_cast<long long>(brow) + row : static_cast<long long>(kb) * C::BK + row;
+      if (n >= p.Nw) return 0.0f;
+      if (W4) {
+        const long long kblk = !B_MN ? kb : (brow + (sub >> 1) * 64) / 64;
+        return kblk < kblocks_w ? __half2float(p.absmax[n * kblocks_w + kblk]) : 0.0f;
+      }
+      return __ldg(p.row_scale + n);
+    };
+    // scales are loaded two code fills ahead so no register waits on a fresh global load
+    auto next_fill = [&](int& t, int& kb) {
+      if (++kb == nkb) { kb = 0; t += npairs; }
+    };
+    int st_t = pair, st_kb = 0;  // the code fill whose scale is loaded next
+    float sq[3] = {0.f, 0.f, 0.f};
+    int sqh = 0;
+    for (int i = 0; i < 2; ++i) {
+      sq[i] = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;
+      next_fill(st_t, st_kb);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = pair; t < ntiles; t += npairs) {
+      bool ok = true;
+      for (int kb = 0; kb < nkb + n_ext; ++kb) {
+        const bool code = kb < nkb;
+        float sc = 0.f;
+        if (code) {
+          sq[(sqh + 2) % 3] = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;
+          next_fill(st_t, st_kb);
+          sc = sq[sqh];
+          sqh = (sqh + 1) % 3;
+        }
+        if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
+        if (code) {
+          uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+          const uint8_t* sC = sB + C::B_BYTES;
+          // destination row (128 bytes = 64 bf16, 128-byte swizzle) and its four 16-byte units
+          uint8_t* rowp;
+          int u0;
+          const uint8_t* cp;
+          if (!B_MN) {
+            rowp = sB + row * 128;
+            u0 = sub * 4;
+            cp = W4 ? sC + row * 32 + sub * 16 : sC + row * 64 + sub * 32;
+          } else {
+            rowp = sB + (sub >> 1) * (C::B_BYTES / 2) + row * 128;
+            u0 = (sub & 1) * 4;
+            cp = W4 ? sC + row * 64 + sub * 16 : sC + row * 128 + sub * 32;
+          }
+          if constexpr (W4) {
+            const uint4 c = *reinterpret_cast<const uint4*>(cp);
+            uint32_t L[4], H[4];
+            block_levels(cb, sc, L, H);
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4*>(rowp + (((u0 + i) ^ (row & 7)) << 4)) = expand8(cw[i], L, H);
+          } else {
+            const uint4 c0 = *reinterpret_cast<const uint4*>(cp);
+            const uint4 c1 = *reinterpret_cast<const uint4*>(cp + 16);
+            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4*>(rowp + (((u0 + i) ^ (row & 7)) << 4)) =
+                  expand8_w8<WF>(cw[2 * i], cw[2 * i + 1], sc);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&deql[stage]));
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace lora

@@ -17,6 +17,7 @@
 #include "lora_linear_testing.h"
 #include "elementwise.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_q.cuh"
 #include "skinny.cuh"
 
 namespace lora {
@@ -142,19 +143,22 @@ lora_status_t dev_info(DevInfo** out) {
   if (!d.attrs_set) {
     bool ok = true;
 #define SET_SMEM(fn, bytes) ok &= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-#define SET_GEMM(WF)                                                                                    \
-  SET_SMEM((lora_gemm_pair_kernel<false, WF, EPI_STORE>), (PairCfg<false, WF>::SMEM_BYTES));           \
-  SET_SMEM((lora_gemm_pair_kernel<true, WF, EPI_STORE>), (PairCfg<true, WF>::SMEM_BYTES));             \
-  SET_SMEM((lora_gemm_pair_kernel<false, WF, EPI_SWIGLU_FWD>), (PairCfg<false, WF>::SMEM_BYTES));      \
-  SET_SMEM((lora_gemm_pair_kernel<true, WF, EPI_SWIGLU_BWD>), (PairCfg<true, WF>::SMEM_BYTES));
-    SET_GEMM(WF_BF16)
-    SET_GEMM(WF_BLOCK4)
-    SET_GEMM(WF_INT8)
-    SET_GEMM(WF_FP8)
-#undef SET_GEMM
-    SET_SMEM((lora_gemm_pair_kernel<false, WF_BF16, EPI_CE_LSE>), (PairCfg<false, WF_BF16>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<false, WF_BF16, EPI_CE_DLOGITS>), (PairCfg<false, WF_BF16>::SMEM_BYTES));
-    SET_SMEM((lora_gemm_pair_kernel<true, WF_BF16, EPI_ACC_F32>), (PairCfg<true, WF_BF16>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, EPI_STORE>), (PairCfg<false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, EPI_STORE>), (PairCfg<true>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, EPI_SWIGLU_FWD>), (PairCfg<false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, EPI_SWIGLU_BWD>), (PairCfg<true>::SMEM_BYTES));
+#define SET_GEMM_Q(WF)                                                                              \
+  SET_SMEM((lora_gemm_q_kernel<false, WF, EPI_STORE>), (QCfg<false, WF>::SMEM_BYTES));             \
+  SET_SMEM((lora_gemm_q_kernel<true, WF, EPI_STORE>), (QCfg<true, WF>::SMEM_BYTES));               \
+  SET_SMEM((lora_gemm_q_kernel<false, WF, EPI_SWIGLU_FWD>), (QCfg<false, WF>::SMEM_BYTES));        \
+  SET_SMEM((lora_gemm_q_kernel<true, WF, EPI_SWIGLU_BWD>), (QCfg<true, WF>::SMEM_BYTES));
+    SET_GEMM_Q(WF_BLOCK4)
+    SET_GEMM_Q(WF_INT8)
+    SET_GEMM_Q(WF_FP8)
+#undef SET_GEMM_Q
+    SET_SMEM((lora_gemm_pair_kernel<false, EPI_CE_LSE>), (PairCfg<false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<false, EPI_CE_DLOGITS>), (PairCfg<false>::SMEM_BYTES));
+    SET_SMEM((lora_gemm_pair_kernel<true, EPI_ACC_F32>), (PairCfg<true>::SMEM_BYTES));
     SET_SMEM((rowproj_kernel<16, false>), (rowproj_smem_bytes<16, false>()));
     SET_SMEM((rowproj_kernel<32, false>), (rowproj_smem_bytes<32, false>()));
     SET_SMEM((rowproj_kernel<64, false>), (rowproj_smem_bytes<64, false>()));
@@ -322,50 +326,78 @@ lora_status_t finalize_cols(const float* part, int splits, int C, int r, float s
 }
 
 // ---------------------------------------------------------------- GEMM launch
-template <bool B_MN, int WF, int EPI>
+template <bool B_MN, int EPI>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
                           const PairParams& p, int sms, cudaStream_t st) {
-  using C = PairCfg<B_MN, WF>;
+  using C = PairCfg<B_MN>;
   const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_pair_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    lora_gemm_pair_kernel<B_MN, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
   }
   count_launch();
   return last_launch();
 }
 
-// Every tensor-map box of the pair GEMM is 64 elements (or 64 code bytes) wide and 128
-// rows high, except the 8-bit code boxes: 64 bytes × 32 rows, one per dequant warp.
-constexpr uint32_t kBoxX = 64, kBoxY = 128, kBoxY8 = 32;
+// Tensor-map boxes of the GEMM operands: 64 elements wide, 128 rows high (the quantized
+// kernel's code and backward-F boxes are set in launch_gemm_w).
+constexpr uint32_t kBoxX = 64, kBoxY = 128;
 
 // The weight operand's tensor map (over the stored [N, K] array, for either direction)
 // and the launch of the GEMM instantiation for the weight's format.
-template <bool B_MN, int EPI>
-lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const CUtensorMap& e, const CUtensorMap& f,
+template <bool B_MN, int WF, int EPI>
+lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CUtensorMap& e, const CUtensorMap& f,
                             const PairParams& p, int sms, cudaStream_t st) {
-  CUtensorMap b;
+  using C = QCfg<B_MN, WF>;
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
+  const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+  const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
+  {
+    TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
+    lora_gemm_q_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, c, e, f, p);
+  }
+  count_launch();
+  return last_launch();
+}
+
+// The LoRA F operand: its array and shape; its tensor map's box depends on the kernel.
+struct FSpec {
+  const void* base;
+  uint64_t inner, rows;
+};
+
+// The weight operand's tensor map (over the stored [N, K] array, for either direction)
+// and the launch of the GEMM for the weight's format: the bf16 pair kernel, or the
+// quantized kernel whose code tiles are 64 deep.
+template <bool B_MN, int EPI>
+lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const CUtensorMap& e, const FSpec& fs,
+                            const PairParams& p, int sms, cudaStream_t st) {
+  CUtensorMap b, f;
+  TRY(tmap_bf16(&f, fs.base, fs.inner, fs.rows, kBoxX, kBoxY));
   if constexpr (EPI == EPI_CE_LSE || EPI == EPI_CE_DLOGITS || EPI == EPI_ACC_F32) {
     // the cross-entropy head is bf16 only (checked by the caller)
     TRY(tmap_bf16(&b, W->data, W->K, W->N, kBoxX, kBoxY));
-    return launch_gemm<B_MN, WF_BF16, EPI>(a, b, e, f, p, sms, st);
+    return launch_gemm<B_MN, EPI>(a, b, e, f, p, sms, st);
   } else {
-  switch (W->fmt) {
-    case LORA_W_BF16:
+    if (W->fmt == LORA_W_BF16) {
       TRY(tmap_bf16(&b, W->data, W->K, W->N, kBoxX, kBoxY));
-      return launch_gemm<B_MN, WF_BF16, EPI>(a, b, e, f, p, sms, st);
-    case LORA_W_BLOCK4:
-      TRY(tmap_u8(&b, W->data, W->K / 2, W->N, kBoxX, kBoxY));
-      return launch_gemm<B_MN, WF_BLOCK4, EPI>(a, b, e, f, p, sms, st);
-    case LORA_W_INT8:
-      TRY(tmap_u8(&b, W->data, W->K, W->N, kBoxX, kBoxY8));
-      return launch_gemm<B_MN, WF_INT8, EPI>(a, b, e, f, p, sms, st);
-    default:
-      TRY(tmap_u8(&b, W->data, W->K, W->N, kBoxX, kBoxY8));
-      return launch_gemm<B_MN, WF_FP8, EPI>(a, b, e, f, p, sms, st);
-  }
+      return launch_gemm<B_MN, EPI>(a, b, e, f, p, sms, st);
+    }
+    // the quantized kernel's backward LoRA fill takes 64 ranks per box
+    if (B_MN) TRY(tmap_bf16(&f, fs.base, fs.inner, fs.rows, kBoxX, 64));
+    const bool w4 = W->fmt == LORA_W_BLOCK4;
+    const uint64_t row_bytes = w4 ? W->K / 2 : W->K;
+    // code boxes: forward 128 weight rows × one 64-deep fill; backward 64 weight rows × 128 columns
+    const uint32_t bx = B_MN ? (w4 ? 64 : 128) : (w4 ? 32 : 64);
+    const uint32_t by = B_MN ? 64 : 128;
+    TRY(tmap_u8(&b, W->data, row_bytes, W->N, bx, by));
+    switch (W->fmt) {
+      case LORA_W_BLOCK4: return launch_gemm_q<B_MN, WF_BLOCK4, EPI>(a, b, e, f, p, sms, st);
+      case LORA_W_INT8: return launch_gemm_q<B_MN, WF_INT8, EPI>(a, b, e, f, p, sms, st);
+      default: return launch_gemm_q<B_MN, WF_FP8, EPI>(a, b, e, f, p, sms, st);
+    }
   }
 }
 
@@ -452,10 +484,10 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   TRY(launch_rowproj<false>(Xb, Ki, static_cast<const __nv_bfloat16*>(A), part, Mi, Ki, rt, sp, st));
   TRY(finalize_rows(part, sp.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
 
-  CUtensorMap ta, te, tf;
+  CUtensorMap ta, te;
   TRY(tmap_bf16(&ta, X, K, M, kBoxX, kBoxY));
   TRY(tmap_bf16(&te, sXA, rt, M, kBoxX, kBoxY));
-  TRY(tmap_bf16(&tf, B, r, N, kBoxX, kBoxY));
+  const FSpec tf{B, static_cast<uint64_t>(r), static_cast<uint64_t>(N)};
   PairParams p = gemm_params(M, N, K, r, Y, status, W);
   set_segments(p, sg, r);
   return launch_gemm_w<false, EPI_STORE>(W, ta, te, tf, p, dev->sms, st);
@@ -494,10 +526,10 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
   }
   if (dX) {
     // dX = dY·W + (s·dY·B)·A with the LoRA fill over all G·r ranks
-    CUtensorMap ta, te, tf;
+    CUtensorMap ta, te;
     TRY(tmap_bf16(&ta, dY, N, M, kBoxX, kBoxY));
     TRY(tmap_bf16(&te, sdYB, rt, M, kBoxX, kBoxY));
-    TRY(tmap_bf16(&tf, A, K, rt, kBoxX, kBoxY));
+    const FSpec tf{A, static_cast<uint64_t>(K), static_cast<uint64_t>(rt)};
     PairParams p = gemm_params(M, K, N, rt, dX, status, W);
     TRY((launch_gemm_w<true, EPI_STORE>(W, ta, te, tf, p, dev->sms, st)));
   }
@@ -629,10 +661,10 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
                             static_cast<const __nv_bfloat16*>(m->A_gate_up), part, Mi, Di, r2, sp, st));
   TRY(finalize_rows(part, sp.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
 
-  CUtensorMap ta, te, tf;
+  CUtensorMap ta, te;
   TRY(tmap_bf16(&ta, X, D, M, kBoxX, kBoxY));
   TRY(tmap_bf16(&te, skinny, r2, M, kBoxX, kBoxY));
-  TRY(tmap_bf16(&tf, m->B_gate_up, r, 2 * I, kBoxX, kBoxY));
+  const FSpec tf{m->B_gate_up, static_cast<uint64_t>(r), static_cast<uint64_t>(2 * I)};
   PairParams p = gemm_params(M, I, D, r2, H, status, &m->gate_up);
   p.half_rows = static_cast<int>(I);
   p.f_shift = r;
@@ -668,10 +700,10 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
   TRY(finalize_cols(part, sp.splits, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
   // dH = dZ·W_d + (s·dZ·B_d)·A_d, consumed by the epilogue: GU <- [dG | dU]
   {
-    CUtensorMap ta, te, tf;
+    CUtensorMap ta, te;
     TRY(tmap_bf16(&ta, dZ, D, M, kBoxX, kBoxY));
     TRY(tmap_bf16(&te, skinny, r, M, kBoxX, kBoxY));
-    TRY(tmap_bf16(&tf, m->A_down, I, r, kBoxX, kBoxY));
+    const FSpec tf{m->A_down, static_cast<uint64_t>(I), static_cast<uint64_t>(r)};
     PairParams p = gemm_params(M, I, D, r, nullptr, status, &m->down);
     p.aux = static_cast<__nv_bfloat16*>(GU);
     p.ld_aux = static_cast<int>(2 * I);
@@ -892,7 +924,8 @@ lora_status_t lora_ce_fwd(const void* X, int64_t M, const lora_weight_t* W, cons
   p.ignore_index = ignore_index;
   p.lse_part = reinterpret_cast<float*>(ws + c.part_off);
   p.label_logit = zy;
-  TRY((launch_gemm_w<false, EPI_CE_LSE>(W, ta, ta, ta, p, dev->sms, st)));
+  TRY((launch_gemm_w<false, EPI_CE_LSE>(W, ta, ta, FSpec{X, static_cast<uint64_t>(D), static_cast<uint64_t>(M)}, p,
+                                         dev->sms, st)));
   ce_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(reinterpret_cast<const float2*>(ws + c.part_off),
                                                    cdiv(V, 256), static_cast<int>(M), zy, labels, ignore_index, loss,
                                                    lse);
@@ -940,14 +973,16 @@ lora_status_t lora_ce_bwd(const void* X, int64_t M, const lora_weight_t* W, cons
     p.v0 = static_cast<int>(v0);
     p.lse = lse;
     p.dloss = dloss;
-    TRY((launch_gemm_w<false, EPI_CE_DLOGITS>(&Wc, tx, tx, tx, p, dev->sms, st)));
+    TRY((launch_gemm_w<false, EPI_CE_DLOGITS>(&Wc, tx, tx, FSpec{X, static_cast<uint64_t>(D), static_cast<uint64_t>(M)},
+                                              p, dev->sms, st)));
     // dX (+)= dlogits_slice · W_slice, summed over slices in fp32
     CUtensorMap ta;
     TRY(tmap_bf16(&ta, dlog, w, M, kBoxX, kBoxY));
     PairParams q = ce_params(M, D, w, dX, status, &Wc);
     q.acc32 = acc;
     q.acc_mode = (i > 0 ? 1 : 0) | (i == nslices - 1 ? 2 : 0);
-    TRY((launch_gemm_w<true, EPI_ACC_F32>(&Wc, ta, ta, ta, q, dev->sms, st)));
+    TRY((launch_gemm_w<true, EPI_ACC_F32>(&Wc, ta, ta, FSpec{dlog, static_cast<uint64_t>(w), static_cast<uint64_t>(M)},
+                                          q, dev->sms, st)));
   }
   return LORA_OK;
 }
