@@ -1,0 +1,162 @@
+// gemm_common.cuh — what the two tcgen05 GEMM kernels share: the launch parameters,
+// the tile order, the epilogue modes and their per-chunk arithmetic.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace lora {
+
+struct PairParams {
+  int M;               // rows of Aop / out
+  int Nout;            // columns of out
+  int Kred;            // reduction length (K forward, N backward)
+  int r;               // rank of the LoRA fill (<= 128): one extra K fill
+  // Grouped projections (forward): output tile columns [seg_end[g-1], seg_end[g]) (in
+  // 256-column tiles) belong to segment g, whose E columns start at g * e_seg_stride.
+  int nseg;            // 1 for a single projection
+  int e_seg_stride;
+  int seg_end_tile[8];
+  int group_m;         // 256-row tiles per raster group (L2 reuse of the B operand)
+  // SwiGLU epilogues (feed-forward block).  Forward: the even CTA of a pair takes gate
+  // rows nb*128.., the odd CTA the up rows half_rows further on, and the odd CTA's LoRA
+  // F tile starts f_shift columns to the left, so it meets the up half of E.
+  int half_rows;
+  int f_shift;
+  __nv_bfloat16* aux;  // [M, ld_aux]: gate pre-activations, up pre-activations aux_off columns on
+  int ld_aux;
+  int aux_off;
+  // Cross-entropy over an LM head (logits = the GEMM's output columns, vocabulary index
+  // v0 + column).
+  const int32_t* labels;   // [M]
+  int ignore_index;
+  int v0;
+  float* lse_part;         // EPI_CE_LSE: [num_n][M][2] (max, sum of exp(z - max)) per 256-column tile
+  float* label_logit;      // EPI_CE_LSE: [M], written by the tile holding the row's label
+  const float* lse;        // EPI_CE_DLOGITS: [M]
+  const float* dloss;      // EPI_CE_DLOGITS: [M] upstream gradient of each row's loss
+  float* acc32;            // EPI_ACC_F32: [M, Nout] fp32 running sum
+  int acc_mode;            // EPI_ACC_F32: bit 0 add the running sum, bit 1 write bf16 to out instead
+  __nv_bfloat16* out;  // [M, Nout] row-major
+  uint32_t* status;    // device status word, may be null
+  uint64_t wait_ns;    // bound of every mbarrier wait
+  // quantized weights only
+  const __half* absmax;      // 4-bit: fp16 [Nw*Kw/64]
+  const float* codebook;     // 4-bit: [16]
+  const float* row_scale;    // 8-bit: fp32 [Nw]
+  int Nw, Kw;                // logical weight shape [Nw, Kw]
+};
+
+// Epilogue of the GEMMs.
+enum : int {
+  EPI_STORE = 0,       // out = accumulator (bf16)
+  EPI_SWIGLU_FWD = 1,  // accumulator columns [0,128) gate g, [128,256) up u of the same 128
+                       // output columns: aux <- g, u; out <- silu(g)·u
+  EPI_SWIGLU_BWD = 2,  // accumulator = dH; aux holds g, u and is overwritten in place with
+                       // dG = dH·u·silu'(g), dU = dH·silu(g); out is not written
+  EPI_CE_LSE = 3,      // accumulator = logits: per row and tile (max, Σ exp(z - max)) and the
+                       // label's logit; no logits are written
+  EPI_CE_DLOGITS = 4,  // accumulator = logits: out <- dloss·(exp(z - lse) - [label == column])
+  EPI_ACC_F32 = 5,     // out/acc32 <- accumulator (+ acc32), see acc_mode
+};
+
+template <int EPI>
+struct EpiTile {
+  static constexpr int COLS = EPI == EPI_SWIGLU_FWD ? 128 : 256;  // output columns per pair tile
+};
+
+// First row of this CTA's half of the B tile (and of its LoRA F tile).
+template <int EPI>
+__device__ __forceinline__ int pair_brow(int nb, uint32_t rank, const PairParams& p) {
+  if (EPI == EPI_SWIGLU_FWD) return nb * 128 + static_cast<int>(rank) * p.half_rows;
+  return nb * 256 + static_cast<int>(rank) * 128;
+}
+
+// silu(g) = g·sigmoid(g); sigmoid from the exponential intrinsic and a rounded reciprocal
+// (1/(1+e^-g) is 0, not NaN, when e^-g overflows).
+__device__ __forceinline__ float sigmoid_f(float g) { return __frcp_rn(1.0f + __expf(-g)); }
+
+__device__ __forceinline__ void pair_tile_coords(int t, int num_m, int num_n, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * num_n;
+  const int g = t / per_group;
+  const int first_m = g * group_m;
+  const int gm = min(group_m, num_m - first_m);
+  const int within = t - first_m * num_n;
+  mb = first_m + within % gm;
+  nb = within / gm;
+}
+
+// ---------------------------------------------------------------- epilogue pieces
+// 32 accumulator columns of one row to bf16 out[row, col0 ..].
+__device__ __forceinline__ void epi_store_chunk(const PairParams& p, const uint32_t (&v)[32], int row, int col0) {
+  __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      uint4 o;
+      o.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]));
+      o.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]), __uint_as_float(v[q * 8 + 3]));
+      o.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]));
+      o.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]), __uint_as_float(v[q * 8 + 7]));
+      *reinterpret_cast<uint4*>(orow + col0 + q * 8) = o;
+    }
+  }
+}
+
+// SwiGLU forward: gate g and up u of 32 output columns -> aux (g, u) and out silu(g)·u.
+__device__ __forceinline__ void epi_swiglu_fwd_chunk(const PairParams& p, const uint32_t (&g)[32],
+                                                     const uint32_t (&u)[32], int row, int col0) {
+  __nv_bfloat16* hrow = p.out + static_cast<size_t>(row) * p.Nout;
+  __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      uint32_t og[4], ou[4], oh[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float g0 = __uint_as_float(g[q * 8 + 2 * e]), g1 = __uint_as_float(g[q * 8 + 2 * e + 1]);
+        const float u0 = __uint_as_float(u[q * 8 + 2 * e]), u1 = __uint_as_float(u[q * 8 + 2 * e + 1]);
+        og[e] = pack_bf16x2(g0, g1);
+        ou[e] = pack_bf16x2(u0, u1);
+        oh[e] = pack_bf16x2(g0 * sigmoid_f(g0) * u0, g1 * sigmoid_f(g1) * u1);
+      }
+      *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(og[0], og[1], og[2], og[3]);
+      *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+      *reinterpret_cast<uint4*>(hrow + col0 + q * 8) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    }
+  }
+}
+
+// SwiGLU backward: dH of 32 columns; aux (g, u) overwritten with dG, dU.
+__device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const uint32_t (&v)[32], int row,
+                                                     int col0) {
+  __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      const uint4 gq = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
+      const uint4 uq = *reinterpret_cast<const uint4*>(grow + p.aux_off + col0 + q * 8);
+      const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+      const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+      uint32_t odg[4], odu[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float dg[2], du[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float gv = __uint_as_float(h2 ? (gw[e] & 0xffff0000u) : (gw[e] << 16));
+          const float uv = __uint_as_float(h2 ? (uw[e] & 0xffff0000u) : (uw[e] << 16));
+          const float dh = __uint_as_float(v[q * 8 + 2 * e + h2]);
+          const float sg = sigmoid_f(gv);
+          du[h2] = dh * gv * sg;
+          dg[h2] = dh * uv * sg * (1.0f + gv * (1.0f - sg));
+        }
+        odg[e] = pack_bf16x2(dg[0], dg[1]);
+        odu[e] = pack_bf16x2(du[0], du[1]);
+      }
+      *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(odg[0], odg[1], odg[2], odg[3]);
+      *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(odu[0], odu[1], odu[2], odu[3]);
+    }
+  }
+}
+
+}  // namespace lora

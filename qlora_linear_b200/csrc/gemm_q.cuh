@@ -25,7 +25,8 @@
 // of each fill to the leader.  Every wait is bounded.
 #pragma once
 
-#include "gemm_pair.cuh"
+#include "dequant.cuh"
+#include "gemm_common.cuh"
 
 namespace lora {
 
@@ -51,80 +52,6 @@ struct QCfg {
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
-
-// ---------------------------------------------------------------- epilogue pieces
-// 32 accumulator columns of one row to bf16 out[row, col0 ..].
-__device__ __forceinline__ void epi_store_chunk(const PairParams& p, const uint32_t (&v)[32], int row, int col0) {
-  __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (col0 + q * 8 < p.Nout) {
-      uint4 o;
-      o.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]));
-      o.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]), __uint_as_float(v[q * 8 + 3]));
-      o.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]));
-      o.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]), __uint_as_float(v[q * 8 + 7]));
-      *reinterpret_cast<uint4*>(orow + col0 + q * 8) = o;
-    }
-  }
-}
-
-// SwiGLU forward: gate g and up u of 32 output columns -> aux (g, u) and out silu(g)·u.
-__device__ __forceinline__ void epi_swiglu_fwd_chunk(const PairParams& p, const uint32_t (&g)[32],
-                                                     const uint32_t (&u)[32], int row, int col0) {
-  __nv_bfloat16* hrow = p.out + static_cast<size_t>(row) * p.Nout;
-  __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (col0 + q * 8 < p.Nout) {
-      uint32_t og[4], ou[4], oh[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float g0 = __uint_as_float(g[q * 8 + 2 * e]), g1 = __uint_as_float(g[q * 8 + 2 * e + 1]);
-        const float u0 = __uint_as_float(u[q * 8 + 2 * e]), u1 = __uint_as_float(u[q * 8 + 2 * e + 1]);
-        og[e] = pack_bf16x2(g0, g1);
-        ou[e] = pack_bf16x2(u0, u1);
-        oh[e] = pack_bf16x2(g0 * sigmoid_f(g0) * u0, g1 * sigmoid_f(g1) * u1);
-      }
-      *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(og[0], og[1], og[2], og[3]);
-      *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
-      *reinterpret_cast<uint4*>(hrow + col0 + q * 8) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-    }
-  }
-}
-
-// SwiGLU backward: dH of 32 columns; aux (g, u) overwritten with dG, dU.
-__device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const uint32_t (&v)[32], int row,
-                                                     int col0) {
-  __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (col0 + q * 8 < p.Nout) {
-      const uint4 gq = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
-      const uint4 uq = *reinterpret_cast<const uint4*>(grow + p.aux_off + col0 + q * 8);
-      const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-      const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
-      uint32_t odg[4], odu[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float dg[2], du[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const float gv = __uint_as_float(h2 ? (gw[e] & 0xffff0000u) : (gw[e] << 16));
-          const float uv = __uint_as_float(h2 ? (uw[e] & 0xffff0000u) : (uw[e] << 16));
-          const float dh = __uint_as_float(v[q * 8 + 2 * e + h2]);
-          const float sg = sigmoid_f(gv);
-          du[h2] = dh * gv * sg;
-          dg[h2] = dh * uv * sg * (1.0f + gv * (1.0f - sg));
-        }
-        odg[e] = pack_bf16x2(dg[0], dg[1]);
-        odu[e] = pack_bf16x2(du[0], du[1]);
-      }
-      *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(odg[0], odg[1], odg[2], odg[3]);
-      *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(odu[0], odu[1], odu[2], odu[3]);
-    }
-  }
-}
 
 template <bool B_MN, int WF, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_THREADS, 1)
