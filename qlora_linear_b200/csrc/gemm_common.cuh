@@ -126,17 +126,30 @@ __device__ __forceinline__ void epi_swiglu_fwd_chunk(const PairParams& p, const 
   }
 }
 
-// SwiGLU backward: dH of 32 columns; aux (g, u) overwritten with dG, dU.
-__device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const uint32_t (&v)[32], int row,
-                                                     int col0) {
+// SwiGLU backward: the saved g and u of 32 columns (loaded one chunk ahead of use) ...
+struct GU32 {
+  uint4 g[4], u[4];
+};
+__device__ __forceinline__ void epi_swiglu_bwd_load(const PairParams& p, int row, int col0, GU32& x) {
+  const __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      x.g[q] = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
+      x.u[q] = *reinterpret_cast<const uint4*>(grow + p.aux_off + col0 + q * 8);
+    }
+  }
+}
+
+// ... and dH of the same columns: aux (g, u) overwritten with dG = dH·u·silu'(g), dU = dH·silu(g).
+__device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const uint32_t (&v)[32], int row, int col0,
+                                                     const GU32& x) {
   __nv_bfloat16* grow = p.aux + static_cast<size_t>(row) * p.ld_aux;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     if (col0 + q * 8 < p.Nout) {
-      const uint4 gq = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
-      const uint4 uq = *reinterpret_cast<const uint4*>(grow + p.aux_off + col0 + q * 8);
-      const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-      const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+      const uint32_t gw[4] = {x.g[q].x, x.g[q].y, x.g[q].z, x.g[q].w};
+      const uint32_t uw[4] = {x.u[q].x, x.u[q].y, x.u[q].z, x.u[q].w};
       uint32_t odg[4], odu[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -156,6 +169,30 @@ __device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const 
       *reinterpret_cast<uint4*>(grow + col0 + q * 8) = make_uint4(odg[0], odg[1], odg[2], odg[3]);
       *reinterpret_cast<uint4*>(grow + p.aux_off + col0 + q * 8) = make_uint4(odu[0], odu[1], odu[2], odu[3]);
     }
+  }
+}
+
+// The SwiGLU-backward epilogue of one row over a 256-column accumulator at tbase: the
+// saved g, u of chunk c + 1 are loaded while chunk c is converted, two chunks per step
+// so both register sets stay named.
+__device__ __forceinline__ void epi_swiglu_bwd_row(const PairParams& p, uint32_t tbase, int row, int colbase) {
+  const bool in = row < p.M;
+  GU32 x0, x1;
+  if (in && colbase < p.Nout) epi_swiglu_bwd_load(p, row, colbase, x0);
+#pragma unroll 1
+  for (int c = 0; c < 8; c += 2) {
+    const int col0 = colbase + c * 32, col1 = col0 + 32;
+    if (col0 >= p.Nout) break;  // warp-uniform
+    if (in && col1 < p.Nout) epi_swiglu_bwd_load(p, row, col1, x1);
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tbase + c * 32, v);
+    tmem_ld_wait();
+    if (in) epi_swiglu_bwd_chunk(p, v, row, col0, x0);
+    if (col1 >= p.Nout) break;
+    if (in && col1 + 32 < p.Nout && c + 2 < 8) epi_swiglu_bwd_load(p, row, col1 + 32, x0);
+    tmem_ld_32x32b_x32(tbase + (c + 1) * 32, v);
+    tmem_ld_wait();
+    if (in) epi_swiglu_bwd_chunk(p, v, row, col1, x1);
   }
 }
 

@@ -243,7 +243,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
           tmem_ld_wait();
           if (row < p.M) epi_swiglu_fwd_chunk(p, g, u, row, col0);
         }
-      } else if constexpr (EPI == EPI_STORE || EPI == EPI_SWIGLU_BWD) {
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        epi_swiglu_bwd_row(p, tbase, row, nb * C::BN);
+      } else if constexpr (EPI == EPI_STORE) {
 #pragma unroll 1
         for (int c = 0; c < C::BN / 32; ++c) {
           const int col0 = nb * C::BN + c * 32;
@@ -251,10 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
           uint32_t v[32];
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (row < p.M) {
-            if constexpr (EPI == EPI_SWIGLU_BWD) epi_swiglu_bwd_chunk(p, v, row, col0);
-            else epi_store_chunk(p, v, row, col0);
-          }
+          if (row < p.M) epi_store_chunk(p, v, row, col0);
         }
       } else if constexpr (EPI == EPI_CE_LSE) {
         float m = -INFINITY, sum = 0.0f;

@@ -250,6 +250,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
             tmem_ld_wait();
             if (row < p.M) epi_swiglu_fwd_chunk(p, g, u, row, col0);
           }
+        } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+          epi_swiglu_bwd_row(p, tbase, row, nb * C::BN);
         } else {
 #pragma unroll 1
           for (int c = 0; c < C::BN / 32; ++c) {
@@ -258,10 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
             uint32_t v[32];
             tmem_ld_32x32b_x32(tbase + c * 32, v);
             tmem_ld_wait();
-            if (row < p.M) {
-              if constexpr (EPI == EPI_SWIGLU_BWD) epi_swiglu_bwd_chunk(p, v, row, col0);
-              else epi_store_chunk(p, v, row, col0);
-            }
+            if (row < p.M) epi_store_chunk(p, v, row, col0);
           }
         }
         tc_fence_before();
