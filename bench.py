@@ -256,7 +256,7 @@ def traffic_record():
 def source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "dequant.cuh", "ptx.cuh"):
+    for f in ("gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "dequant.cuh", "ptx.cuh", "lora_api.cu"):
         with open(os.path.join(ROOT, "qlora_linear_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
