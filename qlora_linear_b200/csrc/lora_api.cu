@@ -354,9 +354,12 @@ lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CU
   const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
+  // the raster group counts tiles; 512-row tiles take half as many for the same rows
+  PairParams q = p;
+  q.group_m = p.group_m > 1 ? p.group_m / 2 : 1;
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_q_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, c, e, f, p);
+    lora_gemm_q_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, c, e, f, q);
   }
   count_launch();
   return last_launch();
