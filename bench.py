@@ -4,7 +4,7 @@ One step = forward and backward of every projection of the workload (default: th
 Llama-8B MLP projections gate, up and down at M = 16384 tokens, r = 16, bf16 weight),
 with inputs resident in device memory.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|qkv|mlp|ce] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|c4s|qkv|mlp|ce] [--impl ours|reference]
 
 Multi-GPU (one process per GPU under torch.distributed.run): data parallel over tokens,
 every rank runs the full per-rank workload (weak scaling) and the adapter gradients dA
@@ -35,6 +35,8 @@ def workload(name: str):
     if name == "mlp":
         blk = MlpCase("mlp_llama8b", 16384, 4096, 14336, 16, 32.0, "bf16", 7000)
         cases = [blk.gate_up_case(), blk.down_case()]
+    elif name == "c4s":
+        cases = [c for c in CONFIGS["c4"] if c.M == 512 and c.r == 16 and c.fmt == "bf16"]
     elif name == "ce":
         # the LM head as a projection: M tokens, K = D, N = V (no adapter; r only sizes nothing)
         from synth import LoraCase
@@ -47,6 +49,8 @@ def workload(name: str):
               "M=16384, r=16, alpha=32, bf16 weight",
         "c3": "QLoRA 4-bit blockwise weight K=4096 N=14336 (16-level codebook, fp16 absmax per 64), "
               "M=8192, r=16, alpha=32",
+        "c4s": "rank-sweep shapes at the smallest batch: M=512, K=N=8192 and K=8192 N=28672, r=16, alpha=32, "
+               "bf16 weight (the most weight-heavy cases; L2 flushed before every step)",
         "ce": "cross-entropy over the Llama-3 LM head (V=128256, D=4096), M=16384 tokens, backward in "
               "16384-column vocabulary slices, bf16 head, no [M, V] logits",
         "mlp": "Llama-8B feed-forward block (D=4096, I=14336) with LoRA on gate, up and down and SwiGLU, "
@@ -67,6 +71,14 @@ def case_flops(c) -> float:
     """Algorithmic FLOPs of one forward + backward: 4MNK + 6Mr(N+K) per projection
     (a grouped case sums this over its projections: 4MNK + 6Mr(N + G·K))."""
     return 4.0 * c.M * c.N * c.K + 6.0 * c.M * c.r * (c.N + c.G * c.K)
+
+
+def case_bytes(c) -> float:
+    """HBM floor of one forward + backward: the frozen weight read twice (bf16 2·NK·2,
+    4-bit 2·(NK/2 + NK/32), 8-bit 2·(NK + 4N)) plus X, dY and XA read and Y, dX, dA, dB
+    written once, 2·(3MK + 2MN) + 4Mr."""
+    w = {"bf16": 2 * c.N * c.K, "block4": c.N * c.K / 2 + c.N * c.K / 32}.get(c.fmt, c.N * c.K + 4 * c.N)
+    return 2.0 * w + 2.0 * (3 * c.M * c.K + 2 * c.M * c.N) + 4.0 * c.M * c.r
 
 
 def gemm_flops(c) -> tuple[float, float]:
@@ -626,10 +638,19 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = args.workload == "c4s"  # working set near the L2 size: flush it before every step
+    if flush:
+        flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks.mark("t_start")
     e0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        if flush:
+            flush_buf.fill_(i & 0xFF)  # outside the step's events
+            ev[i][0].record(stream)
         step()
+        if flush:
+            ev[i][1].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     clocks.mark("t_end")
@@ -639,7 +660,7 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     fwd_ms, fwd_n = q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
     bwd_ms, bwd_n = q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = (sum(a.elapsed_time(b) for a, b in ev) if flush else e0.elapsed_time(e1)) / args.steps
     if world > 1:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -692,6 +713,11 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     elif world == 1 and any(c.rows is not None for c in cases):
         separate = time_separate(args, cases, data, dev)
 
+    # ---- forward and backward timed on their own (single-projection workloads)
+    split = None
+    if isinstance(ws, LinearSet):
+        split = time_split(args, ws, stream)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -714,7 +740,8 @@ def run_ours(args, cases, desc, rank, world, local_rank):
             "config": {"workload": desc, "tokens_per_rank_per_step": tokens_step,
                        "global_batch_tokens": tokens_step * world, "r": cases[0].r,
                        "projections": [c.name for c in cases], "parallelism": f"dp{world}",
-                       "l2": "inputs larger than L2 (step working set several GB >> 126 MB)"},
+                       "l2": ("L2 flushed (512 MB written) before every timed step, outside its events" if flush
+                              else "inputs larger than L2 (step working set several GB >> 126 MB)")},
             "tokens_per_s": world * tokens_step / (ms * 1e-3),
             "pct_peak_burst": value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
             "pct_peak_sustained": value / world / peak_sust,
@@ -724,6 +751,13 @@ def run_ours(args, cases, desc, rank, world, local_rank):
         }
         if separate is not None:
             line["separate_layers"] = separate
+        if split is not None:
+            line["split"] = split
+        if isinstance(ws, LinearSet):
+            line["algorithmic_gbs"] = world * sum(case_bytes(c) for c in cases) / (ms * 1e-3) / 1e9
+            line["algorithmic_gbs_note"] = ("HBM floor of the step (weights read twice, activations and outputs once) "
+                                            "over its time, against the measured copy bandwidth "
+                                            f"{peaks.get('hbm_gbs', FALLBACK_PEAKS['hbm_gbs'])} GB/s")
         print(json.dumps(line), flush=True)
 
 
@@ -769,6 +803,27 @@ def time_separate(args, cases, data, dev):
     flops_step = sum(case_flops(c) for c in cases)
     return {"ms_per_step": ms, "value": flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "note": "the same projections as separate layers (dX of each written separately, not summed)"}
+
+
+def time_split(args, ws, stream):
+    """Forward alone and backward alone over the step's projections (CUDA events)."""
+    import torch
+
+    res = {}
+    for name in ("fwd", "bwd"):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(3, args.steps // 2)
+        e0.record(stream)
+        for _ in range(n):
+            for layer, (d, o) in zip(ws.layers, ws.data):
+                if name == "fwd":
+                    layer.forward(d["X"], Y=o["Y"], XA=o["XA"])
+                else:
+                    layer.backward(d["dY"], d["X"], o["XA"], out=(o["dX"], o["dA"], o["dB"]))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[name + "_ms"] = e0.elapsed_time(e1) / n
+    return res
 
 
 def run_e2e(args, cases, layers, data, step, world, dev):
@@ -880,7 +935,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "qkv", "mlp", "ce"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "c4s", "qkv", "mlp", "ce"])
     ap.add_argument("--only", default=None, help="run a single projection of the workload (e.g. c2_gate)")
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
