@@ -65,3 +65,28 @@ def test_full_size_parity(lib, case):
     check("dA", host_f64(out["dA"].index_select(1, torch.from_numpy(k_idx).cuda())), dA_s)
     del out
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "block4"])
+def test_large_token_count(lib, fmt):
+    """2^17 tokens through a 1024 x 1024 projection: row offsets, tile counts and the split
+    partials of the token reductions at a size far past the configurations."""
+    from synth import LoraCase
+    case = LoraCase(f"large_M_{fmt}", 131072, 1024, 1024, 16, 32.0, fmt, 4242 + (fmt == "block4"))
+    inp = make_case(case)
+    out = run_layer(lib, inp)
+    rng = np.random.default_rng(case.seed)
+    rows = _sample(rng, case.M)
+    n_idx = _sample(rng, case.N)
+    k_idx = _sample(rng, case.K)
+    W = O.weight_f64(inp)
+    A, B = O.bf16_to_f64(inp["A"]), O.bf16_to_f64(inp["B"])
+    Yr, XAr = O.lora_forward_rows(O.bf16_to_f64(inp["X"][rows]), W, A, B, case.s)
+    dXr = O.lora_backward_rows(O.bf16_to_f64(inp["dY"][rows]), W, A, B, case.s)
+    dB_s, dA_s = O.lora_adapter_grads_sampled(inp["dY"], inp["X"], A, B, case.s, n_idx, k_idx)
+    ridx = torch.from_numpy(rows).cuda()
+    check("Y", host_f64(out["Y"].index_select(0, ridx)), Yr)
+    check("XA", host_f64(out["XA"].index_select(0, ridx)), XAr)
+    check("dX", host_f64(out["dX"].index_select(0, ridx)), dXr)
+    check("dB", host_f64(out["dB"].index_select(0, torch.from_numpy(n_idx).cuda())), dB_s)
+    check("dA", host_f64(out["dA"].index_select(1, torch.from_numpy(k_idx).cuda())), dA_s)
