@@ -141,3 +141,21 @@ def test_w8_full_size(lib, fmt):
     check("dX", host_f64(out["dX"].index_select(0, t)), dXr)
     check("dB", host_f64(out["dB"].index_select(0, torch.from_numpy(n_idx).cuda())), dB_s)
     check("dA", host_f64(out["dA"].index_select(1, torch.from_numpy(k_idx).cuda())), dA_s)
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "block4"])
+def test_lora_dequant_other_formats(lib, fmt):
+    """lora_dequant copies a bf16 weight and expands a 4-bit one exactly like
+    dequant_blockwise4; an output overlapping the stored weight is refused."""
+    case = LoraCase(f"dq_{fmt}", 1, 264, 320, 8, 16.0, fmt, 8500)
+    inp = make_case(case, want=("W",))
+    W, keep = make_weight(lib, inp)
+    out = torch.empty((case.N, case.K), dtype=torch.bfloat16, device="cuda")
+    lib.lora_dequant(W, out)
+    torch.cuda.synchronize()
+    ref = inp["W"] if fmt == "bf16" else O.dequant_blockwise4(inp["codes"], inp["absmax"], inp["codebook"], case.N,
+                                                                case.K)
+    assert np.array_equal(host_bits(out), ref)
+    if fmt == "bf16":
+        with pytest.raises(lib.LoraError):
+            lib.lora_dequant(W, keep[0])
