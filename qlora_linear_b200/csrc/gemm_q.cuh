@@ -313,17 +313,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       }
       return __ldg(p.row_scale + n);
     };
-    // scales are loaded two code fills ahead so no register waits on a fresh global load
+    // Scales are loaded two code fills ahead into named registers: a fill's scale is read
+    // two fills after its load was issued, and the rotation moves a value loaded one fill
+    // earlier, so no instruction waits on a fresh global load.  (An indexed array here
+    // would live in local memory, and storing a just-loaded value there waits for it.)
     auto next_fill = [&](int& t, int& kb) {
       if (++kb == nkb) { kb = 0; t += npairs; }
     };
     int st_t = pair, st_kb = 0;  // the code fill whose scale is loaded next
-    float sq[3] = {0.f, 0.f, 0.f};
-    int sqh = 0;
-    for (int i = 0; i < 2; ++i) {
-      sq[i] = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;
-      next_fill(st_t, st_kb);
-    }
+    float s_n1 = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;  // scale of the next code fill
+    next_fill(st_t, st_kb);
+    float s_n2 = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;  // and of the one after
+    next_fill(st_t, st_kb);
     int stage = 0;
     uint32_t phase = 0;
     for (int t = pair; t < ntiles; t += npairs) {
@@ -332,10 +333,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
         const bool code = kb < nkb;
         float sc = 0.f;
         if (code) {
-          sq[(sqh + 2) % 3] = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;
+          sc = s_n1;
+          s_n1 = s_n2;
+          s_n2 = st_t < ntiles ? scale_at(st_t, st_kb) : 0.f;
           next_fill(st_t, st_kb);
-          sc = sq[sqh];
-          sqh = (sqh + 1) % 3;
         }
         if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
         if (code) {
