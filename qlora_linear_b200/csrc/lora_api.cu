@@ -15,6 +15,7 @@
 #include "lora_linear.h"
 #include "lora_linear_profiling.h"
 #include "lora_linear_testing.h"
+#include "dualproj.cuh"
 #include "elementwise.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_q.cuh"
@@ -106,11 +107,52 @@ Split colproj_split(long long M, long long Kout) {
   return make_split(cdiv(Kout, SK_BM), cdiv(M, SK_BK));
 }
 
+// Blocking of the one-pass dY·B / dYᵀ·XA kernel: a × b blocks of row_tiles × col_tiles
+// tiles, one CTA per SM (its shared memory), at most one wave.  The cost model counts
+// the slowest block's bytes at the rate of an even share of HBM (below ~136 CTAs a CTA
+// cannot pull more than that share: measured streaming rates fall off below that) plus
+// the partials written and read back; the two separate passes stream dY twice at ~0.8 of
+// this kernel's rate.
+constexpr int kDualCtas = 148;
+struct DualSplit {
+  bool use = false;
+  int a = 0, b = 0, row_tiles = 0, col_tiles = 0;
+};
+DualSplit dual_split(long long M, long long C, int r) {
+  DualSplit best;
+  if (r > DP_RPAD || M <= 0 || C <= 0) return best;
+  const int ntr = cdiv(M, DP_TR), ntc = cdiv(C, DP_TC);
+  const double tile = double(DP_TR) * DP_TC * 2;
+  double best_cost = 2.4 * ntr * double(ntc) * tile;
+  for (int rt = 1; rt <= DP_MAX_ROW_TILES && rt <= ntr; ++rt) {
+    const int a = cdiv(ntr, rt);
+    if (a > kDualCtas) continue;
+    for (int ct = 1; ct <= ntc; ++ct) {
+      const int b = cdiv(ntc, ct);
+      if (static_cast<long long>(a) * b > kDualCtas) continue;
+      const int n = a * b;
+      const double cost = double(rt) * ct * tile * (n > 136 ? n : 136) + 2.0 * (double(a) * C + double(b) * M) * r * 4;
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = DualSplit{true, a, b, rt, ct};
+      }
+    }
+  }
+  return best;
+}
+size_t dual_part_t_bytes(const DualSplit& d, long long M, int r) {
+  return align256(static_cast<size_t>(d.b) * M * r * 4);
+}
+size_t dual_part_bytes(const DualSplit& d, long long M, long long C, int r) {
+  return d.use ? dual_part_t_bytes(d, M, r) + align256(static_cast<size_t>(d.a) * C * r * 4) : 0;
+}
+
 struct WsLayout {
   size_t skinny_off, part_off, total;
 };
-WsLayout ws_layout(long long M, long long N, long long K, int r) {
+WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg) {
   WsLayout w;
+  const int r = nseg * r1;
   w.skinny_off = kStatusBytes;
   const size_t skinny = align256(static_cast<size_t>(M) * r * 2);
   w.part_off = w.skinny_off + skinny;
@@ -120,6 +162,7 @@ WsLayout ws_layout(long long M, long long N, long long K, int r) {
   upd(static_cast<size_t>(rowproj_split(M, N).splits) * M * r * 4);  // dY·B
   upd(static_cast<size_t>(colproj_split(M, N).splits) * N * r * 4);  // dB
   upd(static_cast<size_t>(colproj_split(M, K).splits) * K * r * 4);  // dA
+  upd(dual_part_bytes(dual_split(M, N, r1), M, N, r1));              // dY·B and dYᵀ·XA in one pass
   w.total = w.part_off + align256(part);
   return w;
 }
@@ -156,6 +199,7 @@ lora_status_t dev_info(DevInfo** out) {
     SET_GEMM_Q(WF_INT8)
     SET_GEMM_Q(WF_FP8)
 #undef SET_GEMM_Q
+    SET_SMEM(dualproj_kernel, dual_smem_bytes());
     SET_SMEM((lora_gemm_pair_kernel<false, EPI_CE_LSE>), (PairCfg<false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<false, EPI_CE_DLOGITS>), (PairCfg<false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<true, EPI_ACC_F32>), (PairCfg<true>::SMEM_BYTES));
@@ -198,10 +242,12 @@ lora_status_t get_encode() {
 }
 
 // Row-major [rows][inner] matrix with row pitch = inner * elem bytes.
+// pitch_elems = 0: rows are packed (pitch = inner).
 lora_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
-                      uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+                      uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw,
+                      uint64_t pitch_elems = 0) {
   cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+  cuuint64_t strides[1] = {(pitch_elems ? pitch_elems : inner) * static_cast<uint64_t>(elem_bytes)};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
@@ -302,6 +348,22 @@ lora_status_t launch_colproj(const __nv_bfloat16* P, int ldp, const __nv_bfloat1
   else
     colproj_kernel<128><<<grid, SK_THREADS, colproj_smem_bytes<128>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
                                                                              sp.tiles_per_split);
+  count_launch();
+  return last_launch();
+}
+
+// partT [d.b][M][r] = dY·B summed per column block, partD [d.a][C][r] = dYᵀ·XA summed per
+// row block, for dY with row pitch ldp, B [C][r] and XA with row pitch ldr.
+lora_status_t launch_dual(const __nv_bfloat16* dY, long long ldp, const __nv_bfloat16* B, const __nv_bfloat16* XA,
+                          long long ldr, long long M, long long C, int r, const DualSplit& d, float* partT,
+                          float* partD, uint32_t* status, cudaStream_t st) {
+  CUtensorMap tp, tq, tr;
+  TRY(tmap_2d(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dY, C, M, 64, DP_TR, CU_TENSOR_MAP_SWIZZLE_128B, ldp));
+  TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, r, C, DP_RPAD, DP_TC, CU_TENSOR_MAP_SWIZZLE_NONE));
+  TRY(tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, XA, r, M, DP_RPAD, DP_TR, CU_TENSOR_MAP_SWIZZLE_32B, ldr));
+  const DualParams dp{partT, partD, static_cast<int>(M), static_cast<int>(C), r, d.row_tiles, d.col_tiles, status,
+                      wait_limit_ns()};
+  dualproj_kernel<<<dim3(d.a, d.b), DP_THREADS, dual_smem_bytes(), st>>>(tp, tq, tr, dp);
   count_launch();
   return last_launch();
 }
@@ -499,7 +561,8 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
 // ---------------------------------------------------------------- backward core
 lora_status_t backward_core(const void* dY, const void* X, const void* XA, long long M, const lora_weight_t* W,
                             const Segs& sg, const void* A, const void* B, int r, float s, void* dX, void* dA,
-                            void* dB, __nv_bfloat16* sdYB, float* part, uint32_t* status, cudaStream_t st) {
+                            void* dB, __nv_bfloat16* sdYB, float* part, size_t part_cap, uint32_t* status,
+                            cudaStream_t st) {
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
   TRY(get_encode());
@@ -514,18 +577,24 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
   for (int g = 0; g < sg.n; ++g) {
     const int rows = static_cast<int>(sg.rows[g]);
     const long long o = sg.off[g];
+    auto* dBg = static_cast<__nv_bfloat16*>(dB) + o * r;
+    const DualSplit ds = dual_split(M, rows, r);
+    if (ds.use && dual_part_bytes(ds, M, rows, r) <= part_cap) {
+      // one pass over dY_g for s·dY_g·B_g (columns [g·r, g·r + r) of s·dY·B) and dB_g = s·dY_gᵀ·XA_g
+      float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
+      TRY(launch_dual(dYb + o, N, Bb + o * r, XAb + g * r, rt, M, rows, r, ds, part, partD, status, st));
+      TRY(finalize_rows(part, ds.b, M, r, rt, s, nullptr, sdYB + g * r, st));
+      TRY(finalize_cols(partD, ds.a, rows, r, s, false, dBg, st));
+      continue;
+    }
     // s·dY_g·B_g -> columns [g·r, g·r + r) of s·dY·B
-    const Split sp = rowproj_split(M, rows);
+    Split sp = rowproj_split(M, rows);
     TRY(launch_rowproj<true>(dYb + o, Ni, Bb + o * r, part, Mi, rows, r, sp, st));
     TRY(finalize_rows(part, sp.splits, M, r, rt, s, nullptr, sdYB + g * r, st));
-  }
-  for (int g = 0; g < sg.n; ++g) {
-    const int rows = static_cast<int>(sg.rows[g]);
-    const long long o = sg.off[g];
     // dB_g = s·dY_gᵀ·XA_g
-    const Split sp = colproj_split(M, rows);
+    sp = colproj_split(M, rows);
     TRY(launch_colproj(dYb + o, Ni, XAb + g * r, rt, part, Mi, rows, r, sp, st));
-    TRY(finalize_cols(part, sp.splits, rows, r, s, false, static_cast<__nv_bfloat16*>(dB) + o * r, st));
+    TRY(finalize_cols(part, sp.splits, rows, r, s, false, dBg, st));
   }
   if (dX) {
     // dX = dY·W + (s·dY·B)·A with the LoRA fill over all G·r ranks
@@ -564,7 +633,7 @@ lora_status_t fwd_entry(const void* X, int64_t M, const lora_weight_t* W, const 
   TRY(check_ptr(X));
   TRY(check_ptr(Y));
   TRY(check_ptr(XA));
-  const WsLayout wl = ws_layout(M, W->N, W->K, sg.n * r);
+  const WsLayout wl = ws_layout(M, W->N, W->K, r, sg.n);
   if (!workspace) return LORA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
   if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
@@ -593,14 +662,14 @@ lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M
   TRY(check_ptr(X));
   TRY(check_ptr(XA));
   if (dX && !aligned16(dX)) return LORA_ERR_ALIGNMENT;
-  const WsLayout wl = ws_layout(M, N, K, rt);
+  const WsLayout wl = ws_layout(M, N, K, r, sg.n);
   if (!workspace) return LORA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
   if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return backward_core(dY, X, XA, M, W, sg, A, B, r, s, dX, dA, dB,
                        reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off), reinterpret_cast<float*>(ws + wl.part_off),
-                       reinterpret_cast<uint32_t*>(ws), st);
+                       wl.total - wl.part_off, reinterpret_cast<uint32_t*>(ws), st);
 }
 
 // ---------------------------------------------------------------- feed-forward block
@@ -618,6 +687,8 @@ WsLayout mlp_ws_layout(long long M, long long D, long long I, int r) {
   upd(static_cast<size_t>(colproj_split(M, D).splits) * D * r * 4);      // dB_d
   upd(static_cast<size_t>(colproj_split(M, I).splits) * I * r * 4);      // dA_d, dB_g, dB_u
   upd(static_cast<size_t>(colproj_split(M, D).splits) * D * 2 * r * 4);  // [dA_g; dA_u]
+  upd(dual_part_bytes(dual_split(M, D, r), M, D, r));                    // dZ·B_d and dZᵀ·(H·A_dᵀ)
+  upd(dual_part_bytes(dual_split(M, I, r), M, I, r));                    // dG·B_g and dGᵀ·XA_g (and the up half)
   w.total = w.part_off + align256(part);
   return w;
 }
@@ -686,21 +757,33 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
 lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const void* H, const void* XAgu,
                                 const void* XAd, long long M, const lora_mlp_t* m, int r, float s, void* dX,
                                 void* dAgu, void* dBgu, void* dAd, void* dBd, __nv_bfloat16* skinny, float* part,
-                                uint32_t* status, cudaStream_t st) {
+                                size_t part_cap, uint32_t* status, cudaStream_t st) {
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
   TRY(get_encode());
   const long long D = m->gate_up.K, I = m->down.K;
   const int Mi = static_cast<int>(M), Di = static_cast<int>(D), Ii = static_cast<int>(I);
   const auto* dZb = static_cast<const __nv_bfloat16*>(dZ);
-  // s·dZ·B_d
-  Split sp = rowproj_split(M, D);
-  TRY(launch_rowproj<true>(dZb, Di, static_cast<const __nv_bfloat16*>(m->B_down), part, Mi, Di, r, sp, st));
-  TRY(finalize_rows(part, sp.splits, M, r, r, s, nullptr, skinny, st));
-  // dB_d = s·dZᵀ·(H·A_dᵀ)
-  sp = colproj_split(M, D);
-  TRY(launch_colproj(dZb, Di, static_cast<const __nv_bfloat16*>(XAd), r, part, Mi, Di, r, sp, st));
-  TRY(finalize_cols(part, sp.splits, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
+  const auto* Bd = static_cast<const __nv_bfloat16*>(m->B_down);
+  const auto* XAdb = static_cast<const __nv_bfloat16*>(XAd);
+  Split sp;
+  const DualSplit ds = dual_split(M, D, r);
+  if (ds.use && dual_part_bytes(ds, M, D, r) <= part_cap) {
+    // one pass over dZ for s·dZ·B_d and dB_d = s·dZᵀ·(H·A_dᵀ)
+    float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
+    TRY(launch_dual(dZb, D, Bd, XAdb, r, M, D, r, ds, part, partD, status, st));
+    TRY(finalize_rows(part, ds.b, M, r, r, s, nullptr, skinny, st));
+    TRY(finalize_cols(partD, ds.a, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
+  } else {
+    // s·dZ·B_d
+    sp = rowproj_split(M, D);
+    TRY(launch_rowproj<true>(dZb, Di, Bd, part, Mi, Di, r, sp, st));
+    TRY(finalize_rows(part, sp.splits, M, r, r, s, nullptr, skinny, st));
+    // dB_d = s·dZᵀ·(H·A_dᵀ)
+    sp = colproj_split(M, D);
+    TRY(launch_colproj(dZb, Di, XAdb, r, part, Mi, Di, r, sp, st));
+    TRY(finalize_cols(part, sp.splits, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
+  }
   // dH = dZ·W_d + (s·dZ·B_d)·A_d, consumed by the epilogue: GU <- [dG | dU]
   {
     CUtensorMap ta, te;
@@ -718,7 +801,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
   TRY(launch_colproj(static_cast<const __nv_bfloat16*>(H), Ii, skinny, r, part, Mi, Ii, r, sp, st));
   TRY(finalize_cols(part, sp.splits, Ii, r, 1.0f, true, static_cast<__nv_bfloat16*>(dAd), st));
   return backward_core(GU, X, XAgu, M, &m->gate_up, gate_up_segs(I), m->A_gate_up, m->B_gate_up, r, s, dX, dAgu,
-                       dBgu, skinny, part, status, st);
+                       dBgu, skinny, part, part_cap, status, st);
 }
 
 lora_status_t mlp_ws_check(long long M, const lora_mlp_t* m, int r, void* workspace, size_t ws_bytes) {
@@ -769,7 +852,7 @@ size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K, int32_t r, int32_t n
   if (nseg < 1 || nseg > LORA_MAX_SEGMENTS || nseg * r > 128) return 0;
   if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3) return 0;
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 30)) return 0;
-  return ws_layout(M, N, K, nseg * r).total;
+  return ws_layout(M, N, K, r, nseg).total;
 }
 
 }  // namespace
@@ -887,7 +970,8 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return mlp_backward_core(dZ, X, GU, H, XA_gate_up, XA_down, M, mlp, r, s, dX, dA_gate_up, dB_gate_up, dA_down,
                            dB_down, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
-                           reinterpret_cast<float*>(ws + wl.part_off), reinterpret_cast<uint32_t*>(ws), st);
+                           reinterpret_cast<float*>(ws + wl.part_off), wl.total - wl.part_off,
+                           reinterpret_cast<uint32_t*>(ws), st);
 }
 
 size_t lora_ce_workspace_bytes(int64_t M, int64_t D, int64_t V, int64_t chunk) {

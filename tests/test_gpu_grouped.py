@@ -45,6 +45,8 @@ GROUPS = [
     (129, [768, 256, 256, 256], 136, 8, "bf16"),
     (300, [512, 256, 256], 192, 32, "block4"),
     (64, [256, 8], 64, 40, "bf16"),
+    # large enough for the one-pass dY·B / dYᵀ·XA kernel on every segment, the last ragged
+    (3000, [1024, 512, 776], 136, 8, "bf16"),
 ]
 
 
