@@ -37,6 +37,11 @@ struct PairParams {
   float* acc32;            // EPI_ACC_F32: [M, Nout] fp32 running sum
   int acc_mode;            // EPI_ACC_F32: bit 0 add the running sum, bit 1 write bf16 to out instead
   __nv_bfloat16* out;  // [M, Nout] row-major
+  // Split reduction (EPI_STORE only): ksplit > 1 cuts the fills of every output tile into
+  // ksplit consecutive ranges, each a work unit of its own whose fp32 accumulator goes to
+  // kpart [ksplit][M][Nout] instead of out; splitk_finalize_kernel sums them in order.
+  int ksplit;          // 1: no split
+  float* kpart;
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
   // quantized weights only
@@ -85,7 +90,58 @@ __device__ __forceinline__ void pair_tile_coords(int t, int num_m, int num_n, in
   nb = within / gm;
 }
 
+// Work unit u of a launch: output tile u % ntiles, split u / ntiles, which covers fills
+// [kb0, kb1) of the nkb over the reduction (and, for split 0, the LoRA fills after them).
+__device__ __forceinline__ void unit_split(int u, int ntiles, int nkb, int ksplit, int& t, int& j, int& kb0, int& kb1) {
+  if (ksplit == 1) {
+    t = u;
+    j = 0;
+    kb0 = 0;
+    kb1 = nkb;
+    return;
+  }
+  t = u % ntiles;
+  j = u / ntiles;
+  kb0 = static_cast<int>(static_cast<long long>(j) * nkb / ksplit);
+  kb1 = static_cast<int>(static_cast<long long>(j + 1) * nkb / ksplit);
+}
+
 // ---------------------------------------------------------------- epilogue pieces
+// 32 accumulator columns of one row to the fp32 partials of split j.
+__device__ __forceinline__ void epi_part_chunk(const PairParams& p, const uint32_t (&v)[32], int j, int row, int col0) {
+  float* prow = p.kpart + (static_cast<size_t>(j) * p.M + row) * p.Nout;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < p.Nout) {
+      float4* d = reinterpret_cast<float4*>(prow + col0 + q * 8);
+      d[0] = make_float4(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]), __uint_as_float(v[q * 8 + 2]),
+                         __uint_as_float(v[q * 8 + 3]));
+      d[1] = make_float4(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]), __uint_as_float(v[q * 8 + 6]),
+                         __uint_as_float(v[q * 8 + 7]));
+    }
+  }
+}
+
+// out[i] = bf16(Σ_j part[j][i]) over n = M·Nout elements (n % 8 == 0), the splits added in
+// order 0, 1, ... so the result does not depend on which unit finished first.
+__global__ void splitk_finalize_kernel(const float* __restrict__ part, int ksplit, size_t n,
+                                       __nv_bfloat16* __restrict__ out) {
+  const size_t groups = n / 8;
+  for (size_t g = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
+       g += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(part) + 2 * g;
+    float4 a = src[0], b = src[1];
+    for (int j = 1; j < ksplit; ++j) {
+      const float4* sj = reinterpret_cast<const float4*>(part + static_cast<size_t>(j) * n) + 2 * g;
+      const float4 c = sj[0], d = sj[1];
+      a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
+      b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
+    }
+    *reinterpret_cast<uint4*>(out + 8 * g) =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
 // 32 accumulator columns of one row to bf16 out[row, col0 ..].
 __device__ __forceinline__ void epi_store_chunk(const PairParams& p, const uint32_t (&v)[32], int row, int col0) {
   __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;

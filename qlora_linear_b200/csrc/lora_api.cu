@@ -147,10 +147,49 @@ size_t dual_part_bytes(const DualSplit& d, long long M, long long C, int r) {
   return d.use ? dual_part_t_bytes(d, M, r) + align256(static_cast<size_t>(d.a) * C * r * 4) : 0;
 }
 
+// Splits of a GEMM's reduction.  When an output has fewer tiles than the GPU has CTA
+// pairs, each tile's fills are cut into S consecutive ranges computed by different pairs
+// into fp32 partials, which a second kernel adds in split order (deterministic).  The
+// choice is a pure function of the sizes and the weight's format (its tile shape), made
+// against a fixed 74 pairs, so the workspace size follows from the sizes alone.  Cost of
+// S: the waves of S-way units times the fills per unit at the kernel's per-pair rate,
+// plus the partials written and read back and the finalize launch; a split must save
+// at least a tenth of the unsplit time.
+constexpr int kGemmPairs = 74;
+int gemm_ksplit(long long M, long long Nout, long long Kred, bool quantized) {
+  if (M <= 0 || Nout <= 0 || Kred <= 0) return 1;
+  const int bm = quantized ? 512 : 256, bk = quantized ? 64 : 128;
+  const long long tiles = static_cast<long long>(cdiv(M, bm)) * cdiv(Nout, 256);
+  if (tiles >= kGemmPairs) return 1;
+  const int nkb = cdiv(Kred, bk);
+  const double fill_s = 2.0 * bm * 256 * bk / ((quantized ? 1.0e15 : 1.5e15) / kGemmPairs);
+  auto cost = [&](int S) {
+    const long long waves = (tiles * S + kGemmPairs - 1) / kGemmPairs;
+    double c = double(waves) * cdiv(nkb, S) * fill_s;
+    if (S > 1) c += double(M) * Nout * (8.0 * S + 2.0) / 5.0e12 + 4.0e-6;
+    return c;
+  };
+  const double c1 = cost(1);
+  int best = 1;
+  double bc = 0.9 * c1;
+  for (int S = 2; S <= 4 && nkb / S >= 8; ++S) {
+    const double c = cost(S);
+    if (c < bc) {
+      best = S;
+      bc = c;
+    }
+  }
+  return best;
+}
+size_t gemm_split_bytes(long long M, long long Nout, long long Kred, bool quantized) {
+  const int S = gemm_ksplit(M, Nout, Kred, quantized);
+  return S > 1 ? static_cast<size_t>(S) * M * Nout * 4 : 0;
+}
+
 struct WsLayout {
   size_t skinny_off, part_off, total;
 };
-WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg) {
+WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg, bool quantized) {
   WsLayout w;
   const int r = nseg * r1;
   w.skinny_off = kStatusBytes;
@@ -163,6 +202,8 @@ WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg) {
   upd(static_cast<size_t>(colproj_split(M, N).splits) * N * r * 4);  // dB
   upd(static_cast<size_t>(colproj_split(M, K).splits) * K * r * 4);  // dA
   upd(dual_part_bytes(dual_split(M, N, r1), M, N, r1));              // dY·B and dYᵀ·XA in one pass
+  upd(gemm_split_bytes(M, N, K, quantized));                         // Y GEMM split partials
+  upd(gemm_split_bytes(M, K, N, quantized));                         // dX GEMM split partials
   w.total = w.part_off + align256(part);
   return w;
 }
@@ -392,7 +433,7 @@ template <bool B_MN, int EPI>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
                           const PairParams& p, int sms, cudaStream_t st) {
   using C = PairCfg<B_MN>;
-  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS) * p.ksplit;
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
@@ -413,7 +454,7 @@ template <bool B_MN, int WF, int EPI>
 lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CUtensorMap& e, const CUtensorMap& f,
                             const PairParams& p, int sms, cudaStream_t st) {
   using C = QCfg<B_MN, WF>;
-  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS) * p.ksplit;
   const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   // the raster group counts tiles; 512-row tiles take half as many for the same rows
@@ -514,6 +555,8 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   p.Kred = static_cast<int>(Kred);
   p.r = r;
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.ksplit = 1;
+  p.kpart = nullptr;
   p.status = status;
   p.wait_ns = wait_limit_ns();
   p.group_m = group_m_default();
@@ -531,12 +574,32 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   return p;
 }
 
+// A split reduction for the plain store epilogue when the size calls for one and its
+// partials fit in the caller's part region (callers without room keep one unit per tile).
+void set_ksplit(PairParams& p, const lora_weight_t* W, float* part, size_t part_cap) {
+  const bool q = W->fmt != LORA_W_BF16;
+  const int S = gemm_ksplit(p.M, p.Nout, p.Kred, q);
+  if (S > 1 && part && gemm_split_bytes(p.M, p.Nout, p.Kred, q) <= part_cap) {
+    p.ksplit = S;
+    p.kpart = part;
+  }
+}
+
+// out = Σ over the splits of the partials, in split order (nothing to do without a split).
+lora_status_t finalize_ksplit(const PairParams& p, cudaStream_t st) {
+  if (p.ksplit <= 1) return LORA_OK;
+  const size_t n = static_cast<size_t>(p.M) * p.Nout;
+  splitk_finalize_kernel<<<finalize_grid(n / 8), 256, 0, st>>>(p.kpart, p.ksplit, n, p.out);
+  count_launch();
+  return last_launch();
+}
+
 // ---------------------------------------------------------------- forward core
 // XA = X·Aᵀ for all segments at once (rank G·r), then Y = X·Wᵀ + s·XA_g·B_gᵀ with the
 // LoRA fill of each output tile taking its segment's columns of s·XA.
 lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, const Segs& sg, const void* A,
                            const void* B, int r, float s, void* Y, void* XA, __nv_bfloat16* sXA, float* part,
-                           uint32_t* status, cudaStream_t st) {
+                           size_t part_cap, uint32_t* status, cudaStream_t st) {
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
   TRY(get_encode());
@@ -555,7 +618,9 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   const FSpec tf{B, static_cast<uint64_t>(r), static_cast<uint64_t>(N)};
   PairParams p = gemm_params(M, N, K, r, Y, status, W);
   set_segments(p, sg, r);
-  return launch_gemm_w<false, EPI_STORE>(W, ta, te, tf, p, dev->sms, st);
+  set_ksplit(p, W, part, part_cap);
+  TRY((launch_gemm_w<false, EPI_STORE>(W, ta, te, tf, p, dev->sms, st)));
+  return finalize_ksplit(p, st);
 }
 
 // ---------------------------------------------------------------- backward core
@@ -603,7 +668,9 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     TRY(tmap_bf16(&te, sdYB, rt, M, kBoxX, kBoxY));
     const FSpec tf{A, static_cast<uint64_t>(K), static_cast<uint64_t>(rt)};
     PairParams p = gemm_params(M, K, N, rt, dX, status, W);
+    set_ksplit(p, W, part, part_cap);
     TRY((launch_gemm_w<true, EPI_STORE>(W, ta, te, tf, p, dev->sms, st)));
+    TRY(finalize_ksplit(p, st));
   }
   // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
   const Split sp = colproj_split(M, K);
@@ -633,14 +700,14 @@ lora_status_t fwd_entry(const void* X, int64_t M, const lora_weight_t* W, const 
   TRY(check_ptr(X));
   TRY(check_ptr(Y));
   TRY(check_ptr(XA));
-  const WsLayout wl = ws_layout(M, W->N, W->K, r, sg.n);
+  const WsLayout wl = ws_layout(M, W->N, W->K, r, sg.n, W->fmt != LORA_W_BF16);
   if (!workspace) return LORA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
   if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return forward_core(X, M, W, sg, A, B, r, s, Y, XA, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
-                      reinterpret_cast<float*>(ws + wl.part_off), reinterpret_cast<uint32_t*>(ws),
-                      static_cast<cudaStream_t>(stream));
+                      reinterpret_cast<float*>(ws + wl.part_off), wl.total - wl.part_off,
+                      reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
@@ -662,7 +729,7 @@ lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M
   TRY(check_ptr(X));
   TRY(check_ptr(XA));
   if (dX && !aligned16(dX)) return LORA_ERR_ALIGNMENT;
-  const WsLayout wl = ws_layout(M, N, K, r, sg.n);
+  const WsLayout wl = ws_layout(M, N, K, r, sg.n, W->fmt != LORA_W_BF16);
   if (!workspace) return LORA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
   if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
@@ -749,7 +816,7 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
   Segs one;
   one.rows[0] = D;
   one.off[1] = D;
-  return forward_core(H, M, &m->down, one, m->A_down, m->B_down, r, s, Z, XAd, skinny, part, status, st);
+  return forward_core(H, M, &m->down, one, m->A_down, m->B_down, r, s, Z, XAd, skinny, part, 0, status, st);
 }
 
 // Down projection's backward with SwiGLU's derivative in the dH GEMM's epilogue (GU
@@ -852,7 +919,7 @@ size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K, int32_t r, int32_t n
   if (nseg < 1 || nseg > LORA_MAX_SEGMENTS || nseg * r > 128) return 0;
   if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3) return 0;
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 30)) return 0;
-  return ws_layout(M, N, K, r, nseg).total;
+  return ws_layout(M, N, K, r, nseg, fmt != LORA_W_BF16).total;
 }
 
 }  // namespace
@@ -1180,6 +1247,11 @@ lora_status_t lora_testing_bounded_wait(void* workspace, uint64_t limit_ns, void
   return last_launch();
 }
 
+int32_t lora_testing_gemm_ksplit(int64_t M, int64_t Nout, int64_t Kred, int32_t fmt) {
+  if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3) return 0;
+  return gemm_ksplit(M, Nout, Kred, fmt != LORA_W_BF16);
+}
+
 lora_status_t lora_timing_enable(int32_t on) {
   g_timing_on.store(on != 0);
   return LORA_OK;
@@ -1270,7 +1342,7 @@ lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weigh
   // every scratch byte read below (the split partials, then s·XA) is written earlier in
   // the same call; no status word: an expired device wait ends the kernel silently
   return forward_core(X, M, W, sg, A, B, r, s, Y, XA, reinterpret_cast<__nv_bfloat16*>(scratch + nl.sxa_off),
-                      reinterpret_cast<float*>(scratch + nl.part_off), nullptr, static_cast<cudaStream_t>(stream));
+                      reinterpret_cast<float*>(scratch + nl.part_off), 0, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -127,6 +127,25 @@ def test_workspace_bytes_is_a_pure_function_of_sizes():
     assert q.workspace_bytes(4096, 4096, 4096, 16) < q.workspace_bytes(4096, 4096, 4096, 128)
 
 
+def test_gemm_split_only_for_outputs_that_leave_pairs_idle():
+    k = q.lora_testing_gemm_ksplit
+    B4, I8 = q.LORA_W_BLOCK4, q.LORA_W_INT8
+    # the rank sweep's small batch with quantized weights: 32 output tiles of 512 x 256
+    # for 74 CTA pairs, forward (K = N = 8192) and the dX of the 8192 -> 28672 projection
+    assert k(512, 8192, 8192, B4) == 2 and k(512, 8192, 28672, B4) == 2 and k(512, 8192, 8192, I8) == 2
+    # a wave or more of tiles: no split (112 tiles; bf16 tiles are 256 rows: 64 of them)
+    assert k(512, 28672, 8192, B4) == 1 and k(512, 8192, 8192) == 1
+    assert k(16384, 14336, 4096) == 1 and k(8192, 14336, 4096, B4) == 1 and k(8192, 4096, 14336, B4) == 1
+    # a split needs at least 8 fills per range: the tiny configuration has 4
+    assert k(256, 512, 512) == 1
+    assert 1 <= k(100, 1024, 8192) <= 4 and k(100, 1024, 8192, 9) == 0
+    assert k(300, 2048, 4096, B4) == k(300, 2048, 4096, B4)
+    # the workspace holds the fp32 partials of the split
+    S = k(512, 8192, 8192, B4)
+    assert q.workspace_bytes(512, 8192, 8192, 16, B4) >= 256 + S * 512 * 8192 * 4
+    assert q.workspace_bytes(512, 8192, 8192, 16) < 512 * 8192 * 4
+
+
 def test_grouped_validation():
     from qlora_linear_b200.binding import segments
     lib = q.lib()
