@@ -25,14 +25,15 @@ extern "C" {
 lora_status_t lora_testing_bounded_wait(void* workspace, uint64_t limit_ns, void* stream);
 
 /*
- * Number of ranges the Y or dX GEMM of lora_linear_fwd / lora_linear_bwd cuts its
- * reduction into for an output of M × Nout over a reduction of length Kred, with a
- * weight of format `fmt` (a lora_wfmt_t): 1 for no split, up to 4 when the output has
- * too few tiles to occupy the GPU.  A pure function of its arguments (lora_workspace_bytes
- * includes the split's fp32 partials); 0 for an unknown format.  Lets tests check that a
- * case takes the split path.
+ * Schedule of the Y or dX GEMM of lora_linear_fwd / lora_linear_bwd for an output of
+ * M × Nout over a reduction of length Kred, LoRA rank r (0..128; the rank of the GEMM's
+ * LoRA fill) and a weight of format `fmt` (a lora_wfmt_t): the number of output tiles the
+ * stream-K schedule shares out among the CTA pairs as pieces, 0 when every tile is
+ * computed whole, -1 for an invalid format or rank.  A pure function of its arguments
+ * (lora_workspace_bytes includes the schedule's fp32 slots); lets tests check that a case
+ * takes the stream-K path.
  */
-int32_t lora_testing_gemm_ksplit(int64_t M, int64_t Nout, int64_t Kred, int32_t fmt);
+int32_t lora_testing_gemm_streamk(int64_t M, int64_t Nout, int64_t Kred, int32_t r, int32_t fmt);
 
 #ifdef __cplusplus
 }

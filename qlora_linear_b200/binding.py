@@ -34,7 +34,7 @@ LORA_W_FP8_E4M3 = 3
 EXPORTED = (
     "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
-    "lora_testing_bounded_wait", "lora_testing_gemm_ksplit", "lora_timing_enable", "lora_timing_read",
+    "lora_testing_bounded_wait", "lora_testing_gemm_streamk", "lora_timing_enable", "lora_timing_read",
     "lora_launch_count",
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
     "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
@@ -125,8 +125,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_version.restype = i32
     lib.lora_testing_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
     lib.lora_testing_bounded_wait.restype = i32
-    lib.lora_testing_gemm_ksplit.argtypes = [i64, i64, i64, i32]
-    lib.lora_testing_gemm_ksplit.restype = i32
+    lib.lora_testing_gemm_streamk.argtypes = [i64, i64, i64, i32, i32]
+    lib.lora_testing_gemm_streamk.restype = i32
     lib.lora_timing_enable.argtypes = [i32]
     lib.lora_timing_enable.restype = i32
     lib.lora_timing_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
@@ -270,9 +270,9 @@ def lora_testing_bounded_wait(workspace, limit_ns: int, stream=None) -> int:
     return int(_lib.lora_testing_bounded_wait(_ptr(workspace), int(limit_ns), _stream(stream)))
 
 
-def lora_testing_gemm_ksplit(M: int, Nout: int, Kred: int, fmt: int = LORA_W_BF16) -> int:
-    """Ranges the Y / dX GEMM splits its reduction into for this output and format."""
-    return int(_lib.lora_testing_gemm_ksplit(int(M), int(Nout), int(Kred), int(fmt)))
+def lora_testing_gemm_streamk(M: int, Nout: int, Kred: int, r: int, fmt: int = LORA_W_BF16) -> int:
+    """Output tiles the Y / dX GEMM shares out as stream-K pieces (0: all tiles whole)."""
+    return int(_lib.lora_testing_gemm_streamk(int(M), int(Nout), int(Kred), int(r), int(fmt)))
 
 
 

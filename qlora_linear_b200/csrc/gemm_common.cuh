@@ -37,10 +37,11 @@ struct PairParams {
   float* acc32;            // EPI_ACC_F32: [M, Nout] fp32 running sum
   int acc_mode;            // EPI_ACC_F32: bit 0 add the running sum, bit 1 write bf16 to out instead
   __nv_bfloat16* out;  // [M, Nout] row-major
-  // Split reduction (EPI_STORE only): ksplit > 1 cuts the fills of every output tile into
-  // ksplit consecutive ranges, each a work unit of its own whose fp32 accumulator goes to
-  // kpart [ksplit][M][Nout] instead of out; splitk_finalize_kernel sums them in order.
-  int ksplit;          // 1: no split
+  // Stream-K schedule (EPI_STORE only, see UnitWalk): sk_on != 0 runs the first
+  // sk_dp_tiles tiles whole and cuts the fill sequence of the rest into one range per CTA
+  // pair; pieces of tiles go to the fp32 slots kpart [2 · pairs][tile rows][256].
+  int sk_on;
+  int sk_dp_tiles;
   float* kpart;
   uint32_t* status;    // device status word, may be null
   uint64_t wait_ns;    // bound of every mbarrier wait
@@ -90,55 +91,96 @@ __device__ __forceinline__ void pair_tile_coords(int t, int num_m, int num_n, in
   nb = within / gm;
 }
 
-// Work unit u of a launch: output tile u % ntiles, split u / ntiles, which covers fills
-// [kb0, kb1) of the nkb over the reduction (and, for split 0, the LoRA fills after them).
-__device__ __forceinline__ void unit_split(int u, int ntiles, int nkb, int ksplit, int& t, int& j, int& kb0, int& kb1) {
-  if (ksplit == 1) {
-    t = u;
-    j = 0;
-    kb0 = 0;
-    kb1 = nkb;
-    return;
+// Work units of a launch, walked in the same order by every role of a CTA pair.
+// A unit is fills [f0, f1) of output tile t, out of the tile's L = nkb + n_ext fills (the
+// code fills of the reduction, then the LoRA fills), and either covers the tile whole
+// (slot < 0: the epilogue writes the output) or is a piece whose fp32 accumulator goes to
+// slot `slot` of kpart.
+//   Data-parallel (sk off): pair p takes tiles p, p + P, p + 2P, ... whole.
+//   Stream-K (sk on): pair p takes tiles p, p + P, ... below dp_tiles (a multiple of P)
+//   whole, then range [p·F/P, (p+1)·F/P) of the F = (ntiles − dp_tiles)·L fills of the
+//   remaining tiles laid end to end.  The pair's first piece goes to slot 2p, its last to
+//   slot 2p + 1 (a range inside one tile is a single piece in slot 2p); every range holds
+//   at least one fill, so the pieces of a tile are those of consecutive pairs.
+struct Unit {
+  int t, f0, f1, slot;
+};
+struct UnitWalk {
+  int p, P, ntiles, L, dp_left, k;
+  long long g, g0, g1;
+  bool sk;
+  __device__ __forceinline__ UnitWalk(int p_, int P_, int ntiles_, int L_, bool sk_, int dp_tiles)
+      : p(p_), P(P_), ntiles(ntiles_), L(L_), dp_left(sk_ ? dp_tiles / P_ : 0), k(0), g(0), g0(0), g1(0), sk(sk_) {
+    if (sk) {
+      const long long F = static_cast<long long>(ntiles - dp_tiles) * L;
+      g0 = static_cast<long long>(p) * F / P;
+      g1 = static_cast<long long>(p + 1) * F / P;
+      g = g0;
+    }
   }
-  t = u % ntiles;
-  j = u / ntiles;
-  kb0 = static_cast<int>(static_cast<long long>(j) * nkb / ksplit);
-  kb1 = static_cast<int>(static_cast<long long>(j + 1) * nkb / ksplit);
-}
+  __device__ __forceinline__ bool next(Unit& u) {
+    if (!sk || k < dp_left) {
+      const int t = p + k * P;
+      if (t >= ntiles) return false;
+      ++k;
+      u = Unit{t, 0, L, -1};
+      return true;
+    }
+    if (g >= g1) return false;
+    const long long tr = g / L;
+    const int f0 = static_cast<int>(g - tr * L);
+    const int f1 = static_cast<int>(min(static_cast<long long>(L), f0 + (g1 - g)));
+    const int slot = (f0 == 0 && f1 == L) ? -1 : (g == g0 ? 2 * p : 2 * p + 1);
+    u = Unit{dp_left * P + static_cast<int>(tr), f0, f1, slot};
+    g += f1 - f0;
+    return true;
+  }
+};
 
 // ---------------------------------------------------------------- epilogue pieces
-// 32 accumulator columns of one row to the fp32 partials of split j.
-__device__ __forceinline__ void epi_part_chunk(const PairParams& p, const uint32_t (&v)[32], int j, int row, int col0) {
-  float* prow = p.kpart + (static_cast<size_t>(j) * p.M + row) * p.Nout;
+// 32 accumulator columns of tile-local row lrow, columns [lc0, lc0 + 32), to a stream-K
+// slot (tile-shaped: TILE_ROWS × 256 fp32).
+template <int TILE_ROWS>
+__device__ __forceinline__ void epi_slot_chunk(const PairParams& p, const uint32_t (&v)[32], int slot, int lrow, int lc0) {
+  float* d = p.kpart + (static_cast<size_t>(slot) * TILE_ROWS + lrow) * 256 + lc0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (col0 + q * 8 < p.Nout) {
-      float4* d = reinterpret_cast<float4*>(prow + col0 + q * 8);
-      d[0] = make_float4(__uint_as_float(v[q * 8 + 0]), __uint_as_float(v[q * 8 + 1]), __uint_as_float(v[q * 8 + 2]),
-                         __uint_as_float(v[q * 8 + 3]));
-      d[1] = make_float4(__uint_as_float(v[q * 8 + 4]), __uint_as_float(v[q * 8 + 5]), __uint_as_float(v[q * 8 + 6]),
-                         __uint_as_float(v[q * 8 + 7]));
-    }
-  }
+  for (int q = 0; q < 8; ++q)
+    reinterpret_cast<float4*>(d)[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                  __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
 }
 
-// out[i] = bf16(Σ_j part[j][i]) over n = M·Nout elements (n % 8 == 0), the splits added in
-// order 0, 1, ... so the result does not depend on which unit finished first.
-__global__ void splitk_finalize_kernel(const float* __restrict__ part, int ksplit, size_t n,
-                                       __nv_bfloat16* __restrict__ out) {
-  const size_t groups = n / 8;
-  for (size_t g = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
-       g += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float4* src = reinterpret_cast<const float4*>(part) + 2 * g;
-    float4 a = src[0], b = src[1];
-    for (int j = 1; j < ksplit; ++j) {
-      const float4* sj = reinterpret_cast<const float4*>(part + static_cast<size_t>(j) * n) + 2 * g;
-      const float4 c = sj[0], d = sj[1];
-      a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
-      b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
+// Output tiles that stream-K cut into pieces: block (x, y) handles the tile in which the
+// boundary between pairs x and x + 1 falls (if that boundary is the tile's first), rows
+// [y·TILE_ROWS/gridDim.y, ...) of it, and writes out = bf16(Σ of the tile's pieces) with
+// the pieces added in pair order.
+template <int TILE_ROWS>
+__global__ void streamk_fixup_kernel(const float* __restrict__ kpart, __nv_bfloat16* __restrict__ out, int M, int Nout,
+                                     int num_m, int num_n, int group_m, int dp_tiles, int ntiles, int L, int P) {
+  const int p = blockIdx.x + 1;
+  const long long F = static_cast<long long>(ntiles - dp_tiles) * L;
+  const long long b = static_cast<long long>(p) * F / P;
+  if (b % L == 0) return;  // the boundary falls between two tiles
+  const long long ts = (b / L) * L, te = ts + L;
+  if (static_cast<long long>(p - 1) * F / P > ts) return;  // an earlier boundary lies in this tile
+  int mb, nb;
+  pair_tile_coords(dp_tiles + static_cast<int>(b / L), num_m, num_n, group_m, mb, nb);
+  const int rows = TILE_ROWS / gridDim.y;
+  for (int e = threadIdx.x; e < rows * 32; e += blockDim.x) {
+    const int lr = blockIdx.y * rows + e / 32, lc = (e % 32) * 8;
+    const int row = mb * TILE_ROWS + lr, col = nb * 256 + lc;
+    if (row >= M || col >= Nout) continue;
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int q = p - 1; q < P; ++q) {
+      const long long gq = static_cast<long long>(q) * F / P;
+      if (gq >= te) break;
+      const int slot = gq >= ts ? 2 * q : 2 * q + 1;
+      const float4* src = reinterpret_cast<const float4*>(kpart + (static_cast<size_t>(slot) * TILE_ROWS + lr) * 256 + lc);
+      const float4 x = src[0], y = src[1];
+      a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
+      a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
     }
-    *reinterpret_cast<uint4*>(out + 8 * g) =
-        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * Nout + col) =
+        make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
   }
 }
 

@@ -24,9 +24,9 @@
 // 0b11); both CTAs' epilogue warps arrive on the leader's `tempty` barriers through
 // cluster addresses.  Every wait is bounded.
 //
-// Work units.  A launch walks ntiles · ksplit units; with ksplit > 1 (small outputs that
-// would leave CTA pairs idle) each unit is one consecutive range of a tile's fills, its
-// accumulator stored as fp32 partials, and the LoRA fill belongs to split 0.
+// Work units (UnitWalk, gemm_common.cuh): whole tiles, or under the stream-K schedule
+// (plain store epilogue only) also pieces of tiles, whose fp32 accumulators go to slots
+// that streamk_fixup_kernel adds up.
 //
 // Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
 // warps 2-5 epilogue.
@@ -81,10 +81,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
   const int num_m = (p.M + C::BM - 1) / C::BM;
   const int num_n = (p.Nout + EpiTile<EPI>::COLS - 1) / EpiTile<EPI>::COLS;
   const int ntiles = num_m * num_n;
-  const int ksplit = EPI == EPI_STORE ? p.ksplit : 1;  // only the plain store epilogue splits
-  const int nunits = ntiles * ksplit;
+  const bool sk = EPI == EPI_STORE && p.sk_on != 0;  // only the plain store epilogue runs stream-K
   const int nkb = (p.Kred + C::BK - 1) / C::BK;
   const int n_ext = p.r > 0 ? 1 : 0;         // one fill holds the whole LoRA block (r <= 128)
+  const int tile_fills = nkb + n_ext;        // fills per tile
   const int ext_atoms = p.r > 64 ? 2 : 1;   // 64-wide rank atoms actually loaded
   const WaitCtl wc{abort_flag, p.status, p.wait_ns};
 
@@ -124,17 +124,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
       uint32_t phase = 0;
       long long fills = 0;
       bool ok = true;
-      for (int u = pair; u < nunits && ok; u += npairs) {
-        int t, j, kb0, kb1, mb, nb;
-        unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-        pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+      UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+      Unit un;
+      while (ok && w.next(un)) {
+        int mb, nb;
+        pair_tile_coords(un.t, num_m, num_n, p.group_m, mb, nb);
         const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A
         const int brow = pair_brow<EPI>(nb, rank, p);  // this CTA's rows of the B tile
-        const int nf = kb1 - kb0 + (j == 0 ? n_ext : 0);
-        for (int i = 0; i < nf; ++i) {
+        for (int kb = un.f0; kb < un.f1; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
-          const int kb = kb0 + i;
-          const bool ext = kb >= kb1;
+          const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const uint32_t full_l = mapa_shared(smem_u32(&full[stage]), 0);
@@ -197,17 +196,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = pair; u < nunits && ok; u += npairs) {
-        int t, j, kb0, kb1;
-        unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
+      UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+      Unit un;
+      while (ok && w.next(un)) {
         if (!mbar_wait<true>(smem_u32(&tempty[acc]), acc_phase ^ 1u, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::BN);
-        const int nf = kb1 - kb0 + (j == 0 ? n_ext : 0);
-        for (int i = 0; i < nf; ++i) {
+        for (int kb = un.f0; kb < un.f1; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
           tc_fence_after();
-          const bool ext = kb0 + i >= kb1;
+          const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const int nk = ext ? (p.r + 15) / 16 : C::BK / 16;
@@ -217,7 +215,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
             const uint32_t koff = (k >> 2) * (C::A_BYTES / 2) + (k & 3) * 32;
             const uint64_t ad = sdesc_sw128(sA + koff, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(sB + k * 2048, C::B_BYTES / 2, 1024) : sdesc_sw128(sB + koff, 16, 1024);
-            tc_mma_bf16_pair(d, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+            tc_mma_bf16_pair(d, ad, bd, idesc, (kb > un.f0 || k > 0) ? 1u : 0u);
           }
           tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -236,10 +234,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = pair; u < nunits; u += npairs) {
-      int t, j, kb0, kb1, mb, nb;
-      unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+    UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+    Unit un;
+    while (w.next(un)) {
+      int mb, nb;
+      pair_tile_coords(un.t, num_m, num_n, p.group_m, mb, nb);
       if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, wc)) break;
       tc_fence_after();
       const int row = mb * C::BM + static_cast<int>(rank) * C::HM + quarter * 32 + lane;
@@ -267,7 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
           if (row < p.M) {
-            if (ksplit > 1) epi_part_chunk(p, v, j, row, col0);
+            if (un.slot >= 0) epi_slot_chunk<C::BM>(p, v, un.slot, row - mb * C::BM, c * 32);
             else epi_store_chunk(p, v, row, col0);
           }
         }

@@ -20,8 +20,9 @@
 // has its own full/empty barrier pair, so the next tile's MMAs into the first
 // accumulator start while the epilogue still drains the second.
 //
-// Work units as in lora_gemm_pair_kernel: ntiles · ksplit of them, split j of a tile
-// covering one consecutive range of its code fills (split 0 also the LoRA fills).
+// Work units as in lora_gemm_pair_kernel (UnitWalk): whole tiles, and under the stream-K
+// schedule pieces of tiles, a piece being any consecutive range of the tile's code fills
+// and LoRA fills.
 //
 // Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
 // warps 2-5 epilogue, warps 6-13 dequant, warp 14 forwards the dequant warps' completion
@@ -87,10 +88,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
   const int num_m = (p.M + C::BM - 1) / C::BM;
   const int num_n = (p.Nout + EpiTile<EPI>::COLS - 1) / EpiTile<EPI>::COLS;
   const int ntiles = num_m * num_n;
-  const int ksplit = EPI == EPI_STORE ? p.ksplit : 1;  // only the plain store epilogue splits
-  const int nunits = ntiles * ksplit;
+  const bool sk = EPI == EPI_STORE && p.sk_on != 0;  // only the plain store epilogue runs stream-K
   const int nkb = (p.Kred + C::BK - 1) / C::BK;
   const int n_ext = p.r > 0 ? (p.r + C::ATOM - 1) / C::ATOM : 0;  // 64 ranks per LoRA fill
+  const int tile_fills = nkb + n_ext;  // fills per tile
   const WaitCtl wc{abort_flag, p.status, p.wait_ns};
 
   if (threadIdx.x == 0) {
@@ -132,17 +133,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       uint32_t phase = 0;
       long long fills = 0;
       bool ok = true;
-      for (int u = pair; u < nunits && ok; u += npairs) {
-        int t, j, kb0, kb1, mb, nb;
-        unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-        pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+      UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+      Unit un;
+      while (ok && w.next(un)) {
+        int mb, nb;
+        pair_tile_coords(un.t, num_m, num_n, p.group_m, mb, nb);
         const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A block 0
         const int brow = pair_brow<EPI>(nb, rank, p);
-        const int nf = kb1 - kb0 + (j == 0 ? n_ext : 0);
-        for (int i = 0; i < nf; ++i) {
+        for (int kb = un.f0; kb < un.f1; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
-          const int kb = kb0 + i;
-          const bool ext = kb >= kb1;
+          const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const uint32_t sC = sB + C::B_BYTES;
@@ -161,7 +161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
               else tma_load_2d(sC, &tmC, cb, brow, kb * C::BK);             // 128 B × 64 rows
             }
           } else {
-            const int e = kb - kb1;
+            const int e = kb - nkb;
             int seg = 0;
             while (seg + 1 < p.nseg && nb >= p.seg_end_tile[seg]) ++seg;
             const int e0 = seg * p.e_seg_stride + e * C::ATOM;  // this fill's columns of E
@@ -199,21 +199,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       uint32_t phase = 0;
       uint32_t tphase = 0;  // parity of the accumulator barriers for this tile
       bool ok = true;
-      for (int u = pair; u < nunits && ok; u += npairs) {
-        int t, j, kb0, kb1;
-        unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-        const int nf = kb1 - kb0 + (j == 0 ? n_ext : 0);
-        for (int i = 0; i < nf; ++i) {
+      UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+      Unit un;
+      while (ok && w.next(un)) {
+        for (int kb = un.f0; kb < un.f1; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
           if (!mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
           tc_fence_after();
-          const int kb = kb0 + i;
-          const bool ext = kb >= kb1;
+          const bool ext = kb >= nkb;
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
-          const int nk = ext ? min(C::BK / 16, (p.r - (kb - kb1) * C::ATOM + 15) / 16) : C::BK / 16;
+          const int nk = ext ? min(C::BK / 16, (p.r - (kb - nkb) * C::ATOM + 15) / 16) : C::BK / 16;
           for (int b = 0; b < C::MB; ++b) {
-            if (i == 0) {
+            if (kb == un.f0) {
               // the epilogue must have drained accumulator b of the previous tile
               if (!mbar_wait<true>(smem_u32(&tempty[b]), tphase ^ 1u, wc)) { ok = false; break; }
               tc_fence_after();
@@ -222,7 +220,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
             for (int k = 0; k < nk; ++k) {
               const uint64_t ad = sdesc_sw128(sA + b * C::A_BLOCK_BYTES + k * 32, 16, 1024);
               const uint64_t bd = B_MN ? sdesc_sw128(sB + k * 2048, C::B_BYTES / 2, 1024) : sdesc_sw128(sB + k * 32, 16, 1024);
-              tc_mma_bf16_pair(d, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+              tc_mma_bf16_pair(d, ad, bd, idesc, (kb > un.f0 || k > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
@@ -242,10 +240,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     uint32_t tphase = 0;
     bool ok = true;
-    for (int u = pair; u < nunits && ok; u += npairs) {
-      int t, j, kb0, kb1, mb, nb;
-      unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
+    UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+    Unit un;
+    while (ok && w.next(un)) {
+      int mb, nb;
+      pair_tile_coords(un.t, num_m, num_n, p.group_m, mb, nb);
       for (int b = 0; b < C::MB; ++b) {
         if (!mbar_wait_warp(smem_u32(&tfull[b]), tphase, wc)) { ok = false; break; }
         tc_fence_after();
@@ -274,7 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
             tmem_ld_32x32b_x32(tbase + c * 32, v);
             tmem_ld_wait();
             if (row < p.M) {
-              if (ksplit > 1) epi_part_chunk(p, v, j, row, col0);
+              if (un.slot >= 0) epi_slot_chunk<C::BM>(p, v, un.slot, row - mb * C::BM, c * 32);
               else epi_store_chunk(p, v, row, col0);
             }
           }
@@ -295,11 +294,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = pair; u < nunits && ok; u += npairs) {
-        int t, j, kb0, kb1;
-        unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-        const int nf = kb1 - kb0 + (j == 0 ? n_ext : 0);
-        for (int i = 0; i < nf; ++i) {
+      UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+      Unit un;
+      while (ok && w.next(un)) {
+        for (int kb = un.f0; kb < un.f1; ++kb) {
           if (!mbar_wait(smem_u32(&deql[stage]), phase, wc)) { ok = false; break; }
           mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -319,10 +317,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
     }
     const long long kblocks_w = p.Kw / 64;  // 4-bit scale blocks per weight row
-    // scale for code fill kb of unit u: a fp16 block scale (4-bit) or a fp32 row scale (8-bit)
-    auto scale_at = [&](int u, int kb) -> float {
+    // scale for code fill kb of tile t: a fp16 block scale (4-bit) or a fp32 row scale (8-bit)
+    auto scale_at = [&](int t, int kb) -> float {
       int mb, nb;
-      pair_tile_coords(ksplit == 1 ? u : u % ntiles, num_m, num_n, p.group_m, mb, nb);
+      pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
       const int brow = pair_brow<EPI>(nb, rank, p);
       const long long n = !B_MN ? static_cast<long long>(brow) + row : static_cast<long long>(kb) * C::BK + row;
       if (n >= p.Nw) return 0.0f;
@@ -336,36 +334,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     // two fills after its load was issued, and the rotation moves a value loaded one fill
     // earlier, so no instruction waits on a fresh global load.  (An indexed array here
     // would live in local memory, and storing a just-loaded value there waits for it.)
-    auto first_kb = [&](int u) {
-      return ksplit == 1 ? 0 : static_cast<int>(static_cast<long long>(u / ntiles) * nkb / ksplit);
-    };
-    auto next_fill = [&](int& u, int& kb) {
-      const int kb1 = ksplit == 1 ? nkb : static_cast<int>(static_cast<long long>(u / ntiles + 1) * nkb / ksplit);
-      if (++kb == kb1) {
-        u += npairs;
-        kb = u < nunits ? first_kb(u) : 0;
+    // A second walk of the units tracks the code fill whose scale is loaded next.
+    UnitWalk sw(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+    Unit su;
+    bool s_more = sw.next(su);
+    int s_kb = s_more ? su.f0 : 0;
+    auto skip_ext = [&]() {  // move past LoRA fills (and units made of them only)
+      while (s_more && s_kb >= min(su.f1, nkb)) {
+        s_more = sw.next(su);
+        if (s_more) s_kb = su.f0;
       }
     };
-    int st_u = pair, st_kb = pair < nunits ? first_kb(pair) : 0;  // the code fill whose scale is loaded next
-    float s_n1 = st_u < nunits ? scale_at(st_u, st_kb) : 0.f;  // scale of the next code fill
-    next_fill(st_u, st_kb);
-    float s_n2 = st_u < nunits ? scale_at(st_u, st_kb) : 0.f;  // and of the one after
-    next_fill(st_u, st_kb);
+    auto load_next = [&]() -> float {
+      skip_ext();
+      const float v = s_more ? scale_at(su.t, s_kb) : 0.f;
+      ++s_kb;
+      return v;
+    };
+    float s_n1 = load_next();  // scale of the next code fill
+    float s_n2 = load_next();  // and of the one after
     int stage = 0;
     uint32_t phase = 0;
-    for (int u = pair; u < nunits; u += npairs) {
+    UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
+    Unit un;
+    while (w.next(un)) {
       bool ok = true;
-      int t, j, kb0, kb1;
-      unit_split(u, ntiles, nkb, ksplit, t, j, kb0, kb1);
-      const int nf = kb1 - kb0 + (j == 0 ? n_ext : 0);
-      for (int f = 0; f < nf; ++f) {
-        const bool code = kb0 + f < kb1;
+      for (int kb = un.f0; kb < un.f1; ++kb) {
+        const bool code = kb < nkb;
         float sc = 0.f;
         if (code) {
           sc = s_n1;
           s_n1 = s_n2;
-          s_n2 = st_u < nunits ? scale_at(st_u, st_kb) : 0.f;
-          next_fill(st_u, st_kb);
+          s_n2 = load_next();
         }
         if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
         if (code) {

@@ -147,43 +147,50 @@ size_t dual_part_bytes(const DualSplit& d, long long M, long long C, int r) {
   return d.use ? dual_part_t_bytes(d, M, r) + align256(static_cast<size_t>(d.a) * C * r * 4) : 0;
 }
 
-// Splits of a GEMM's reduction.  When an output has fewer tiles than the GPU has CTA
-// pairs, each tile's fills are cut into S consecutive ranges computed by different pairs
-// into fp32 partials, which a second kernel adds in split order (deterministic).  The
-// choice is a pure function of the sizes and the weight's format (its tile shape), made
-// against a fixed 74 pairs, so the workspace size follows from the sizes alone.  Cost of
-// S: the waves of S-way units times the fills per unit at the kernel's per-pair rate,
-// plus the partials written and read back and the finalize launch; a split must save
-// at least a tenth of the unsplit time.
+// Schedule of a GEMM launch.  Whole tiles round-robin over the CTA pairs leave pairs
+// idle in the last wave when the tile count is not a multiple of the pairs (an output of
+// 1.5 waves runs two full ones).  Stream-K evens that out: every pair first runs the same
+// number of whole tiles (all waves but the last full one), then an equal share of the
+// fills of the remaining tiles, pieces of tiles going to fp32 slots that a second kernel
+// adds in pair order (deterministic).  The choice is a pure function of the sizes, the
+// rank and the weight's format (its tile shape), made against a fixed 74 pairs, so the
+// workspace size follows from the sizes alone.  Cost model: fills per pair at the
+// kernel's per-pair rate (plus three for the extra epilogue of a piece), slots written
+// and read back at 5 TB/s, and the fixup launch; stream-K must save a twentieth.
 constexpr int kGemmPairs = 74;
-int gemm_ksplit(long long M, long long Nout, long long Kred, bool quantized) {
-  if (M <= 0 || Nout <= 0 || Kred <= 0) return 1;
-  const int bm = quantized ? 512 : 256, bk = quantized ? 64 : 128;
-  const long long tiles = static_cast<long long>(cdiv(M, bm)) * cdiv(Nout, 256);
-  if (tiles >= kGemmPairs) return 1;
-  const int nkb = cdiv(Kred, bk);
-  const double fill_s = 2.0 * bm * 256 * bk / ((quantized ? 1.0e15 : 1.5e15) / kGemmPairs);
-  auto cost = [&](int S) {
-    const long long waves = (tiles * S + kGemmPairs - 1) / kGemmPairs;
-    double c = double(waves) * cdiv(nkb, S) * fill_s;
-    if (S > 1) c += double(M) * Nout * (8.0 * S + 2.0) / 5.0e12 + 4.0e-6;
-    return c;
-  };
-  const double c1 = cost(1);
-  int best = 1;
-  double bc = 0.9 * c1;
-  for (int S = 2; S <= 4 && nkb / S >= 8; ++S) {
-    const double c = cost(S);
-    if (c < bc) {
-      best = S;
-      bc = c;
-    }
+struct GemmSched {
+  bool sk = false;
+  int dp_tiles = 0;
+  int tile_rows = 256;
+  int tile_fills = 0;
+};
+GemmSched gemm_sched(long long M, long long Nout, long long Kred, int r, bool quantized) {
+  GemmSched g;
+  g.tile_rows = quantized ? 512 : 256;
+  if (M <= 0 || Nout <= 0 || Kred <= 0) return g;
+  const int bk = quantized ? 64 : 128;
+  const long long tiles = static_cast<long long>(cdiv(M, g.tile_rows)) * cdiv(Nout, 256);
+  const long long L = cdiv(Kred, bk) + (r > 0 ? (quantized ? cdiv(r, 64) : 1) : 0);
+  g.tile_fills = static_cast<int>(L);
+  const int P = kGemmPairs;
+  const long long full = tiles / P;
+  const long long dp = full > 1 ? (full - 1) * P : 0;
+  const long long rest = tiles - dp;
+  if (rest * L < 8LL * P) return g;  // every pair's range must hold at least 8 fills
+  const double fill_s = 2.0 * g.tile_rows * 256 * bk / ((quantized ? 1.0e15 : 1.5e15) / P);
+  const double slot_bytes = double(g.tile_rows) * 256 * 4;
+  const double t_dp = double((tiles + P - 1) / P) * L * fill_s;
+  const double t_sk = (double(dp / P) * L + double((rest * L + P - 1) / P) + 3.0) * fill_s +
+                      2.0 * double(rest + P) * slot_bytes / 5.0e12 + 4.0e-6;
+  if (t_sk < 0.95 * t_dp) {
+    g.sk = true;
+    g.dp_tiles = static_cast<int>(dp);
   }
-  return best;
+  return g;
 }
-size_t gemm_split_bytes(long long M, long long Nout, long long Kred, bool quantized) {
-  const int S = gemm_ksplit(M, Nout, Kred, quantized);
-  return S > 1 ? static_cast<size_t>(S) * M * Nout * 4 : 0;
+size_t gemm_sched_bytes(long long M, long long Nout, long long Kred, int r, bool quantized) {
+  const GemmSched g = gemm_sched(M, Nout, Kred, r, quantized);
+  return g.sk ? static_cast<size_t>(2) * kGemmPairs * g.tile_rows * 256 * 4 : 0;
 }
 
 struct WsLayout {
@@ -202,8 +209,8 @@ WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg, bool
   upd(static_cast<size_t>(colproj_split(M, N).splits) * N * r * 4);  // dB
   upd(static_cast<size_t>(colproj_split(M, K).splits) * K * r * 4);  // dA
   upd(dual_part_bytes(dual_split(M, N, r1), M, N, r1));              // dY·B and dYᵀ·XA in one pass
-  upd(gemm_split_bytes(M, N, K, quantized));                         // Y GEMM split partials
-  upd(gemm_split_bytes(M, K, N, quantized));                         // dX GEMM split partials
+  upd(gemm_sched_bytes(M, N, K, r1, quantized));                    // Y GEMM stream-K slots
+  upd(gemm_sched_bytes(M, K, N, r, quantized));                      // dX GEMM stream-K slots
   w.total = w.part_off + align256(part);
   return w;
 }
@@ -433,8 +440,8 @@ template <bool B_MN, int EPI>
 lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e, const CUtensorMap& f,
                           const PairParams& p, int sms, cudaStream_t st) {
   using C = PairCfg<B_MN>;
-  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS) * p.ksplit;
-  const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
+  const long long pairs = p.sk_on ? kGemmPairs : (tiles < sms / 2 ? tiles : sms / 2);
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
@@ -454,8 +461,8 @@ template <bool B_MN, int WF, int EPI>
 lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CUtensorMap& e, const CUtensorMap& f,
                             const PairParams& p, int sms, cudaStream_t st) {
   using C = QCfg<B_MN, WF>;
-  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS) * p.ksplit;
-  const long long pairs = tiles < sms / 2 ? tiles : sms / 2;
+  const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
+  const long long pairs = p.sk_on ? kGemmPairs : (tiles < sms / 2 ? tiles : sms / 2);
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   // the raster group counts tiles; 512-row tiles take half as many for the same rows
   PairParams q = p;
@@ -555,7 +562,8 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   p.Kred = static_cast<int>(Kred);
   p.r = r;
   p.out = static_cast<__nv_bfloat16*>(out);
-  p.ksplit = 1;
+  p.sk_on = 0;
+  p.sk_dp_tiles = 0;
   p.kpart = nullptr;
   p.status = status;
   p.wait_ns = wait_limit_ns();
@@ -574,22 +582,34 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   return p;
 }
 
-// A split reduction for the plain store epilogue when the size calls for one and its
-// partials fit in the caller's part region (callers without room keep one unit per tile).
-void set_ksplit(PairParams& p, const lora_weight_t* W, float* part, size_t part_cap) {
+// The stream-K schedule for the plain store epilogue when the sizes call for it, the GPU
+// runs the 74 CTA pairs it is planned for, and its slots fit in the caller's part region
+// (callers without room keep whole tiles).
+GemmSched set_sched(PairParams& p, const lora_weight_t* W, float* part, size_t part_cap, int sms) {
   const bool q = W->fmt != LORA_W_BF16;
-  const int S = gemm_ksplit(p.M, p.Nout, p.Kred, q);
-  if (S > 1 && part && gemm_split_bytes(p.M, p.Nout, p.Kred, q) <= part_cap) {
-    p.ksplit = S;
+  GemmSched g = gemm_sched(p.M, p.Nout, p.Kred, p.r, q);
+  if (g.sk && part && sms / 2 >= kGemmPairs && gemm_sched_bytes(p.M, p.Nout, p.Kred, p.r, q) <= part_cap) {
+    p.sk_on = 1;
+    p.sk_dp_tiles = g.dp_tiles;
     p.kpart = part;
+  } else {
+    g.sk = false;
   }
+  return g;
 }
 
-// out = Σ over the splits of the partials, in split order (nothing to do without a split).
-lora_status_t finalize_ksplit(const PairParams& p, cudaStream_t st) {
-  if (p.ksplit <= 1) return LORA_OK;
-  const size_t n = static_cast<size_t>(p.M) * p.Nout;
-  splitk_finalize_kernel<<<finalize_grid(n / 8), 256, 0, st>>>(p.kpart, p.ksplit, n, p.out);
+// The tiles stream-K cut into pieces: out = Σ of their slots in pair order.
+lora_status_t streamk_fixup(const PairParams& p, const GemmSched& g, cudaStream_t st) {
+  if (!g.sk) return LORA_OK;
+  const int num_m = cdiv(p.M, g.tile_rows), num_n = cdiv(p.Nout, 256);
+  const int group_m = g.tile_rows == 512 ? (p.group_m > 1 ? p.group_m / 2 : 1) : p.group_m;
+  const dim3 grid(kGemmPairs - 1, 8);
+  if (g.tile_rows == 512)
+    streamk_fixup_kernel<512><<<grid, 256, 0, st>>>(p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m, g.dp_tiles,
+                                                    num_m * num_n, g.tile_fills, kGemmPairs);
+  else
+    streamk_fixup_kernel<256><<<grid, 256, 0, st>>>(p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m, g.dp_tiles,
+                                                    num_m * num_n, g.tile_fills, kGemmPairs);
   count_launch();
   return last_launch();
 }
@@ -618,9 +638,9 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   const FSpec tf{B, static_cast<uint64_t>(r), static_cast<uint64_t>(N)};
   PairParams p = gemm_params(M, N, K, r, Y, status, W);
   set_segments(p, sg, r);
-  set_ksplit(p, W, part, part_cap);
+  const GemmSched g = set_sched(p, W, part, part_cap, dev->sms);
   TRY((launch_gemm_w<false, EPI_STORE>(W, ta, te, tf, p, dev->sms, st)));
-  return finalize_ksplit(p, st);
+  return streamk_fixup(p, g, st);
 }
 
 // ---------------------------------------------------------------- backward core
@@ -668,9 +688,9 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     TRY(tmap_bf16(&te, sdYB, rt, M, kBoxX, kBoxY));
     const FSpec tf{A, static_cast<uint64_t>(K), static_cast<uint64_t>(rt)};
     PairParams p = gemm_params(M, K, N, rt, dX, status, W);
-    set_ksplit(p, W, part, part_cap);
+    const GemmSched g = set_sched(p, W, part, part_cap, dev->sms);
     TRY((launch_gemm_w<true, EPI_STORE>(W, ta, te, tf, p, dev->sms, st)));
-    TRY(finalize_ksplit(p, st));
+    TRY(streamk_fixup(p, g, st));
   }
   // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
   const Split sp = colproj_split(M, K);
@@ -1247,9 +1267,12 @@ lora_status_t lora_testing_bounded_wait(void* workspace, uint64_t limit_ns, void
   return last_launch();
 }
 
-int32_t lora_testing_gemm_ksplit(int64_t M, int64_t Nout, int64_t Kred, int32_t fmt) {
-  if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3) return 0;
-  return gemm_ksplit(M, Nout, Kred, fmt != LORA_W_BF16);
+int32_t lora_testing_gemm_streamk(int64_t M, int64_t Nout, int64_t Kred, int32_t r, int32_t fmt) {
+  if (fmt < LORA_W_BF16 || fmt > LORA_W_FP8_E4M3 || r < 0 || r > 128) return -1;
+  const GemmSched g = gemm_sched(M, Nout, Kred, r, fmt != LORA_W_BF16);
+  if (!g.sk) return 0;
+  const long long tiles = static_cast<long long>(cdiv(M, g.tile_rows)) * cdiv(Nout, 256);
+  return static_cast<int32_t>(tiles - g.dp_tiles);
 }
 
 lora_status_t lora_timing_enable(int32_t on) {

@@ -127,22 +127,23 @@ def test_workspace_bytes_is_a_pure_function_of_sizes():
     assert q.workspace_bytes(4096, 4096, 4096, 16) < q.workspace_bytes(4096, 4096, 4096, 128)
 
 
-def test_gemm_split_only_for_outputs_that_leave_pairs_idle():
-    k = q.lora_testing_gemm_ksplit
+def test_gemm_streamk_only_where_the_last_wave_leaves_pairs_idle():
+    k = q.lora_testing_gemm_streamk
     B4, I8 = q.LORA_W_BLOCK4, q.LORA_W_INT8
-    # the rank sweep's small batch with quantized weights: 32 output tiles of 512 x 256
-    # for 74 CTA pairs, forward (K = N = 8192) and the dX of the 8192 -> 28672 projection
-    assert k(512, 8192, 8192, B4) == 2 and k(512, 8192, 28672, B4) == 2 and k(512, 8192, 8192, I8) == 2
-    # a wave or more of tiles: no split (112 tiles; bf16 tiles are 256 rows: 64 of them)
-    assert k(512, 28672, 8192, B4) == 1 and k(512, 8192, 8192) == 1
-    assert k(16384, 14336, 4096) == 1 and k(8192, 14336, 4096, B4) == 1 and k(8192, 4096, 14336, B4) == 1
-    # a split needs at least 8 fills per range: the tiny configuration has 4
-    assert k(256, 512, 512) == 1
-    assert 1 <= k(100, 1024, 8192) <= 4 and k(100, 1024, 8192, 9) == 0
-    assert k(300, 2048, 4096, B4) == k(300, 2048, 4096, B4)
-    # the workspace holds the fp32 partials of the split
-    S = k(512, 8192, 8192, B4)
-    assert q.workspace_bytes(512, 8192, 8192, 16, B4) >= 256 + S * 512 * 8192 * 4
+    # the rank sweep's 512-token shapes with quantized weights: 32 or 112 tiles of
+    # 512 x 256 for 74 CTA pairs, all shared out as pieces
+    assert k(512, 8192, 8192, 16, B4) == 32 and k(512, 28672, 8192, 16, B4) == 112
+    assert k(512, 8192, 28672, 16, B4) == 32 and k(512, 8192, 8192, 16, I8) == 32
+    # the QLoRA dX GEMM: 256 tiles = 3.46 waves; two waves whole, 108 tiles as pieces
+    assert k(8192, 4096, 14336, 16, B4) == 256 - 148
+    # bf16 at 512 tokens and N = 28672: 224 tiles, 76 as pieces; N = 8192: 64 tiles, whole
+    assert k(512, 28672, 8192, 16) == 76 and k(512, 8192, 8192, 16) == 0
+    # many waves, or too little work per pair: whole tiles
+    assert k(16384, 14336, 4096, 16) == 0 and k(16384, 4096, 14336, 16) == 0 and k(8192, 4096, 4096, 16) == 0
+    assert k(8192, 14336, 4096, 16, B4) == 0 and k(256, 512, 512, 8) == 0
+    assert k(512, 8192, 8192, 16, 9) == -1 and k(512, 8192, 8192, 129, 0) == -1
+    # the workspace holds the schedule's fp32 slots: two tiles of 512 x 256 per pair
+    assert q.workspace_bytes(512, 8192, 8192, 16, B4) >= 256 + 2 * 74 * 512 * 256 * 4
     assert q.workspace_bytes(512, 8192, 8192, 16) < 512 * 8192 * 4
 
 
