@@ -691,7 +691,9 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     if tr and tr.get("source_hash") == source_hash() and tr.get("workload") == args.workload:
         traffic = tr.get("bytes_per_launch")
     roofline = {
-        "kernel": "lora_gemm_pair_kernel (Y and dX GEMMs)",
+        "kernel": ("lora_gemm_pair_kernel" if all(c.fmt == "bf16" for c in cases) else
+                   "lora_gemm_q_kernel" if all(c.fmt != "bf16" for c in cases) else
+                   "lora_gemm_pair_kernel / lora_gemm_q_kernel") + " (Y and dX GEMMs)",
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": achieved / peak if achieved else None, "traffic": traffic,
         "peak_source": f"{peak_src} bf16 dense, " + ("sustained (power cap or low clock seen)" if capped
