@@ -99,6 +99,10 @@ typedef struct {
  * buffer serves both).  The workspace must be zero-filled once before its first use
  * (it holds the device status word read by lora_device_status()); afterwards calls
  * leave that word alone unless a kernel reports an error.  Returns 0 for invalid sizes.
+ * It holds the rank-r operand s·XA or s·dY·B, the fp32 split partials of the rank-r
+ * passes and, for sizes whose output tiles would leave the GPU's CTA pairs idle in the
+ * last wave, the fp32 slots of the GEMM's stream-K schedule (up to 2·74 tiles of
+ * 512 × 256 fp32, 77.6 MB, for a quantized weight).
  */
 size_t lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int32_t fmt);
 
@@ -293,8 +297,10 @@ lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, i
  * latency-critical code that must not call cudaMalloc/cudaFree because those calls
  * can synchronize the whole device and may fail under a fixed memory budget.
  *
- * Computes exactly what lora_linear_fwd computes (same kernels, same arguments apart
- * from the workspace), but keeps its scratch (s·XA and the split partial sums of X·Aᵀ)
+ * Computes what lora_linear_fwd computes with the same kernels, except that every
+ * output tile of the GEMM is computed whole (the stream-K schedule, which lora_linear_fwd
+ * takes for some small outputs, needs more scratch; results then agree to the last few
+ * bits of fp32 summation order), and keeps its scratch (s·XA and the split partial sums of X·Aᵀ)
  * in one fixed array of LORA_NOALLOC_SCRATCH_BYTES bytes that is part of the library
  * image: every GPU that loads the library holds that array until the process exits.
  * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
