@@ -35,6 +35,15 @@ lora_status_t lora_testing_bounded_wait(void* workspace, uint64_t limit_ns, void
  */
 int32_t lora_testing_gemm_streamk(int64_t M, int64_t Nout, int64_t Kred, int32_t r, int32_t fmt);
 
+/*
+ * Which passes over X run on the TMA-fed stream (the kernel of the one-pass dY·B / dYᵀ·XA
+ * products in a single-product mode) rather than the cp.async passes, for M tokens, K
+ * input features and LoRA rank r (the grouped layers' G·r): bit 0 the forward's X·Aᵀ,
+ * bit 1 the backward's Xᵀ·(s·dY·B) for dA; -1 for invalid sizes.  A pure function of
+ * its arguments; lets tests check that a case takes those paths.
+ */
+int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,7 +34,7 @@ LORA_W_FP8_E4M3 = 3
 EXPORTED = (
     "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
-    "lora_testing_bounded_wait", "lora_testing_gemm_streamk", "lora_timing_enable", "lora_timing_read",
+    "lora_testing_bounded_wait", "lora_testing_gemm_streamk", "lora_testing_xpass_tma", "lora_timing_enable", "lora_timing_read",
     "lora_launch_count",
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
     "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
@@ -127,6 +127,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_testing_bounded_wait.restype = i32
     lib.lora_testing_gemm_streamk.argtypes = [i64, i64, i64, i32, i32]
     lib.lora_testing_gemm_streamk.restype = i32
+    lib.lora_testing_xpass_tma.argtypes = [i64, i64, i32]
+    lib.lora_testing_xpass_tma.restype = i32
     lib.lora_timing_enable.argtypes = [i32]
     lib.lora_timing_enable.restype = i32
     lib.lora_timing_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
@@ -268,6 +270,11 @@ def lora_device_status(workspace, stream=None) -> int:
 
 def lora_testing_bounded_wait(workspace, limit_ns: int, stream=None) -> int:
     return int(_lib.lora_testing_bounded_wait(_ptr(workspace), int(limit_ns), _stream(stream)))
+
+
+def lora_testing_xpass_tma(M: int, K: int, r: int) -> int:
+    """Bit 0: the forward's X·Aᵀ, bit 1: the backward's pass for dA run on the TMA stream."""
+    return int(_lib.lora_testing_xpass_tma(int(M), int(K), int(r)))
 
 
 def lora_testing_gemm_streamk(M: int, Nout: int, Kred: int, r: int, fmt: int = LORA_W_BF16) -> int:

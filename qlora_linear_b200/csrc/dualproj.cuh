@@ -19,6 +19,10 @@
 //   D columns of the tile -> register accumulators, written once per column tile
 // Each block writes fp32 partials, T for its column block and D for its row block; the
 // finalize kernels add them in split order, so results do not depend on scheduling.
+//
+// The same stream serves the two passes over X, one product each (MODE):
+//   DP_ROWS  T = X·Aᵀ      (the forward's XA; Q read from A [r][K] as stored)
+//   DP_COLS  D = Xᵀ·R      (dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and finalized transposed)
 #pragma once
 
 #include "ptx.cuh"
@@ -39,6 +43,8 @@ constexpr int DP_TPITCH = DP_RPAD + 8;                    // fp32 words per T ac
 constexpr int DP_MAX_ROW_TILES = 16;                      // the T accumulator of 16 × 64 rows fills the rest
 static_assert(DP_STAGE_BYTES % 1024 == 0, "stage size must keep the 128-byte swizzle atoms aligned");
 
+enum : int { DP_BOTH = 0, DP_ROWS = 1, DP_COLS = 2 };
+
 constexpr int dual_smem_bytes() {
   return 1024 + DP_STAGES * DP_STAGE_BYTES + 2 * DP_Q_BYTES + DP_MAX_ROW_TILES * DP_TR * DP_TPITCH * 4;
 }
@@ -53,11 +59,16 @@ struct DualParams {
 };
 
 // tmP: dY block [M rows][C columns] (row pitch of dY), box 64 × 64, 128-byte swizzle.
-// tmQ: B [C rows][r], box 16 × 256.  tmR: XA [M rows][r] (row pitch of XA), box 16 × 64,
-// 32-byte swizzle (16-byte chunk index ^= bit 2 of the row: conflict-free ldmatrix).
+// tmQ: B [C rows][r], box 16 × 256 (DP_ROWS: A [r rows][C], box 256 × 16).  tmR: XA
+// [M rows][r] (row pitch of XA), box 16 × 64, 32-byte swizzle (16-byte chunk index ^= bit
+// 2 of the row: conflict-free ldmatrix).  A mode that skips a product never touches its
+// operand's map or its partials.
+template <int MODE>
 __global__ void __launch_bounds__(DP_THREADS, 1)
     dualproj_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmR, const DualParams p) {
+  constexpr bool DO_T = MODE != DP_COLS, DO_D = MODE != DP_ROWS;
+  constexpr int STAGE_TX = DP_P_BYTES + (DO_D ? DP_R_BYTES : 0);
   extern __shared__ uint8_t dp_raw[];
   __shared__ __align__(8) uint64_t full[DP_STAGES], empty[DP_STAGES], qfull[2], qempty[2];
   __shared__ uint32_t abort_s, never_s;
@@ -86,10 +97,11 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
     never_s = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmP);
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmR);
+    if (DO_T) tma_prefetch_desc(&tmQ);
+    if (DO_D) tma_prefetch_desc(&tmR);
   }
-  for (int i = threadIdx.x; i < max(nrt, 0) * DP_TR * DP_TPITCH; i += DP_THREADS) tacc_s[i] = 0.f;
+  if (DO_T)
+    for (int i = threadIdx.x; i < max(nrt, 0) * DP_TR * DP_TPITCH; i += DP_THREADS) tacc_s[i] = 0.f;
   __syncthreads();
   if (nrt <= 0 || nct <= 0) return;
 
@@ -100,14 +112,17 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
       int qloads = 0;
       bool ok = true;
       for (int ci = 0; ci < nct && ok; ++ci) {
-        const int qb = ci & 1;
-        if (ci >= 2 && !mbar_wait(smem_u32(&qempty[qb]), static_cast<uint32_t>(((ci >> 1) - 1) & 1), wc)) {
-          ok = false;
-          break;
+        if (DO_T) {
+          const int qb = ci & 1;
+          if (ci >= 2 && !mbar_wait(smem_u32(&qempty[qb]), static_cast<uint32_t>(((ci >> 1) - 1) & 1), wc)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(smem_u32(&qfull[qb]), DP_Q_BYTES);
+          if (MODE == DP_ROWS) tma_load_2d(sQ + qb * DP_Q_BYTES, &tmQ, smem_u32(&qfull[qb]), (ct0 + ci) * DP_TC, 0);
+          else tma_load_2d(sQ + qb * DP_Q_BYTES, &tmQ, smem_u32(&qfull[qb]), 0, (ct0 + ci) * DP_TC);
+          ++qloads;
         }
-        mbar_arrive_expect_tx(smem_u32(&qfull[qb]), DP_Q_BYTES);
-        tma_load_2d(sQ + qb * DP_Q_BYTES, &tmQ, smem_u32(&qfull[qb]), 0, (ct0 + ci) * DP_TC);
-        ++qloads;
         for (int ri = 0; ri < nrt; ++ri) {
           const int s = static_cast<int>(fills % DP_STAGES);
           const uint32_t ph = static_cast<uint32_t>((fills / DP_STAGES) & 1);
@@ -117,11 +132,11 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
           }
           const uint32_t st = sbase + s * DP_STAGE_BYTES;
           const uint32_t bar = smem_u32(&full[s]);
-          mbar_arrive_expect_tx(bar, DP_STAGE_BYTES);
+          mbar_arrive_expect_tx(bar, STAGE_TX);
           const int y = (rt0 + ri) * DP_TR;
 #pragma unroll
           for (int b = 0; b < DP_TC / 64; ++b) tma_load_2d(st + b * DP_BOX_BYTES, &tmP, bar, (ct0 + ci) * DP_TC + b * 64, y);
-          tma_load_2d(st + DP_P_BYTES, &tmR, bar, 0, y);
+          if (DO_D) tma_load_2d(st + DP_P_BYTES, &tmR, bar, 0, y);
           ++fills;
         }
       }
@@ -143,21 +158,32 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
   bool ok = true;
   float* outD = p.partD + static_cast<size_t>(blockIdx.x) * p.C * p.r;
   for (int ci = 0; ci < nct && ok; ++ci) {
-    const int qb = ci & 1;
-    if (!mbar_wait_warp(smem_u32(&qfull[qb]), static_cast<uint32_t>((ci >> 1) & 1), wc)) {
-      ok = false;
-      break;
-    }
-    // B of this column tile as the MMA's second operand, 16 k-steps of 16 columns
+    // B (or Aᵀ) of this column tile as the MMA's second operand, 16 k-steps of 16 columns
     uint32_t qf[DP_TC / 16][4];
-    {
+    if (DO_T) {
+      const int qb = ci & 1;
+      if (!mbar_wait_warp(smem_u32(&qfull[qb]), static_cast<uint32_t>((ci >> 1) & 1), wc)) {
+        ok = false;
+        break;
+      }
       const uint32_t qa = sQ + qb * DP_Q_BYTES;
 #pragma unroll
       for (int kk = 0; kk < DP_TC / 16; ++kk) {
-        const int kr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int jc = ((lane >> 4) & 1) * 8;
-        ldsm_x4_t(qa + (kr * DP_RPAD + jc) * 2, qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+        if (MODE == DP_ROWS) {
+          // A [16 ranks][256 columns] as stored: rank j's row holds the k values, the
+          // fragment layout of the MMA's second operand without a transpose
+          const int j = (lane & 7) + ((lane >> 4) & 1) * 8;
+          const int kc = kk * 16 + ((lane >> 3) & 1) * 8;
+          ldsm_x4(qa + (j * DP_TC + kc) * 2, qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+        } else {
+          const int kr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int jc = ((lane >> 4) & 1) * 8;
+          ldsm_x4_t(qa + (kr * DP_RPAD + jc) * 2, qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+        }
       }
+      // the next TMA load into this buffer (async proxy) must follow these ordinary
+      // shared-memory reads: without the proxy fence it can overwrite them first
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&qempty[qb]));
     }
@@ -185,7 +211,7 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) tacc[t][e] = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < DP_TC / 16; ++kk) {
+      for (int kk = 0; kk < (DO_T ? DP_TC / 16 : 0); ++kk) {
         const int row = w * 16 + (lane & 15);
         const int chunk = ((kk & 3) << 1) | (lane >> 4);
         uint32_t a0, a1, a2, a3;
@@ -195,7 +221,7 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
       }
       // D: columns 64w .. 64w+63 (TMA box w) against all 64 rows
 #pragma unroll
-      for (int kk = 0; kk < DP_TR / 16; ++kk) {
+      for (int kk = 0; kk < (DO_D ? DP_TR / 16 : 0); ++kk) {
         const int mr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
         const int jchunk = (lane >> 4) & 1;
         uint32_t b0, b1, b2, b3;
@@ -210,6 +236,7 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
           mma_bf16_16816(dacc[f][1], a0, a1, a2, a3, b2, b3);
         }
       }
+      fence_proxy_async_smem();  // as for the B buffer: reads of the stage before its next TMA load
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
       ++fills;
@@ -217,7 +244,7 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
       // this warp owns rows 16w .. 16w+15 of every tile of the block
       float* trow = tacc_s + (ri * DP_TR + w * 16 + (lane >> 2)) * DP_TPITCH + (lane & 3) * 2;
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
+      for (int t = 0; t < (DO_T ? 2 : 0); ++t) {
         float2* lo = reinterpret_cast<float2*>(trow + t * 8);
         float2* hi = reinterpret_cast<float2*>(trow + 8 * DP_TPITCH + t * 8);
         float2 v = *lo;
@@ -234,7 +261,7 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
 
     // D over this block's rows for the warp's 64 columns
 #pragma unroll
-    for (int f = 0; f < 4; ++f) {
+    for (int f = 0; f < (DO_D ? 4 : 0); ++f) {
       const int c = (ct0 + ci) * DP_TC + w * 64 + f * 16 + (lane >> 2);
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
@@ -249,7 +276,7 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
       }
     }
   }
-  if (!ok) return;
+  if (!ok || !DO_T) return;
 
   // T over this block's columns for the warp's rows
   __syncwarp();

@@ -118,12 +118,14 @@ struct DualSplit {
   bool use = false;
   int a = 0, b = 0, row_tiles = 0, col_tiles = 0;
 };
-DualSplit dual_split(long long M, long long C, int r) {
+DualSplit dual_split(long long M, long long C, int r, int mode = DP_BOTH) {
   DualSplit best;
   if (r > DP_RPAD || M <= 0 || C <= 0) return best;
   const int ntr = cdiv(M, DP_TR), ntc = cdiv(C, DP_TC);
   const double tile = double(DP_TR) * DP_TC * 2;
-  double best_cost = 2.4 * ntr * double(ntc) * tile;
+  // against the cp.async passes: two of them for both products, one for a single product
+  double best_cost = (mode == DP_BOTH ? 2.4 : 1.2) * ntr * double(ntc) * tile;
+  const double wT = mode == DP_COLS ? 0.0 : 1.0, wD = mode == DP_ROWS ? 0.0 : 1.0;
   for (int rt = 1; rt <= DP_MAX_ROW_TILES && rt <= ntr; ++rt) {
     const int a = cdiv(ntr, rt);
     if (a > kDualCtas) continue;
@@ -131,7 +133,7 @@ DualSplit dual_split(long long M, long long C, int r) {
       const int b = cdiv(ntc, ct);
       if (static_cast<long long>(a) * b > kDualCtas) continue;
       const int n = a * b;
-      const double cost = double(rt) * ct * tile * (n > 136 ? n : 136) + 2.0 * (double(a) * C + double(b) * M) * r * 4;
+      const double cost = double(rt) * ct * tile * (n > 136 ? n : 136) + 2.0 * (wD * a * C + wT * b * M) * r * 4;
       if (cost < best_cost) {
         best_cost = cost;
         best = DualSplit{true, a, b, rt, ct};
@@ -142,6 +144,9 @@ DualSplit dual_split(long long M, long long C, int r) {
 }
 size_t dual_part_t_bytes(const DualSplit& d, long long M, int r) {
   return align256(static_cast<size_t>(d.b) * M * r * 4);
+}
+size_t dual_part_d_bytes(const DualSplit& d, long long C, int r) {
+  return align256(static_cast<size_t>(d.a) * C * r * 4);
 }
 size_t dual_part_bytes(const DualSplit& d, long long M, long long C, int r) {
   return d.use ? dual_part_t_bytes(d, M, r) + align256(static_cast<size_t>(d.a) * C * r * 4) : 0;
@@ -209,6 +214,9 @@ WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg, bool
   upd(static_cast<size_t>(colproj_split(M, N).splits) * N * r * 4);  // dB
   upd(static_cast<size_t>(colproj_split(M, K).splits) * K * r * 4);  // dA
   upd(dual_part_bytes(dual_split(M, N, r1), M, N, r1));              // dY·B and dYᵀ·XA in one pass
+  const DualSplit xr = dual_split(M, K, r, DP_ROWS), xc = dual_split(M, K, r, DP_COLS);
+  if (xr.use) upd(dual_part_t_bytes(xr, M, r));                      // X·Aᵀ on the TMA stream
+  if (xc.use) upd(dual_part_d_bytes(xc, K, r));                      // Xᵀ·(s·dY·B) on the TMA stream
   upd(gemm_sched_bytes(M, N, K, r1, quantized));                    // Y GEMM stream-K slots
   upd(gemm_sched_bytes(M, K, N, r, quantized));                      // dX GEMM stream-K slots
   w.total = w.part_off + align256(part);
@@ -247,7 +255,9 @@ lora_status_t dev_info(DevInfo** out) {
     SET_GEMM_Q(WF_INT8)
     SET_GEMM_Q(WF_FP8)
 #undef SET_GEMM_Q
-    SET_SMEM(dualproj_kernel, dual_smem_bytes());
+    SET_SMEM(dualproj_kernel<DP_BOTH>, dual_smem_bytes());
+    SET_SMEM(dualproj_kernel<DP_ROWS>, dual_smem_bytes());
+    SET_SMEM(dualproj_kernel<DP_COLS>, dual_smem_bytes());
     SET_SMEM((lora_gemm_pair_kernel<false, EPI_CE_LSE>), (PairCfg<false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<false, EPI_CE_DLOGITS>), (PairCfg<false>::SMEM_BYTES));
     SET_SMEM((lora_gemm_pair_kernel<true, EPI_ACC_F32>), (PairCfg<true>::SMEM_BYTES));
@@ -400,18 +410,28 @@ lora_status_t launch_colproj(const __nv_bfloat16* P, int ldp, const __nv_bfloat1
   return last_launch();
 }
 
-// partT [d.b][M][r] = dY·B summed per column block, partD [d.a][C][r] = dYᵀ·XA summed per
-// row block, for dY with row pitch ldp, B [C][r] and XA with row pitch ldr.
-lora_status_t launch_dual(const __nv_bfloat16* dY, long long ldp, const __nv_bfloat16* B, const __nv_bfloat16* XA,
+// partT [d.b][M][r] = P·Q summed per column block, partD [d.a][C][r] = Pᵀ·R summed per row
+// block, for P [M][C] with row pitch ldp, Q = B [C][r] (DP_ROWS: Q = Aᵀ with A [r][C] as
+// stored) and R with row pitch ldr; a single-product mode leaves the other partials alone.
+template <int MODE>
+lora_status_t launch_dual(const __nv_bfloat16* P, long long ldp, const __nv_bfloat16* Q, const __nv_bfloat16* R,
                           long long ldr, long long M, long long C, int r, const DualSplit& d, float* partT,
                           float* partD, uint32_t* status, cudaStream_t st) {
   CUtensorMap tp, tq, tr;
-  TRY(tmap_2d(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dY, C, M, 64, DP_TR, CU_TENSOR_MAP_SWIZZLE_128B, ldp));
-  TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, r, C, DP_RPAD, DP_TC, CU_TENSOR_MAP_SWIZZLE_NONE));
-  TRY(tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, XA, r, M, DP_RPAD, DP_TR, CU_TENSOR_MAP_SWIZZLE_32B, ldr));
+  TRY(tmap_2d(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, C, M, 64, DP_TR, CU_TENSOR_MAP_SWIZZLE_128B, ldp));
+  if (MODE == DP_ROWS)
+    TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Q, C, r, DP_TC, DP_RPAD, CU_TENSOR_MAP_SWIZZLE_NONE));
+  else if (MODE == DP_BOTH)
+    TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Q, r, C, DP_RPAD, DP_TC, CU_TENSOR_MAP_SWIZZLE_NONE));
+  else
+    tq = tp;  // not read
+  if (MODE != DP_ROWS)
+    TRY(tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, r, M, DP_RPAD, DP_TR, CU_TENSOR_MAP_SWIZZLE_32B, ldr));
+  else
+    tr = tp;  // not read
   const DualParams dp{partT, partD, static_cast<int>(M), static_cast<int>(C), r, d.row_tiles, d.col_tiles, status,
                       wait_limit_ns()};
-  dualproj_kernel<<<dim3(d.a, d.b), DP_THREADS, dual_smem_bytes(), st>>>(tp, tq, tr, dp);
+  dualproj_kernel<MODE><<<dim3(d.a, d.b), DP_THREADS, dual_smem_bytes(), st>>>(tp, tq, tr, dp);
   count_launch();
   return last_launch();
 }
@@ -628,9 +648,17 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   const int Mi = static_cast<int>(M), Ki = static_cast<int>(K);
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
 
-  const Split sp = rowproj_split(M, K);
-  TRY(launch_rowproj<false>(Xb, Ki, static_cast<const __nv_bfloat16*>(A), part, Mi, Ki, rt, sp, st));
-  TRY(finalize_rows(part, sp.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
+  const DualSplit ds = dual_split(M, K, rt, DP_ROWS);
+  if (ds.use && dual_part_t_bytes(ds, M, rt) <= part_cap) {
+    // one TMA-fed pass over X
+    TRY(launch_dual<DP_ROWS>(Xb, K, static_cast<const __nv_bfloat16*>(A), nullptr, 0, M, K, rt, ds, part, nullptr,
+                             status, st));
+    TRY(finalize_rows(part, ds.b, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
+  } else {
+    const Split sp = rowproj_split(M, K);
+    TRY(launch_rowproj<false>(Xb, Ki, static_cast<const __nv_bfloat16*>(A), part, Mi, Ki, rt, sp, st));
+    TRY(finalize_rows(part, sp.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
+  }
 
   CUtensorMap ta, te;
   TRY(tmap_bf16(&ta, X, K, M, kBoxX, kBoxY));
@@ -667,7 +695,7 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     if (ds.use && dual_part_bytes(ds, M, rows, r) <= part_cap) {
       // one pass over dY_g for s·dY_g·B_g (columns [g·r, g·r + r) of s·dY·B) and dB_g = s·dY_gᵀ·XA_g
       float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
-      TRY(launch_dual(dYb + o, N, Bb + o * r, XAb + g * r, rt, M, rows, r, ds, part, partD, status, st));
+      TRY(launch_dual<DP_BOTH>(dYb + o, N, Bb + o * r, XAb + g * r, rt, M, rows, r, ds, part, partD, status, st));
       TRY(finalize_rows(part, ds.b, M, r, rt, s, nullptr, sdYB + g * r, st));
       TRY(finalize_cols(partD, ds.a, rows, r, s, false, dBg, st));
       continue;
@@ -693,6 +721,12 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     TRY(streamk_fixup(p, g, st));
   }
   // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
+  const DualSplit dsa = dual_split(M, K, rt, DP_COLS);
+  if (dsa.use && dual_part_d_bytes(dsa, K, rt) <= part_cap) {
+    // one TMA-fed pass over X
+    TRY(launch_dual<DP_COLS>(Xb, K, nullptr, sdYB, rt, M, K, rt, dsa, nullptr, part, status, st));
+    return finalize_cols(part, dsa.a, Ki, rt, 1.0f, true, static_cast<__nv_bfloat16*>(dA), st);
+  }
   const Split sp = colproj_split(M, K);
   TRY(launch_colproj(Xb, Ki, sdYB, rt, part, Mi, Ki, rt, sp, st));
   return finalize_cols(part, sp.splits, Ki, rt, 1.0f, true, static_cast<__nv_bfloat16*>(dA), st);
@@ -858,7 +892,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
   if (ds.use && dual_part_bytes(ds, M, D, r) <= part_cap) {
     // one pass over dZ for s·dZ·B_d and dB_d = s·dZᵀ·(H·A_dᵀ)
     float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
-    TRY(launch_dual(dZb, D, Bd, XAdb, r, M, D, r, ds, part, partD, status, st));
+    TRY(launch_dual<DP_BOTH>(dZb, D, Bd, XAdb, r, M, D, r, ds, part, partD, status, st));
     TRY(finalize_rows(part, ds.b, M, r, r, s, nullptr, skinny, st));
     TRY(finalize_cols(partD, ds.a, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
   } else {
@@ -1273,6 +1307,11 @@ int32_t lora_testing_gemm_streamk(int64_t M, int64_t Nout, int64_t Kred, int32_t
   if (!g.sk) return 0;
   const long long tiles = static_cast<long long>(cdiv(M, g.tile_rows)) * cdiv(Nout, 256);
   return static_cast<int32_t>(tiles - g.dp_tiles);
+}
+
+int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r) {
+  if (M <= 0 || K <= 0 || r < 1 || r > 128) return -1;
+  return (dual_split(M, K, r, DP_ROWS).use ? 1 : 0) | (dual_split(M, K, r, DP_COLS).use ? 2 : 0);
 }
 
 lora_status_t lora_timing_enable(int32_t on) {

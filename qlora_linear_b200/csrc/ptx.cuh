@@ -154,8 +154,9 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(m)), "r"(cluster_bar), "r"(x), "r"(y)
       : "memory");
 }
-// Orders this thread's generic-proxy shared-memory writes before later async-proxy
-// (tensor core / TMA) reads of the same bytes.
+// Orders this thread's generic-proxy shared-memory accesses before later async-proxy
+// (tensor core / TMA) accesses of the same bytes: writes before their reads, and reads
+// before a TMA load that overwrites the buffer.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
