@@ -270,15 +270,17 @@ __device__ __forceinline__ void epi_swiglu_bwd_chunk(const PairParams& p, const 
   }
 }
 
-// The SwiGLU-backward epilogue of one row over a 256-column accumulator at tbase: the
-// saved g, u of chunk c + 1 are loaded while chunk c is converted, two chunks per step
-// so both register sets stay named.
-__device__ __forceinline__ void epi_swiglu_bwd_row(const PairParams& p, uint32_t tbase, int row, int colbase) {
+// The SwiGLU-backward epilogue of one row over 32-column chunks [c_begin, c_end) of a
+// 256-column accumulator at tbase: the saved g, u of chunk c + 1 are loaded while chunk c
+// is converted, two chunks per step so both register sets stay named (the range holds an
+// even number of chunks).
+__device__ __forceinline__ void epi_swiglu_bwd_row(const PairParams& p, uint32_t tbase, int row, int colbase,
+                                                   int c_begin = 0, int c_end = 8) {
   const bool in = row < p.M;
   GU32 x0, x1;
-  if (in && colbase < p.Nout) epi_swiglu_bwd_load(p, row, colbase, x0);
+  if (in && colbase + c_begin * 32 < p.Nout) epi_swiglu_bwd_load(p, row, colbase + c_begin * 32, x0);
 #pragma unroll 1
-  for (int c = 0; c < 8; c += 2) {
+  for (int c = c_begin; c < c_end; c += 2) {
     const int col0 = colbase + c * 32, col1 = col0 + 32;
     if (col0 >= p.Nout) break;  // warp-uniform
     if (in && col1 < p.Nout) epi_swiglu_bwd_load(p, row, col1, x1);
@@ -287,7 +289,7 @@ __device__ __forceinline__ void epi_swiglu_bwd_row(const PairParams& p, uint32_t
     tmem_ld_wait();
     if (in) epi_swiglu_bwd_chunk(p, v, row, col0, x0);
     if (col1 >= p.Nout) break;
-    if (in && col1 + 32 < p.Nout && c + 2 < 8) epi_swiglu_bwd_load(p, row, col1 + 32, x0);
+    if (in && col1 + 32 < p.Nout && c + 2 < c_end) epi_swiglu_bwd_load(p, row, col1 + 32, x0);
     tmem_ld_32x32b_x32(tbase + (c + 1) * 32, v);
     tmem_ld_wait();
     if (in) epi_swiglu_bwd_chunk(p, v, row, col1, x1);

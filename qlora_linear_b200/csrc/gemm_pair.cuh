@@ -47,6 +47,13 @@ struct PairCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NUM_EPI_WARPS = 4;
   static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS);
+  // The SwiGLU-backward epilogue reads the saved gate and up values and rewrites them (four
+  // times the bytes of a plain store): two warps per TMEM lane quarter, each draining half
+  // of the columns, keep twice the loads in flight.
+  template <int EPI>
+  static constexpr int epi_warps() { return EPI == EPI_SWIGLU_BWD ? 8 : NUM_EPI_WARPS; }
+  template <int EPI>
+  static constexpr int threads() { return 32 * (2 + epi_warps<EPI>()); }
   static constexpr int TMEM_COLS = 512;
   static constexpr int NUM_BARS = 2 * STAGES + 5;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
@@ -55,11 +62,12 @@ struct PairCfg {
 };
 
 template <bool B_MN, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::template threads<EPI>(), 1)
     lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
                           const PairParams p) {
   using C = PairCfg<B_MN>;
+  constexpr int NEPI = C::template epi_warps<EPI>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -95,7 +103,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 2 * C::NUM_EPI_WARPS);
+      mbar_init(smem_u32(&tempty[a]), 2 * NEPI);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -229,7 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
       const WaitCtl drain_wc{never_flag, nullptr, p.wait_ns};
       mbar_wait(smem_u32(drain), 0, drain_wc);
     }
-  } else if (warp < 2 + C::NUM_EPI_WARPS) {
+  } else if (warp < 2 + NEPI) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
@@ -256,7 +264,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::NUM_T
           if (row < p.M) epi_swiglu_fwd_chunk(p, g, u, row, col0);
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-        epi_swiglu_bwd_row(p, tbase, row, nb * C::BN);
+        // with 8 epilogue warps, warps 2-5 and 6-9 split the 8 column chunks
+        const int half = (warp - 2) >> 2;
+        epi_swiglu_bwd_row(p, tbase, row, nb * C::BN, NEPI == 8 ? 4 * half : 0, NEPI == 8 ? 4 * half + 4 : 8);
       } else if constexpr (EPI == EPI_STORE) {
 #pragma unroll 1
         for (int c = 0; c < C::BN / 32; ++c) {

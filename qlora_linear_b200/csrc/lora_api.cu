@@ -465,7 +465,7 @@ lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUte
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_pair_kernel<B_MN, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    lora_gemm_pair_kernel<B_MN, EPI><<<grid, C::template threads<EPI>(), C::SMEM_BYTES, st>>>(a, b, e, f, p);
   }
   count_launch();
   return last_launch();
