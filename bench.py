@@ -723,8 +723,12 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = ws.e2e(args, step) if args.workload in ("mlp", "ce") else run_e2e(args, cases, layers, data, step, world,
-                                                                               dev)
+        if args.workload in ("mlp", "ce"):
+            e2e = ws.e2e(args, step)
+        else:
+            e2e = run_e2e(args, cases, layers, data, step, world, dev)
+            # the same with every output (Y and dX too) read back each step
+            e2e["all_outputs"] = run_e2e(args, cases, layers, data, step, world, dev, outs=("Y", "dX", "dA", "dB"))
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
@@ -828,12 +832,14 @@ def time_split(args, ws, stream):
     return res
 
 
-def run_e2e(args, cases, layers, data, step, world, dev):
+def run_e2e(args, cases, layers, data, step, world, dev, outs=("dA", "dB")):
     """Same metric through the public API with host buffers: each step copies that
     step's inputs (X, dY and the adapter A, B) from pinned host memory and reads the
-    outputs (Y, dX, dA, dB) back; the frozen weight stays resident.  Uploads, compute
-    and read-backs run on three streams over two sets of device buffers, so one step's
-    copies overlap the neighbouring steps' compute (the bytes moved are unchanged)."""
+    step's result back: by default the adapter gradients dA, dB, the trainable outputs
+    of a LoRA training step (Y and dX are activations that a model keeps on the device);
+    outs=("Y", "dX", "dA", "dB") reads every output back.  The frozen weight stays
+    resident.  Uploads, compute and read-backs run on three streams over two sets of
+    device buffers, so one step's copies overlap the neighbouring steps' compute."""
     import torch
     import torch.distributed as dist
 
@@ -858,7 +864,7 @@ def run_e2e(args, cases, layers, data, step, world, dev):
         hi = {"dY": d["dY"].cpu().pin_memory(), "A": d["A"].cpu().pin_memory(), "B": d["B"].cpu().pin_memory()}
         h2d += (hi["dY"].numel() + hi["A"].numel() + hi["B"].numel()) * 2
         host_in.append(hi)
-        ho = {k2: torch.empty(o[k2].shape, dtype=o[k2].dtype).pin_memory() for k2 in ("Y", "dX", "dA", "dB")}
+        ho = {k2: torch.empty(o[k2].shape, dtype=o[k2].dtype).pin_memory() for k2 in outs}
         d2h += sum(v.numel() * 2 for v in ho.values())
         host_out.append(ho)
     dev_x = [[torch.empty_like(x) for x, _ in xs_host] for _ in range(NB)]
@@ -896,7 +902,7 @@ def run_e2e(args, cases, layers, data, step, world, dev):
             ev.record(s_comp)
             s_d2h.wait_event(ev)
             with torch.cuda.stream(s_d2h):
-                for k2 in ("Y", "dX", "dA", "dB"):
+                for k2 in outs:
                     host_out[i][k2].copy_(o[k2], non_blocking=True)
                 ev_out[b][i].record(s_d2h)
         ev_comp[b].record(s_comp)
@@ -926,9 +932,9 @@ def run_e2e(args, cases, layers, data, step, world, dev):
     flops_step = sum(case_flops(c) for c in cases)
     return {"value": world * flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
-            "note": "inputs X, dY, A, B copied from pinned host memory and Y, dX, dA, dB read back every step; "
-                    "the frozen weight stays resident; uploads, compute and read-backs on three streams over two "
-                    "buffer sets"}
+            "note": "inputs X, dY, A, B copied from pinned host memory and " + ", ".join(outs) +
+                    " read back every step; the frozen weight stays resident; uploads, compute and read-backs on "
+                    "three streams over two buffer sets"}
 
 
 def main(argv=None):
