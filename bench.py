@@ -869,6 +869,18 @@ def run_e2e(args, cases, layers, data, step, world, dev, outs=("dA", "dB")):
         host_out.append(ho)
     dev_x = [[torch.empty_like(x) for x, _ in xs_host] for _ in range(NB)]
     dev_dy = [[torch.empty_like(d["dY"]) for d, _ in data] for _ in range(NB)]
+    # each buffer set has its own adapter tensors, uploaded on the upload stream with X and
+    # dY (an upload on the compute stream would queue behind the next step's large copies);
+    # the layer copies share the weight and the workspace (their calls are stream-ordered)
+    import copy
+    lay_b = []
+    for _ in range(NB):
+        row = []
+        for layer in layers:
+            lb = copy.copy(layer)
+            lb.A, lb.B = torch.empty_like(layer.A), torch.empty_like(layer.B)
+            row.append(lb)
+        lay_b.append(row)
     dev_out = [[{k2: torch.empty_like(o[k2]) for k2 in ("Y", "XA", "dX", "dA", "dB")} for _, o in data]
                for _ in range(NB)]
     ev_in = [[torch.cuda.Event() for _ in data] for _ in range(NB)]
@@ -886,13 +898,13 @@ def run_e2e(args, cases, layers, data, step, world, dev, outs=("dA", "dB")):
                     dev_x[b][x_of[i]].copy_(xs_host[x_of[i]][1], non_blocking=True)
                     done.add(x_of[i])
                 dev_dy[b][i].copy_(host_in[i]["dY"], non_blocking=True)
+                lay_b[b][i].A.copy_(host_in[i]["A"], non_blocking=True)
+                lay_b[b][i].B.copy_(host_in[i]["B"], non_blocking=True)
                 ev_in[b][i].record(s_h2d)
-        for i, layer in enumerate(layers):
+        for i, layer in enumerate(lay_b[b]):
             o = dev_out[b][i]
             s_comp.wait_event(ev_in[b][i])
             s_comp.wait_event(ev_out[b][i])  # this buffer's previous outputs have been read back
-            layer.A.copy_(host_in[i]["A"], non_blocking=True)
-            layer.B.copy_(host_in[i]["B"], non_blocking=True)
             X = dev_x[b][x_of[i]]
             layer.forward(X, Y=o["Y"], XA=o["XA"], stream=s_comp)
             layer.backward(dev_dy[b][i], X, o["XA"], out=(o["dX"], o["dA"], o["dB"]), stream=s_comp)
