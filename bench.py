@@ -382,8 +382,9 @@ class MlpSet:
         return [q.lora_device_status(self.mlp.workspace(self.M))]
 
     def e2e(self, args, step):
-        """End to end with host buffers: X, dZ and the four adapters in, Z, dX and the four
-        adapter gradients out, every step; the frozen weights stay resident."""
+        """End to end with host buffers: X, dZ and the four adapters in and the step's result,
+        the four adapter gradients, out every step (Z and dX are activations a model keeps on
+        the device); the frozen weights stay resident."""
         import torch
         import torch.distributed as dist
 
@@ -393,7 +394,7 @@ class MlpSet:
                                                        ("A_gate_up", m.A_gate_up), ("B_gate_up", m.B_gate_up),
                                                        ("A_down", m.A_down), ("B_down", m.B_down))}
         d_in = {"X": torch.empty_like(self.inputs["X"]), "dZ": torch.empty_like(self.inputs["dZ"])}
-        outs = (self.Z,) + tuple(self.grads)
+        outs = tuple(self.grads[1:])  # dA_gate_up, dB_gate_up, dA_down, dB_down (not dX)
         h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
         h2d = sum(t.numel() * 2 for t in h_in.values())
         d2h = sum(t.numel() * 2 for t in h_out)
@@ -428,8 +429,8 @@ class MlpSet:
         flops_step = sum(case_flops(c) for c in self.cases)
         return {"value": self.world * flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
-                "note": "X, dZ and the four adapters copied from pinned host memory and Z, dX and the four adapter "
-                        "gradients read back every step; the frozen weights stay resident"}
+                "note": "X, dZ and the four adapters copied from pinned host memory and the four adapter gradients "
+                        "read back every step; the frozen weights stay resident"}
 
 
 class CeSet:
@@ -466,20 +467,18 @@ class CeSet:
         return [q.lora_device_status(self.ce.workspace(self.M))]
 
     def e2e(self, args, step):
-        """X in from pinned host memory and the per-row losses and dX out, every step."""
+        """X in from pinned host memory and the per-row losses (the step's result) out, every step."""
         import torch
 
         stream = torch.cuda.current_stream()
         hX = self.X.cpu().pin_memory()
         dXin = torch.empty_like(self.X)
         hloss = torch.empty(self.M, dtype=torch.float32).pin_memory()
-        hdX = torch.empty(self.dX.shape, dtype=self.dX.dtype).pin_memory()
 
         def e2e_step():
             dXin.copy_(hX, non_blocking=True)
             step(inputs={"X": dXin})
             hloss.copy_(self.loss, non_blocking=True)
-            hdX.copy_(self.dX, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -493,10 +492,10 @@ class CeSet:
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / steps
         return {"value": self.world * ce_flops(self.cases[0]) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": hX.numel() * 2, "d2h_bytes_per_step": hloss.numel() * 4 + hdX.numel() * 2,
+                "h2d_bytes_per_step": hX.numel() * 2, "d2h_bytes_per_step": hloss.numel() * 4,
                 "ms_per_step": ms, "steps": steps,
-                "note": "X copied from pinned host memory and the per-row losses and dX read back every step; "
-                        "head, labels and dloss resident"}
+                "note": "X copied from pinned host memory and the step's result, the per-row losses, read back "
+                        "every step (dX stays on the device for the layers below); head, labels and dloss resident"}
 
 
 def time_separate_ce(args, cases, ws, dev):
