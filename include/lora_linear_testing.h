@@ -44,6 +44,16 @@ int32_t lora_testing_gemm_streamk(int64_t M, int64_t Nout, int64_t Kred, int32_t
  */
 int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r);
 
+/*
+ * Blocking of the one-pass kernel over a [M, C] activation at rank r: mode 0 both
+ * products (dY·B and dYᵀ·XA), 1 the row product only (X·Aᵀ), 2 the column product only.
+ * Writes {a, b, row_tiles, col_tiles} to out4 (host memory, 4 int32): an a × b grid of
+ * blocks of row_tiles × 64 rows by col_tiles × 256 columns.  Returns 1 when the kernel is
+ * used for these sizes, 0 when the cp.async passes are (out4 then holds zeros), -1 for
+ * invalid arguments.  A pure function of its arguments.
+ */
+int32_t lora_testing_dual_blocking(int64_t M, int64_t C, int32_t r, int32_t mode, int32_t* out4);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,7 +34,7 @@ LORA_W_FP8_E4M3 = 3
 EXPORTED = (
     "lora_workspace_bytes", "lora_linear_fwd", "lora_linear_bwd", "dequant_blockwise4",
     "lora_merge", "lora_device_status", "lora_status_string", "lora_version",
-    "lora_testing_bounded_wait", "lora_testing_gemm_streamk", "lora_testing_xpass_tma", "lora_timing_enable", "lora_timing_read",
+    "lora_testing_bounded_wait", "lora_testing_gemm_streamk", "lora_testing_xpass_tma", "lora_testing_dual_blocking", "lora_timing_enable", "lora_timing_read",
     "lora_launch_count",
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
     "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
@@ -129,6 +129,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_testing_gemm_streamk.restype = i32
     lib.lora_testing_xpass_tma.argtypes = [i64, i64, i32]
     lib.lora_testing_xpass_tma.restype = i32
+    lib.lora_testing_dual_blocking.argtypes = [i64, i64, i32, i32, ctypes.POINTER(i32)]
+    lib.lora_testing_dual_blocking.restype = i32
     lib.lora_timing_enable.argtypes = [i32]
     lib.lora_timing_enable.restype = i32
     lib.lora_timing_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
@@ -270,6 +272,13 @@ def lora_device_status(workspace, stream=None) -> int:
 
 def lora_testing_bounded_wait(workspace, limit_ns: int, stream=None) -> int:
     return int(_lib.lora_testing_bounded_wait(_ptr(workspace), int(limit_ns), _stream(stream)))
+
+
+def lora_testing_dual_blocking(M: int, C: int, r: int, mode: int = 0):
+    """(used, (a, b, row_tiles, col_tiles)) of the one-pass kernel over [M, C] at rank r."""
+    out = (ctypes.c_int32 * 4)()
+    used = int(_lib.lora_testing_dual_blocking(int(M), int(C), int(r), int(mode), out))
+    return used, tuple(int(v) for v in out)
 
 
 def lora_testing_xpass_tma(M: int, K: int, r: int) -> int:

@@ -1309,6 +1309,16 @@ int32_t lora_testing_gemm_streamk(int64_t M, int64_t Nout, int64_t Kred, int32_t
   return static_cast<int32_t>(tiles - g.dp_tiles);
 }
 
+int32_t lora_testing_dual_blocking(int64_t M, int64_t C, int32_t r, int32_t mode, int32_t* out4) {
+  if (!out4 || M <= 0 || C <= 0 || r < 1 || r > 128 || mode < DP_BOTH || mode > DP_COLS) return -1;
+  const DualSplit d = dual_split(M, C, r, mode);
+  out4[0] = d.a;
+  out4[1] = d.b;
+  out4[2] = d.row_tiles;
+  out4[3] = d.col_tiles;
+  return d.use ? 1 : 0;
+}
+
 int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r) {
   if (M <= 0 || K <= 0 || r < 1 || r > 128) return -1;
   return (dual_split(M, K, r, DP_ROWS).use ? 1 : 0) | (dual_split(M, K, r, DP_COLS).use ? 2 : 0);
