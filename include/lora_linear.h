@@ -30,6 +30,11 @@
  *     anything is enqueued; on a validation error nothing is enqueued.
  *   - Device pointers must be 16-byte aligned (LORA_ERR_ALIGNMENT otherwise).
  *   - Results are deterministic: the same inputs give the same bits on every call.
+ *   - lora_linear_fwd / lora_linear_bwd (and the grouped, feed-forward and cross-entropy
+ *     calls) only enqueue kernels on `stream`, so a CUDA stream capture records them; the
+ *     first call on a device sets kernel attributes and looks up a driver entry point
+ *     and must come before any capture.  A replay reads and writes the buffers given at
+ *     capture time.
  *   - Limits: 8 <= r <= 128 with r % 8 == 0; N % 8 == 0 and K % 8 == 0 (bf16 weight),
  *     K % 64 == 0 (4-bit weight) or K % 16 == 0 (8-bit weights); M >= 0 (M == 0 is an empty batch);
  *     s finite.  Sizes outside these give LORA_ERR_UNSUPPORTED (r, alignment of sizes)
