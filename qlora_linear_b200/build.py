@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblora_linear.so")
 SOURCES = ["lora_api.cu"]
-HEADERS = ["ptx.cuh", "dequant.cuh", "gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "skinny.cuh", "dualproj.cuh", "elementwise.cuh"]
+HEADERS = ["ptx.cuh", "dequant.cuh", "gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "skinny.cuh", "dualproj.cuh", "elementwise.cuh", "streamk.cuh"]
 
 
 def nvcc_path() -> str:

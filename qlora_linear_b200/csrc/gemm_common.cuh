@@ -149,41 +149,6 @@ __device__ __forceinline__ void epi_slot_chunk(const PairParams& p, const uint32
                                                   __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
 }
 
-// Output tiles that stream-K cut into pieces: block (x, y) handles the tile in which the
-// boundary between pairs x and x + 1 falls (if that boundary is the tile's first), rows
-// [y·TILE_ROWS/gridDim.y, ...) of it, and writes out = bf16(Σ of the tile's pieces) with
-// the pieces added in pair order.
-template <int TILE_ROWS>
-__global__ void streamk_fixup_kernel(const float* __restrict__ kpart, __nv_bfloat16* __restrict__ out, int M, int Nout,
-                                     int num_m, int num_n, int group_m, int dp_tiles, int ntiles, int L, int P) {
-  const int p = blockIdx.x + 1;
-  const long long F = static_cast<long long>(ntiles - dp_tiles) * L;
-  const long long b = static_cast<long long>(p) * F / P;
-  if (b % L == 0) return;  // the boundary falls between two tiles
-  const long long ts = (b / L) * L, te = ts + L;
-  if (static_cast<long long>(p - 1) * F / P > ts) return;  // an earlier boundary lies in this tile
-  int mb, nb;
-  pair_tile_coords(dp_tiles + static_cast<int>(b / L), num_m, num_n, group_m, mb, nb);
-  const int rows = TILE_ROWS / gridDim.y;
-  for (int e = threadIdx.x; e < rows * 32; e += blockDim.x) {
-    const int lr = blockIdx.y * rows + e / 32, lc = (e % 32) * 8;
-    const int row = mb * TILE_ROWS + lr, col = nb * 256 + lc;
-    if (row >= M || col >= Nout) continue;
-    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int q = p - 1; q < P; ++q) {
-      const long long gq = static_cast<long long>(q) * F / P;
-      if (gq >= te) break;
-      const int slot = gq >= ts ? 2 * q : 2 * q + 1;
-      const float4* src = reinterpret_cast<const float4*>(kpart + (static_cast<size_t>(slot) * TILE_ROWS + lr) * 256 + lc);
-      const float4 x = src[0], y = src[1];
-      a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
-      a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
-    }
-    *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * Nout + col) =
-        make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
-  }
-}
-
 // 32 accumulator columns of one row to bf16 out[row, col0 ..].
 __device__ __forceinline__ void epi_store_chunk(const PairParams& p, const uint32_t (&v)[32], int row, int col0) {
   __nv_bfloat16* orow = p.out + static_cast<size_t>(row) * p.Nout;

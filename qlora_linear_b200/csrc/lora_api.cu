@@ -20,6 +20,7 @@
 #include "gemm_pair.cuh"
 #include "gemm_q.cuh"
 #include "skinny.cuh"
+#include "streamk.cuh"
 
 namespace lora {
 namespace {
@@ -623,7 +624,7 @@ lora_status_t streamk_fixup(const PairParams& p, const GemmSched& g, cudaStream_
   if (!g.sk) return LORA_OK;
   const int num_m = cdiv(p.M, g.tile_rows), num_n = cdiv(p.Nout, 256);
   const int group_m = g.tile_rows == 512 ? (p.group_m > 1 ? p.group_m / 2 : 1) : p.group_m;
-  const dim3 grid(kGemmPairs - 1, 8);
+  const dim3 grid(kGemmPairs - 1, g.tile_rows / 8);  // 8 tile rows per block
   if (g.tile_rows == 512)
     streamk_fixup_kernel<512><<<grid, 256, 0, st>>>(p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m, g.dp_tiles,
                                                     num_m * num_n, g.tile_fills, kGemmPairs);
