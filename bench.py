@@ -4,11 +4,13 @@ One step = forward and backward of every projection of the workload (default: th
 Llama-8B MLP projections gate, up and down at M = 16384 tokens, r = 16, bf16 weight),
 with inputs resident in device memory.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|c4s|qkv|mlp|ce] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c1|c3|c4|c4s|qkv|mlp|ce] [--impl ours|reference]
+    python bench.py --workload c4 [--select M=512,r=16,fmt=block4,N=28672]   (rank sweep, one line for the set)
 
 Multi-GPU (one process per GPU under torch.distributed.run): data parallel over tokens,
 every rank runs the full per-rank workload (weak scaling) and the adapter gradients dA
-and dB are summed across ranks with NCCL, the layer's one exchange step.
+and dB, written in fp32, are summed across ranks with one NCCL all-reduce per step (the
+layer's one exchange step) and rounded to bf16 once.
 """
 from __future__ import annotations
 
@@ -28,6 +30,7 @@ if ROOT not in sys.path:
 
 METRIC = "LoRA linear fwd+bwd TFLOP/s & tokens/s; % of B200 BF16 tensor peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, datasheet figure
 
 
 def workload(name: str):
@@ -37,6 +40,8 @@ def workload(name: str):
         cases = [blk.gate_up_case(), blk.down_case()]
     elif name == "c4s":
         cases = [c for c in CONFIGS["c4"] if c.M == 512 and c.r == 16 and c.fmt == "bf16"]
+    elif name == "c4":
+        cases = list(CONFIGS["c4"])
     elif name == "ce":
         # the LM head as a projection: M tokens, K = D, N = V (no adapter; r only sizes nothing)
         from synth import LoraCase
@@ -49,6 +54,8 @@ def workload(name: str):
               "M=16384, r=16, alpha=32, bf16 weight",
         "c3": "QLoRA 4-bit blockwise weight K=4096 N=14336 (16-level codebook, fp16 absmax per 64), "
               "M=8192, r=16, alpha=32",
+        "c4": "wide-model rank sweep: K=N=8192 and K=8192 N=28672, M in {512, 4096, 16384}, r in {8, 16, 64, 128}, "
+              "alpha=2r, bf16 and 4-bit blockwise weights (each case timed on its own, L2 flushed before every step)",
         "c4s": "rank-sweep shapes at the smallest batch: M=512, K=N=8192 and K=8192 N=28672, r=16, alpha=32, "
                "bf16 weight (the most weight-heavy cases; L2 flushed before every step)",
         "ce": "cross-entropy over the Llama-3 LM head (V=128256, D=4096), M=16384 tokens, backward in "
@@ -59,6 +66,21 @@ def workload(name: str):
                "M=8192, r=16 per projection, alpha=32, bf16 weight",
     }[name]
     return cases, desc
+
+
+def select_cases(cases, spec: str):
+    """Cases whose fields match every key of `spec` ("M=512,r=16,fmt=block4"); a key
+    given more than once matches any of its values."""
+    want: dict[str, set] = {}
+    for item in spec.split(","):
+        if not item.strip():
+            continue
+        k, _, v = item.partition("=")
+        k, v = k.strip(), v.strip()
+        if k not in ("M", "N", "K", "r", "fmt"):
+            raise SystemExit(f"--select: unknown key {k!r} (M, N, K, r, fmt)")
+        want.setdefault(k, set()).add(v if k == "fmt" else int(v))
+    return [c for c in cases if all(getattr(c, k) in vs for k, vs in want.items())]
 
 
 def ce_flops(c) -> float:
@@ -107,20 +129,49 @@ def cpu_threads() -> int:
 
 
 # ---------------------------------------------------------------------------- clocks
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+MIN_CLOCK_SAMPLES = 10
+
+
 class ClockSampler:
-    """Samples SM clock and throttle reasons with nvidia-smi while running."""
+    """Samples the SM clock, its maximum, board power and the active clock-event
+    (throttle) reasons while the benchmark runs: through NVML every 10 ms (read-only
+    queries), else through `nvidia-smi -lms 100`.  Each sample is a tuple
+    (time, sm_mhz, sm_max_mhz, power_w, set of reason names)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
+    def __init__(self, gpu_id: str, index: int = 0, period_s: float = 0.01):
         self.gpu_id = gpu_id
+        self.index = index
+        self.period_s = period_s
         self.proc = None
-        self.lines = []
+        self.samples = []
         self.thread = None
+        self.stop_ev = threading.Event()
+        self.source = None
+        self.marks = {}
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h, bits), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -128,49 +179,73 @@ class ClockSampler:
         except Exception:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi"
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    def _poll_nvml(self, nv, h, bits):
+        smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop_ev.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rb = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.time(), sm, smax, pw, {n for n, b in bits.items() if rb & b}))
+            except Exception:
+                pass
+            self.stop_ev.wait(self.period_s)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
-
-    def mark(self, which: str):
-        setattr(self, which, time.time())
-
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        if self.thread:
-            self.thread.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        t0 = getattr(self, "t_start", 0.0)
-        t1 = getattr(self, "t_end", float("inf"))
-        window = [ln for ts, ln in self.lines if t0 <= ts <= t1 + 0.1]
-        if not window:  # timed region shorter than the sampling period: nearest samples
-            window = [ln for ts, ln in self.lines if ts >= t0][:2] or [ln for _, ln in self.lines[-2:]]
-        for ln in window:
-            parts = [p.strip() for p in ln.split(",")]
+            parts = [p.strip() for p in line.strip().split(",")]
             if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
+                sm, smax = float(parts[0]), float(parts[1])
+                pw = float(parts[2]) if parts[2] not in ("", "[N/A]") else 0.0
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+            reasons = {nm for nm, v in zip(REASON_NAMES, parts[4:8]) if v.lower() == "active"}
+            self.samples.append((time.time(), sm, smax, pw, reasons))
+
+    def mark(self, which: str):
+        self.marks[which] = time.time()
+
+    def stop(self):
+        self.stop_ev.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0_mark: str, t1_mark: str, wide_mark: str | None = None):
+        """Clock record of the region between two marks.  When that region holds fewer
+        than MIN_CLOCK_SAMPLES samples, the window opens back to `wide_mark` (the start
+        of the warm-up steps, which run the same work) and says so."""
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        t0, t1 = self.marks.get(t0_mark, 0.0), self.marks.get(t1_mark, float("inf"))
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(win) < MIN_CLOCK_SAMPLES and wide_mark is not None:
+            tw = self.marks.get(wide_mark, t0)
+            win = [s for s in self.samples if tw <= s[0] <= t1]
+            window = "warm-up and timed region (the timed region alone held fewer than " \
+                     f"{MIN_CLOCK_SAMPLES} samples)"
+        if not win:
+            win = self.samples[-MIN_CLOCK_SAMPLES:]
+            window = "last samples before the end of the timed region"
+        reasons = set().union(*(s[4] for s in win))
+        capped = sum(1 for s in win if "sw_power_cap" in s[4])
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": max(s[2] for s in win),
+                "sm_min_mhz": min(s[1] for s in win), "power_w_max": max(s[3] for s in win),
+                "reasons": sorted(reasons), "samples": len(win), "samples_power_capped": capped,
+                "window": window, "source": self.source,
+                "period_ms": self.period_s * 1e3 if self.source == "nvml" else 100.0}
 
 
 def gpu_uuid(dev) -> str:
@@ -321,16 +396,26 @@ class LinearSet:
             }
             self.layers.append(layer)
             self.data.append((d, out))
+        # data parallel: every projection's fp32 adapter gradients in one exchange buffer,
+        # summed over ranks by one all-reduce per step and rounded to bf16 once
+        self.exchange = None
+        if world > 1:
+            shapes = [s for _, o in self.data for s in (o["dA"].shape, o["dB"].shape)]
+            self.exchange = q.AdapterGradExchange(shapes, dev)
 
     def step(self, inputs=None):
-        import qlora_linear_b200 as q
         for i, (layer, (d, o)) in enumerate(zip(self.layers, self.data)):
             X = d["X"] if inputs is None else inputs[i]["X"]
             dY = d["dY"] if inputs is None else inputs[i]["dY"]
             layer.forward(X, Y=o["Y"], XA=o["XA"])
-            layer.backward(dY, X, o["XA"], out=(o["dX"], o["dA"], o["dB"]))
-            if self.world > 1:
-                q.allreduce_adapter_grads(o["dA"], o["dB"])
+            if self.exchange is None:
+                layer.backward(dY, X, o["XA"], out=(o["dX"], o["dA"], o["dB"]))
+            else:
+                v = self.exchange.views
+                layer.backward(dY, X, o["XA"], out=(o["dX"], v[2 * i], v[2 * i + 1]), grads_f32=True)
+        if self.exchange is not None:
+            self.exchange.allreduce()
+            self.exchange.round_into([t for _, o in self.data for t in (o["dA"], o["dB"])])
 
     def statuses(self):
         import qlora_linear_b200 as q
@@ -366,16 +451,18 @@ class MlpSet:
                       torch.empty((self.D, self.r), dtype=bf, device=dev))
         self.layers = [self.mlp]
         self.data = []
+        self.exchange = q.AdapterGradExchange([g.shape for g in self.grads[1:]], dev) if world > 1 else None
 
     def step(self, inputs=None):
-        import qlora_linear_b200 as q
         X = self.inputs["X"] if inputs is None else inputs["X"]
         dZ = self.inputs["dZ"] if inputs is None else inputs["dZ"]
         self.mlp.forward(X, Z=self.Z, saved=self.saved)
-        self.mlp.backward(dZ, X, self.saved, out=self.grads)
-        if self.world > 1:
-            q.allreduce_adapter_grads(self.grads[1], self.grads[2])
-            q.allreduce_adapter_grads(self.grads[3], self.grads[4])
+        if self.exchange is None:
+            self.mlp.backward(dZ, X, self.saved, out=self.grads)
+        else:
+            self.mlp.backward(dZ, X, self.saved, out=(self.grads[0], *self.exchange.views), grads_f32=True)
+            self.exchange.allreduce()
+            self.exchange.round_into(list(self.grads[1:]))
 
     def statuses(self):
         import qlora_linear_b200 as q
@@ -594,12 +681,152 @@ def time_separate_mlp(args, cases, ws, dev):
                     "torch elementwise ops in fp32, dX of gate and up summed by torch"}
 
 
+def gemm_roofline(cases, ce, steps, fwd_ms, bwd_ms, g_launches, step_ms, peaks, clk):
+    """Roofline of the dominant kernel, the tcgen05 GEMM (its Y and dX launches):
+    algorithmic FLOPs of those launches over their summed CUDA-event time, against the
+    measured dense bf16 peak.  `frac` is always against the burst peak (the GEMM is timed
+    inside a region of well under a minute); the sustained peak and a clock-normalised
+    figure (the same launches at the maximum SM clock, time x median MHz / max MHz) are
+    reported beside it."""
+    gflops = (ce_flops(cases[0]) if ce else sum(sum(gemm_flops(c)) for c in cases)) * steps
+    g_ms = fwd_ms + bwd_ms
+    achieved = gflops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    at_max = None
+    if achieved and clk and clk.get("sm_mhz"):
+        at_max = achieved * clk["sm_max_mhz"] / clk["sm_mhz"]
+    return {
+        "bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+        "frac": achieved / peak_burst if achieved else None,
+        "peak_source": "bf16_tflops (burst) of MEASURED_PEAKS.json" if "bf16_tflops" in peaks
+                       else "fallback burst figure",
+        "frac_of_sustained": achieved / peak_sust if achieved else None,
+        "achieved_at_max_clock": at_max,
+        "frac_at_max_clock": at_max / peak_burst if at_max else None,
+        "launches": g_launches, "avg_launch_ms": g_ms / g_launches if g_launches else None,
+        "gemm_share_of_step": g_ms / (step_ms * steps) if step_ms > 0 else None,
+    }
+
+
+def time_steps(q, torch, step, steps, stream, flush_buf=None):
+    """Runs `steps` steps between two CUDA events on `stream` and returns (ms per step,
+    GEMM fwd ms, GEMM bwd ms, GEMM launches, library launches).  With `flush_buf`, a
+    buffer larger than L2 is rewritten before every step, outside that step's events."""
+    q.lora_timing_enable(True)
+    q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
+    q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
+    launches0 = q.lora_launch_count()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    e0.record(stream)
+    for i in range(steps):
+        if flush_buf is not None:
+            flush_buf.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+        step()
+        if flush_buf is not None:
+            ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = q.lora_launch_count() - launches0
+    q.lora_timing_enable(False)
+    fwd_ms, fwd_n = q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
+    bwd_ms, bwd_n = q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
+    ms = (sum(a.elapsed_time(b) for a, b in ev) if flush_buf is not None else e0.elapsed_time(e1)) / steps
+    return ms, fwd_ms, bwd_ms, fwd_n + bwd_n, launches
+
+
+def run_sweep(args, cases, desc, rank, world, local_rank):
+    """The rank sweep (one projection per case): each case is built, warmed up and timed
+    on its own (forward + backward per step, L2 flushed before every step, outside the
+    step's events), then freed.  The line's value is the algorithmic FLOPs of one pass
+    over every selected case divided by the sum of their per-step times; `sweep` lists
+    each case."""
+    import torch
+    import torch.distributed as dist
+
+    import qlora_linear_b200 as q
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    clocks = ClockSampler(gpu_uuid(dev), local_rank)
+    clocks.start()
+    rows, tot_ms, tot_flops, tot_launches = [], 0.0, 0.0, 0
+    g_ms_all, g_fl_all = 0.0, 0.0
+    clocks.mark("t_warm")
+    clocks.mark("t_start")
+    for c in cases:
+        ws = LinearSet([c], dev, rank, world)
+        for _ in range(args.warmup):
+            ws.step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms, fwd_ms, bwd_ms, g_n, launches = time_steps(q, torch, ws.step, args.steps, stream, flush_buf)
+        if world > 1:
+            t = torch.tensor([ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        for st in ws.statuses():
+            if st != q.LORA_OK:
+                raise RuntimeError(f"device status after {c.name}: " + q.status_string(st))
+        fl = case_flops(c)
+        gfl = sum(gemm_flops(c)) * args.steps
+        g_ms = fwd_ms + bwd_ms
+        rows.append({
+            "case": c.name, "M": c.M, "N": c.N, "K": c.K, "r": c.r, "fmt": c.fmt, "ms_per_step": ms,
+            "tflops": fl / (ms * 1e-3) / 1e12, "frac_of_burst": fl / (ms * 1e-3) / 1e12 / peaks.get(
+                "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+            "tokens_per_s": c.M / (ms * 1e-3),
+            "gemm_tflops": gfl / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None,
+            "gemm_share": g_ms / (ms * args.steps) if ms > 0 else None,
+            "rank_r_passes_share": 1.0 - g_ms / (ms * args.steps) if ms > 0 else None,
+            "hbm_floor_gbs": case_bytes(c) / (ms * 1e-3) / 1e9,
+            "hbm_floor_frac": case_bytes(c) / (ms * 1e-3) / 1e9 / hbm,
+            "launches_per_step": launches / args.steps,
+        })
+        tot_ms += ms
+        tot_flops += fl
+        tot_launches += launches
+        g_ms_all += g_ms
+        g_fl_all += gfl
+        del ws
+        torch.cuda.empty_cache()
+    clocks.mark("t_end")
+    clocks.stop()
+    clk = clocks.summary("t_start", "t_end", "t_warm")
+    achieved = g_fl_all / (g_ms_all * 1e-3) / 1e12 if g_ms_all > 0 else None
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * tot_flops / (tot_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, drawn on device)",
+            "config": {"workload": desc, "cases": len(cases), "parallelism": f"dp{world}",
+                       "l2": "L2 flushed (512 MB written) before every timed step, outside its events",
+                       "step": "one forward + backward of every selected case, each timed on its own"},
+            "tokens_per_s": world * sum(c.M for c in cases) / (tot_ms * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                         "frac": achieved / peak_burst if achieved else None, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 dense, burst"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": tot_launches, "clocks": clk,
+            "sweep": rows,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, cases, desc, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
     import qlora_linear_b200 as q
-    from synth.device import make_case_device
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -619,6 +846,12 @@ def run_ours(args, cases, desc, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    # the clock record covers the warm-up steps too (the same work), so a short timed
+    # region still has enough samples
+    clocks = ClockSampler(gpu_uuid(dev), local_rank)
+    clocks.start()
+    time.sleep(0.05)
+    clocks.mark("t_warm")
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -627,39 +860,16 @@ def run_ours(args, cases, desc, rank, world, local_rank):
             raise RuntimeError("device status after warm-up: " + q.status_string(st))
 
     # ---- timed region: K steps, device time (CUDA events), max over ranks
-    clocks = ClockSampler(gpu_uuid(dev))
-    clocks.start()
-    time.sleep(0.3)
-    q.lora_timing_enable(True)
-    q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
-    q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
-    launches0 = q.lora_launch_count()
+    flush = args.workload == "c4s"  # working set near the L2 size: flush it before every step
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if flush else None
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    flush = args.workload == "c4s"  # working set near the L2 size: flush it before every step
-    if flush:
-        flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks.mark("t_start")
-    e0.record(stream)
-    for i in range(args.steps):
-        if flush:
-            flush_buf.fill_(i & 0xFF)  # outside the step's events
-            ev[i][0].record(stream)
-        step()
-        if flush:
-            ev[i][1].record(stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    ms, fwd_ms, bwd_ms, g_launches, launches = time_steps(q, torch, step, args.steps, stream, flush_buf)
     clocks.mark("t_end")
     barrier()
-    launches = q.lora_launch_count() - launches0
-    q.lora_timing_enable(False)
-    fwd_ms, fwd_n = q.lora_timing_read(q.LORA_KERNEL_FWD_GEMM)
-    bwd_ms, bwd_n = q.lora_timing_read(q.LORA_KERNEL_BWD_GEMM)
-    clk = clocks.stop()
-    ms = (sum(a.elapsed_time(b) for a, b in ev) if flush else e0.elapsed_time(e1)) / args.steps
+    clocks.stop()
+    clk = clocks.summary("t_start", "t_end", "t_warm")
     if world > 1:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -673,35 +883,17 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     tokens_step = cases[0].M
     value = world * flops_step / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
+    peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
 
     # ---- roofline of the dominant kernel (the tcgen05 GEMM: Y and dX launches)
-    gflops = (ce_flops(cases[0]) if ce else sum(sum(gemm_flops(c)) for c in cases)) * args.steps
-    g_ms = fwd_ms + bwd_ms
-    g_launches = fwd_n + bwd_n
-    achieved = gflops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
-    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    # burst peak while the clocks stayed up; the sustained one once the power cap bit or a
-    # clock well below max was seen during the timed region
-    capped = bool(clk) and ("sw_power_cap" in clk["reasons"] or clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])
-    peak = peak_sust if capped else peak_burst
+    roofline = gemm_roofline(cases, ce, args.steps, fwd_ms, bwd_ms, g_launches, ms, peaks, clk)
+    roofline["kernel"] = ("lora_gemm_pair_kernel" if all(c.fmt == "bf16" for c in cases) else
+                          "lora_gemm_q_kernel" if all(c.fmt != "bf16" for c in cases) else
+                          "lora_gemm_pair_kernel / lora_gemm_q_kernel") + " (Y and dX GEMMs)"
     tr = traffic_record()
-    traffic = None
+    roofline["traffic"] = None
     if tr and tr.get("source_hash") == source_hash() and tr.get("workload") == args.workload:
-        traffic = tr.get("bytes_per_launch")
-    roofline = {
-        "kernel": ("lora_gemm_pair_kernel" if all(c.fmt == "bf16" for c in cases) else
-                   "lora_gemm_q_kernel" if all(c.fmt != "bf16" for c in cases) else
-                   "lora_gemm_pair_kernel / lora_gemm_q_kernel") + " (Y and dX GEMMs)",
-        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-        "frac": achieved / peak if achieved else None, "traffic": traffic,
-        "peak_source": f"{peak_src} bf16 dense, " + ("sustained (power cap or low clock seen)" if capped
-                                                     else "burst (clocks stayed at max)"),
-        "frac_of_burst": achieved / peak_burst if achieved else None,
-        "frac_of_sustained": achieved / peak_sust if achieved else None,
-        "launches": g_launches, "avg_launch_ms": g_ms / g_launches if g_launches else None,
-        "gemm_share_of_step": g_ms / (ms * args.steps) if ms > 0 else None,
-    }
+        roofline["traffic"] = tr.get("bytes_per_launch")
 
     # ---- grouped workloads: the same projections as separate layers, for comparison
     separate = None
@@ -750,6 +942,7 @@ def run_ours(args, cases, desc, rank, world, local_rank):
             "tokens_per_s": world * tokens_step / (ms * 1e-3),
             "pct_peak_burst": value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
             "pct_peak_sustained": value / world / peak_sust,
+            "pct_peak_nominal": value / world / NOMINAL_BF16_TFLOPS,
             "peak_source": peak_src,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk,
@@ -882,6 +1075,8 @@ def run_e2e(args, cases, layers, data, step, world, dev, outs=("dA", "dB")):
         lay_b.append(row)
     dev_out = [[{k2: torch.empty_like(o[k2]) for k2 in ("Y", "XA", "dX", "dA", "dB")} for _, o in data]
                for _ in range(NB)]
+    ex = [[q.AdapterGradExchange([o["dA"].shape, o["dB"].shape], dev) for _, o in data] for _ in range(NB)] \
+        if world > 1 else None
     ev_in = [[torch.cuda.Event() for _ in data] for _ in range(NB)]
     ev_comp = [torch.cuda.Event() for _ in range(NB)]
     ev_out = [[torch.cuda.Event() for _ in data] for _ in range(NB)]
@@ -906,9 +1101,14 @@ def run_e2e(args, cases, layers, data, step, world, dev, outs=("dA", "dB")):
             s_comp.wait_event(ev_out[b][i])  # this buffer's previous outputs have been read back
             X = dev_x[b][x_of[i]]
             layer.forward(X, Y=o["Y"], XA=o["XA"], stream=s_comp)
-            layer.backward(dev_dy[b][i], X, o["XA"], out=(o["dX"], o["dA"], o["dB"]), stream=s_comp)
-            if world > 1:
-                q.allreduce_adapter_grads(o["dA"], o["dB"])
+            if world == 1:
+                layer.backward(dev_dy[b][i], X, o["XA"], out=(o["dX"], o["dA"], o["dB"]), stream=s_comp)
+            else:
+                v = ex[b][i].views
+                layer.backward(dev_dy[b][i], X, o["XA"], out=(o["dX"], v[0], v[1]), stream=s_comp, grads_f32=True)
+                with torch.cuda.stream(s_comp):
+                    ex[b][i].allreduce()
+                    ex[b][i].round_into([o["dA"], o["dB"]])
             ev = torch.cuda.Event()
             ev.record(s_comp)
             s_d2h.wait_event(ev)
@@ -954,7 +1154,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "c4s", "qkv", "mlp", "ce"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "c4", "c4s", "qkv", "mlp", "ce"])
+    ap.add_argument("--select", default=None,
+                    help="rank sweep only: comma-separated key=value filters on M, N, K, r and fmt "
+                         "(a key may repeat: M=512,M=4096)")
     ap.add_argument("--only", default=None, help="run a single projection of the workload (e.g. c2_gate)")
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -974,6 +1177,11 @@ def main(argv=None):
         import dataclasses
         cases = [dataclasses.replace(c, fmt=args.weight) for c in cases]
         desc = f"{desc}; frozen weights stored as {args.weight}"
+    if args.select:
+        cases = select_cases(cases, args.select)
+        if not cases:
+            raise SystemExit(f"no case of {args.workload} matches {args.select}")
+        desc = f"{desc}; selected {args.select}"
     if args.only:
         cases = [c for c in cases if c.name == args.only]
         if not cases:
@@ -990,7 +1198,10 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, cases, desc, rank, world, local_rank)
+        if args.workload == "c4":
+            run_sweep(args, cases, desc, rank, world, local_rank)
+        else:
+            run_ours(args, cases, desc, rank, world, local_rank)
     finally:
         if world > 1 and dist.is_initialized():
             dist.destroy_process_group()

@@ -138,6 +138,36 @@ lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int
                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Adapter gradients in fp32, for data-parallel training.  When the tokens of a batch are
+ * split over several GPUs (data parallelism over M), dA and dB are sums over tokens and
+ * therefore sums over the GPUs' partial results; summing those partials in bf16 would
+ * round every rank's gradient and the sum again.  With flags = LORA_GRADS_F32 the
+ * backward writes dA [G·r, K] and dB [N, r] as fp32 (the same sums, scaled by s, without
+ * the final rounding); the caller sums them over ranks (e.g. one NCCL all-reduce of a
+ * buffer holding both) and rounds the sum once with lora_round_bf16.  On one GPU,
+ * lora_round_bf16 of these fp32 gradients gives lora_linear_bwd's bf16 gradients bit for
+ * bit.  flags = 0 is exactly lora_linear_bwd; other bits give LORA_ERR_INVALID_ARG.
+ * Everything else (arguments, workspace, dX) is as for lora_linear_bwd.  The data-parallel
+ * layout — each rank holds the frozen weight and the adapter and processes its own
+ * tokens, the adapter gradients being the one exchange step — follows the distributed
+ * training paragraph of "Unsloth vs The Stack v2" (a data-parallel wrapper with a custom
+ * all-reduce), which names no precision for the exchange; fp32 is this library's choice.
+ */
+#define LORA_GRADS_F32 1u
+lora_status_t lora_linear_bwd_ex(const void* dY, const void* X, const void* XA, int64_t M,
+                                 const lora_weight_t* W, const void* A, const void* B,
+                                 int32_t r, float s,
+                                 void* dX, void* dA, void* dB, uint32_t flags,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * dst = bf16_rn(src) for n elements: src fp32 (device), dst bf16 (device, out; must not
+ * overlap src).  The one rounding of adapter gradients summed over ranks in fp32.
+ * n == 0 enqueues nothing; n < 0 gives LORA_ERR_INVALID_ARG.
+ */
+lora_status_t lora_round_bf16(const float* src, void* dst, int64_t n, void* stream);
+
+/*
  * Grouped projections sharing one input — e.g. the q, k and v projections of an
  * attention block, whose six adapter derivatives (dA and dB of each) "Unsloth vs
  * PyTorch: The ONLY Video You Need to Understand the Difference" counts at transcript
@@ -178,6 +208,14 @@ lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, in
                                const void* A, const void* B, int32_t r, float s,
                                void* dX, void* dA, void* dB,
                                void* workspace, size_t ws_bytes, void* stream);
+
+/* As lora_grouped_bwd; flags = LORA_GRADS_F32 writes dA and dB as fp32 (see
+ * lora_linear_bwd_ex). */
+lora_status_t lora_grouped_bwd_ex(const void* dY, const void* X, const void* XA, int64_t M,
+                                  const lora_weight_t* W, const lora_segments_t* segs,
+                                  const void* A, const void* B, int32_t r, float s,
+                                  void* dX, void* dA, void* dB, uint32_t flags,
+                                  void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Feed-forward block with LoRA on all three projections and SwiGLU gating ("Unsloth"
@@ -232,6 +270,13 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
                            const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s,
                            void* dX, void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down,
                            void* workspace, size_t ws_bytes, void* stream);
+
+/* As lora_mlp_bwd; flags = LORA_GRADS_F32 writes the four adapter gradients as fp32 (see
+ * lora_linear_bwd_ex). */
+lora_status_t lora_mlp_bwd_ex(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
+                              const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s,
+                              void* dX, void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down,
+                              uint32_t flags, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Cross-entropy over a frozen LM head without the [M, V] logits ("Unsloth" wiki entry,
@@ -302,12 +347,16 @@ lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, i
  * latency-critical code that must not call cudaMalloc/cudaFree because those calls
  * can synchronize the whole device and may fail under a fixed memory budget.
  *
- * Computes what lora_linear_fwd computes with the same kernels, except that every
- * output tile of the GEMM is computed whole (the stream-K schedule, which lora_linear_fwd
- * takes for some small outputs, needs more scratch; results then agree to the last few
- * bits of fp32 summation order), and keeps its scratch (s·XA and the split partial sums of X·Aᵀ)
- * in one fixed array of LORA_NOALLOC_SCRATCH_BYTES bytes that is part of the library
- * image: every GPU that loads the library holds that array until the process exits.
+ * Computes what lora_linear_fwd computes, with two differences of schedule, both because
+ * the larger partial-sum buffers they need do not fit the fixed scratch: X·Aᵀ always
+ * runs as the split pass over K whose partial sums are added in order (lora_linear_fwd
+ * takes a one-pass TMA-fed kernel for r <= 16 at most sizes), and every output tile of
+ * the GEMM is computed whole (lora_linear_fwd takes the stream-K schedule for some small
+ * outputs).  Both change only the order of fp32 additions, so XA and Y agree with
+ * lora_linear_fwd's within the parity tolerance, not necessarily bit for bit.  Its
+ * scratch (s·XA and the split partial sums of X·Aᵀ) is one fixed array of
+ * LORA_NOALLOC_SCRATCH_BYTES bytes that is part of the library image: every GPU that
+ * loads the library holds that array until the process exits.
  * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  *
  *   - Size limit: the scratch a problem needs is 2·M·r bytes for s·XA plus 4·S·M·r
@@ -317,8 +366,9 @@ lora_status_t lora_merge(const lora_weight_t* W, const void* A, const void* B, i
  *     9 000 tokens at r = 128.  A larger problem gets LORA_ERR_SCRATCH_LIMIT and
  *     nothing is enqueued.  Other arguments are validated as for lora_linear_fwd.
  *   - First call on each device: it looks up the device address of the array on that
- *     device (the current device) once and caches it.  Make this first call before
- *     any stream capture begins on that device.
+ *     device (the current device) and caches it for the current CUDA context; a
+ *     context created anew (after cudaDeviceReset) gets the lookup again on its first
+ *     call.  Make that first call before any stream capture begins on the device.
  *   - Shared state: all calls in the process share the one array per device, and the
  *     array keeps whatever the last call left in it.  Every scratch byte a call reads
  *     is written earlier by the same call, so nothing needs clearing between calls.

@@ -26,6 +26,8 @@ LORA_ERR_DEVICE_TIMEOUT = 6
 LORA_ERR_SCRATCH_LIMIT = 7
 LORA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
+LORA_GRADS_F32 = 1  # flags of the *_bwd_ex calls: adapter gradients as fp32
+
 LORA_W_BF16 = 0
 LORA_W_BLOCK4 = 1
 LORA_W_INT8 = 2
@@ -39,6 +41,7 @@ EXPORTED = (
     "lora_linear_fwd_noalloc", "lora_grouped_workspace_bytes", "lora_grouped_fwd", "lora_grouped_bwd",
     "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
     "lora_ce_workspace_bytes", "lora_ce_fwd", "lora_ce_bwd",
+    "lora_linear_bwd_ex", "lora_grouped_bwd_ex", "lora_mlp_bwd_ex", "lora_round_bf16",
 )
 
 LORA_MAX_SEGMENTS = 8
@@ -105,6 +108,11 @@ def _load() -> ctypes.CDLL:
     lib.lora_linear_fwd.restype = i32
     lib.lora_linear_bwd.argtypes = [vp, vp, vp, i64, W, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
     lib.lora_linear_bwd.restype = i32
+    u32 = ctypes.c_uint32
+    lib.lora_linear_bwd_ex.argtypes = [vp, vp, vp, i64, W, vp, vp, i32, f32, vp, vp, vp, u32, vp, sz, vp]
+    lib.lora_linear_bwd_ex.restype = i32
+    lib.lora_round_bf16.argtypes = [vp, vp, i64, vp]
+    lib.lora_round_bf16.restype = i32
     lib.dequant_blockwise4.argtypes = [W, vp, vp]
     lib.dequant_blockwise4.restype = i32
     lib.lora_dequant.argtypes = [W, vp, vp]
@@ -146,6 +154,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_grouped_fwd.restype = i32
     lib.lora_grouped_bwd.argtypes = [vp, vp, vp, i64, W, S, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
     lib.lora_grouped_bwd.restype = i32
+    lib.lora_grouped_bwd_ex.argtypes = [vp, vp, vp, i64, W, S, vp, vp, i32, f32, vp, vp, vp, u32, vp, sz, vp]
+    lib.lora_grouped_bwd_ex.restype = i32
     P = ctypes.POINTER(lora_mlp_t)
     lib.lora_mlp_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
     lib.lora_mlp_workspace_bytes.restype = sz
@@ -153,6 +163,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_mlp_fwd.restype = i32
     lib.lora_mlp_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, P, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.lora_mlp_bwd.restype = i32
+    lib.lora_mlp_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i64, P, i32, f32, vp, vp, vp, vp, vp, u32, vp, sz, vp]
+    lib.lora_mlp_bwd_ex.restype = i32
     return lib
 
 
@@ -247,6 +259,22 @@ def lora_linear_bwd(dY, X, XA, M: int, W: LoraWeight, A, B, r: int, s: float, dX
     _check(_lib.lora_linear_bwd(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r),
                                 float(s), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), int(nb), _stream(stream)),
            "lora_linear_bwd")
+
+
+def lora_linear_bwd_ex(dY, X, XA, M: int, W: LoraWeight, A, B, r: int, s: float, dX, dA, dB, flags: int, workspace,
+                       ws_bytes=None, stream=None) -> None:
+    """lora_linear_bwd with flags; LORA_GRADS_F32 writes dA and dB as fp32 tensors."""
+    w = W.c_struct()
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_linear_bwd_ex(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), _ptr(A), _ptr(B), int(r),
+                                   float(s), _ptr(dX), _ptr(dA), _ptr(dB), int(flags), _ptr(workspace), int(nb),
+                                   _stream(stream)), "lora_linear_bwd_ex")
+
+
+def lora_round_bf16(src, dst, n: int | None = None, stream=None) -> None:
+    """dst (bf16) = round-to-nearest-even of src (fp32), n elements (default: all of src)."""
+    n = src.numel() if n is None else int(n)
+    _check(_lib.lora_round_bf16(_ptr(src), _ptr(dst), n, _stream(stream)), "lora_round_bf16")
 
 
 def lora_dequant(W: LoraWeight, W_out, stream=None) -> None:
@@ -348,6 +376,16 @@ def lora_grouped_bwd(dY, X, XA, M: int, W: LoraWeight, rows, A, B, r: int, s: fl
                                  _stream(stream)), "lora_grouped_bwd")
 
 
+def lora_grouped_bwd_ex(dY, X, XA, M: int, W: LoraWeight, rows, A, B, r: int, s: float, dX, dA, dB, flags: int,
+                        workspace, ws_bytes=None, stream=None) -> None:
+    w = W.c_struct()
+    seg = segments(rows)
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_grouped_bwd_ex(_ptr(dY), _ptr(X), _ptr(XA), int(M), ctypes.byref(w), ctypes.byref(seg),
+                                    _ptr(A), _ptr(B), int(r), float(s), _ptr(dX), _ptr(dA), _ptr(dB), int(flags),
+                                    _ptr(workspace), int(nb), _stream(stream)), "lora_grouped_bwd_ex")
+
+
 def mlp_workspace_bytes(M: int, D: int, I: int, r: int, fmt: int = LORA_W_BF16) -> int:
     return int(_lib.lora_mlp_workspace_bytes(int(M), int(D), int(I), int(r), int(fmt)))
 
@@ -374,6 +412,15 @@ def lora_mlp_bwd(dZ, X, GU, H, XA_gate_up, XA_down, M: int, mlp: lora_mlp_t, r: 
                              ctypes.byref(mlp), int(r), float(s), _ptr(dX), _ptr(dA_gate_up), _ptr(dB_gate_up),
                              _ptr(dA_down), _ptr(dB_down), _ptr(workspace), int(nb), _stream(stream)),
            "lora_mlp_bwd")
+
+
+def lora_mlp_bwd_ex(dZ, X, GU, H, XA_gate_up, XA_down, M: int, mlp: lora_mlp_t, r: int, s: float, dX, dA_gate_up,
+                    dB_gate_up, dA_down, dB_down, flags: int, workspace, ws_bytes=None, stream=None) -> None:
+    nb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.lora_mlp_bwd_ex(_ptr(dZ), _ptr(X), _ptr(GU), _ptr(H), _ptr(XA_gate_up), _ptr(XA_down), int(M),
+                                ctypes.byref(mlp), int(r), float(s), _ptr(dX), _ptr(dA_gate_up), _ptr(dB_gate_up),
+                                _ptr(dA_down), _ptr(dB_down), int(flags), _ptr(workspace), int(nb), _stream(stream)),
+           "lora_mlp_bwd_ex")
 
 
 def ce_workspace_bytes(M: int, D: int, V: int, slice_: int = 0) -> int:

@@ -225,9 +225,31 @@ WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg, bool
 }
 
 // ---------------------------------------------------------------- device info
+// The current CUDA context (driver API, looked up through the runtime).  Per-device
+// state cached by this library (kernel attributes, the device address of the fixed
+// scratch of lora_linear_fwd_noalloc) belongs to one context: after cudaDeviceReset
+// the primary context is created anew and that state is set up again.
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+
+// The context current on this thread, or nullptr when none is (yet).
+CUcontext current_ctx() {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && fn)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  });
+  CUcontext c = nullptr;
+  if (!g_ctx_current || g_ctx_current(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 struct DevInfo {
   int sms = 0;
   bool attrs_set = false;
+  CUcontext ctx = nullptr;  // context the attributes were set in
 };
 std::mutex g_mu;
 DevInfo g_dev[64];
@@ -235,8 +257,12 @@ DevInfo g_dev[64];
 lora_status_t dev_info(DevInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  // No current context (a thread's first call) or another one than the attributes were
+  // set in: set them again; cudaFuncSetAttribute makes the primary context current.
+  const CUcontext ctx = current_ctx();
   std::lock_guard<std::mutex> lk(g_mu);
   DevInfo& d = g_dev[dev];
+  if (!ctx || d.ctx != ctx) d.attrs_set = false;
   if (d.sms == 0) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LORA_ERR_CUDA;
   }
@@ -276,6 +302,8 @@ lora_status_t dev_info(DevInfo** out) {
     SET_SMEM((colproj_kernel<128>), (colproj_smem_bytes<128>()));
 #undef SET_SMEM
     if (!ok) return LORA_ERR_CUDA;
+    d.ctx = current_ctx();
+    if (!d.ctx) return LORA_ERR_CUDA;
     d.attrs_set = true;
   }
   *out = &d;
@@ -447,13 +475,24 @@ lora_status_t finalize_rows(const float* part, int splits, long long rows, int r
   return last_launch();
 }
 
-// scale · Σ of the split partials [splits][C][r] -> out [C][r], or [r][C] if transpose.
-lora_status_t finalize_cols(const float* part, int splits, int C, int r, float scale, bool transpose,
-                            __nv_bfloat16* out, cudaStream_t st) {
+// scale · Σ of the split partials [splits][C][r] -> out [C][r], or [r][C] if transpose;
+// out is bf16, or fp32 when f32 (adapter gradients summed over ranks before rounding).
+lora_status_t finalize_cols(const float* part, int splits, int C, int r, float scale, bool transpose, void* out,
+                            bool f32, cudaStream_t st) {
   const size_t n = static_cast<size_t>(C) * r;
-  finalize_cols_kernel<<<finalize_grid(n), 256, 0, st>>>(part, splits, C, r, scale, transpose ? 1 : 0, out);
+  if (f32)
+    finalize_cols_kernel<float><<<finalize_grid(n), 256, 0, st>>>(part, splits, C, r, scale, transpose ? 1 : 0,
+                                                                  static_cast<float*>(out));
+  else
+    finalize_cols_kernel<__nv_bfloat16><<<finalize_grid(n), 256, 0, st>>>(
+        part, splits, C, r, scale, transpose ? 1 : 0, static_cast<__nv_bfloat16*>(out));
   count_launch();
   return last_launch();
+}
+
+// Byte pointer `elems` elements into an adapter-gradient array of bf16 or fp32 elements.
+inline void* grad_at(void* base, size_t elems, bool f32) {
+  return static_cast<uint8_t*>(base) + elems * (f32 ? 4 : 2);
 }
 
 // ---------------------------------------------------------------- GEMM launch
@@ -675,7 +714,7 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
 // ---------------------------------------------------------------- backward core
 lora_status_t backward_core(const void* dY, const void* X, const void* XA, long long M, const lora_weight_t* W,
                             const Segs& sg, const void* A, const void* B, int r, float s, void* dX, void* dA,
-                            void* dB, __nv_bfloat16* sdYB, float* part, size_t part_cap, uint32_t* status,
+                            void* dB, bool f32, __nv_bfloat16* sdYB, float* part, size_t part_cap, uint32_t* status,
                             cudaStream_t st) {
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
@@ -691,14 +730,14 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
   for (int g = 0; g < sg.n; ++g) {
     const int rows = static_cast<int>(sg.rows[g]);
     const long long o = sg.off[g];
-    auto* dBg = static_cast<__nv_bfloat16*>(dB) + o * r;
+    void* dBg = grad_at(dB, static_cast<size_t>(o) * r, f32);
     const DualSplit ds = dual_split(M, rows, r);
     if (ds.use && dual_part_bytes(ds, M, rows, r) <= part_cap) {
       // one pass over dY_g for s·dY_g·B_g (columns [g·r, g·r + r) of s·dY·B) and dB_g = s·dY_gᵀ·XA_g
       float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
       TRY(launch_dual<DP_BOTH>(dYb + o, N, Bb + o * r, XAb + g * r, rt, M, rows, r, ds, part, partD, status, st));
       TRY(finalize_rows(part, ds.b, M, r, rt, s, nullptr, sdYB + g * r, st));
-      TRY(finalize_cols(partD, ds.a, rows, r, s, false, dBg, st));
+      TRY(finalize_cols(partD, ds.a, rows, r, s, false, dBg, f32, st));
       continue;
     }
     // s·dY_g·B_g -> columns [g·r, g·r + r) of s·dY·B
@@ -708,7 +747,7 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     // dB_g = s·dY_gᵀ·XA_g
     sp = colproj_split(M, rows);
     TRY(launch_colproj(dYb + o, Ni, XAb + g * r, rt, part, Mi, rows, r, sp, st));
-    TRY(finalize_cols(part, sp.splits, rows, r, s, false, dBg, st));
+    TRY(finalize_cols(part, sp.splits, rows, r, s, false, dBg, f32, st));
   }
   if (dX) {
     // dX = dY·W + (s·dY·B)·A with the LoRA fill over all G·r ranks
@@ -726,11 +765,11 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
   if (dsa.use && dual_part_d_bytes(dsa, K, rt) <= part_cap) {
     // one TMA-fed pass over X
     TRY(launch_dual<DP_COLS>(Xb, K, nullptr, sdYB, rt, M, K, rt, dsa, nullptr, part, status, st));
-    return finalize_cols(part, dsa.a, Ki, rt, 1.0f, true, static_cast<__nv_bfloat16*>(dA), st);
+    return finalize_cols(part, dsa.a, Ki, rt, 1.0f, true, dA, f32, st);
   }
   const Split sp = colproj_split(M, K);
   TRY(launch_colproj(Xb, Ki, sdYB, rt, part, Mi, Ki, rt, sp, st));
-  return finalize_cols(part, sp.splits, Ki, rt, 1.0f, true, static_cast<__nv_bfloat16*>(dA), st);
+  return finalize_cols(part, sp.splits, Ki, rt, 1.0f, true, dA, f32, st);
 }
 
 // ---------------------------------------------------------------- argument checks shared by the entries
@@ -767,17 +806,20 @@ lora_status_t fwd_entry(const void* X, int64_t M, const lora_weight_t* W, const 
 
 lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
                         const lora_segments_t* segs, const void* A, const void* B, int32_t r, float s, void* dX,
-                        void* dA, void* dB, void* workspace, size_t ws_bytes, void* stream) {
+                        void* dA, void* dB, uint32_t flags, void* workspace, size_t ws_bytes, void* stream) {
   Segs sg;
+  if (flags & ~static_cast<uint32_t>(LORA_GRADS_F32)) return LORA_ERR_INVALID_ARG;
+  const bool f32 = (flags & LORA_GRADS_F32) != 0;
   TRY(check_common(W, segs, r, s, M, A, B, &sg));
   TRY(check_ptr(dA));
   TRY(check_ptr(dB));
   const long long N = W->N, K = W->K;
   const int rt = sg.n * r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t esz = f32 ? 4 : 2;
   if (M == 0) {
-    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(rt) * K * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
-    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return LORA_ERR_CUDA;
+    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(rt) * K * esz, st) != cudaSuccess) return LORA_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * esz, st) != cudaSuccess) return LORA_ERR_CUDA;
     return LORA_OK;
   }
   TRY(check_ptr(dY));
@@ -789,7 +831,7 @@ lora_status_t bwd_entry(const void* dY, const void* X, const void* XA, int64_t M
   if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
   if (ws_bytes < wl.total) return LORA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  return backward_core(dY, X, XA, M, W, sg, A, B, r, s, dX, dA, dB,
+  return backward_core(dY, X, XA, M, W, sg, A, B, r, s, dX, dA, dB, f32,
                        reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off), reinterpret_cast<float*>(ws + wl.part_off),
                        wl.total - wl.part_off, reinterpret_cast<uint32_t*>(ws), st);
 }
@@ -878,8 +920,8 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
 // becomes [dG | dU]), then gate and up as two projections of X with dY = [dG | dU].
 lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const void* H, const void* XAgu,
                                 const void* XAd, long long M, const lora_mlp_t* m, int r, float s, void* dX,
-                                void* dAgu, void* dBgu, void* dAd, void* dBd, __nv_bfloat16* skinny, float* part,
-                                size_t part_cap, uint32_t* status, cudaStream_t st) {
+                                void* dAgu, void* dBgu, void* dAd, void* dBd, bool f32, __nv_bfloat16* skinny,
+                                float* part, size_t part_cap, uint32_t* status, cudaStream_t st) {
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
   TRY(get_encode());
@@ -895,7 +937,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
     float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
     TRY(launch_dual<DP_BOTH>(dZb, D, Bd, XAdb, r, M, D, r, ds, part, partD, status, st));
     TRY(finalize_rows(part, ds.b, M, r, r, s, nullptr, skinny, st));
-    TRY(finalize_cols(partD, ds.a, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
+    TRY(finalize_cols(partD, ds.a, Di, r, s, false, dBd, f32, st));
   } else {
     // s·dZ·B_d
     sp = rowproj_split(M, D);
@@ -904,7 +946,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
     // dB_d = s·dZᵀ·(H·A_dᵀ)
     sp = colproj_split(M, D);
     TRY(launch_colproj(dZb, Di, XAdb, r, part, Mi, Di, r, sp, st));
-    TRY(finalize_cols(part, sp.splits, Di, r, s, false, static_cast<__nv_bfloat16*>(dBd), st));
+    TRY(finalize_cols(part, sp.splits, Di, r, s, false, dBd, f32, st));
   }
   // dH = dZ·W_d + (s·dZ·B_d)·A_d, consumed by the epilogue: GU <- [dG | dU]
   {
@@ -921,9 +963,9 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
   // dA_d = (s·dZ·B_d)ᵀ·H
   sp = colproj_split(M, I);
   TRY(launch_colproj(static_cast<const __nv_bfloat16*>(H), Ii, skinny, r, part, Mi, Ii, r, sp, st));
-  TRY(finalize_cols(part, sp.splits, Ii, r, 1.0f, true, static_cast<__nv_bfloat16*>(dAd), st));
+  TRY(finalize_cols(part, sp.splits, Ii, r, 1.0f, true, dAd, f32, st));
   return backward_core(GU, X, XAgu, M, &m->gate_up, gate_up_segs(I), m->A_gate_up, m->B_gate_up, r, s, dX, dAgu,
-                       dBgu, skinny, part, part_cap, status, st);
+                       dBgu, f32, skinny, part, part_cap, status, st);
 }
 
 lora_status_t mlp_ws_check(long long M, const lora_mlp_t* m, int r, void* workspace, size_t ws_bytes) {
@@ -1019,7 +1061,13 @@ lora_status_t lora_linear_fwd(const void* X, int64_t M, const lora_weight_t* W, 
 lora_status_t lora_linear_bwd(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
                               const void* A, const void* B, int32_t r, float s, void* dX, void* dA, void* dB,
                               void* workspace, size_t ws_bytes, void* stream) {
-  return bwd_entry(dY, X, XA, M, W, nullptr, A, B, r, s, dX, dA, dB, workspace, ws_bytes, stream);
+  return bwd_entry(dY, X, XA, M, W, nullptr, A, B, r, s, dX, dA, dB, 0u, workspace, ws_bytes, stream);
+}
+
+lora_status_t lora_linear_bwd_ex(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
+                                 const void* A, const void* B, int32_t r, float s, void* dX, void* dA, void* dB,
+                                 uint32_t flags, void* workspace, size_t ws_bytes, void* stream) {
+  return bwd_entry(dY, X, XA, M, W, nullptr, A, B, r, s, dX, dA, dB, flags, workspace, ws_bytes, stream);
 }
 
 lora_status_t lora_grouped_fwd(const void* X, int64_t M, const lora_weight_t* W, const lora_segments_t* segs,
@@ -1033,7 +1081,38 @@ lora_status_t lora_grouped_bwd(const void* dY, const void* X, const void* XA, in
                                const lora_segments_t* segs, const void* A, const void* B, int32_t r, float s,
                                void* dX, void* dA, void* dB, void* workspace, size_t ws_bytes, void* stream) {
   if (!segs) return LORA_ERR_INVALID_ARG;
-  return bwd_entry(dY, X, XA, M, W, segs, A, B, r, s, dX, dA, dB, workspace, ws_bytes, stream);
+  return bwd_entry(dY, X, XA, M, W, segs, A, B, r, s, dX, dA, dB, 0u, workspace, ws_bytes, stream);
+}
+
+lora_status_t lora_grouped_bwd_ex(const void* dY, const void* X, const void* XA, int64_t M, const lora_weight_t* W,
+                                  const lora_segments_t* segs, const void* A, const void* B, int32_t r, float s,
+                                  void* dX, void* dA, void* dB, uint32_t flags, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  if (!segs) return LORA_ERR_INVALID_ARG;
+  return bwd_entry(dY, X, XA, M, W, segs, A, B, r, s, dX, dA, dB, flags, workspace, ws_bytes, stream);
+}
+
+lora_status_t lora_round_bf16(const float* src, void* dst, int64_t n, void* stream) {
+  if (n < 0) return LORA_ERR_INVALID_ARG;
+  if (n == 0) return LORA_OK;
+  TRY(check_ptr(src));
+  TRY(check_ptr(dst));
+  {
+    // the output may not overlap the input
+    const uint8_t* a0 = reinterpret_cast<const uint8_t*>(src);
+    const uint8_t* b0 = static_cast<const uint8_t*>(dst);
+    if (b0 < a0 + static_cast<size_t>(n) * 4 && a0 < b0 + static_cast<size_t>(n) * 2) return LORA_ERR_INVALID_ARG;
+  }
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  const size_t total = static_cast<size_t>(n);
+  size_t grid = (total + 255) / 256;
+  const size_t cap = static_cast<size_t>(dev->sms) * 8;
+  if (grid > cap) grid = cap;
+  round_bf16_kernel<<<static_cast<int>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      src, static_cast<__nv_bfloat16*>(dst), total);
+  count_launch();
+  return last_launch();
 }
 
 size_t lora_mlp_workspace_bytes(int64_t M, int64_t D, int64_t I, int32_t r, int32_t fmt) {
@@ -1061,10 +1140,12 @@ lora_status_t lora_mlp_fwd(const void* X, int64_t M, const lora_mlp_t* mlp, int3
                           reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
 }
 
-lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
-                           const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s, void* dX,
-                           void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down, void* workspace,
-                           size_t ws_bytes, void* stream) {
+static lora_status_t mlp_bwd_entry(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
+                            const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s, void* dX,
+                            void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down, uint32_t flags,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  if (flags & ~static_cast<uint32_t>(LORA_GRADS_F32)) return LORA_ERR_INVALID_ARG;
+  const bool f32 = (flags & LORA_GRADS_F32) != 0;
   TRY(mlp_check(mlp, r, s, M));
   TRY(check_ptr(dA_gate_up));
   TRY(check_ptr(dB_gate_up));
@@ -1073,8 +1154,9 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
   const long long D = mlp->gate_up.K, I = mlp->down.K;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (M == 0) {
-    const size_t z[4] = {static_cast<size_t>(2 * r) * D * 2, static_cast<size_t>(2 * I) * r * 2,
-                         static_cast<size_t>(r) * I * 2, static_cast<size_t>(D) * r * 2};
+    const size_t esz = f32 ? 4 : 2;
+    const size_t z[4] = {static_cast<size_t>(2 * r) * D * esz, static_cast<size_t>(2 * I) * r * esz,
+                         static_cast<size_t>(r) * I * esz, static_cast<size_t>(D) * r * esz};
     void* ptrs[4] = {dA_gate_up, dB_gate_up, dA_down, dB_down};
     for (int i = 0; i < 4; ++i)
       if (cudaMemsetAsync(ptrs[i], 0, z[i], st) != cudaSuccess) return LORA_ERR_CUDA;
@@ -1091,9 +1173,25 @@ lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* 
   const WsLayout wl = mlp_ws_layout(M, D, I, r);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return mlp_backward_core(dZ, X, GU, H, XA_gate_up, XA_down, M, mlp, r, s, dX, dA_gate_up, dB_gate_up, dA_down,
-                           dB_down, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
+                           dB_down, f32, reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off),
                            reinterpret_cast<float*>(ws + wl.part_off), wl.total - wl.part_off,
                            reinterpret_cast<uint32_t*>(ws), st);
+}
+
+lora_status_t lora_mlp_bwd(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
+                           const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s, void* dX,
+                           void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  return mlp_bwd_entry(dZ, X, GU, H, XA_gate_up, XA_down, M, mlp, r, s, dX, dA_gate_up, dB_gate_up, dA_down,
+                       dB_down, 0u, workspace, ws_bytes, stream);
+}
+
+lora_status_t lora_mlp_bwd_ex(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
+                              const void* XA_down, int64_t M, const lora_mlp_t* mlp, int32_t r, float s, void* dX,
+                              void* dA_gate_up, void* dB_gate_up, void* dA_down, void* dB_down, uint32_t flags,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  return mlp_bwd_entry(dZ, X, GU, H, XA_gate_up, XA_down, M, mlp, r, s, dX, dA_gate_up, dB_gate_up, dA_down,
+                       dB_down, flags, workspace, ws_bytes, stream);
 }
 
 size_t lora_ce_workspace_bytes(int64_t M, int64_t D, int64_t V, int64_t chunk) {
@@ -1378,16 +1476,22 @@ NoAllocLayout noalloc_layout(long long M, long long K, int r) {
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[64] = {};
+CUcontext g_noalloc_ctx[64] = {};
 
-// Device address of the fixed scratch on the current device, looked up on first use.
+// Device address of the fixed scratch on the current device, looked up on the first
+// call in each context (the array lives in the library's module of that context, so a
+// context created anew after cudaDeviceReset has its own copy at another address).
 lora_status_t noalloc_scratch(uint8_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  const CUcontext ctx = current_ctx();  // current: dev_info() ran first
+  if (!ctx) return LORA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  if (!g_noalloc_addr[dev] || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LORA_ERR_CUDA;
     g_noalloc_addr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = static_cast<uint8_t*>(g_noalloc_addr[dev]);
   return LORA_OK;

@@ -255,10 +255,15 @@ __global__ void finalize_rows_kernel(const float* __restrict__ part, int splits,
   }
 }
 
-// out = bf16(scale · Σ_s part[s]) where part is [splits][C][r]; written as [C][r], or as
-// [r][C] when transpose is set.
+// out = scale · Σ_s part[s] where part is [splits][C][r]; written as [C][r], or as [r][C]
+// when transpose is set.  OutT = __nv_bfloat16 rounds to nearest even; OutT = float keeps
+// the fp32 value (adapter gradients that are summed over data-parallel ranks first).
+__device__ __forceinline__ void store_out(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+__device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
+
+template <typename OutT>
 __global__ void finalize_cols_kernel(const float* __restrict__ part, int splits, int C, int r, float scale,
-                                     int transpose, __nv_bfloat16* __restrict__ out) {
+                                     int transpose, OutT* __restrict__ out) {
   const size_t n = static_cast<size_t>(C) * r;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -272,8 +277,15 @@ __global__ void finalize_cols_kernel(const float* __restrict__ part, int splits,
     }
     float acc = part[src];
     for (int s = 1; s < splits; ++s) acc += part[static_cast<size_t>(s) * n + src];
-    out[i] = __float2bfloat16_rn(scale * acc);
+    store_out(out + i, scale * acc);
   }
+}
+
+// dst = bf16_rn(src), n elements (the fp32 adapter gradients after their sum over ranks).
+__global__ void round_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
 }
 
 }  // namespace lora

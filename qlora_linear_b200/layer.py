@@ -38,17 +38,20 @@ class LoraLinear:
         return Y, XA
 
     def backward(self, dY: torch.Tensor, X: torch.Tensor, XA: torch.Tensor, need_dX: bool = True, out=None,
-                 stream=None):
+                 stream=None, grads_f32: bool = False):
+        """dX, dA, dB.  ``grads_f32``: dA and dB are fp32 (unrounded), for a sum over
+        data-parallel ranks before the one rounding to bf16."""
         M = dY.shape[0]
         dev = dY.device
+        gt = torch.float32 if grads_f32 else torch.bfloat16
         if out is None:
             dX = torch.empty((M, self.W.K), dtype=torch.bfloat16, device=dev) if need_dX else None
-            dA = torch.empty((self.r, self.W.K), dtype=torch.bfloat16, device=dev)
-            dB = torch.empty((self.W.N, self.r), dtype=torch.bfloat16, device=dev)
+            dA = torch.empty((self.r, self.W.K), dtype=gt, device=dev)
+            dB = torch.empty((self.W.N, self.r), dtype=gt, device=dev)
         else:
             dX, dA, dB = out
-        _b.lora_linear_bwd(dY, X, XA, M, self.W, self.A, self.B, self.r, self.s, dX, dA, dB, self.workspace(M),
-                           stream=stream)
+        _b.lora_linear_bwd_ex(dY, X, XA, M, self.W, self.A, self.B, self.r, self.s, dX, dA, dB,
+                              _b.LORA_GRADS_F32 if grads_f32 else 0, self.workspace(M), stream=stream)
         return dX, dA, dB
 
 
@@ -89,17 +92,18 @@ class LoraGroupedLinear:
         return Y, XA
 
     def backward(self, dY: torch.Tensor, X: torch.Tensor, XA: torch.Tensor, need_dX: bool = True, out=None,
-                 stream=None):
+                 stream=None, grads_f32: bool = False):
         M = dY.shape[0]
         dev = dY.device
+        gt = torch.float32 if grads_f32 else torch.bfloat16
         if out is None:
             dX = torch.empty((M, self.W.K), dtype=torch.bfloat16, device=dev) if need_dX else None
-            dA = torch.empty((self.G * self.r, self.W.K), dtype=torch.bfloat16, device=dev)
-            dB = torch.empty((self.W.N, self.r), dtype=torch.bfloat16, device=dev)
+            dA = torch.empty((self.G * self.r, self.W.K), dtype=gt, device=dev)
+            dB = torch.empty((self.W.N, self.r), dtype=gt, device=dev)
         else:
             dX, dA, dB = out
-        _b.lora_grouped_bwd(dY, X, XA, M, self.W, self.rows, self.A, self.B, self.r, self.s, dX, dA, dB,
-                            self.workspace(M), stream=stream)
+        _b.lora_grouped_bwd_ex(dY, X, XA, M, self.W, self.rows, self.A, self.B, self.r, self.s, dX, dA, dB,
+                               _b.LORA_GRADS_F32 if grads_f32 else 0, self.workspace(M), stream=stream)
         return dX, dA, dB
 
 
@@ -153,19 +157,22 @@ class LoraMLP:
                         saved["XA_down"], self.workspace(M), stream=stream)
         return Z, saved
 
-    def backward(self, dZ: torch.Tensor, X: torch.Tensor, saved: dict, need_dX: bool = True, out=None, stream=None):
+    def backward(self, dZ: torch.Tensor, X: torch.Tensor, saved: dict, need_dX: bool = True, out=None, stream=None,
+                 grads_f32: bool = False):
         M = dZ.shape[0]
         dev = dZ.device
         bf = torch.bfloat16
+        gt = torch.float32 if grads_f32 else bf
         if out is None:
             out = (torch.empty((M, self.D), dtype=bf, device=dev) if need_dX else None,
-                   torch.empty((2 * self.r, self.D), dtype=bf, device=dev),
-                   torch.empty((2 * self.I, self.r), dtype=bf, device=dev),
-                   torch.empty((self.r, self.I), dtype=bf, device=dev),
-                   torch.empty((self.D, self.r), dtype=bf, device=dev))
+                   torch.empty((2 * self.r, self.D), dtype=gt, device=dev),
+                   torch.empty((2 * self.I, self.r), dtype=gt, device=dev),
+                   torch.empty((self.r, self.I), dtype=gt, device=dev),
+                   torch.empty((self.D, self.r), dtype=gt, device=dev))
         dX, dAgu, dBgu, dAd, dBd = out
-        _b.lora_mlp_bwd(dZ, X, saved["GU"], saved["H"], saved["XA_gate_up"], saved["XA_down"], M, self.c_struct(),
-                        self.r, self.s, dX, dAgu, dBgu, dAd, dBd, self.workspace(M), stream=stream)
+        _b.lora_mlp_bwd_ex(dZ, X, saved["GU"], saved["H"], saved["XA_gate_up"], saved["XA_down"], M,
+                           self.c_struct(), self.r, self.s, dX, dAgu, dBgu, dAd, dBd,
+                           _b.LORA_GRADS_F32 if grads_f32 else 0, self.workspace(M), stream=stream)
         return out
 
 

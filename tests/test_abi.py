@@ -239,3 +239,40 @@ def test_ce_validation():
     assert bwd(nb=fixed + 64 * 255 * 2) == q.LORA_ERR_WORKSPACE
     assert q.ce_workspace_bytes(64, 256, 1000, 512) > q.ce_workspace_bytes(64, 256, 1000, 256)
     assert q.ce_workspace_bytes(64, 256, 1000, 0) == q.ce_workspace_bytes(64, 256, 1000, 1024)
+
+
+def bwd_ex(W, flags=1, M=256, r=8, s=2.0, dY=P, X=P, XA=P, A=P, B=P, dX=P, dA=P, dB=P, ws=P2, nb=1 << 30):
+    return q.lib().lora_linear_bwd_ex(dY, X, XA, M, ctypes.byref(W) if W is not None else None, A, B, r, s, dX, dA,
+                                      dB, flags, ws, nb, None)
+
+
+def test_fp32_gradient_entries_validate_like_the_plain_ones():
+    # the same host checks as lora_linear_bwd, with fp32 or bf16 gradients
+    for flags in (0, q.LORA_GRADS_F32):
+        assert bwd_ex(None, flags) == q.LORA_ERR_INVALID_ARG
+        assert bwd_ex(_w(N=513), flags) == q.LORA_ERR_UNSUPPORTED
+        assert bwd_ex(_w(), flags, dA=0) == q.LORA_ERR_INVALID_ARG
+        assert bwd_ex(_w(), flags, dB=P + 4) == q.LORA_ERR_ALIGNMENT
+        assert bwd_ex(_w(), flags, ws=0) == q.LORA_ERR_WORKSPACE
+    # unknown flag bits are rejected before anything else
+    for bad in (2, 4, 0x80000000, 3):
+        assert bwd_ex(_w(), bad) == q.LORA_ERR_INVALID_ARG, bad
+    lib = q.lib()
+    seg = q.segments([256, 256])
+    assert lib.lora_grouped_bwd_ex(P, P, P, 256, ctypes.byref(_w()), ctypes.byref(seg), P, P, 8, 2.0, P, P, P, 2,
+                                   P2, 1 << 30, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_grouped_bwd_ex(P, P, P, 256, ctypes.byref(_w()), None, P, P, 8, 2.0, P, P, P, 1,
+                                   P2, 1 << 30, None) == q.LORA_ERR_INVALID_ARG
+    m = q.mlp_struct(q.LoraWeight(1024, 512, P), q.LoraWeight(512, 512, P), P, P, P, P)
+    assert lib.lora_mlp_bwd_ex(P, P, P, P, P, P, 256, ctypes.byref(m), 8, 2.0, P, P, P, P, P, 8, P2, 1 << 30,
+                               None) == q.LORA_ERR_INVALID_ARG
+
+
+def test_round_bf16_validation():
+    lib = q.lib()
+    assert lib.lora_round_bf16(P, P2, -1, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_round_bf16(0, P2, 16, None) == q.LORA_ERR_INVALID_ARG
+    assert lib.lora_round_bf16(P + 4, P2, 16, None) == q.LORA_ERR_ALIGNMENT
+    assert lib.lora_round_bf16(P, P2 + 8, 16, None) == q.LORA_ERR_ALIGNMENT
+    assert lib.lora_round_bf16(P, P + 16, 16, None) == q.LORA_ERR_INVALID_ARG  # output overlaps the input
+    assert lib.lora_round_bf16(0, 0, 0, None) == q.LORA_OK  # nothing to do, nothing enqueued
