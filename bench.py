@@ -211,6 +211,10 @@ class ClockSampler:
     def mark(self, which: str):
         self.marks[which] = time.time()
 
+    def count_since(self, which: str) -> int:
+        t0 = self.marks.get(which, 0.0)
+        return sum(1 for s in list(self.samples) if s[0] >= t0)
+
     def stop(self):
         self.stop_ev.set()
         if self.proc is not None:
@@ -855,6 +859,14 @@ def run_ours(args, cases, desc, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # short steps on one GPU: keep warming up (same work) until the clock record holds
+    # enough samples (with several ranks every rank must run the same steps, each with its
+    # collective, so the count is not decided per rank)
+    t_w = time.time()
+    while world == 1 and clocks.source and clocks.count_since("t_warm") < MIN_CLOCK_SAMPLES \
+            and time.time() - t_w < 2.0:
+        step()
+        torch.cuda.synchronize()
     for st in ws.statuses():
         if st != q.LORA_OK:
             raise RuntimeError("device status after warm-up: " + q.status_string(st))

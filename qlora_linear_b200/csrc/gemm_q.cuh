@@ -24,9 +24,14 @@
 // schedule pieces of tiles, a piece being any consecutive range of the tile's code fills
 // and LoRA fills.
 //
-// Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (leader) and TMEM owner,
-// warps 2-5 epilogue, warps 6-13 dequant, warp 14 forwards the dequant warps' completion
-// of each fill to the leader.  Every wait is bounded.
+// Roles per CTA (16 warps; warp w runs on sub-partition w % 4): warp 0 TMA producer,
+// warp 1 MMA issuer (leader) and TMEM owner, warps 2-5 epilogue, warp 9 forwards the
+// dequant warps' completion of each fill to the leader, warp 13 has no role, and warps
+// 6-8, 10-12, 14-15 dequantize.  No dequant warp shares the MMA warp's sub-partition:
+// a tcgen05.mma whose issue waits for room in the tensor core's queue holds up the other
+// warps of its sub-partition, and dequant warps placed there lagged their CTA's others
+// by ~2400 cycles per fill in a timeline of the kernel (untraced: +5% on the QLoRA
+// shape).  Every wait is bounded.
 #pragma once
 
 #include "dequant.cuh"
@@ -49,10 +54,20 @@ struct QCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
   static constexpr int NUM_EPI_WARPS = 4;
   static constexpr int NUM_DEQ_WARPS = 8;
-  static constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS + NUM_DEQ_WARPS + 1);  // + the forwarder warp
+  static constexpr int NUM_THREADS = 32 * 16;
+  static constexpr int FWD_WARP = 9;   // forwarder
+  static constexpr int IDLE_WARP = 13;
+  // dequant warps 6,7,8,10,11,12,14,15 -> dequant index 0..7
+  static __device__ __forceinline__ int deq_index(int warp) { return warp < 9 ? warp - 6 : (warp < 13 ? warp - 7 : warp - 8); }
   static constexpr int TMEM_COLS = 512;  // MB accumulators of BN fp32 columns
   static constexpr int NUM_BARS = 5 * STAGES + 2 * MB + 1;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+  // Output staging of the store epilogue (4-bit weights; the 8-bit formats' larger code
+  // tiles leave no room): two 32-row × 32-column bf16 buffers per epilogue warp, 64-byte
+  // swizzle, written to global memory by TMA stores.
+  static constexpr bool STAGED_STORE = W4;
+  static constexpr int STG_BYTES = 2048;
+  static constexpr int EPI_STG_BYTES = STAGED_STORE ? NUM_EPI_WARPS * 2 * STG_BYTES : 0;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_STG_BYTES + 8 * NUM_BARS + 16;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -61,12 +76,13 @@ template <bool B_MN, int WF, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_THREADS, 1)
     lora_gemm_q_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
-                       const PairParams p) {
+                       const __grid_constant__ CUtensorMap tmO, const PairParams p) {
   using C = QCfg<B_MN, WF>;
   constexpr bool W4 = C::W4;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* stg_base = smem + C::STAGES * C::STAGE_BYTES;  // epilogue staging (1024-aligned)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg_base + C::EPI_STG_BYTES);
   uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
   uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
   uint64_t* cfull = bars + 2 * C::STAGES;   // both: this CTA's code tile landed
@@ -114,6 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     tma_prefetch_desc(&tmC);
     tma_prefetch_desc(&tmE);
     tma_prefetch_desc(&tmF);
+    if (EPI == EPI_STORE && C::STAGED_STORE) tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -238,6 +255,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
   } else if (warp < 2 + C::NUM_EPI_WARPS) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const uint32_t stg = smem_u32(stg_base) + static_cast<uint32_t>((warp - 2) * 2 * C::STG_BYTES);
+    int sb = 0;  // staging buffer of the next staged chunk
     uint32_t tphase = 0;
     bool ok = true;
     UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
@@ -264,6 +283,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
           }
         } else if constexpr (EPI == EPI_SWIGLU_BWD) {
           epi_swiglu_bwd_row(p, tbase, row, nb * C::BN);
+        } else if (C::STAGED_STORE && un.slot < 0) {
+          // 32 rows × 32 columns per chunk through a staging buffer and one TMA store (rows
+          // past M and columns past Nout are not written); chunk c + 1's TMEM load is in
+          // flight while chunk c is converted and staged.  Lane i writes row i, 16-byte unit
+          // u at position u ^ ((i >> 1) & 3), the 64-byte swizzle of the output map.
+          const int row0 = row - lane;  // first of the warp's 32 rows
+          const int nch = min(C::BN / 32, (p.Nout - nb * C::BN + 31) / 32);  // warp-uniform
+          auto stage_chunk = [&](const uint32_t (&v)[32], int c) {
+            const uint32_t buf = stg + static_cast<uint32_t>(sb * C::STG_BYTES);
+            if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t a = buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                           "r"(pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]))),
+                           "r"(pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]))),
+                           "r"(pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]))),
+                           "r"(pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])))
+                           : "memory");
+            }
+            fence_proxy_async_smem();  // the generic writes before the TMA store reads them
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmO, buf, nb * C::BN + c * 32, row0);
+              bulk_commit();
+            }
+            sb ^= 1;
+          };
+          if (row0 < p.M && nch > 0) {
+            uint32_t va[32], vb[32];
+            tmem_ld_32x32b_x32(tbase, va);
+            tmem_ld_wait();
+#pragma unroll 1
+            for (int c = 0; c < nch; c += 2) {
+              if (c + 1 < nch) tmem_ld_32x32b_x32(tbase + (c + 1) * 32, vb);
+              stage_chunk(va, c);
+              if (c + 1 < nch) {
+                tmem_ld_wait();
+                if (c + 2 < nch) tmem_ld_32x32b_x32(tbase + (c + 2) * 32, va);
+                stage_chunk(vb, c + 1);
+                if (c + 2 < nch) tmem_ld_wait();
+              }
+            }
+          }
         } else {
 #pragma unroll 1
           for (int c = 0; c < C::BN / 32; ++c) {
@@ -284,7 +348,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       }
       tphase ^= 1u;
     }
-  } else if (warp == 2 + C::NUM_EPI_WARPS + C::NUM_DEQ_WARPS) {
+  } else if (warp == C::IDLE_WARP) {
+    // no role (keeps the dequant warps off the MMA warp's sub-partition)
+  } else if (warp == C::FWD_WARP) {
     // ------------------------------------------------------------ forwarder (both CTAs)
     // The dequant warps signal a CTA-local barrier (release at CTA scope); this warp turns
     // each completed fill into the one cluster-scope release arrive the leader's MMA
@@ -306,7 +372,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     }
   } else {
     // ------------------------------------------------------------ dequant (both CTAs)
-    const int dt = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..255
+    const int dt = C::deq_index(warp) * 32 + lane;  // 0..255
     // forward: weight row `row` of this CTA's 128, 32-element half `h` of the 64-deep fill;
     // backward: weight row `krow` of the 64-deep fill, 32-column chunk `c4` of this CTA's 128
     const int row = !B_MN ? (dt & 127) : (dt >> 2);
@@ -317,23 +383,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
     }
     const long long kblocks_w = p.Kw / 64;  // 4-bit scale blocks per weight row
-    // scale for code fill kb of tile t: a fp16 block scale (4-bit) or a fp32 row scale (8-bit)
-    auto scale_at = [&](int t, int kb) -> float {
+    // scale for code fill kb of tile t, as raw bits: a fp16 block scale (4-bit) or a fp32
+    // row scale (8-bit); converted only where the fill uses it (sconv)
+    auto scale_at = [&](int t, int kb) -> uint32_t {
       int mb, nb;
       pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
       const int brow = pair_brow<EPI>(nb, rank, p);
       const long long n = !B_MN ? static_cast<long long>(brow) + row : static_cast<long long>(kb) * C::BK + row;
-      if (n >= p.Nw) return 0.0f;
+      if (n >= p.Nw) return 0u;
       if (W4) {
         const long long kblk = !B_MN ? kb : (brow + (sub >> 1) * 64) / 64;
-        return kblk < kblocks_w ? __half2float(p.absmax[n * kblocks_w + kblk]) : 0.0f;
+        return kblk < kblocks_w
+                   ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p.absmax) + n * kblocks_w + kblk))
+                   : 0u;
       }
-      return __ldg(p.row_scale + n);
+      return __float_as_uint(__ldg(p.row_scale + n));
     };
-    // Scales are loaded two code fills ahead into named registers: a fill's scale is read
-    // two fills after its load was issued, and the rotation moves a value loaded one fill
-    // earlier, so no instruction waits on a fresh global load.  (An indexed array here
-    // would live in local memory, and storing a just-loaded value there waits for it.)
+    auto sconv = [](uint32_t b) -> float {
+      return W4 ? __half2float(__ushort_as_half(static_cast<unsigned short>(b))) : __uint_as_float(b);
+    };
+    // Scales are loaded two code fills ahead into named registers as raw bits: a fill's
+    // scale is read (and converted) two fills after its load was issued, and the rotation
+    // moves a value loaded one fill earlier, so no instruction waits on a fresh global
+    // load.  (Converting the fp16 scale right at its load made every fill wait for it; an
+    // indexed array would live in local memory, and storing a just-loaded value there
+    // waits for it too.)
     // A second walk of the units tracks the code fill whose scale is loaded next.
     UnitWalk sw(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
     Unit su;
@@ -345,14 +419,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
         if (s_more) s_kb = su.f0;
       }
     };
-    auto load_next = [&]() -> float {
+    auto load_next = [&]() -> uint32_t {
       skip_ext();
-      const float v = s_more ? scale_at(su.t, s_kb) : 0.f;
+      const uint32_t v = s_more ? scale_at(su.t, s_kb) : 0u;
       ++s_kb;
       return v;
     };
-    float s_n1 = load_next();  // scale of the next code fill
-    float s_n2 = load_next();  // and of the one after
+    uint32_t s_n1 = load_next();  // scale of the next code fill
+    uint32_t s_n2 = load_next();  // and of the one after
     int stage = 0;
     uint32_t phase = 0;
     UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
@@ -363,7 +437,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
         const bool code = kb < nkb;
         float sc = 0.f;
         if (code) {
-          sc = s_n1;
+          sc = sconv(s_n1);
           s_n1 = s_n2;
           s_n2 = load_next();
         }
@@ -410,6 +484,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       if (!ok) break;
     }
   }
+
+  // the staged output stores of this warp are complete before the CTA exits
+  if (EPI == EPI_STORE && C::STAGED_STORE && warp >= 2 && warp < 2 + C::NUM_EPI_WARPS && lane == 0) bulk_wait<0>();
 
   // ------------------------------------------------------------ teardown
   tc_fence_before();

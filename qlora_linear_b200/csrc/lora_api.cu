@@ -527,9 +527,13 @@ lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CU
   // the raster group counts tiles; 512-row tiles take half as many for the same rows
   PairParams q = p;
   q.group_m = p.group_m > 1 ? p.group_m / 2 : 1;
+  // the staged store epilogue's output map: 32 × 32 boxes, 64-byte swizzle
+  CUtensorMap o = a;  // not read by the other epilogues
+  if (EPI == EPI_STORE && C::STAGED_STORE)
+    TRY(tmap_2d(&o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.out, p.Nout, p.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_q_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, c, e, f, q);
+    lora_gemm_q_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, c, e, f, o, q);
   }
   count_launch();
   return last_launch();

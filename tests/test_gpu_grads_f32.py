@@ -60,11 +60,12 @@ def test_layer_f32_grads_round_to_plain_bits(lib, M, N, K, r, fmt):
 
 
 def test_grouped_f32_grads_round_to_plain_bits(lib):
-    case = LoraCase("g32_grouped", 333, 640, 256, 16, 32.0, "bf16", 8200, rows=(256, 256, 128))
-    inp = make_grouped_case(case)
+    rows = [256, 256, 128]
+    case = LoraCase("g32_grouped", 333, 640, 256, 16, 32.0, "bf16", 8200)
+    inp = make_grouped_case(case, rows)
     W = lib.LoraWeight(case.N, case.K, dev_bf16(inp["W"]))
     X, A, B, dY = (dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
-    layer = lib.LoraGroupedLinear(W, inp["rows"], A, B, case.alpha)
+    layer = lib.LoraGroupedLinear(W, rows, A, B, case.alpha)
     Y, XA = layer.forward(X)
     _, dA, dB = layer.backward(dY, X, XA)
     _, dA32, dB32 = layer.backward(dY, X, XA, grads_f32=True)
