@@ -116,7 +116,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       mbar_init(smem_u32(&empty[s]), 1);
       mbar_init(smem_u32(&cfull[s]), 1);
       mbar_init(smem_u32(&deq[s]), 2);
-      mbar_init(smem_u32(&deql[s]), C::NUM_DEQ_WARPS);
+      mbar_init(smem_u32(&deql[s]), C::NUM_DEQ_WARPS / 2);  // the stage's dequant group
     }
     for (int b = 0; b < C::MB; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
@@ -372,11 +372,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     }
   } else {
     // ------------------------------------------------------------ dequant (both CTAs)
-    const int dt = C::deq_index(warp) * 32 + lane;  // 0..255
-    // forward: weight row `row` of this CTA's 128, 32-element half `h` of the 64-deep fill;
-    // backward: weight row `krow` of the 64-deep fill, 32-column chunk `c4` of this CTA's 128
-    const int row = !B_MN ? (dt & 127) : (dt >> 2);
-    const int sub = !B_MN ? (dt >> 7) : (dt & 3);
+    // Two groups of four warps take turns: group g expands the fills held in stages g and
+    // g + 2 (an even number of stages, so every fill of a stage belongs to one group), and a
+    // thread expands one whole 64-element scale block per fill, so each block's 16 levels
+    // are built once:
+    //   forward:  weight row `row` (0..127) of this CTA's B rows, the fill's 64-deep slice;
+    //   backward: weight row `row` (0..63) of the fill, 64-column half `h` of this CTA's 128.
+    static_assert(C::STAGES % 2 == 0, "stages alternate between the two dequant groups");
+    const int dq = C::deq_index(warp);   // 0..7
+    const int grp = dq >> 2;             // 0 or 1
+    const int gt = (dq & 3) * 32 + lane;  // 0..127 within the group
+    const int row = !B_MN ? gt : (gt & 63);
+    const int h = !B_MN ? 0 : (gt >> 6);
     float cb[16];
     if (W4) {
 #pragma unroll
@@ -392,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       const long long n = !B_MN ? static_cast<long long>(brow) + row : static_cast<long long>(kb) * C::BK + row;
       if (n >= p.Nw) return 0u;
       if (W4) {
-        const long long kblk = !B_MN ? kb : (brow + (sub >> 1) * 64) / 64;
+        const long long kblk = !B_MN ? kb : (brow + h * 64) / 64;
         return kblk < kblocks_w
                    ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p.absmax) + n * kblocks_w + kblk))
                    : 0u;
@@ -402,30 +409,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     auto sconv = [](uint32_t b) -> float {
       return W4 ? __half2float(__ushort_as_half(static_cast<unsigned short>(b))) : __uint_as_float(b);
     };
-    // Scales are loaded two code fills ahead into named registers as raw bits: a fill's
-    // scale is read (and converted) two fills after its load was issued, and the rotation
-    // moves a value loaded one fill earlier, so no instruction waits on a fresh global
-    // load.  (Converting the fp16 scale right at its load made every fill wait for it; an
-    // indexed array would live in local memory, and storing a just-loaded value there
-    // waits for it too.)
-    // A second walk of the units tracks the code fill whose scale is loaded next.
+    // Scales are loaded two of this group's code fills ahead into named registers as raw
+    // bits: a fill's scale is read (and converted) two fills after its load was issued, and
+    // the rotation moves a value loaded one fill earlier, so no instruction waits on a fresh
+    // global load.  (Converting the fp16 scale right at its load made every fill wait for
+    // it; an indexed array would live in local memory, and storing a just-loaded value
+    // there waits for it too.)  A second walk of the units tracks the fill whose scale is
+    // loaded next: s_f counts every fill, so its parity tells the group.
     UnitWalk sw(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
     Unit su;
     bool s_more = sw.next(su);
     int s_kb = s_more ? su.f0 : 0;
-    auto skip_ext = [&]() {  // move past LoRA fills (and units made of them only)
-      while (s_more && s_kb >= min(su.f1, nkb)) {
+    long long s_f = 0;
+    auto s_advance = [&]() {
+      ++s_f;
+      if (++s_kb >= su.f1) {
         s_more = sw.next(su);
         if (s_more) s_kb = su.f0;
       }
     };
     auto load_next = [&]() -> uint32_t {
-      skip_ext();
-      const uint32_t v = s_more ? scale_at(su.t, s_kb) : 0u;
-      ++s_kb;
+      while (s_more && (s_kb >= nkb || static_cast<int>(s_f & 1) != grp)) s_advance();  // LoRA fills, other group
+      if (!s_more) return 0u;
+      const uint32_t v = scale_at(su.t, s_kb);
+      s_advance();
       return v;
     };
-    uint32_t s_n1 = load_next();  // scale of the next code fill
+    uint32_t s_n1 = load_next();  // scale of this group's next code fill
     uint32_t s_n2 = load_next();  // and of the one after
     int stage = 0;
     uint32_t phase = 0;
@@ -434,51 +444,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     while (w.next(un)) {
       bool ok = true;
       for (int kb = un.f0; kb < un.f1; ++kb) {
-        const bool code = kb < nkb;
-        float sc = 0.f;
-        if (code) {
-          sc = sconv(s_n1);
-          s_n1 = s_n2;
-          s_n2 = load_next();
-        }
-        if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
-        if (code) {
-          uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-          const uint8_t* sC = sB + C::B_BYTES;
-          // destination row (128 bytes = 64 bf16, 128-byte swizzle) and its four 16-byte units
-          uint8_t* rowp;
-          int u0;
-          const uint8_t* cp;
-          if (!B_MN) {
-            rowp = sB + row * 128;
-            u0 = sub * 4;
-            cp = W4 ? sC + row * 32 + sub * 16 : sC + row * 64 + sub * 32;
-          } else {
-            rowp = sB + (sub >> 1) * (C::B_BYTES / 2) + row * 128;
-            u0 = (sub & 1) * 4;
-            cp = W4 ? sC + row * 64 + sub * 16 : sC + row * 128 + sub * 32;
+        if ((stage & 1) == grp) {
+          const bool code = kb < nkb;
+          float sc = 0.f;
+          if (code) {
+            sc = sconv(s_n1);
+            s_n1 = s_n2;
+            s_n2 = load_next();
           }
-          if constexpr (W4) {
-            const uint4 c = *reinterpret_cast<const uint4*>(cp);
-            uint32_t L[4], H[4];
-            block_levels(cb, sc, L, H);
-            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+          if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
+          if (code) {
+            uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+            const uint8_t* sC = sB + C::B_BYTES;
+            // destination: one 128-byte row (64 bf16, 128-byte swizzle: 16-byte unit u at
+            // u ^ (row & 7)); source: the row's 64 codes (32 bytes 4-bit, 64 bytes 8-bit)
+            uint8_t* rowp;
+            const uint8_t* cp;
+            if (!B_MN) {
+              rowp = sB + row * 128;
+              cp = W4 ? sC + row * 32 : sC + row * 64;
+            } else {
+              rowp = sB + h * (C::B_BYTES / 2) + row * 128;
+              cp = W4 ? sC + row * 64 + h * 32 : sC + row * 128 + h * 64;
+            }
+            if constexpr (W4) {
+              const uint4 c0 = *reinterpret_cast<const uint4*>(cp);
+              const uint4 c1 = *reinterpret_cast<const uint4*>(cp + 16);
+              uint32_t L[4], H[4];
+              block_levels(cb, sc, L, H);
+              const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              *reinterpret_cast<uint4*>(rowp + (((u0 + i) ^ (row & 7)) << 4)) = expand8(cw[i], L, H);
-          } else {
-            const uint4 c0 = *reinterpret_cast<const uint4*>(cp);
-            const uint4 c1 = *reinterpret_cast<const uint4*>(cp + 16);
-            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+              for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) = expand8(cw[u], L, H);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              *reinterpret_cast<uint4*>(rowp + (((u0 + i) ^ (row & 7)) << 4)) =
-                  expand8_w8<WF>(cw[2 * i], cw[2 * i + 1], sc);
+              for (int half = 0; half < 2; ++half) {
+                const uint4 c0 = *reinterpret_cast<const uint4*>(cp + half * 32);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(cp + half * 32 + 16);
+                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  *reinterpret_cast<uint4*>(rowp + (((half * 4 + i) ^ (row & 7)) << 4)) =
+                      expand8_w8<WF>(cw[2 * i], cw[2 * i + 1], sc);
+              }
+            }
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&deql[stage]));
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&deql[stage]));
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
