@@ -21,6 +21,7 @@
 #include "gemm_q.cuh"
 #include "skinny.cuh"
 #include "streamk.cuh"
+#include "tcproj.cuh"
 
 namespace lora {
 namespace {
@@ -194,6 +195,29 @@ GemmSched gemm_sched(long long M, long long Nout, long long Kred, int r, bool qu
   }
   return g;
 }
+// Split of a tensor-core rank-r pass (ranks above 16): output tiles of 128 rows and splits
+// of the reduction so that about two CTAs per SM run, each split at least four 64-deep
+// fills and none empty.  A pure function of the sizes.
+struct TcSplit {
+  int tiles = 0, splits = 1, fps = 1;
+};
+TcSplit tc_split(long long rows, long long red) {
+  TcSplit t;
+  t.tiles = cdiv(rows, TP_BM);
+  const int nkb = cdiv(red, TP_BK);
+  if (t.tiles <= 0 || nkb <= 0) return t;
+  const int want = cdiv(2 * 148, t.tiles);
+  const int cap = nkb / 4 > 1 ? nkb / 4 : 1;
+  const int s = want < cap ? want : cap;
+  t.fps = cdiv(nkb, s > 0 ? s : 1);
+  t.splits = cdiv(nkb, t.fps);
+  return t;
+}
+inline bool tc_rank(int r) { return r > 16; }
+size_t tc_part_bytes(long long rows, long long red, int r) {
+  return align256(static_cast<size_t>(tc_split(rows, red).splits) * rows * r * 4);
+}
+
 size_t gemm_sched_bytes(long long M, long long Nout, long long Kred, int r, bool quantized) {
   const GemmSched g = gemm_sched(M, Nout, Kred, r, quantized);
   return g.sk ? static_cast<size_t>(2) * kGemmPairs * g.tile_rows * 256 * 4 : 0;
@@ -220,6 +244,14 @@ WsLayout ws_layout(long long M, long long N, long long K, int r1, int nseg, bool
   if (xc.use) upd(dual_part_d_bytes(xc, K, r));                      // Xᵀ·(s·dY·B) on the TMA stream
   upd(gemm_sched_bytes(M, N, K, r1, quantized));                    // Y GEMM stream-K slots
   upd(gemm_sched_bytes(M, K, N, r, quantized));                      // dX GEMM stream-K slots
+  if (tc_rank(r)) {
+    upd(tc_part_bytes(M, K, r));   // X·Aᵀ on the tensor cores
+    upd(tc_part_bytes(K, M, r));   // Xᵀ·(s·dY·B) for dA
+  }
+  if (tc_rank(r1)) {
+    upd(tc_part_bytes(M, N, r1));  // dY·B (any segment has at most N rows)
+    upd(tc_part_bytes(N, M, r1));  // dYᵀ·XA for dB
+  }
   w.total = w.part_off + align256(part);
   return w;
 }
@@ -300,6 +332,9 @@ lora_status_t dev_info(DevInfo** out) {
     SET_SMEM((colproj_kernel<32>), (colproj_smem_bytes<32>()));
     SET_SMEM((colproj_kernel<64>), (colproj_smem_bytes<64>()));
     SET_SMEM((colproj_kernel<128>), (colproj_smem_bytes<128>()));
+    SET_SMEM(tcproj_kernel<TP_ROWS_K>, tcproj_smem_bytes());
+    SET_SMEM(tcproj_kernel<TP_ROWS_MN>, tcproj_smem_bytes());
+    SET_SMEM(tcproj_kernel<TP_COLS>, tcproj_smem_bytes());
 #undef SET_SMEM
     if (!ok) return LORA_ERR_CUDA;
     d.ctx = current_ctx();
@@ -461,6 +496,32 @@ lora_status_t launch_dual(const __nv_bfloat16* P, long long ldp, const __nv_bflo
   const DualParams dp{partT, partD, static_cast<int>(M), static_cast<int>(C), r, d.row_tiles, d.col_tiles, status,
                       wait_limit_ns()};
   dualproj_kernel<MODE><<<dim3(d.a, d.b), DP_THREADS, dual_smem_bytes(), st>>>(tp, tq, tr, dp);
+  count_launch();
+  return last_launch();
+}
+
+// Tensor-core rank-r pass (tcproj.cuh).  Row projection: P [rows][red] with row pitch ldp
+// and Q = A [r][red] (TP_ROWS_K) or B [red][r] with row pitch ldq (TP_ROWS_MN).  Column
+// projection (TP_COLS): P [red][rows] with row pitch ldp and R [red][r] with row pitch ldq.
+// Writes part [splits][rows][r].
+template <int MODE>
+lora_status_t launch_tcproj(const __nv_bfloat16* P, long long ldp, const __nv_bfloat16* Q, long long ldq,
+                            long long rows, long long red, int r, const TcSplit& t, float* part, uint32_t* status,
+                            cudaStream_t st) {
+  const int rpad = r <= 64 ? 64 : 128;
+  CUtensorMap tp, tq;
+  if (MODE == TP_COLS) {
+    TRY(tmap_2d(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, rows, red, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, ldp));
+  } else {
+    TRY(tmap_2d(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, red, rows, 64, TP_BM, CU_TENSOR_MAP_SWIZZLE_128B, ldp));
+  }
+  if (MODE == TP_ROWS_K)
+    TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Q, red, r, 64, rpad, CU_TENSOR_MAP_SWIZZLE_128B, ldq));
+  else
+    TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Q, r, red, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, ldq));
+  const TcProjParams tpp{part, static_cast<int>(rows), static_cast<int>(red), r, rpad, t.splits, t.fps, status,
+                         wait_limit_ns()};
+  tcproj_kernel<MODE><<<t.tiles * t.splits, TP_THREADS, tcproj_smem_bytes(), st>>>(tp, tq, tpp);
   count_launch();
   return last_launch();
 }
@@ -693,7 +754,12 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
 
   const DualSplit ds = dual_split(M, K, rt, DP_ROWS);
-  if (ds.use && dual_part_t_bytes(ds, M, rt) <= part_cap) {
+  if (tc_rank(rt) && tc_part_bytes(M, K, rt) <= part_cap) {
+    // X·Aᵀ on the tensor cores
+    const TcSplit t = tc_split(M, K);
+    TRY(launch_tcproj<TP_ROWS_K>(Xb, K, static_cast<const __nv_bfloat16*>(A), K, M, K, rt, t, part, status, st));
+    TRY(finalize_rows(part, t.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
+  } else if (ds.use && dual_part_t_bytes(ds, M, rt) <= part_cap) {
     // one TMA-fed pass over X
     TRY(launch_dual<DP_ROWS>(Xb, K, static_cast<const __nv_bfloat16*>(A), nullptr, 0, M, K, rt, ds, part, nullptr,
                              status, st));
@@ -736,6 +802,16 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     const long long o = sg.off[g];
     void* dBg = grad_at(dB, static_cast<size_t>(o) * r, f32);
     const DualSplit ds = dual_split(M, rows, r);
+    if (tc_rank(r) && tc_part_bytes(M, rows, r) <= part_cap && tc_part_bytes(rows, M, r) <= part_cap) {
+      // s·dY_g·B_g and dB_g = s·dY_gᵀ·XA_g on the tensor cores, one pass each
+      TcSplit t = tc_split(M, rows);
+      TRY(launch_tcproj<TP_ROWS_MN>(dYb + o, N, Bb + o * r, r, M, rows, r, t, part, status, st));
+      TRY(finalize_rows(part, t.splits, M, r, rt, s, nullptr, sdYB + g * r, st));
+      t = tc_split(rows, M);
+      TRY(launch_tcproj<TP_COLS>(dYb + o, N, XAb + g * r, rt, rows, M, r, t, part, status, st));
+      TRY(finalize_cols(part, t.splits, rows, r, s, false, dBg, f32, st));
+      continue;
+    }
     if (ds.use && dual_part_bytes(ds, M, rows, r) <= part_cap) {
       // one pass over dY_g for s·dY_g·B_g (columns [g·r, g·r + r) of s·dY·B) and dB_g = s·dY_gᵀ·XA_g
       float* partD = part + dual_part_t_bytes(ds, M, r) / 4;
@@ -765,6 +841,11 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     TRY(streamk_fixup(p, g, st));
   }
   // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
+  if (tc_rank(rt) && tc_part_bytes(K, M, rt) <= part_cap) {
+    const TcSplit t = tc_split(K, M);
+    TRY(launch_tcproj<TP_COLS>(Xb, K, sdYB, rt, K, M, rt, t, part, status, st));
+    return finalize_cols(part, t.splits, Ki, rt, 1.0f, true, dA, f32, st);
+  }
   const DualSplit dsa = dual_split(M, K, rt, DP_COLS);
   if (dsa.use && dual_part_d_bytes(dsa, K, rt) <= part_cap) {
     // one TMA-fed pass over X
@@ -857,6 +938,16 @@ WsLayout mlp_ws_layout(long long M, long long D, long long I, int r) {
   upd(static_cast<size_t>(colproj_split(M, D).splits) * D * 2 * r * 4);  // [dA_g; dA_u]
   upd(dual_part_bytes(dual_split(M, D, r), M, D, r));                    // dZ·B_d and dZᵀ·(H·A_dᵀ)
   upd(dual_part_bytes(dual_split(M, I, r), M, I, r));                    // dG·B_g and dGᵀ·XA_g (and the up half)
+  if (tc_rank(2 * r)) {
+    upd(tc_part_bytes(M, D, 2 * r));  // [X·A_gᵀ | X·A_uᵀ] on the tensor cores
+    upd(tc_part_bytes(D, M, 2 * r));  // [dA_g; dA_u]
+  }
+  if (tc_rank(r)) {
+    upd(tc_part_bytes(M, I, r));  // H·A_dᵀ, dG·B_g, dU·B_u
+    upd(tc_part_bytes(I, M, r));  // dA_d, dB_g, dB_u
+    upd(tc_part_bytes(M, D, r));  // dZ·B_d
+    upd(tc_part_bytes(D, M, r));  // dB_d
+  }
   w.total = w.part_off + align256(part);
   return w;
 }
@@ -890,18 +981,25 @@ Segs gate_up_segs(long long I) {
 // [X·A_gᵀ | X·A_uᵀ] in one pass over X; one GEMM for gate and up whose epilogue writes
 // G, U and H = silu(G)·U; then the down projection as a LoRA linear of H.
 lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, int r, float s, void* Z, void* GU,
-                               void* H, void* XAgu, void* XAd, __nv_bfloat16* skinny, float* part, uint32_t* status,
-                               cudaStream_t st) {
+                               void* H, void* XAgu, void* XAd, __nv_bfloat16* skinny, float* part, size_t part_cap,
+                               uint32_t* status, cudaStream_t st) {
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
   TRY(get_encode());
   const long long D = m->gate_up.K, I = m->down.K;
   const int r2 = 2 * r;
   const int Mi = static_cast<int>(M), Di = static_cast<int>(D);
-  const Split sp = rowproj_split(M, D);
-  TRY(launch_rowproj<false>(static_cast<const __nv_bfloat16*>(X), Di,
-                            static_cast<const __nv_bfloat16*>(m->A_gate_up), part, Mi, Di, r2, sp, st));
-  TRY(finalize_rows(part, sp.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
+  if (tc_rank(r2) && tc_part_bytes(M, D, r2) <= part_cap) {
+    const TcSplit t = tc_split(M, D);
+    TRY(launch_tcproj<TP_ROWS_K>(static_cast<const __nv_bfloat16*>(X), D,
+                                 static_cast<const __nv_bfloat16*>(m->A_gate_up), D, M, D, r2, t, part, status, st));
+    TRY(finalize_rows(part, t.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
+  } else {
+    const Split sp = rowproj_split(M, D);
+    TRY(launch_rowproj<false>(static_cast<const __nv_bfloat16*>(X), Di,
+                              static_cast<const __nv_bfloat16*>(m->A_gate_up), part, Mi, Di, r2, sp, st));
+    TRY(finalize_rows(part, sp.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
+  }
 
   CUtensorMap ta, te;
   TRY(tmap_bf16(&ta, X, D, M, kBoxX, kBoxY));
@@ -917,7 +1015,7 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
   Segs one;
   one.rows[0] = D;
   one.off[1] = D;
-  return forward_core(H, M, &m->down, one, m->A_down, m->B_down, r, s, Z, XAd, skinny, part, 0, status, st);
+  return forward_core(H, M, &m->down, one, m->A_down, m->B_down, r, s, Z, XAd, skinny, part, part_cap, status, st);
 }
 
 // Down projection's backward with SwiGLU's derivative in the dH GEMM's epilogue (GU
@@ -942,6 +1040,14 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
     TRY(launch_dual<DP_BOTH>(dZb, D, Bd, XAdb, r, M, D, r, ds, part, partD, status, st));
     TRY(finalize_rows(part, ds.b, M, r, r, s, nullptr, skinny, st));
     TRY(finalize_cols(partD, ds.a, Di, r, s, false, dBd, f32, st));
+  } else if (tc_rank(r) && tc_part_bytes(M, D, r) <= part_cap && tc_part_bytes(D, M, r) <= part_cap) {
+    // s·dZ·B_d and dB_d = s·dZᵀ·(H·A_dᵀ) on the tensor cores
+    TcSplit t = tc_split(M, D);
+    TRY(launch_tcproj<TP_ROWS_MN>(dZb, D, Bd, r, M, D, r, t, part, status, st));
+    TRY(finalize_rows(part, t.splits, M, r, r, s, nullptr, skinny, st));
+    t = tc_split(D, M);
+    TRY(launch_tcproj<TP_COLS>(dZb, D, XAdb, r, D, M, r, t, part, status, st));
+    TRY(finalize_cols(part, t.splits, Di, r, s, false, dBd, f32, st));
   } else {
     // s·dZ·B_d
     sp = rowproj_split(M, D);
@@ -965,9 +1071,15 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
     TRY((launch_gemm_w<true, EPI_SWIGLU_BWD>(&m->down, ta, te, tf, p, dev->sms, st)));
   }
   // dA_d = (s·dZ·B_d)ᵀ·H
-  sp = colproj_split(M, I);
-  TRY(launch_colproj(static_cast<const __nv_bfloat16*>(H), Ii, skinny, r, part, Mi, Ii, r, sp, st));
-  TRY(finalize_cols(part, sp.splits, Ii, r, 1.0f, true, dAd, f32, st));
+  if (tc_rank(r) && tc_part_bytes(I, M, r) <= part_cap) {
+    const TcSplit t = tc_split(I, M);
+    TRY(launch_tcproj<TP_COLS>(static_cast<const __nv_bfloat16*>(H), I, skinny, r, I, M, r, t, part, status, st));
+    TRY(finalize_cols(part, t.splits, Ii, r, 1.0f, true, dAd, f32, st));
+  } else {
+    sp = colproj_split(M, I);
+    TRY(launch_colproj(static_cast<const __nv_bfloat16*>(H), Ii, skinny, r, part, Mi, Ii, r, sp, st));
+    TRY(finalize_cols(part, sp.splits, Ii, r, 1.0f, true, dAd, f32, st));
+  }
   return backward_core(GU, X, XAgu, M, &m->gate_up, gate_up_segs(I), m->A_gate_up, m->B_gate_up, r, s, dX, dAgu,
                        dBgu, f32, skinny, part, part_cap, status, st);
 }
@@ -1141,7 +1253,7 @@ lora_status_t lora_mlp_fwd(const void* X, int64_t M, const lora_mlp_t* mlp, int3
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return mlp_forward_core(X, M, mlp, r, s, Z, GU, H, XA_gate_up, XA_down,
                           reinterpret_cast<__nv_bfloat16*>(ws + wl.skinny_off), reinterpret_cast<float*>(ws + wl.part_off),
-                          reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
+                          wl.total - wl.part_off, reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 static lora_status_t mlp_bwd_entry(const void* dZ, const void* X, void* GU, const void* H, const void* XA_gate_up,
