@@ -1177,6 +1177,8 @@ def main(argv=None):
     ap.add_argument("--no-separate", action="store_true", help="skip the unfused comparison of qkv / mlp")
     ap.add_argument("--weight", default=None, choices=["bf16", "block4", "int8", "fp8"],
                     help="store every frozen weight of the workload in this format")
+    ap.add_argument("--rank", type=int, default=None,
+                    help="run every projection at this LoRA rank (alpha = 2·rank) instead of the workload's")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -1189,6 +1191,10 @@ def main(argv=None):
         import dataclasses
         cases = [dataclasses.replace(c, fmt=args.weight) for c in cases]
         desc = f"{desc}; frozen weights stored as {args.weight}"
+    if args.rank:
+        import dataclasses
+        cases = [dataclasses.replace(c, r=args.rank, alpha=2.0 * args.rank) for c in cases]
+        desc = f"{desc}; LoRA rank {args.rank}, alpha {2 * args.rank}"
     if args.select:
         cases = select_cases(cases, args.select)
         if not cases:

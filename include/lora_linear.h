@@ -58,7 +58,9 @@ typedef enum {
   LORA_ERR_WORKSPACE = 4,       /* workspace NULL or smaller than lora_workspace_bytes() */
   LORA_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed (launch error etc.) */
   LORA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up a bounded wait (read with lora_device_status) */
-  LORA_ERR_SCRATCH_LIMIT = 7    /* lora_linear_fwd_noalloc: problem too large for its fixed scratch */
+  LORA_ERR_SCRATCH_LIMIT = 7,   /* lora_linear_fwd_noalloc: problem too large for its fixed scratch */
+  LORA_ERR_DEVICE_BOUNDS = 8    /* checked build only: a kernel found a tile or copy origin out of range
+                                   and skipped it (read with lora_device_status) */
 } lora_status_t;
 
 typedef enum {
@@ -386,7 +388,10 @@ lora_status_t lora_linear_fwd_noalloc(const void* X, int64_t M, const lora_weigh
 /*
  * Reads and clears the device status word in `workspace` (synchronizes `stream`).
  * Returns LORA_OK, or LORA_ERR_DEVICE_TIMEOUT if a kernel of an earlier call gave up a
- * bounded wait (its outputs are then undefined), or LORA_ERR_CUDA.
+ * bounded wait (its outputs are then undefined), or LORA_ERR_DEVICE_BOUNDS if a kernel of
+ * the checked build (compiled with -DLORA_CHECKED=1) found a tile or TMA box origin out of
+ * range and skipped that copy (outputs undefined; the regular build does not test), or
+ * LORA_ERR_CUDA.
  */
 lora_status_t lora_device_status(void* workspace, void* stream);
 

@@ -54,6 +54,26 @@ int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r);
  */
 int32_t lora_testing_dual_blocking(int64_t M, int64_t C, int32_t r, int32_t mode, int32_t* out4);
 
+/*
+ * Launches the tensor-core rank-r row projection (X·Aᵀ at rank r, 16 < r <= 128, r % 8 == 0)
+ * over P [rows, red] (device bf16, row-major) and A [r, red] (device bf16) with one output
+ * tile more than `rows` holds: that tile starts at row 128·ceil(rows/128), past the last
+ * row.  Its TMA loads lie wholly outside P, so the hardware fills them with zeros, and its
+ * epilogue writes no row at or past `rows`; nothing out of range is read or written.  The
+ * regular build computes the real tiles into part (device fp32, at least part_bytes =
+ * splits·rows·r·4 bytes for the pass's split count, which this call checks) and returns
+ * LORA_OK from lora_device_status; the checked build (-DLORA_CHECKED=1) also rejects the
+ * extra tile before its first copy, so lora_device_status(workspace, stream) then returns
+ * LORA_ERR_DEVICE_BOUNDS.  workspace: device, zero-filled, at least 256 bytes.  Lets the
+ * tests see the checked build's bounds test fire.
+ */
+/* Split count of the tensor-core rank-r pass for an output of `rows` rows over a
+ * reduction of length `red` (a pure function of the two); -1 for invalid sizes. */
+int32_t lora_testing_tcproj_splits(int64_t rows, int64_t red);
+
+lora_status_t lora_testing_tcproj_extra_tile(const void* P, const void* A, int64_t rows, int64_t red, int32_t r,
+                                             float* part, size_t part_bytes, void* workspace, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,7 @@ LORA_ERR_WORKSPACE = 4
 LORA_ERR_CUDA = 5
 LORA_ERR_DEVICE_TIMEOUT = 6
 LORA_ERR_SCRATCH_LIMIT = 7
+LORA_ERR_DEVICE_BOUNDS = 8
 LORA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 LORA_GRADS_F32 = 1  # flags of the *_bwd_ex calls: adapter gradients as fp32
@@ -42,6 +43,7 @@ EXPORTED = (
     "lora_mlp_workspace_bytes", "lora_mlp_fwd", "lora_mlp_bwd", "lora_dequant",
     "lora_ce_workspace_bytes", "lora_ce_fwd", "lora_ce_bwd",
     "lora_linear_bwd_ex", "lora_grouped_bwd_ex", "lora_mlp_bwd_ex", "lora_round_bf16",
+    "lora_testing_tcproj_extra_tile", "lora_testing_tcproj_splits",
 )
 
 LORA_MAX_SEGMENTS = 8
@@ -139,6 +141,10 @@ def _load() -> ctypes.CDLL:
     lib.lora_testing_xpass_tma.restype = i32
     lib.lora_testing_dual_blocking.argtypes = [i64, i64, i32, i32, ctypes.POINTER(i32)]
     lib.lora_testing_dual_blocking.restype = i32
+    lib.lora_testing_tcproj_extra_tile.argtypes = [vp, vp, i64, i64, i32, vp, sz, vp, vp]
+    lib.lora_testing_tcproj_extra_tile.restype = i32
+    lib.lora_testing_tcproj_splits.argtypes = [i64, i64]
+    lib.lora_testing_tcproj_splits.restype = i32
     lib.lora_timing_enable.argtypes = [i32]
     lib.lora_timing_enable.restype = i32
     lib.lora_timing_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
@@ -312,6 +318,17 @@ def lora_testing_dual_blocking(M: int, C: int, r: int, mode: int = 0):
 def lora_testing_xpass_tma(M: int, K: int, r: int) -> int:
     """Bit 0: the forward's X·Aᵀ, bit 1: the backward's pass for dA run on the TMA stream."""
     return int(_lib.lora_testing_xpass_tma(int(M), int(K), int(r)))
+
+
+def lora_testing_tcproj_splits(rows: int, red: int) -> int:
+    return int(_lib.lora_testing_tcproj_splits(int(rows), int(red)))
+
+
+def lora_testing_tcproj_extra_tile(P, A, rows: int, red: int, r: int, part, workspace, stream=None) -> int:
+    """Rank-r row projection with one output tile past the last row (see lora_linear_testing.h)."""
+    return int(_lib.lora_testing_tcproj_extra_tile(_ptr(P), _ptr(A), int(rows), int(red), int(r), _ptr(part),
+                                                   int(part.numel() * part.element_size()), _ptr(workspace),
+                                                   _stream(stream)))
 
 
 def lora_testing_gemm_streamk(M: int, Nout: int, Kred: int, r: int, fmt: int = LORA_W_BF16) -> int:

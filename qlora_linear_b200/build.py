@@ -14,8 +14,13 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblora_linear.so")
+# The checked build: every TMA producer tests its tile coordinates and box origins before
+# a copy and reports LORA_ERR_DEVICE_BOUNDS instead of issuing an out-of-range one
+# (select it with LORA_LIB_PATH; the tests run the ragged shapes on it).
+LIB_CHECKED = os.path.join(PKG, "liblora_linear_checked.so")
 SOURCES = ["lora_api.cu"]
-HEADERS = ["ptx.cuh", "dequant.cuh", "gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "skinny.cuh", "dualproj.cuh", "elementwise.cuh", "streamk.cuh"]
+HEADERS = ["ptx.cuh", "dequant.cuh", "gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "skinny.cuh", "dualproj.cuh",
+           "elementwise.cuh", "streamk.cuh", "tcproj.cuh"]
 
 
 def nvcc_path() -> str:
@@ -36,21 +41,25 @@ def flags(extra=()) -> list[str]:
     ]
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile the library if any source is newer than it; returns the .so path."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
+def build(force: bool = False, verbose: bool = False, extra=(), checked: bool = False) -> str:
+    """Compile the library (or its checked build) if any source is newer than it; returns
+    the .so path."""
+    lib = LIB_CHECKED if checked else LIB
+    if checked:
+        extra = (*extra, "-DLORA_CHECKED=1")
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + ".tmp"
     cmd = [nvcc_path(), *flags(extra), "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd), flush=True)
@@ -59,10 +68,10 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
-          extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())
+          extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else (), checked="--checked" in sys.argv)

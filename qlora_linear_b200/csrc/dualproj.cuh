@@ -132,8 +132,13 @@ __global__ void __launch_bounds__(DP_THREADS, 1)
           }
           const uint32_t st = sbase + s * DP_STAGE_BYTES;
           const uint32_t bar = smem_u32(&full[s]);
-          mbar_arrive_expect_tx(bar, STAGE_TX);
           const int y = (rt0 + ri) * DP_TR;
+          // checked build: the tile's first row and column exist
+          if (!lora_check(y < p.M && (ct0 + ci) * DP_TC < p.C, wc)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar, STAGE_TX);
 #pragma unroll
           for (int b = 0; b < DP_TC / 64; ++b) tma_load_2d(st + b * DP_BOX_BYTES, &tmP, bar, (ct0 + ci) * DP_TC + b * 64, y);
           if (DO_D) tma_load_2d(st + DP_P_BYTES, &tmR, bar, 0, y);

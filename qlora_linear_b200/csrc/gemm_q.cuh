@@ -157,9 +157,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
         pair_tile_coords(un.t, num_m, num_n, p.group_m, mb, nb);
         const int arow = mb * C::BM + static_cast<int>(rank) * C::HM;  // this CTA's rows of A block 0
         const int brow = pair_brow<EPI>(nb, rank, p);
+        // checked build: the tile exists and starts inside the output (a CTA's half of a
+        // ragged tile may lie wholly past M or N: its boxes are TMA zero fills)
+        if (!lora_check(mb < num_m && nb < num_n && mb * C::BM < p.M && nb * EpiTile<EPI>::COLS < p.Nout, wc)) {
+          ok = false;
+          break;
+        }
         for (int kb = un.f0; kb < un.f1; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
           const bool ext = kb >= nkb;
+          if (!lora_check(ext ? kb - nkb < n_ext : kb * C::BK < p.Kred, wc)) { ok = false; break; }
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const uint32_t sC = sB + C::B_BYTES;

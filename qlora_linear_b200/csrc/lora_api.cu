@@ -1153,6 +1153,8 @@ const char* lora_status_string(int32_t status) {
     case LORA_ERR_WORKSPACE: return "workspace missing or smaller than lora_workspace_bytes()";
     case LORA_ERR_CUDA: return "a CUDA call failed";
     case LORA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait; outputs of that call are undefined";
+    case LORA_ERR_DEVICE_BOUNDS:
+      return "checked build: a kernel found a tile or copy origin out of range and skipped it; outputs undefined";
     case LORA_ERR_SCRATCH_LIMIT:
       return "problem needs more scratch than the fixed LORA_NOALLOC_SCRATCH_BYTES of lora_linear_fwd_noalloc";
     default: return "unknown status";
@@ -1504,6 +1506,7 @@ lora_status_t lora_device_status(void* workspace, void* stream) {
   if (word == 0) return LORA_OK;
   if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return LORA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return LORA_ERR_CUDA;
+  if (word & kDevErrBounds) return LORA_ERR_DEVICE_BOUNDS;
   return (word & kDevErrTimeout) ? LORA_ERR_DEVICE_TIMEOUT : LORA_ERR_CUDA;
 }
 
@@ -1532,6 +1535,31 @@ int32_t lora_testing_dual_blocking(int64_t M, int64_t C, int32_t r, int32_t mode
   out4[2] = d.row_tiles;
   out4[3] = d.col_tiles;
   return d.use ? 1 : 0;
+}
+
+lora_status_t lora_testing_tcproj_extra_tile(const void* P, const void* A, int64_t rows, int64_t red, int32_t r,
+                                             float* part, size_t part_bytes, void* workspace, void* stream) {
+  if (rows <= 0 || red <= 0 || red % 8 != 0 || rows > (1LL << 30) || red > (1LL << 30)) return LORA_ERR_INVALID_ARG;
+  if (r <= 16 || r > 128 || r % 8 != 0) return LORA_ERR_UNSUPPORTED;
+  TRY(check_ptr(P));
+  TRY(check_ptr(A));
+  TRY(check_ptr(part));
+  if (!workspace) return LORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
+  TcSplit t = tc_split(rows, red);
+  if (part_bytes < static_cast<size_t>(t.splits) * rows * r * 4) return LORA_ERR_WORKSPACE;
+  DevInfo* dev = nullptr;
+  TRY(dev_info(&dev));
+  TRY(get_encode());
+  t.tiles += 1;  // one tile past the last row
+  return launch_tcproj<TP_ROWS_K>(static_cast<const __nv_bfloat16*>(P), red, static_cast<const __nv_bfloat16*>(A),
+                                  red, rows, red, r, t, part, static_cast<uint32_t*>(workspace),
+                                  static_cast<cudaStream_t>(stream));
+}
+
+int32_t lora_testing_tcproj_splits(int64_t rows, int64_t red) {
+  if (rows <= 0 || red <= 0) return -1;
+  return tc_split(rows, red).splits;
 }
 
 int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r) {

@@ -11,6 +11,7 @@ namespace lora {
 
 // Device status word bits (workspace word 0).
 constexpr uint32_t kDevErrTimeout = 1u;
+constexpr uint32_t kDevErrBounds = 2u;  // checked build: a tile or box origin out of range
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -72,6 +73,25 @@ struct WaitCtl {
 __device__ __noinline__ void wait_timed_out(const WaitCtl& w) {
   *w.abort_flag = 1u;
   if (w.status) atomicOr(w.status, kDevErrTimeout);
+}
+
+// Checked build (compiled with -DLORA_CHECKED=1): the TMA producers test every tile
+// coordinate and box origin before the copy; a failed test raises the CTA's abort flag
+// (its other roles leave through their bounded waits), sets kDevErrBounds in the status
+// word and skips the copy.  Without the flag the tests compile to nothing.
+#ifndef LORA_CHECKED
+#define LORA_CHECKED 0
+#endif
+__device__ __noinline__ void bounds_failed(const WaitCtl& w) {
+  *w.abort_flag = 1u;
+  if (w.status) atomicOr(w.status, kDevErrBounds);
+}
+__device__ __forceinline__ bool lora_check(bool ok, const WaitCtl& w) {
+  if (LORA_CHECKED && !ok) {
+    bounds_failed(w);
+    return false;
+  }
+  return true;
 }
 
 // Single-thread bounded wait for the phase with the given parity to complete.

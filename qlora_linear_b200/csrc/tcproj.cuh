@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(TP_THREADS, 1)
         const int s = fills % TP_STAGES;
         const uint32_t ph = static_cast<uint32_t>((fills / TP_STAGES) & 1);
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, wc)) { ok = false; break; }
+        // checked build: the output tile and the fill's reduction slice exist
+        if (!lora_check(row0 < p.rows && kb * TP_BK < p.red && split < p.splits, wc)) { ok = false; break; }
         const uint32_t sP = smem_u32(smem + s * TP_STAGE_BYTES);
         const uint32_t sQ = sP + TP_P_BYTES;
         const uint32_t bar = smem_u32(&full[s]);

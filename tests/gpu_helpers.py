@@ -50,14 +50,23 @@ def make_weight(q, inp):
     return q.LoraWeight(case.N, case.K, codes, absmax, cb), (codes, absmax, cb)
 
 
+def nan_canary(shape) -> torch.Tensor:
+    """A bf16 output buffer filled with NaN: an element the kernels never write stays NaN
+    and fails the parity check (which rejects non-finite values)."""
+    return torch.full(shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+
+
 def run_layer(q, inp, need_dX=True):
-    """Forward and backward of one case through the library; returns device tensors."""
+    """Forward and backward of one case through the library, every output buffer
+    NaN-filled first; returns device tensors."""
     case = inp["case"]
     W, keep = make_weight(q, inp)
     X, A, B, dY = (dev_bf16(inp[k]) for k in ("X", "A", "B", "dY"))
     layer = q.LoraLinear(W, A, B, case.alpha)
-    Y, XA = layer.forward(X)
-    dX, dA, dB = layer.backward(dY, X, XA, need_dX=need_dX)
+    M, N, K, r = case.M, case.N, case.K, case.r
+    Y, XA = layer.forward(X, Y=nan_canary((M, N)), XA=nan_canary((M, r)))
+    dX, dA, dB = layer.backward(dY, X, XA, out=(nan_canary((M, K)) if need_dX else None, nan_canary((r, K)),
+                                                nan_canary((N, r))))
     torch.cuda.synchronize()
     st = q.lora_device_status(layer.workspace(case.M))
     assert st == q.LORA_OK, q.status_string(st)
