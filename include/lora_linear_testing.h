@@ -68,8 +68,9 @@ int32_t lora_testing_dual_blocking(int64_t M, int64_t C, int32_t r, int32_t mode
  * tests see the checked build's bounds test fire.
  */
 /* Split count of the tensor-core rank-r pass for an output of `rows` rows over a
- * reduction of length `red` (a pure function of the two); -1 for invalid sizes. */
-int32_t lora_testing_tcproj_splits(int64_t rows, int64_t red);
+ * reduction of length `red` at rank r (a pure function of the three); -1 for invalid
+ * sizes. */
+int32_t lora_testing_tcproj_splits(int64_t rows, int64_t red, int32_t r);
 
 lora_status_t lora_testing_tcproj_extra_tile(const void* P, const void* A, int64_t rows, int64_t red, int32_t r,
                                              float* part, size_t part_bytes, void* workspace, void* stream);

@@ -143,7 +143,7 @@ def _load() -> ctypes.CDLL:
     lib.lora_testing_dual_blocking.restype = i32
     lib.lora_testing_tcproj_extra_tile.argtypes = [vp, vp, i64, i64, i32, vp, sz, vp, vp]
     lib.lora_testing_tcproj_extra_tile.restype = i32
-    lib.lora_testing_tcproj_splits.argtypes = [i64, i64]
+    lib.lora_testing_tcproj_splits.argtypes = [i64, i64, i32]
     lib.lora_testing_tcproj_splits.restype = i32
     lib.lora_timing_enable.argtypes = [i32]
     lib.lora_timing_enable.restype = i32
@@ -320,8 +320,8 @@ def lora_testing_xpass_tma(M: int, K: int, r: int) -> int:
     return int(_lib.lora_testing_xpass_tma(int(M), int(K), int(r)))
 
 
-def lora_testing_tcproj_splits(rows: int, red: int) -> int:
-    return int(_lib.lora_testing_tcproj_splits(int(rows), int(red)))
+def lora_testing_tcproj_splits(rows: int, red: int, r: int) -> int:
+    return int(_lib.lora_testing_tcproj_splits(int(rows), int(red), int(r)))
 
 
 def lora_testing_tcproj_extra_tile(P, A, rows: int, red: int, r: int, part, workspace, stream=None) -> int:

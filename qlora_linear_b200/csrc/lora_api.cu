@@ -46,6 +46,12 @@ uint64_t wait_limit_ns() {
 }
 
 // 256-row output tiles per raster group of the GEMMs; LORA_GROUP_M overrides (1..64).
+// The tiles of a group walk the output column by column, re-reading the group's A panels
+// (256 × Kred bf16 each) from L2 for every column.  16 keeps a reduction-over-4096
+// launch at ~1.2 GB of DRAM traffic (0.77 GB read; ~1.1 GB read with 8).  A reduction
+// over 14336 reads 2.5-3.4 GB with either 8 or 16: the group's panels and the 117 MB
+// weight exceed the 126 MB L2 whatever the group, and the pairs drift apart in k over the
+// 14 waves.  16 was ~1.4% faster than 8 in 100-step power-capped runs of the c2 step.
 int group_m_default() {
   static int v = [] {
     const char* e = std::getenv("LORA_GROUP_M");
@@ -53,7 +59,7 @@ int group_m_default() {
       const long x = std::strtol(e, nullptr, 10);
       if (x >= 1 && x <= 64) return static_cast<int>(x);
     }
-    return 16;  // 8 and 16 were level in short runs; 16 was ~1.4% faster in 100-step power-capped runs
+    return 16;
   }();
   return v;
 }
@@ -195,27 +201,41 @@ GemmSched gemm_sched(long long M, long long Nout, long long Kred, int r, bool qu
   }
   return g;
 }
-// Split of a tensor-core rank-r pass (ranks above 16): output tiles of 128 rows and splits
-// of the reduction so that about two CTAs per SM run, each split at least four 64-deep
-// fills and none empty.  A pure function of the sizes.
+// Split of a tensor-core rank-r pass (ranks above 16): output tiles of 128 rows and the
+// number of splits of the reduction that minimises the estimated time in 64-deep fills:
+// (waves of two CTAs per SM) × (fills per split + 3 for a CTA's ramp-up and epilogue)
+// plus the fp32 partials written and read back (2·splits·rows·r·4 bytes) at the bytes one
+// fill of every resident CTA streams (296 × 16 KB).  A second, mostly empty wave costs as
+// much as a full one.  Splits hold at least four fills, none is empty.  A pure function of
+// the sizes (made for 148 SMs).
 struct TcSplit {
   int tiles = 0, splits = 1, fps = 1;
 };
-TcSplit tc_split(long long rows, long long red) {
+TcSplit tc_split(long long rows, long long red, int r) {
   TcSplit t;
   t.tiles = cdiv(rows, TP_BM);
   const int nkb = cdiv(red, TP_BK);
   if (t.tiles <= 0 || nkb <= 0) return t;
-  const int want = cdiv(2 * 148, t.tiles);
+  constexpr int kResident = 2 * 148;
+  const double fill_bytes = kResident * static_cast<double>(TP_P_BYTES);
   const int cap = nkb / 4 > 1 ? nkb / 4 : 1;
-  const int s = want < cap ? want : cap;
-  t.fps = cdiv(nkb, s > 0 ? s : 1);
-  t.splits = cdiv(nkb, t.fps);
+  double best = -1.0;
+  for (int s = 1; s <= cap && s <= 256; ++s) {
+    const int fps = cdiv(nkb, s);
+    const int splits = cdiv(nkb, fps);
+    const double waves = cdiv(static_cast<long long>(t.tiles) * splits, kResident);
+    const double cost = waves * (fps + 3) + 2.0 * splits * static_cast<double>(rows) * r * 4 / fill_bytes;
+    if (best < 0 || cost < best) {
+      best = cost;
+      t.fps = fps;
+      t.splits = splits;
+    }
+  }
   return t;
 }
 inline bool tc_rank(int r) { return r > 16; }
 size_t tc_part_bytes(long long rows, long long red, int r) {
-  return align256(static_cast<size_t>(tc_split(rows, red).splits) * rows * r * 4);
+  return align256(static_cast<size_t>(tc_split(rows, red, r).splits) * rows * r * 4);
 }
 
 size_t gemm_sched_bytes(long long M, long long Nout, long long Kred, int r, bool quantized) {
@@ -756,7 +776,7 @@ lora_status_t forward_core(const void* X, long long M, const lora_weight_t* W, c
   const DualSplit ds = dual_split(M, K, rt, DP_ROWS);
   if (tc_rank(rt) && tc_part_bytes(M, K, rt) <= part_cap) {
     // X·Aᵀ on the tensor cores
-    const TcSplit t = tc_split(M, K);
+    const TcSplit t = tc_split(M, K, rt);
     TRY(launch_tcproj<TP_ROWS_K>(Xb, K, static_cast<const __nv_bfloat16*>(A), K, M, K, rt, t, part, status, st));
     TRY(finalize_rows(part, t.splits, M, rt, rt, s, static_cast<__nv_bfloat16*>(XA), sXA, st));
   } else if (ds.use && dual_part_t_bytes(ds, M, rt) <= part_cap) {
@@ -804,10 +824,10 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
     const DualSplit ds = dual_split(M, rows, r);
     if (tc_rank(r) && tc_part_bytes(M, rows, r) <= part_cap && tc_part_bytes(rows, M, r) <= part_cap) {
       // s·dY_g·B_g and dB_g = s·dY_gᵀ·XA_g on the tensor cores, one pass each
-      TcSplit t = tc_split(M, rows);
+      TcSplit t = tc_split(M, rows, r);
       TRY(launch_tcproj<TP_ROWS_MN>(dYb + o, N, Bb + o * r, r, M, rows, r, t, part, status, st));
       TRY(finalize_rows(part, t.splits, M, r, rt, s, nullptr, sdYB + g * r, st));
-      t = tc_split(rows, M);
+      t = tc_split(rows, M, r);
       TRY(launch_tcproj<TP_COLS>(dYb + o, N, XAb + g * r, rt, rows, M, r, t, part, status, st));
       TRY(finalize_cols(part, t.splits, rows, r, s, false, dBg, f32, st));
       continue;
@@ -842,7 +862,7 @@ lora_status_t backward_core(const void* dY, const void* X, const void* XA, long 
   }
   // dA = (s·dY·B)ᵀ·X, computed as Xᵀ·(s·dY·B) and written transposed [G·r, K]
   if (tc_rank(rt) && tc_part_bytes(K, M, rt) <= part_cap) {
-    const TcSplit t = tc_split(K, M);
+    const TcSplit t = tc_split(K, M, rt);
     TRY(launch_tcproj<TP_COLS>(Xb, K, sdYB, rt, K, M, rt, t, part, status, st));
     return finalize_cols(part, t.splits, Ki, rt, 1.0f, true, dA, f32, st);
   }
@@ -990,7 +1010,7 @@ lora_status_t mlp_forward_core(const void* X, long long M, const lora_mlp_t* m, 
   const int r2 = 2 * r;
   const int Mi = static_cast<int>(M), Di = static_cast<int>(D);
   if (tc_rank(r2) && tc_part_bytes(M, D, r2) <= part_cap) {
-    const TcSplit t = tc_split(M, D);
+    const TcSplit t = tc_split(M, D, r2);
     TRY(launch_tcproj<TP_ROWS_K>(static_cast<const __nv_bfloat16*>(X), D,
                                  static_cast<const __nv_bfloat16*>(m->A_gate_up), D, M, D, r2, t, part, status, st));
     TRY(finalize_rows(part, t.splits, M, r2, r2, s, static_cast<__nv_bfloat16*>(XAgu), skinny, st));
@@ -1042,10 +1062,10 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
     TRY(finalize_cols(partD, ds.a, Di, r, s, false, dBd, f32, st));
   } else if (tc_rank(r) && tc_part_bytes(M, D, r) <= part_cap && tc_part_bytes(D, M, r) <= part_cap) {
     // s·dZ·B_d and dB_d = s·dZᵀ·(H·A_dᵀ) on the tensor cores
-    TcSplit t = tc_split(M, D);
+    TcSplit t = tc_split(M, D, r);
     TRY(launch_tcproj<TP_ROWS_MN>(dZb, D, Bd, r, M, D, r, t, part, status, st));
     TRY(finalize_rows(part, t.splits, M, r, r, s, nullptr, skinny, st));
-    t = tc_split(D, M);
+    t = tc_split(D, M, r);
     TRY(launch_tcproj<TP_COLS>(dZb, D, XAdb, r, D, M, r, t, part, status, st));
     TRY(finalize_cols(part, t.splits, Di, r, s, false, dBd, f32, st));
   } else {
@@ -1072,7 +1092,7 @@ lora_status_t mlp_backward_core(const void* dZ, const void* X, void* GU, const v
   }
   // dA_d = (s·dZ·B_d)ᵀ·H
   if (tc_rank(r) && tc_part_bytes(I, M, r) <= part_cap) {
-    const TcSplit t = tc_split(I, M);
+    const TcSplit t = tc_split(I, M, r);
     TRY(launch_tcproj<TP_COLS>(static_cast<const __nv_bfloat16*>(H), I, skinny, r, I, M, r, t, part, status, st));
     TRY(finalize_cols(part, t.splits, Ii, r, 1.0f, true, dAd, f32, st));
   } else {
@@ -1546,7 +1566,7 @@ lora_status_t lora_testing_tcproj_extra_tile(const void* P, const void* A, int64
   TRY(check_ptr(part));
   if (!workspace) return LORA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return LORA_ERR_ALIGNMENT;
-  TcSplit t = tc_split(rows, red);
+  TcSplit t = tc_split(rows, red, r);
   if (part_bytes < static_cast<size_t>(t.splits) * rows * r * 4) return LORA_ERR_WORKSPACE;
   DevInfo* dev = nullptr;
   TRY(dev_info(&dev));
@@ -1557,9 +1577,9 @@ lora_status_t lora_testing_tcproj_extra_tile(const void* P, const void* A, int64
                                   static_cast<cudaStream_t>(stream));
 }
 
-int32_t lora_testing_tcproj_splits(int64_t rows, int64_t red) {
-  if (rows <= 0 || red <= 0) return -1;
-  return tc_split(rows, red).splits;
+int32_t lora_testing_tcproj_splits(int64_t rows, int64_t red, int32_t r) {
+  if (rows <= 0 || red <= 0 || r < 1 || r > 128) return -1;
+  return tc_split(rows, red, r).splits;
 }
 
 int32_t lora_testing_xpass_tma(int64_t M, int64_t K, int32_t r) {

@@ -22,7 +22,7 @@ def out_of_range_tile(q, torch):
     rows, red, r = 300, 520, 72
     P = torch.randn((rows, red), device="cuda").to(torch.bfloat16)
     A = torch.randn((r, red), device="cuda").to(torch.bfloat16)
-    splits = q.lora_testing_tcproj_splits(rows, red)
+    splits = q.lora_testing_tcproj_splits(rows, red, r)
     part = torch.zeros(splits * rows * r, dtype=torch.float32, device="cuda")
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     st = q.lora_testing_tcproj_extra_tile(P, A, rows, red, r, part, ws)
