@@ -67,6 +67,7 @@ template <int MODE>
 __global__ void __launch_bounds__(DP_THREADS, 1)
     dualproj_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmR, const DualParams p) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   constexpr bool DO_T = MODE != DP_COLS, DO_D = MODE != DP_ROWS;
   constexpr int STAGE_TX = DP_P_BYTES + (DO_D ? DP_R_BYTES : 0);
   extern __shared__ uint8_t dp_raw[];

@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(MG_THREADS)
 __global__ void ce_finalize_kernel(const float2* __restrict__ part, int ntiles, int M,
                                    const float* __restrict__ label_logit, const int32_t* __restrict__ labels,
                                    int ignore_index, float* __restrict__ loss, float* __restrict__ lse) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= M) return;
   float m = -INFINITY;

@@ -66,6 +66,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<B_MN>::templ
     lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
                           const PairParams p) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   using C = PairCfg<B_MN>;
   constexpr int NEPI = C::template epi_warps<EPI>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];

@@ -77,6 +77,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     lora_gemm_q_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
                        const __grid_constant__ CUtensorMap tmO, const PairParams p) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   using C = QCfg<B_MN, WF>;
   constexpr bool W4 = C::W4;
   extern __shared__ __align__(1024) uint8_t smem_raw[];

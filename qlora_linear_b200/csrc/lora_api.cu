@@ -92,6 +92,35 @@ struct TimedRegion {
   }
 };
 
+// ---------------------------------------------------------------- kernel launch
+// The layer's kernels are launched with programmatic stream serialization: a kernel may
+// start launching while the previous kernel in the stream finishes (its CTA set-up
+// overlaps that kernel's tail); each waits (griddepcontrol.wait) for the previous grid to
+// complete before its first global-memory access, so the stream order of every read and
+// write is kept.  LORA_PDL=0 launches them plainly.
+bool pdl_enabled() {
+  static bool v = [] {
+    const char* e = std::getenv("LORA_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+template <typename... Params, typename... Args>
+void launch_k(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // a launch error stays pending for cudaGetLastError (last_launch) like one of <<<>>>
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------- split heuristics
 // Pure functions of the sizes, so the workspace size and the summation order are
 // fixed by the problem alone.
@@ -458,38 +487,40 @@ int finalize_grid(size_t n) {
 template <bool Q_T>
 lora_status_t launch_rowproj(const __nv_bfloat16* P, int ldp, const __nv_bfloat16* Q, float* part, int M, int Kred,
                              int r, Split sp, cudaStream_t st) {
-  dim3 grid(cdiv(M, SK_BM), sp.splits);
+  const dim3 grid(cdiv(M, SK_BM), sp.splits);
+  const int tps = sp.tiles_per_split;
   if (r <= 16)
-    rowproj_kernel<16, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<16, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
-                                                                                     sp.tiles_per_split);
+    launch_k(rowproj_kernel<16, Q_T>, grid, dim3(SK_THREADS), rowproj_smem_bytes<16, Q_T>(), st, P, ldp, Q, part, M,
+             Kred, r, tps);
   else if (r <= 32)
-    rowproj_kernel<32, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<32, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
-                                                                                     sp.tiles_per_split);
+    launch_k(rowproj_kernel<32, Q_T>, grid, dim3(SK_THREADS), rowproj_smem_bytes<32, Q_T>(), st, P, ldp, Q, part, M,
+             Kred, r, tps);
   else if (r <= 64)
-    rowproj_kernel<64, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<64, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
-                                                                                     sp.tiles_per_split);
+    launch_k(rowproj_kernel<64, Q_T>, grid, dim3(SK_THREADS), rowproj_smem_bytes<64, Q_T>(), st, P, ldp, Q, part, M,
+             Kred, r, tps);
   else
-    rowproj_kernel<128, Q_T><<<grid, SK_THREADS, rowproj_smem_bytes<128, Q_T>(), st>>>(P, ldp, Q, part, M, Kred, r,
-                                                                                       sp.tiles_per_split);
+    launch_k(rowproj_kernel<128, Q_T>, grid, dim3(SK_THREADS), rowproj_smem_bytes<128, Q_T>(), st, P, ldp, Q, part, M,
+             Kred, r, tps);
   count_launch();
   return last_launch();
 }
 
 lora_status_t launch_colproj(const __nv_bfloat16* P, int ldp, const __nv_bfloat16* R, int ldr, float* part, int M,
                              int Kout, int r, Split sp, cudaStream_t st) {
-  dim3 grid(cdiv(Kout, SK_BM), sp.splits);
+  const dim3 grid(cdiv(Kout, SK_BM), sp.splits);
+  const int tps = sp.tiles_per_split;
   if (r <= 16)
-    colproj_kernel<16><<<grid, SK_THREADS, colproj_smem_bytes<16>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
-                                                                           sp.tiles_per_split);
+    launch_k(colproj_kernel<16>, grid, dim3(SK_THREADS), colproj_smem_bytes<16>(), st, P, ldp, R, ldr, part, M, Kout,
+             r, tps);
   else if (r <= 32)
-    colproj_kernel<32><<<grid, SK_THREADS, colproj_smem_bytes<32>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
-                                                                           sp.tiles_per_split);
+    launch_k(colproj_kernel<32>, grid, dim3(SK_THREADS), colproj_smem_bytes<32>(), st, P, ldp, R, ldr, part, M, Kout,
+             r, tps);
   else if (r <= 64)
-    colproj_kernel<64><<<grid, SK_THREADS, colproj_smem_bytes<64>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
-                                                                           sp.tiles_per_split);
+    launch_k(colproj_kernel<64>, grid, dim3(SK_THREADS), colproj_smem_bytes<64>(), st, P, ldp, R, ldr, part, M, Kout,
+             r, tps);
   else
-    colproj_kernel<128><<<grid, SK_THREADS, colproj_smem_bytes<128>(), st>>>(P, ldp, R, ldr, part, M, Kout, r,
-                                                                             sp.tiles_per_split);
+    launch_k(colproj_kernel<128>, grid, dim3(SK_THREADS), colproj_smem_bytes<128>(), st, P, ldp, R, ldr, part, M, Kout,
+             r, tps);
   count_launch();
   return last_launch();
 }
@@ -515,7 +546,7 @@ lora_status_t launch_dual(const __nv_bfloat16* P, long long ldp, const __nv_bflo
     tr = tp;  // not read
   const DualParams dp{partT, partD, static_cast<int>(M), static_cast<int>(C), r, d.row_tiles, d.col_tiles, status,
                       wait_limit_ns()};
-  dualproj_kernel<MODE><<<dim3(d.a, d.b), DP_THREADS, dual_smem_bytes(), st>>>(tp, tq, tr, dp);
+  launch_k(dualproj_kernel<MODE>, dim3(d.a, d.b), dim3(DP_THREADS), dual_smem_bytes(), st, tp, tq, tr, dp);
   count_launch();
   return last_launch();
 }
@@ -541,7 +572,7 @@ lora_status_t launch_tcproj(const __nv_bfloat16* P, long long ldp, const __nv_bf
     TRY(tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Q, r, red, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, ldq));
   const TcProjParams tpp{part, static_cast<int>(rows), static_cast<int>(red), r, rpad, t.splits, t.fps, status,
                          wait_limit_ns()};
-  tcproj_kernel<MODE><<<t.tiles * t.splits, TP_THREADS, tcproj_smem_bytes(), st>>>(tp, tq, tpp);
+  launch_k(tcproj_kernel<MODE>, dim3(t.tiles * t.splits), dim3(TP_THREADS), tcproj_smem_bytes(), st, tp, tq, tpp);
   count_launch();
   return last_launch();
 }
@@ -551,7 +582,7 @@ lora_status_t launch_tcproj(const __nv_bfloat16* P, long long ldp, const __nv_bf
 lora_status_t finalize_rows(const float* part, int splits, long long rows, int r, int opitch, float scale,
                             __nv_bfloat16* out1, __nv_bfloat16* out2, cudaStream_t st) {
   const size_t n = static_cast<size_t>(rows) * r;
-  finalize_rows_kernel<<<finalize_grid(n / 2), 256, 0, st>>>(part, splits, n, r, opitch, scale, out1, out2);
+  launch_k(finalize_rows_kernel, dim3(finalize_grid(n / 2)), dim3(256), 0, st, part, splits, n, r, opitch, scale, out1, out2);
   count_launch();
   return last_launch();
 }
@@ -562,11 +593,11 @@ lora_status_t finalize_cols(const float* part, int splits, int C, int r, float s
                             bool f32, cudaStream_t st) {
   const size_t n = static_cast<size_t>(C) * r;
   if (f32)
-    finalize_cols_kernel<float><<<finalize_grid(n), 256, 0, st>>>(part, splits, C, r, scale, transpose ? 1 : 0,
-                                                                  static_cast<float*>(out));
+    launch_k(finalize_cols_kernel<float>, dim3(finalize_grid(n)), dim3(256), 0, st, part, splits, C, r, scale,
+             transpose ? 1 : 0, static_cast<float*>(out));
   else
-    finalize_cols_kernel<__nv_bfloat16><<<finalize_grid(n), 256, 0, st>>>(
-        part, splits, C, r, scale, transpose ? 1 : 0, static_cast<__nv_bfloat16*>(out));
+    launch_k(finalize_cols_kernel<__nv_bfloat16>, dim3(finalize_grid(n)), dim3(256), 0, st, part, splits, C, r, scale,
+             transpose ? 1 : 0, static_cast<__nv_bfloat16*>(out));
   count_launch();
   return last_launch();
 }
@@ -586,7 +617,8 @@ lora_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUte
   const int grid = static_cast<int>(2 * (pairs > 0 ? pairs : 1));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_pair_kernel<B_MN, EPI><<<grid, C::template threads<EPI>(), C::SMEM_BYTES, st>>>(a, b, e, f, p);
+    launch_k(lora_gemm_pair_kernel<B_MN, EPI>, dim3(grid), dim3(C::template threads<EPI>()), C::SMEM_BYTES, st, a, b,
+             e, f, p);
   }
   count_launch();
   return last_launch();
@@ -614,7 +646,8 @@ lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CU
     TRY(tmap_2d(&o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.out, p.Nout, p.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    lora_gemm_q_kernel<B_MN, WF, EPI><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, c, e, f, o, q);
+    launch_k(lora_gemm_q_kernel<B_MN, WF, EPI>, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, st, a, c, e, f, o,
+             q);
   }
   count_launch();
   return last_launch();
@@ -750,11 +783,11 @@ lora_status_t streamk_fixup(const PairParams& p, const GemmSched& g, cudaStream_
   const int group_m = g.tile_rows == 512 ? (p.group_m > 1 ? p.group_m / 2 : 1) : p.group_m;
   const dim3 grid(kGemmPairs - 1, g.tile_rows / 8);  // 8 tile rows per block
   if (g.tile_rows == 512)
-    streamk_fixup_kernel<512><<<grid, 256, 0, st>>>(p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m, g.dp_tiles,
-                                                    num_m * num_n, g.tile_fills, kGemmPairs);
+    launch_k(streamk_fixup_kernel<512>, grid, dim3(256), 0, st, p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m,
+             g.dp_tiles, num_m * num_n, g.tile_fills, kGemmPairs);
   else
-    streamk_fixup_kernel<256><<<grid, 256, 0, st>>>(p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m, g.dp_tiles,
-                                                    num_m * num_n, g.tile_fills, kGemmPairs);
+    launch_k(streamk_fixup_kernel<256>, grid, dim3(256), 0, st, p.kpart, p.out, p.M, p.Nout, num_m, num_n, group_m,
+             g.dp_tiles, num_m * num_n, g.tile_fills, kGemmPairs);
   count_launch();
   return last_launch();
 }
@@ -1247,8 +1280,8 @@ lora_status_t lora_round_bf16(const float* src, void* dst, int64_t n, void* stre
   size_t grid = (total + 255) / 256;
   const size_t cap = static_cast<size_t>(dev->sms) * 8;
   if (grid > cap) grid = cap;
-  round_bf16_kernel<<<static_cast<int>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      src, static_cast<__nv_bfloat16*>(dst), total);
+  launch_k(round_bf16_kernel, dim3(static_cast<int>(grid)), dim3(256), 0, static_cast<cudaStream_t>(stream), src,
+           static_cast<__nv_bfloat16*>(dst), total);
   count_launch();
   return last_launch();
 }
@@ -1371,9 +1404,8 @@ lora_status_t lora_ce_fwd(const void* X, int64_t M, const lora_weight_t* W, cons
   p.label_logit = zy;
   TRY((launch_gemm_w<false, EPI_CE_LSE>(W, ta, ta, FSpec{X, static_cast<uint64_t>(D), static_cast<uint64_t>(M)}, p,
                                          dev->sms, st)));
-  ce_finalize_kernel<<<cdiv(M, 256), 256, 0, st>>>(reinterpret_cast<const float2*>(ws + c.part_off),
-                                                   cdiv(V, 256), static_cast<int>(M), zy, labels, ignore_index, loss,
-                                                   lse);
+  launch_k(ce_finalize_kernel, dim3(cdiv(M, 256)), dim3(256), 0, st, reinterpret_cast<const float2*>(ws + c.part_off),
+           cdiv(V, 256), static_cast<int>(M), zy, labels, ignore_index, loss, lse);
   count_launch();
   return last_launch();
 }

@@ -13,6 +13,21 @@ namespace lora {
 constexpr uint32_t kDevErrTimeout = 1u;
 constexpr uint32_t kDevErrBounds = 2u;  // checked build: a tile or box origin out of range
 
+// Programmatic dependent launch: the library launches its layer kernels so that each
+// may start while the previous kernel in the stream finishes; every such kernel calls
+// griddep_wait() before its first global-memory access, which waits for the previous
+// grid's completion and the visibility of its writes, and then lets the next kernel
+// start launching (griddep_launch_dependents).  Both are no-ops without the launch
+// attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_enter() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

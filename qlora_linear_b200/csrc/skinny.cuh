@@ -75,6 +75,7 @@ template <int RPAD, bool Q_T>
 __global__ void __launch_bounds__(SK_THREADS)
     rowproj_kernel(const __nv_bfloat16* __restrict__ P, int ldp, const __nv_bfloat16* __restrict__ Q,
                    float* __restrict__ part, int M, int Kred, int r, int ktiles_per_split) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   using S = SkinnyCfg<RPAD>;
   constexpr int QE = Q_T ? S::QT_ELEMS : S::QN_ELEMS;
   extern __shared__ __align__(16) uint8_t sk_smem[];
@@ -161,6 +162,7 @@ template <int RPAD>
 __global__ void __launch_bounds__(SK_THREADS)
     colproj_kernel(const __nv_bfloat16* __restrict__ P, int ldp, const __nv_bfloat16* __restrict__ R, int ldr,
                    float* __restrict__ part, int M, int Kout, int r, int mtiles_per_split) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   using S = SkinnyCfg<RPAD>;
   extern __shared__ __align__(16) uint8_t sk_smem[];
   const uint32_t sbase = smem_u32(sk_smem);
@@ -241,6 +243,7 @@ __global__ void __launch_bounds__(SK_THREADS)
 // wider matrix).
 __global__ void finalize_rows_kernel(const float* __restrict__ part, int splits, size_t n, int r, int opitch,
                                      float scale, __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   for (size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x * 2) {
     const size_t o = (opitch == r) ? i : (i / r) * opitch + i % r;
@@ -264,6 +267,7 @@ __device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
 template <typename OutT>
 __global__ void finalize_cols_kernel(const float* __restrict__ part, int splits, int C, int r, float scale,
                                      int transpose, OutT* __restrict__ out) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   const size_t n = static_cast<size_t>(C) * r;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -283,6 +287,7 @@ __global__ void finalize_cols_kernel(const float* __restrict__ part, int splits,
 
 // dst = bf16_rn(src), n elements (the fp32 adapter gradients after their sum over ranks).
 __global__ void round_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     dst[i] = __float2bfloat16_rn(src[i]);

@@ -15,6 +15,7 @@ template <int TILE_ROWS>
 __global__ void __launch_bounds__(256) streamk_fixup_kernel(const float* __restrict__ kpart, __nv_bfloat16* __restrict__ out,
                                                             int M, int Nout, int num_m, int num_n, int group_m,
                                                             int dp_tiles, int ntiles, int L, int P) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   const int p = blockIdx.x + 1;
   const long long F = static_cast<long long>(ntiles - dp_tiles) * L;
   const long long b = static_cast<long long>(p) * F / P;

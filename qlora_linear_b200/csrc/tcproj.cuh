@@ -62,6 +62,7 @@ template <int MODE>
 __global__ void __launch_bounds__(TP_THREADS, 1)
     tcproj_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                   const TcProjParams p) {
+  griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   extern __shared__ __align__(1024) uint8_t tp_raw[];
   __shared__ __align__(8) uint64_t full[TP_STAGES], empty[TP_STAGES], tfull;
   __shared__ uint32_t tmem_slot, abort_s, never_s;
