@@ -49,6 +49,7 @@ struct PairParams {
   const __half* absmax;      // 4-bit: fp16 [Nw*Kw/64]
   const float* codebook;     // 4-bit: [16]
   const float* row_scale;    // 8-bit: fp32 [Nw]
+  const uint8_t* codes;      // [Nw][Kw/2] (4-bit, two codes a byte) or [Nw][Kw] (8-bit)
   int Nw, Kw;                // logical weight shape [Nw, Kw]
 };
 

@@ -24,10 +24,20 @@
 // schedule pieces of tiles, a piece being any consecutive range of the tile's code fills
 // and LoRA fills.
 //
+// Codes do not pass through shared memory.  Each dequant thread loads the 32 (4-bit) or
+// 64 (8-bit) code bytes it expands, with its block scale, into registers two of its
+// group's fills ahead, and writes the stage's B tile as soon as the MMAs of the stage's
+// previous fill have completed (the `empty` barrier the producer waits for too).  With the
+// codes in the stage's TMA load instead, every fill's expansion waited for a load issued
+// only when the stage came free, and the four-stage ring spent ~1.5k more cycles per
+// round trip than its fills' MMA time covers: two stages ran 37% slower than four, and
+// the kernel ran ~10% slower than the same kernel with the expansion skipped.
+//
 // Roles per CTA (16 warps; warp w runs on sub-partition w % 4): warp 0 TMA producer,
-// warp 1 MMA issuer (leader) and TMEM owner, warps 2-5 epilogue, warp 9 forwards the
-// dequant warps' completion of each fill to the leader, warp 13 has no role, and warps
-// 6-8, 10-12, 14-15 dequantize.  No dequant warp shares the MMA warp's sub-partition:
+// warp 1 MMA issuer (leader) and TMEM owner, warps 2-5 epilogue, warps 9 and 13 forward
+// the dequant warps' completion of each fill to the leader (one per dequant group: the
+// cluster-scope arrive holds its thread for ~1000 cycles), and warps 6-8, 10-12, 14-15
+// dequantize.  No dequant warp shares the MMA warp's sub-partition:
 // a tcgen05.mma whose issue waits for room in the tensor core's queue holds up the other
 // warps of its sub-partition, and dequant warps placed there lagged their CTA's others
 // by ~2400 cycles per fill in a timeline of the kernel (untraced: +5% on the QLoRA
@@ -50,23 +60,23 @@ struct QCfg {
   static constexpr int A_BLOCK_BYTES = HM * BK * 2;     // 16 KB
   static constexpr int A_BYTES = MB * A_BLOCK_BYTES;    // 32 KB
   static constexpr int B_BYTES = HN * BK * 2;           // 16 KB (two 8 KB MN atoms when B is MN-major)
-  static constexpr int C_BYTES = W4 ? HN * BK / 2 : HN * BK;  // codes: 4 KB (4-bit) or 8 KB (8-bit)
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int CODE_WORDS = W4 ? 2 : 4;         // 16-byte code words a dequant thread expands per fill
   static constexpr int NUM_EPI_WARPS = 4;
   static constexpr int NUM_DEQ_WARPS = 8;
   static constexpr int NUM_THREADS = 32 * 16;
-  static constexpr int FWD_WARP = 9;   // forwarder
-  static constexpr int IDLE_WARP = 13;
+  static constexpr int FWD_WARP = 9;    // forwarder of dequant group 0
+  static constexpr int FWD_WARP2 = 13;  // forwarder of dequant group 1
   // dequant warps 6,7,8,10,11,12,14,15 -> dequant index 0..7
   static __device__ __forceinline__ int deq_index(int warp) { return warp < 9 ? warp - 6 : (warp < 13 ? warp - 7 : warp - 8); }
   static constexpr int TMEM_COLS = 512;  // MB accumulators of BN fp32 columns
-  static constexpr int NUM_BARS = 5 * STAGES + 2 * MB + 1;
-  // Output staging of the store epilogue (4-bit weights; the 8-bit formats' larger code
-  // tiles leave no room): two 32-row × 32-column bf16 buffers per epilogue warp, 64-byte
-  // swizzle, written to global memory by TMA stores.
-  static constexpr bool STAGED_STORE = W4;
+  static constexpr int NUM_BARS = 4 * STAGES + 2 * MB + 1;
+  // Output staging of the store epilogue: two 32-row × 32-column bf16 buffers per epilogue
+  // warp, 64-byte swizzle, written to global memory by TMA stores.
+  static constexpr bool STAGED_STORE = true;
   static constexpr int STG_BYTES = 2048;
-  static constexpr int EPI_STG_BYTES = STAGED_STORE ? NUM_EPI_WARPS * 2 * STG_BYTES : 0;
+  static constexpr int NSTG = 2;  // staging buffers per epilogue warp (a power of two)
+  static constexpr int EPI_STG_BYTES = STAGED_STORE ? NUM_EPI_WARPS * NSTG * STG_BYTES : 0;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_STG_BYTES + 8 * NUM_BARS + 16;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -74,8 +84,8 @@ struct QCfg {
 
 template <bool B_MN, int WF, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_THREADS, 1)
-    lora_gemm_q_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
-                       const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
+    lora_gemm_q_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmE,
+                       const __grid_constant__ CUtensorMap tmF,
                        const __grid_constant__ CUtensorMap tmO, const PairParams p) {
   griddep_enter();  // the previous kernel in the stream completed (see ptx.cuh)
   using C = QCfg<B_MN, WF>;
@@ -86,9 +96,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
   uint64_t* bars = reinterpret_cast<uint64_t*>(stg_base + C::EPI_STG_BYTES);
   uint64_t* full = bars;                    // leader: TMA bytes of both CTAs landed
   uint64_t* empty = bars + C::STAGES;       // both: the pair MMA finished reading the stage
-  uint64_t* cfull = bars + 2 * C::STAGES;   // both: this CTA's code tile landed
-  uint64_t* deq = bars + 3 * C::STAGES;     // leader: both CTAs' expanded tiles written (one forward each)
-  uint64_t* tfull = bars + 4 * C::STAGES;   // both: accumulator b ready for the epilogue
+  uint64_t* deq = bars + 2 * C::STAGES;     // leader: both CTAs' expanded tiles written (one forward each)
+  uint64_t* tfull = bars + 3 * C::STAGES;   // both: accumulator b ready for the epilogue
   uint64_t* tempty = tfull + C::MB;         // leader: both CTAs drained accumulator b
   uint64_t* drain = tempty + C::MB;         // leader: final commit before TMEM release
   uint64_t* deql = drain + 1;               // both: this CTA's dequant warps wrote the stage
@@ -115,7 +124,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
-      mbar_init(smem_u32(&cfull[s]), 1);
       mbar_init(smem_u32(&deq[s]), 2);
       mbar_init(smem_u32(&deql[s]), C::NUM_DEQ_WARPS / 2);  // the stage's dequant group
     }
@@ -128,7 +136,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     *never_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmC);
     tma_prefetch_desc(&tmE);
     tma_prefetch_desc(&tmF);
     if (EPI == EPI_STORE && C::STAGED_STORE) tma_prefetch_desc(&tmO);
@@ -170,21 +177,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
           if (!lora_check(ext ? kb - nkb < n_ext : kb * C::BK < p.Kred, wc)) { ok = false; break; }
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
-          const uint32_t sC = sB + C::B_BYTES;
           const uint32_t full_l = mapa_shared(smem_u32(&full[stage]), 0);
           if (leader) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + (ext ? C::B_BYTES : 0)));
           if (!ext) {
             for (int b = 0; b < C::MB; ++b)
               tma_load_2d_pair(sA + b * C::A_BLOCK_BYTES, &tmA, full_l, kb * C::BK, arow + b * 256);
-            const uint32_t cb = smem_u32(&cfull[stage]);
-            mbar_arrive_expect_tx(cb, C::C_BYTES);
-            if (W4) {
-              if (!B_MN) tma_load_2d(sC, &tmC, cb, kb * (C::BK / 2), brow);  // 32 B × 128 rows
-              else tma_load_2d(sC, &tmC, cb, brow / 2, kb * C::BK);         // 64 B × 64 rows
-            } else {
-              if (!B_MN) tma_load_2d(sC, &tmC, cb, kb * C::BK, brow);       // 64 B × 128 rows
-              else tma_load_2d(sC, &tmC, cb, brow, kb * C::BK);             // 128 B × 64 rows
-            }
           } else {
             const int e = kb - nkb;
             int seg = 0;
@@ -199,7 +196,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
               tma_load_2d_pair(sB, &tmF, full_l, brow, e * C::ATOM);       // 64 columns × 64 ranks
               tma_load_2d_pair(sB + C::B_BYTES / 2, &tmF, full_l, brow + C::ATOM, e * C::ATOM);
             }
-            mbar_arrive(smem_u32(&cfull[stage]));  // nothing to expand in this fill
           }
           ++fills;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -212,7 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
           const int s = static_cast<int>(f % C::STAGES);
           const uint32_t ph = static_cast<uint32_t>((f / C::STAGES) & 1);
           if (leader) mbar_wait(smem_u32(&full[s]), ph, drain_wc);
-          mbar_wait(smem_u32(&cfull[s]), ph, drain_wc);
         }
       }
     }
@@ -263,7 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
   } else if (warp < 2 + C::NUM_EPI_WARPS) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-    const uint32_t stg = smem_u32(stg_base) + static_cast<uint32_t>((warp - 2) * 2 * C::STG_BYTES);
+    const uint32_t stg = smem_u32(stg_base) + static_cast<uint32_t>((warp - 2) * C::NSTG * C::STG_BYTES);
     int sb = 0;  // staging buffer of the next staged chunk
     uint32_t tphase = 0;
     bool ok = true;
@@ -300,7 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
           const int nch = min(C::BN / 32, (p.Nout - nb * C::BN + 31) / 32);  // warp-uniform
           auto stage_chunk = [&](const uint32_t (&v)[32], int c) {
             const uint32_t buf = stg + static_cast<uint32_t>(sb * C::STG_BYTES);
-            if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer
+            if (lane == 0) bulk_wait_read<C::NSTG - 1>();  // the store that last read this buffer
             __syncwarp();
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -318,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
               tma_store_2d(&tmO, buf, nb * C::BN + c * 32, row0);
               bulk_commit();
             }
-            sb ^= 1;
+            sb = (sb + 1) & (C::NSTG - 1);
           };
           if (row0 < p.M && nch > 0) {
             uint32_t va[32], vb[32];
@@ -356,14 +351,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       }
       tphase ^= 1u;
     }
-  } else if (warp == C::IDLE_WARP) {
-    // no role (keeps the dequant warps off the MMA warp's sub-partition)
-  } else if (warp == C::FWD_WARP) {
-    // ------------------------------------------------------------ forwarder (both CTAs)
-    // The dequant warps signal a CTA-local barrier (release at CTA scope); this warp turns
+  } else if (warp == C::FWD_WARP || warp == C::FWD_WARP2) {
+    // ------------------------------------------------------------ forwarders (both CTAs)
+    // The dequant warps signal a CTA-local barrier (release at CTA scope); these warps turn
     // each completed fill into the one cluster-scope release arrive the leader's MMA
-    // issuer waits for.  A release at cluster scope costs about a fill's worth of cycles
-    // when every dequant warp issues its own.
+    // issuer waits for, warp 9 for the stages of dequant group 0, warp 13 for group 1.  A
+    // release at cluster scope costs about a fill's worth of cycles when every dequant
+    // warp issues its own, and holds the forwarding thread for ~1000 cycles.
+    const int fgrp = warp == C::FWD_WARP ? 0 : 1;
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -372,8 +367,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       Unit un;
       while (ok && w.next(un)) {
         for (int kb = un.f0; kb < un.f1; ++kb) {
-          if (!mbar_wait(smem_u32(&deql[stage]), phase, wc)) { ok = false; break; }
-          mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
+          if ((stage & 1) == fgrp) {
+            if (!mbar_wait(smem_u32(&deql[stage]), phase, wc)) { ok = false; break; }
+            mbar_arrive_cluster(mapa_shared(smem_u32(&deq[stage]), 0));
+          }
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -387,6 +384,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
     //   forward:  weight row `row` (0..127) of this CTA's B rows, the fill's 64-deep slice;
     //   backward: weight row `row` (0..63) of the fill, 64-column half `h` of this CTA's 128.
     static_assert(C::STAGES % 2 == 0, "stages alternate between the two dequant groups");
+    constexpr int NW = C::CODE_WORDS;
     const int dq = C::deq_index(warp);   // 0..7
     const int grp = dq >> 2;             // 0 or 1
     const int gt = (dq & 3) * 32 + lane;  // 0..127 within the group
@@ -398,32 +396,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       for (int i = 0; i < 16; ++i) cb[i] = __ldg(p.codebook + i);
     }
     const long long kblocks_w = p.Kw / 64;  // 4-bit scale blocks per weight row
-    // scale for code fill kb of tile t, as raw bits: a fp16 block scale (4-bit) or a fp32
-    // row scale (8-bit); converted only where the fill uses it (sconv)
-    auto scale_at = [&](int t, int kb) -> uint32_t {
+    const long long row_bytes = W4 ? p.Kw / 2 : p.Kw;
+    // What this thread expands in one code fill: the scale as raw bits (a fp16 block scale
+    // for 4-bit, a fp32 row scale for 8-bit; converted only where the fill uses it) and the
+    // code bytes, the same bytes a TMA box of the fill would hold, zero outside the weight
+    // (weight rows >= Nw, columns >= Kw: 16-byte words, Kw being a multiple of 16 codes).
+    struct FillCodes {
+      uint32_t s;
+      uint4 c[NW];
+    };
+    auto fill_codes = [&](int t, int kb, FillCodes& q) {
       int mb, nb;
       pair_tile_coords(t, num_m, num_n, p.group_m, mb, nb);
       const int brow = pair_brow<EPI>(nb, rank, p);
+      // forward: weight row brow + row, bytes of the fill's 64 columns; backward: weight
+      // row kb·64 + row, bytes of this thread's 64 of the CTA's output columns
       const long long n = !B_MN ? static_cast<long long>(brow) + row : static_cast<long long>(kb) * C::BK + row;
-      if (n >= p.Nw) return 0u;
-      if (W4) {
-        const long long kblk = !B_MN ? kb : (brow + h * 64) / 64;
-        return kblk < kblocks_w
-                   ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p.absmax) + n * kblocks_w + kblk))
-                   : 0u;
+      const long long x = !B_MN ? static_cast<long long>(kb) * (NW * 16)
+                                : static_cast<long long>(W4 ? brow / 2 : brow) + h * (NW * 16);
+      const bool in_rows = n < p.Nw;
+      const uint4* src = reinterpret_cast<const uint4*>(p.codes + (in_rows ? n : 0) * row_bytes + x);
+#pragma unroll
+      for (int i = 0; i < NW; ++i)
+        q.c[i] = in_rows && x + i * 16 < row_bytes ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      q.s = 0u;
+      if (in_rows) {
+        if (W4) {
+          const long long kblk = !B_MN ? kb : (brow + h * 64) / 64;
+          if (kblk < kblocks_w)
+            q.s = static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p.absmax) + n * kblocks_w + kblk));
+        } else {
+          q.s = __float_as_uint(__ldg(p.row_scale + n));
+        }
       }
-      return __float_as_uint(__ldg(p.row_scale + n));
     };
     auto sconv = [](uint32_t b) -> float {
       return W4 ? __half2float(__ushort_as_half(static_cast<unsigned short>(b))) : __uint_as_float(b);
     };
-    // Scales are loaded two of this group's code fills ahead into named registers as raw
-    // bits: a fill's scale is read (and converted) two fills after its load was issued, and
-    // the rotation moves a value loaded one fill earlier, so no instruction waits on a fresh
+    // Codes and scales are loaded two of this group's code fills ahead into named
+    // registers: a fill's values are used two fills after their loads were issued, and the
+    // rotation moves values loaded one fill earlier, so no instruction waits on a fresh
     // global load.  (Converting the fp16 scale right at its load made every fill wait for
     // it; an indexed array would live in local memory, and storing a just-loaded value
-    // there waits for it too.)  A second walk of the units tracks the fill whose scale is
-    // loaded next: s_f counts every fill, so its parity tells the group.
+    // there waits for it too.)  A second walk of the units tracks the fill loaded next:
+    // s_f counts every fill, so its parity tells the group.
     UnitWalk sw(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
     Unit su;
     bool s_more = sw.next(su);
@@ -436,15 +452,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
         if (s_more) s_kb = su.f0;
       }
     };
-    auto load_next = [&]() -> uint32_t {
+    auto load_next = [&](FillCodes& q) {
       while (s_more && (s_kb >= nkb || static_cast<int>(s_f & 1) != grp)) s_advance();  // LoRA fills, other group
-      if (!s_more) return 0u;
-      const uint32_t v = scale_at(su.t, s_kb);
+      if (!s_more) {
+        q.s = 0u;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) q.c[i] = make_uint4(0u, 0u, 0u, 0u);
+        return;
+      }
+      fill_codes(su.t, s_kb, q);
       s_advance();
-      return v;
     };
-    uint32_t s_n1 = load_next();  // scale of this group's next code fill
-    uint32_t s_n2 = load_next();  // and of the one after
+    FillCodes n1, n2;  // this group's next code fill and the one after
+    load_next(n1);
+    load_next(n2);
     int stage = 0;
     uint32_t phase = 0;
     UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
@@ -454,47 +475,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       for (int kb = un.f0; kb < un.f1; ++kb) {
         if ((stage & 1) == grp) {
           const bool code = kb < nkb;
-          float sc = 0.f;
+          FillCodes cur;
           if (code) {
-            sc = sconv(s_n1);
-            s_n1 = s_n2;
-            s_n2 = load_next();
+            cur = n1;
+            n1 = n2;
+            load_next(n2);
           }
-          if (!mbar_wait(smem_u32(&cfull[stage]), phase, wc)) { ok = false; break; }
+          // the MMAs of the stage's previous fill completed: its B tile may be rewritten
+          // (a LoRA fill waits too, so no group runs a ring ahead of the MMA)
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wc)) { ok = false; break; }
           if (code) {
+            const float sc = sconv(cur.s);
             uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-            const uint8_t* sC = sB + C::B_BYTES;
             // destination: one 128-byte row (64 bf16, 128-byte swizzle: 16-byte unit u at
-            // u ^ (row & 7)); source: the row's 64 codes (32 bytes 4-bit, 64 bytes 8-bit)
-            uint8_t* rowp;
-            const uint8_t* cp;
-            if (!B_MN) {
-              rowp = sB + row * 128;
-              cp = W4 ? sC + row * 32 : sC + row * 64;
-            } else {
-              rowp = sB + h * (C::B_BYTES / 2) + row * 128;
-              cp = W4 ? sC + row * 64 + h * 32 : sC + row * 128 + h * 64;
+            // u ^ (row & 7))
+            uint8_t* rowp = !B_MN ? sB + row * 128 : sB + h * (C::B_BYTES / 2) + row * 128;
+            uint32_t cw[4 * NW];  // the row's codes as 32-bit words, in memory order
+#pragma unroll
+            for (int i = 0; i < NW; ++i) {
+              cw[4 * i] = cur.c[i].x;
+              cw[4 * i + 1] = cur.c[i].y;
+              cw[4 * i + 2] = cur.c[i].z;
+              cw[4 * i + 3] = cur.c[i].w;
             }
             if constexpr (W4) {
-              const uint4 c0 = *reinterpret_cast<const uint4*>(cp);
-              const uint4 c1 = *reinterpret_cast<const uint4*>(cp + 16);
               uint32_t L[4], H[4];
               block_levels(cb, sc, L, H);
-              const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
               for (int u = 0; u < 8; ++u)
                 *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) = expand8(cw[u], L, H);
             } else {
 #pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                const uint4 c0 = *reinterpret_cast<const uint4*>(cp + half * 32);
-                const uint4 c1 = *reinterpret_cast<const uint4*>(cp + half * 32 + 16);
-                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  *reinterpret_cast<uint4*>(rowp + (((half * 4 + i) ^ (row & 7)) << 4)) =
-                      expand8_w8<WF>(cw[2 * i], cw[2 * i + 1], sc);
-              }
+              for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) =
+                    expand8_w8<WF>(cw[2 * u], cw[2 * u + 1], sc);
             }
             fence_proxy_async_smem();
           }

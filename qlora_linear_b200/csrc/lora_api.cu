@@ -428,9 +428,6 @@ lora_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, co
 lora_status_t tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t bi, uint32_t br) {
   return tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, rows, bi, br, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-lora_status_t tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t bi, uint32_t br) {
-  return tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, inner, rows, bi, br, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
 
 // ---------------------------------------------------------------- validation
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -631,8 +628,8 @@ constexpr uint32_t kBoxX = 64, kBoxY = 128;
 // The weight operand's tensor map (over the stored [N, K] array, for either direction)
 // and the launch of the GEMM instantiation for the weight's format.
 template <bool B_MN, int WF, int EPI>
-lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CUtensorMap& e, const CUtensorMap& f,
-                            const PairParams& p, int sms, cudaStream_t st) {
+lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& e, const CUtensorMap& f, const PairParams& p,
+                            int sms, cudaStream_t st) {
   using C = QCfg<B_MN, WF>;
   const long long tiles = static_cast<long long>(cdiv(p.M, C::BM)) * cdiv(p.Nout, EpiTile<EPI>::COLS);
   const long long pairs = p.sk_on ? kGemmPairs : (tiles < sms / 2 ? tiles : sms / 2);
@@ -646,8 +643,7 @@ lora_status_t launch_gemm_q(const CUtensorMap& a, const CUtensorMap& c, const CU
     TRY(tmap_2d(&o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.out, p.Nout, p.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
   {
     TimedRegion tr(B_MN ? LORA_KERNEL_BWD_GEMM : LORA_KERNEL_FWD_GEMM, st);
-    launch_k(lora_gemm_q_kernel<B_MN, WF, EPI>, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, st, a, c, e, f, o,
-             q);
+    launch_k(lora_gemm_q_kernel<B_MN, WF, EPI>, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, st, a, e, f, o, q);
   }
   count_launch();
   return last_launch();
@@ -661,7 +657,7 @@ struct FSpec {
 
 // The weight operand's tensor map (over the stored [N, K] array, for either direction)
 // and the launch of the GEMM for the weight's format: the bf16 pair kernel, or the
-// quantized kernel whose code tiles are 64 deep.
+// quantized kernel, whose fills are 64 deep.
 template <bool B_MN, int EPI>
 lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const CUtensorMap& e, const FSpec& fs,
                             const PairParams& p, int sms, cudaStream_t st) {
@@ -676,18 +672,13 @@ lora_status_t launch_gemm_w(const lora_weight_t* W, const CUtensorMap& a, const 
       TRY(tmap_bf16(&b, W->data, W->K, W->N, kBoxX, kBoxY));
       return launch_gemm<B_MN, EPI>(a, b, e, f, p, sms, st);
     }
-    // the quantized kernel's backward LoRA fill takes 64 ranks per box
+    // the quantized kernel's backward LoRA fill takes 64 ranks per box; its dequant
+    // threads load the codes themselves (PairParams::codes)
     if (B_MN) TRY(tmap_bf16(&f, fs.base, fs.inner, fs.rows, kBoxX, 64));
-    const bool w4 = W->fmt == LORA_W_BLOCK4;
-    const uint64_t row_bytes = w4 ? W->K / 2 : W->K;
-    // code boxes: forward 128 weight rows × one 64-deep fill; backward 64 weight rows × 128 columns
-    const uint32_t bx = B_MN ? (w4 ? 64 : 128) : (w4 ? 32 : 64);
-    const uint32_t by = B_MN ? 64 : 128;
-    TRY(tmap_u8(&b, W->data, row_bytes, W->N, bx, by));
     switch (W->fmt) {
-      case LORA_W_BLOCK4: return launch_gemm_q<B_MN, WF_BLOCK4, EPI>(a, b, e, f, p, sms, st);
-      case LORA_W_INT8: return launch_gemm_q<B_MN, WF_INT8, EPI>(a, b, e, f, p, sms, st);
-      default: return launch_gemm_q<B_MN, WF_FP8, EPI>(a, b, e, f, p, sms, st);
+      case LORA_W_BLOCK4: return launch_gemm_q<B_MN, WF_BLOCK4, EPI>(a, e, f, p, sms, st);
+      case LORA_W_INT8: return launch_gemm_q<B_MN, WF_INT8, EPI>(a, e, f, p, sms, st);
+      default: return launch_gemm_q<B_MN, WF_FP8, EPI>(a, e, f, p, sms, st);
     }
   }
 }
@@ -751,6 +742,7 @@ PairParams gemm_params(long long M, long long Nout, long long Kred, int r, void*
   for (int g = 0; g < LORA_MAX_SEGMENTS; ++g) p.seg_end_tile[g] = 0x7fffffff;
   p.Nw = static_cast<int>(W->N);
   p.Kw = static_cast<int>(W->K);
+  p.codes = W->fmt != LORA_W_BF16 ? static_cast<const uint8_t*>(W->data) : nullptr;
   if (W->fmt == LORA_W_BLOCK4) {
     p.absmax = static_cast<const __half*>(W->absmax);
     p.codebook = W->codebook;
