@@ -192,13 +192,16 @@ size_t dual_part_bytes(const DualSplit& d, long long M, long long C, int r) {
 // Schedule of a GEMM launch.  Whole tiles round-robin over the CTA pairs leave pairs
 // idle in the last wave when the tile count is not a multiple of the pairs (an output of
 // 1.5 waves runs two full ones).  Stream-K evens that out: every pair first runs the same
-// number of whole tiles (all waves but the last full one), then an equal share of the
-// fills of the remaining tiles, pieces of tiles going to fp32 slots that a second kernel
-// adds in pair order (deterministic).  The choice is a pure function of the sizes, the
-// rank and the weight's format (its tile shape), made against a fixed 74 pairs, so the
-// workspace size follows from the sizes alone.  Cost model: fills per pair at the
-// kernel's per-pair rate (plus three for the extra epilogue of a piece), slots written
-// and read back at 5 TB/s, and the fixup launch; stream-K must save a twentieth.
+// number of whole tiles, then an equal share of the fills of the remaining tiles, pieces
+// of tiles going to fp32 slots that a second kernel adds in pair order (deterministic).
+// The whole tiles are either all full waves (only the partial last wave is cut) or all
+// full waves but one (the last full wave is cut too, for longer ranges); of the two the
+// model takes the cheaper.  The choice is a pure function of the sizes, the rank and the
+// weight's format (its tile shape), made against a fixed 74 pairs, so the workspace size
+// follows from the sizes alone.  Cost model: fills per pair at the kernel's per-pair
+// rate (plus three for the extra epilogue of a piece), slots (about one per cut tile and
+// one per pair) written and read back at 5 TB/s, and the fixup launch; stream-K must
+// save 3%, and every pair's range holds at least four fills.
 constexpr int kGemmPairs = 74;
 struct GemmSched {
   bool sk = false;
@@ -216,17 +219,21 @@ GemmSched gemm_sched(long long M, long long Nout, long long Kred, int r, bool qu
   g.tile_fills = static_cast<int>(L);
   const int P = kGemmPairs;
   const long long full = tiles / P;
-  const long long dp = full > 1 ? (full - 1) * P : 0;
-  const long long rest = tiles - dp;
-  if (rest * L < 8LL * P) return g;  // every pair's range must hold at least 8 fills
-  const double fill_s = 2.0 * g.tile_rows * 256 * bk / ((quantized ? 1.0e15 : 1.5e15) / P);
+  const double fill_s = 2.0 * g.tile_rows * 256 * bk / ((quantized ? 1.2e15 : 1.5e15) / P);
   const double slot_bytes = double(g.tile_rows) * 256 * 4;
   const double t_dp = double((tiles + P - 1) / P) * L * fill_s;
-  const double t_sk = (double(dp / P) * L + double((rest * L + P - 1) / P) + 3.0) * fill_s +
-                      2.0 * double(rest + P) * slot_bytes / 5.0e12 + 4.0e-6;
-  if (t_sk < 0.95 * t_dp) {
-    g.sk = true;
-    g.dp_tiles = static_cast<int>(dp);
+  double best = 0.97 * t_dp;
+  for (long long waves = full > 1 ? full - 1 : 0; waves <= full; ++waves) {
+    const long long dp = waves * P;
+    const long long rest = tiles - dp;
+    if (rest <= 0 || rest * L < 4LL * P) continue;
+    const double t_sk = (double(waves) * L + double((rest * L + P - 1) / P) + 3.0) * fill_s +
+                        2.0 * double(rest + P) * slot_bytes / 5.0e12 + 4.0e-6;
+    if (t_sk < best) {
+      best = t_sk;
+      g.sk = true;
+      g.dp_tiles = static_cast<int>(dp);
+    }
   }
   return g;
 }

@@ -96,7 +96,7 @@ def test_streamk_walk_covers_every_fill_once(M, Nout, Kred, r, fmt):
         pytest.skip("whole tiles for this shape")
     dp_tiles = ntiles - shared
     assert 0 <= dp_tiles < ntiles and dp_tiles % PAIRS == 0
-    assert shared * L >= 8 * PAIRS  # every pair's range holds fills (the kernels need one or more)
+    assert shared * L >= 4 * PAIRS  # every pair's range holds four fills or more (the kernels need one)
 
     cover = {t: [] for t in range(ntiles)}
     for p in range(PAIRS):
