@@ -132,17 +132,20 @@ def test_workspace_bytes_is_a_pure_function_of_sizes():
 def test_gemm_streamk_only_where_the_last_wave_leaves_pairs_idle():
     k = q.lora_testing_gemm_streamk
     B4, I8 = q.LORA_W_BLOCK4, q.LORA_W_INT8
-    # the rank sweep's 512-token shapes with quantized weights: 32 or 112 tiles of
-    # 512 x 256 for 74 CTA pairs, all shared out as pieces
-    assert k(512, 8192, 8192, 16, B4) == 32 and k(512, 28672, 8192, 16, B4) == 112
+    # the rank sweep's 512-token shapes with quantized weights: 32 tiles of 512 x 256 for
+    # 74 CTA pairs, all shared out as pieces; 112 tiles: one wave whole, 38 as pieces
+    assert k(512, 8192, 8192, 16, B4) == 32 and k(512, 28672, 8192, 16, B4) == 112 - 74
     assert k(512, 8192, 28672, 16, B4) == 32 and k(512, 8192, 8192, 16, I8) == 32
-    # the QLoRA dX GEMM: 256 tiles = 3.46 waves; two waves whole, 108 tiles as pieces
-    assert k(8192, 4096, 14336, 16, B4) == 256 - 148
+    # the QLoRA dX GEMM: 256 tiles = 3.46 waves; three waves whole, the last 34 tiles as
+    # pieces (fewer fp32 slots than cutting the third wave too)
+    assert k(8192, 4096, 14336, 16, B4) == 256 - 222
+    # the QLoRA Y GEMM: 896 tiles = 12.1 waves; the 8 tiles of the partial wave as pieces
+    assert k(8192, 14336, 4096, 16, B4) == 8
     # bf16 at 512 tokens and N = 28672: 224 tiles, 76 as pieces; N = 8192: 64 tiles, whole
     assert k(512, 28672, 8192, 16) == 76 and k(512, 8192, 8192, 16) == 0
     # many waves, or too little work per pair: whole tiles
     assert k(16384, 14336, 4096, 16) == 0 and k(16384, 4096, 14336, 16) == 0 and k(8192, 4096, 4096, 16) == 0
-    assert k(8192, 14336, 4096, 16, B4) == 0 and k(256, 512, 512, 8) == 0
+    assert k(256, 512, 512, 8) == 0
     assert k(512, 8192, 8192, 16, 9) == -1 and k(512, 8192, 8192, 129, 0) == -1
     # the workspace holds the schedule's fp32 slots: two tiles of 512 x 256 per pair
     assert q.workspace_bytes(512, 8192, 8192, 16, B4) >= 256 + 2 * 74 * 512 * 256 * 4
