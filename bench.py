@@ -689,25 +689,20 @@ def gemm_roofline(cases, ce, steps, fwd_ms, bwd_ms, g_launches, step_ms, peaks, 
     """Roofline of the dominant kernel, the tcgen05 GEMM (its Y and dX launches):
     algorithmic FLOPs of those launches over their summed CUDA-event time, against the
     measured dense bf16 peak.  `frac` is always against the burst peak (the GEMM is timed
-    inside a region of well under a minute); the sustained peak and a clock-normalised
-    figure (the same launches at the maximum SM clock, time x median MHz / max MHz) are
-    reported beside it."""
+    inside a region of well under a minute); the fraction of the sustained peak is reported
+    beside it.  (No clock-scaled figure: the median of sampled SM clocks misses the power
+    limiter's short slowdowns, and scaling by it overstates the rate at the top clock.)"""
     gflops = (ce_flops(cases[0]) if ce else sum(sum(gemm_flops(c)) for c in cases)) * steps
     g_ms = fwd_ms + bwd_ms
     achieved = gflops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    at_max = None
-    if achieved and clk and clk.get("sm_mhz"):
-        at_max = achieved * clk["sm_max_mhz"] / clk["sm_mhz"]
     return {
         "bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
         "frac": achieved / peak_burst if achieved else None,
         "peak_source": "bf16_tflops (burst) of MEASURED_PEAKS.json" if "bf16_tflops" in peaks
                        else "fallback burst figure",
         "frac_of_sustained": achieved / peak_sust if achieved else None,
-        "achieved_at_max_clock": at_max,
-        "frac_at_max_clock": at_max / peak_burst if at_max else None,
         "launches": g_launches, "avg_launch_ms": g_ms / g_launches if g_launches else None,
         "gemm_share_of_step": g_ms / (step_ms * steps) if step_ms > 0 else None,
     }

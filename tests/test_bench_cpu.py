@@ -56,7 +56,7 @@ def test_roofline_frac_is_against_burst_peak():
     assert abs(r["achieved"] - 1200.0) < 1e-6
     assert r["peak"] == 1600.0 and abs(r["frac"] - 0.75) < 1e-12  # power cap seen: still the burst peak
     assert abs(r["frac_of_sustained"] - 1200.0 / 1400.0) < 1e-12
-    assert abs(r["achieved_at_max_clock"] - 1200.0 * 1965.0 / 1500.0) < 1e-6
+    assert "achieved_at_max_clock" not in r
     assert abs(r["gemm_share_of_step"] - g_ms / 10.0) < 1e-12
 
 
