@@ -221,34 +221,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(QCfg<B_MN, WF>::NUM_
       bool ok = true;
       UnitWalk w(pair, npairs, ntiles, tile_fills, sk, p.sk_dp_tiles);
       Unit un;
-      while (ok && w.next(un)) {
-        for (int kb = un.f0; kb < un.f1; ++kb) {
-          if (!mbar_wait(smem_u32(&full[stage]), phase, wc)) { ok = false; break; }
-          if (!mbar_wait<true>(smem_u32(&deq[stage]), phase, wc)) { ok = false; break; }
+      // the MMAs of one fill into accumulator b (the fill's first MMA overwrites it when the
+      // fill is the unit's first)
+      auto issue = [&](int st, int kb, int b, bool first_fill) {
+        const bool ext = kb >= nkb;
+        const uint32_t sA = smem_u32(smem + st * C::STAGE_BYTES);
+        const uint32_t sB = sA + C::A_BYTES;
+        const int nk = ext ? min(C::BK / 16, (p.r - (kb - nkb) * C::ATOM + 15) / 16) : C::BK / 16;
+        const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::BN);
+        for (int k = 0; k < nk; ++k) {
+          const uint64_t ad = sdesc_sw128(sA + b * C::A_BLOCK_BYTES + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? sdesc_sw128(sB + k * 2048, C::B_BYTES / 2, 1024) : sdesc_sw128(sB + k * 32, 16, 1024);
+          tc_mma_bf16_pair(d, ad, bd, idesc, (!first_fill || k > 0) ? 1u : 0u);
+        }
+      };
+      auto ready = [&](int st, uint32_t ph) -> bool {  // the fill's tiles of both CTAs are in place
+        if (!mbar_wait(smem_u32(&full[st]), ph, wc)) return false;
+        if (!mbar_wait<true>(smem_u32(&deq[st]), ph, wc)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto advance = [](int& st, uint32_t& ph) {
+        if (++st == C::STAGES) { st = 0; ph ^= 1u; }
+      };
+      // A unit's first and last fills (up to a stage ring's worth each) are issued one
+      // accumulator at a time.  First fills: accumulator 0's MMAs of all of them start as
+      // soon as the epilogue has drained accumulator 0 of the previous tile, while it still
+      // drains accumulator 1.  Last fills: accumulator 0 is complete, and handed to the
+      // epilogue, while accumulator 1's last MMAs still run.  Fills in between alternate the
+      // accumulators fill by fill and release each stage at once.  Each accumulator sums its
+      // fills in the same order either way.
+      auto group = [&](int lo, int hi, bool first, bool last) -> bool {
+        int st = stage;
+        uint32_t ph = phase;
+        if (first) {
+          if (!mbar_wait<true>(smem_u32(&tempty[0]), tphase ^ 1u, wc)) return false;
           tc_fence_after();
-          const bool ext = kb >= nkb;
-          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
-          const int nk = ext ? min(C::BK / 16, (p.r - (kb - nkb) * C::ATOM + 15) / 16) : C::BK / 16;
-          for (int b = 0; b < C::MB; ++b) {
-            if (kb == un.f0) {
-              // the epilogue must have drained accumulator b of the previous tile
-              if (!mbar_wait<true>(smem_u32(&tempty[b]), tphase ^ 1u, wc)) { ok = false; break; }
-              tc_fence_after();
-            }
-            const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::BN);
-            for (int k = 0; k < nk; ++k) {
-              const uint64_t ad = sdesc_sw128(sA + b * C::A_BLOCK_BYTES + k * 32, 16, 1024);
-              const uint64_t bd = B_MN ? sdesc_sw128(sB + k * 2048, C::B_BYTES / 2, 1024) : sdesc_sw128(sB + k * 32, 16, 1024);
-              tc_mma_bf16_pair(d, ad, bd, idesc, (kb > un.f0 || k > 0) ? 1u : 0u);
-            }
-          }
-          if (!ok) break;
+        }
+        for (int j = lo; j < hi; ++j) {
+          if (!ready(st, ph)) return false;
+          issue(st, un.f0 + j, 0, j == 0);
+          advance(st, ph);
+        }
+        if (last) tc_commit_pair_mc(smem_u32(&tfull[0]), 0x3);
+        if (first) {
+          if (!mbar_wait<true>(smem_u32(&tempty[1]), tphase ^ 1u, wc)) return false;
+          tc_fence_after();
+        }
+        for (int j = lo; j < hi; ++j) {
+          issue(stage, un.f0 + j, 1, j == 0);
           tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          advance(stage, phase);
+        }
+        if (last) tc_commit_pair_mc(smem_u32(&tfull[1]), 0x3);
+        return true;
+      };
+      static_assert(C::MB == 2, "the issue order is written for two accumulators");
+      while (ok && w.next(un)) {
+        const int n = un.f1 - un.f0;
+        const int g0 = min(n, C::STAGES);          // first fills [0, g0)
+        const int g1 = max(g0, n - C::STAGES);     // last fills [g1, n)
+        if (!group(0, g0, true, g0 == n)) { ok = false; break; }
+        for (int j = g0; j < g1; ++j) {
+          if (!ready(stage, phase)) { ok = false; break; }
+          issue(stage, un.f0 + j, 0, false);
+          issue(stage, un.f0 + j, 1, false);
+          tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
+          advance(stage, phase);
         }
         if (!ok) break;
-        for (int b = 0; b < C::MB; ++b) tc_commit_pair_mc(smem_u32(&tfull[b]), 0x3);
+        if (g1 < n && !group(g1, n, false, true)) { ok = false; break; }
         tphase ^= 1u;
       }
       tc_commit_pair(smem_u32(drain));
