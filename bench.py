@@ -131,6 +131,7 @@ def cpu_threads() -> int:
 # ---------------------------------------------------------------------------- clocks
 REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 MIN_CLOCK_SAMPLES = 10
+CASE_GAP_S = 1.0  # idle time before each case of the rank sweep
 
 
 class ClockSampler:
@@ -153,6 +154,7 @@ class ClockSampler:
         self.stop_ev = threading.Event()
         self.source = None
         self.marks = {}
+        self.idle_spans = []
 
     def start(self):
         try:
@@ -211,6 +213,12 @@ class ClockSampler:
     def mark(self, which: str):
         self.marks[which] = time.time()
 
+    def idle(self, seconds: float):
+        """Sleeps with the GPU idle; the summaries leave the samples of that time out."""
+        t0 = time.time()
+        time.sleep(seconds)
+        self.idle_spans.append((t0, time.time()))
+
     def count_since(self, which: str) -> int:
         t0 = self.marks.get(which, 0.0)
         return sum(1 for s in list(self.samples) if s[0] >= t0)
@@ -233,11 +241,15 @@ class ClockSampler:
         if not self.samples:
             return None
         t0, t1 = self.marks.get(t0_mark, 0.0), self.marks.get(t1_mark, float("inf"))
-        win = [s for s in self.samples if t0 <= s[0] <= t1]
+
+        def busy(s):
+            return not any(a <= s[0] <= b for a, b in self.idle_spans)
+
+        win = [s for s in self.samples if t0 <= s[0] <= t1 and busy(s)]
         window = "timed region"
         if len(win) < MIN_CLOCK_SAMPLES and wide_mark is not None:
             tw = self.marks.get(wide_mark, t0)
-            win = [s for s in self.samples if tw <= s[0] <= t1]
+            win = [s for s in self.samples if tw <= s[0] <= t1 and busy(s)]
             window = "warm-up and timed region (the timed region alone held fewer than " \
                      f"{MIN_CLOCK_SAMPLES} samples)"
         if not win:
@@ -740,9 +752,12 @@ def time_steps(q, torch, step, steps, stream, flush_buf=None):
 def run_sweep(args, cases, desc, rank, world, local_rank):
     """The rank sweep (one projection per case): each case is built, warmed up and timed
     on its own (forward + backward per step, L2 flushed before every step, outside the
-    step's events), then freed.  The line's value is the algorithmic FLOPs of one pass
-    over every selected case divided by the sum of their per-step times; `sweep` lists
-    each case."""
+    step's events), then freed.  Each case starts after the GPU has been idle for
+    CASE_GAP_S, so a small case does not inherit the clock the power limiter holds after a
+    large one (measured: the 512-token 4-bit cases ran at half speed right after the
+    16384-token cases, and at full speed on their own).  The line's value is the
+    algorithmic FLOPs of one pass over every selected case divided by the sum of their
+    per-step times; `sweep` lists each case."""
     import torch
     import torch.distributed as dist
 
@@ -761,6 +776,8 @@ def run_sweep(args, cases, desc, rank, world, local_rank):
     clocks.mark("t_warm")
     clocks.mark("t_start")
     for c in cases:
+        torch.cuda.synchronize()
+        clocks.idle(CASE_GAP_S)
         ws = LinearSet([c], dev, rank, world)
         for _ in range(args.warmup):
             ws.step()

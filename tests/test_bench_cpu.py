@@ -78,6 +78,21 @@ def test_clock_summary_window_opens_to_warmup_when_short():
     assert d["window"] == "timed region" and d["samples"] == 17
 
 
+def test_clock_summary_leaves_idle_gaps_out():
+    b = _bench()
+    s = b.ClockSampler("GPU-x")
+    s.source = "nvml"
+    s.marks = {"t_start": 0.0, "t_end": 3.0}
+    # loaded samples at 1500 MHz, idle ones (between sweep cases) at the top clock
+    s.samples = [(0.01 * i, 1500.0, 1965.0, 950.0, {"sw_power_cap"}) for i in range(100)]
+    s.samples += [(1.0 + 0.01 * i, 1965.0, 1965.0, 120.0, set()) for i in range(150)]
+    s.samples += [(2.5 + 0.01 * i, 1400.0, 1965.0, 990.0, {"sw_power_cap"}) for i in range(50)]
+    s.idle_spans = [(0.995, 2.495)]
+    d = s.summary("t_start", "t_end")
+    assert d["samples"] == 150 and d["samples_power_capped"] == 150
+    assert d["sm_mhz"] == 1500.0 and d["power_w_max"] == 990.0
+
+
 def test_select_cases_filters_the_rank_sweep():
     b = _bench()
     from synth import CONFIGS
