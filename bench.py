@@ -357,9 +357,11 @@ def traffic_record():
 
 
 def source_hash() -> str:
+    """Hash of the sources the bf16 GEMM (the kernel of the traffic record) and its launch
+    are built from; the record counts only while they are unchanged."""
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemm_common.cuh", "gemm_pair.cuh", "gemm_q.cuh", "dequant.cuh", "ptx.cuh", "lora_api.cu"):
+    for f in ("gemm_common.cuh", "gemm_pair.cuh", "ptx.cuh", "lora_api.cu"):
         with open(os.path.join(ROOT, "qlora_linear_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -916,7 +918,8 @@ def run_ours(args, cases, desc, rank, world, local_rank):
                           "lora_gemm_pair_kernel / lora_gemm_q_kernel") + " (Y and dX GEMMs)"
     tr = traffic_record()
     roofline["traffic"] = None
-    if tr and tr.get("source_hash") == source_hash() and tr.get("workload") == args.workload:
+    if tr and tr.get("source_hash") == source_hash() and tr.get("workload") == args.workload and \
+            args.weight in (None, "bf16") and not args.rank and not args.only:
         roofline["traffic"] = tr.get("bytes_per_launch")
 
     # ---- grouped workloads: the same projections as separate layers, for comparison
